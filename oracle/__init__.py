@@ -1,0 +1,10 @@
+"""fp64 CPU oracle for low-rank compressed-KV decode attention.
+
+Test infrastructure only: ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline / reference arm may import it; the CUDA library
+and its Python binding never do.
+"""
+from .bf16 import bf16_round, bf16_bits, bf16_from_bits, bf16_ulp
+from .lrkv_oracle import (Dims, Cache, project, reconstruct, rel_error, route,
+                          compress, effective_kv, softmax, decode_attn,
+                          decode_attn_coef, FULL_OVERFLOW, SEQ_OVERFLOW)
