@@ -1,1 +1,180 @@
-"""Low-rank compressed-KV decode attention on B200 (placeholder; binding follows)."""
+"""Low-rank compressed-KV decode attention for NVIDIA B200 (sm_100a).
+
+A thin Python binding over the C ABI of ``liblrkv.so`` (declared in
+``include/lrkv.h``).  It only marshals arguments: PyTorch supplies device
+memory and the stream, every step of the computation runs in the library's
+CUDA kernels, and there is no CPU fallback -- importing works without a
+GPU, but every compute call needs the built library and a CUDA device.
+
+Entry points (same names as the C ABI):
+    lrkv_workspace_size(dims) -> int
+    lrkv_compress(dims, cache, k_new, v_new, tau, t_new_b=None, err_out=None, ws=...)
+    lrkv_decode_attn(dims, cache, q, out, ws=...)
+    lrkv_status_str(code) -> str
+plus ``LayerCache`` (allocates one layer's buffers with torch) and
+``make_workspace``.
+"""
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+from . import accounting  # noqa: F401  (host-side byte accounting)
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblrkv.so")
+
+LRKV_OK = 0
+STATUS_NAMES = {0: "LRKV_OK", 1: "LRKV_ERR_INVALID_ARG", 2: "LRKV_ERR_UNSUPPORTED",
+                3: "LRKV_ERR_ALIGNMENT", 4: "LRKV_ERR_CUDA"}
+DEV_FULL_OVERFLOW = 0x1
+DEV_SEQ_OVERFLOW = 0x2
+DEV_BAD_COUNT = 0x4
+
+
+class LrkvError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)} ({lrkv_status_str(code)})")
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hq", "Hkv", "d", "r_k", "r_v", "T_cap", "F_cap")]
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "U_k", "U_v", "coef_k", "coef_v", "route_mask", "full_idx", "full_k", "full_v",
+        "full_cnt", "seq_len", "dev_status")]
+
+
+_lib = None
+
+
+def load_library(path=None):
+    """Load liblrkv.so (built in-tree).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: build it with `python -m decode_attention_lrkv_b200.build`")
+    lib = ctypes.CDLL(p)
+    P = ctypes.c_void_p
+    lib.lrkv_workspace_size.argtypes = [ctypes.POINTER(_Dims)]
+    lib.lrkv_workspace_size.restype = ctypes.c_size_t
+    lib.lrkv_compress.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Cache), P, P,
+                                  ctypes.c_int32, P, ctypes.c_float, P, P, ctypes.c_size_t, P]
+    lib.lrkv_compress.restype = ctypes.c_int
+    lib.lrkv_decode_attn.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Cache), P, P, P,
+                                     ctypes.c_size_t, P]
+    lib.lrkv_decode_attn.restype = ctypes.c_int
+    lib.lrkv_status_str.argtypes = [ctypes.c_int]
+    lib.lrkv_status_str.restype = ctypes.c_char_p
+    if path is None:
+        _lib = lib
+    return lib
+
+
+@dataclass(frozen=True)
+class Dims:
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    r_k: int
+    r_v: int
+    T_cap: int
+    F_cap: int
+
+    @property
+    def g(self):
+        return self.Hq // self.Hkv
+
+    def c(self):
+        return _Dims(self.B, self.Hq, self.Hkv, self.d, self.r_k, self.r_v, self.T_cap, self.F_cap)
+
+
+class LayerCache:
+    """One layer of compressed cache as torch tensors, in the C ABI's layout.
+
+    bf16 tensors: U_k [Hkv,d,r_k], U_v [Hkv,d,r_v], coef_k [B,Hkv,T_cap,r_k],
+    coef_v [B,Hkv,T_cap,r_v], full_k/full_v [B,Hkv,F_cap,d];
+    int32: route_mask [B,Hkv,T_cap/32] (bit patterns), full_idx [B,Hkv,F_cap],
+    full_cnt [B,Hkv], seq_len [B]; dev_status int32 [4] (word 0 used).
+    """
+    FIELDS = ("U_k", "U_v", "coef_k", "coef_v", "route_mask", "full_idx", "full_k", "full_v",
+              "full_cnt", "seq_len", "dev_status")
+
+    def __init__(self, dims, U_k, U_v, device="cuda"):
+        D = dims
+        self.dims = D
+        z = lambda *s, dt=torch.bfloat16: torch.zeros(*s, dtype=dt, device=device)
+        self.U_k = U_k.to(device=device, dtype=torch.bfloat16).contiguous()
+        self.U_v = U_v.to(device=device, dtype=torch.bfloat16).contiguous()
+        assert tuple(self.U_k.shape) == (D.Hkv, D.d, D.r_k) and tuple(self.U_v.shape) == (D.Hkv, D.d, D.r_v)
+        self.coef_k = z(D.B, D.Hkv, D.T_cap, D.r_k)
+        self.coef_v = z(D.B, D.Hkv, D.T_cap, D.r_v)
+        self.route_mask = z(D.B, D.Hkv, D.T_cap // 32, dt=torch.int32)
+        self.full_idx = z(D.B, D.Hkv, max(D.F_cap, 1), dt=torch.int32)
+        self.full_k = z(D.B, D.Hkv, max(D.F_cap, 1), D.d)
+        self.full_v = z(D.B, D.Hkv, max(D.F_cap, 1), D.d)
+        self.full_cnt = z(D.B, D.Hkv, dt=torch.int32)
+        self.seq_len = z(D.B, dt=torch.int32)
+        self.dev_status = z(4, dt=torch.int32)
+
+    def c(self):
+        return _Cache(*[getattr(self, f).data_ptr() for f in self.FIELDS])
+
+    def nbytes(self):
+        return sum(getattr(self, f).numel() * getattr(self, f).element_size() for f in self.FIELDS)
+
+
+def lrkv_status_str(code):
+    return load_library().lrkv_status_str(int(code)).decode()
+
+
+def lrkv_workspace_size(dims):
+    return int(load_library().lrkv_workspace_size(ctypes.byref(dims.c())))
+
+
+def make_workspace(dims, device="cuda"):
+    """A zero-filled workspace tensor of lrkv_workspace_size(dims) bytes."""
+    n = lrkv_workspace_size(dims)
+    if n == 0:
+        raise ValueError(f"invalid dims {dims}")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def lrkv_compress(dims, cache, k_new, v_new, tau, t_new_b=None, err_out=None, ws=None,
+                  stream=None, check=True):
+    """Append k_new/v_new [B,t_new,Hkv,d] (bf16, device) to ``cache``; see include/lrkv.h."""
+    lib = load_library()
+    t_new = int(k_new.shape[1])
+    code = lib.lrkv_compress(ctypes.byref(dims.c()), ctypes.byref(cache.c()), _ptr(k_new),
+                             _ptr(v_new), t_new, _ptr(t_new_b), float(tau), _ptr(err_out),
+                             _ptr(ws), 0 if ws is None else ws.numel(), _stream_ptr(stream))
+    if check and code != LRKV_OK:
+        raise LrkvError(code, "lrkv_compress")
+    return code
+
+
+def lrkv_decode_attn(dims, cache, q, out, ws=None, stream=None, check=True):
+    """out [B,Hq,d] fp32 <- decode attention of q [B,Hq,d] (bf16) over ``cache``."""
+    lib = load_library()
+    code = lib.lrkv_decode_attn(ctypes.byref(dims.c()), ctypes.byref(cache.c()), _ptr(q), _ptr(out),
+                                _ptr(ws), 0 if ws is None else ws.numel(), _stream_ptr(stream))
+    if check and code != LRKV_OK:
+        raise LrkvError(code, "lrkv_decode_attn")
+    return code

@@ -1,0 +1,155 @@
+/*
+ * lrkv.h -- C ABI of liblrkv.so: low-rank compressed-KV decode attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (one transformer layer per call):
+ *
+ *   Write path -- OjaKV repository README, "Method Summary > StaticPCA"
+ *   (a fixed offline per-head basis) and "Method Summary > OjaKV" (hybrid
+ *   storage: tokens with a high reconstruction error stay in full rank, the
+ *   rest are compressed).  For every new token t of kv head h:
+ *       c_k = U_k[h]^T k_t,  c_v = U_v[h]^T v_t             (fp32 accumulate)
+ *       e_k = ||k_t - U_k c_k|| / ||k_t||,  e_v likewise,  e_t = max(e_k, e_v)
+ *       the coefficients are stored as bf16 (round to nearest even) at the
+ *       token's position; if e_t > tau the token is also appended, in
+ *       ascending position order, to the full-rank list (its k and v rows
+ *       copied) and its route-mask bit is set.
+ *
+ *   Read path -- decode attention directly over the compressed cache, the
+ *   coefficient-space form of "reconstruct on the fly, then attend":
+ *       q~_h = U_k^T q_h
+ *       s_t  = q~_h . c_k,t / sqrt(d)   (t compressed)
+ *       s_t  = q_h  . k_t   / sqrt(d)   (t full rank)
+ *       p    = softmax over all tokens of the sequence, both sets together
+ *       o_h  = U_v sum_{t compressed} p_t c_v,t + sum_{t full} p_t v_t
+ *   Query head h reads kv head floor(h / g), g = Hq / Hkv (grouped-query).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, caller-allocated and
+ *     caller-owned; the library never allocates, frees or synchronises.
+ *     All work is enqueued on the given stream (a cudaStream_t passed as
+ *     void*; NULL is the legacy default stream).
+ *   - bf16 values are raw bfloat16 bit patterns (uint16_t), row-major,
+ *     densely packed in the shapes given below.
+ *   - Every pointer must be 16-byte aligned.
+ *   - Synchronous errors (returned, nothing launched): null pointers, d != 128,
+ *     r_k or r_v not a multiple of 16 or outside [16, d], Hq % Hkv != 0,
+ *     T_cap not a positive multiple of 32, F_cap < 0, workspace too small,
+ *     misaligned pointers, a launch failure (LRKV_ERR_CUDA).
+ *   - Asynchronous conditions are OR-ed into *dev_status (device word),
+ *     read by the caller after synchronising; kernels never trap.
+ *   - A sequence with no tokens attends to nothing: its output rows are 0.
+ *   - Non-finite inputs give undefined (but memory-safe) results.
+ *   - Two calls that share a cache or a workspace must not overlap in time
+ *     (issue them on one stream, or order them with events).
+ */
+#ifndef LRKV_H
+#define LRKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LRKV_API __attribute__((visibility("default")))
+#else
+#define LRKV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t lrkv_bf16; /* raw bfloat16 bits */
+
+typedef enum {
+  LRKV_OK = 0,
+  LRKV_ERR_INVALID_ARG = 1, /* null pointer, bad size, workspace too small */
+  LRKV_ERR_UNSUPPORTED = 2, /* a shape this build does not handle (d != 128, ...) */
+  LRKV_ERR_ALIGNMENT = 3,   /* a pointer not 16-byte aligned */
+  LRKV_ERR_CUDA = 4         /* a CUDA launch failed; cudaGetLastError() was cleared */
+} lrkv_status;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define LRKV_DEV_FULL_OVERFLOW 0x1u /* a routed token found the full-rank list full: it was
+                                       kept compressed (mask bit clear) instead */
+#define LRKV_DEV_SEQ_OVERFLOW 0x2u  /* seq_len + new tokens exceeded T_cap: the tokens past
+                                       T_cap were dropped */
+#define LRKV_DEV_BAD_COUNT 0x4u     /* a t_new_b entry outside [0, t_new]: clamped into it */
+
+/* Problem sizes of one layer. */
+typedef struct {
+  int32_t B;     /* batch rows (sequences) */
+  int32_t Hq;    /* query heads */
+  int32_t Hkv;   /* kv heads; Hq % Hkv == 0 */
+  int32_t d;     /* head dimension; 128 in this build */
+  int32_t r_k;   /* key rank, multiple of 16 in [16, d] */
+  int32_t r_v;   /* value rank, multiple of 16 in [16, d] */
+  int32_t T_cap; /* positions per sequence the cache can hold, multiple of 32 */
+  int32_t F_cap; /* full-rank rows per (sequence, kv head) the list can hold, >= 0 */
+} lrkv_dims;
+
+/* One layer of compressed cache.  Every pointer is a device pointer. */
+typedef struct {
+  const lrkv_bf16* U_k; /* [Hkv][d][r_k] key basis (orthonormal columns, rounded to bf16) */
+  const lrkv_bf16* U_v; /* [Hkv][d][r_v] value basis */
+  lrkv_bf16* coef_k;    /* [B][Hkv][T_cap][r_k] key coefficients, indexed by position */
+  lrkv_bf16* coef_v;    /* [B][Hkv][T_cap][r_v] value coefficients */
+  uint32_t* route_mask; /* [B][Hkv][T_cap/32]; bit p%32 of word p/32 = position p is full rank */
+  int32_t* full_idx;    /* [B][Hkv][F_cap] positions of the full-rank rows, ascending */
+  lrkv_bf16* full_k;    /* [B][Hkv][F_cap][d] key rows of full-rank tokens */
+  lrkv_bf16* full_v;    /* [B][Hkv][F_cap][d] value rows of full-rank tokens */
+  int32_t* full_cnt;    /* [B][Hkv] rows in use in the full-rank list */
+  int32_t* seq_len;     /* [B] tokens already in the cache (positions 0..seq_len-1) */
+  uint32_t* dev_status; /* 1 word, LRKV_DEV_* bits */
+} lrkv_cache;
+/* A new cache is all zeros (seq_len = full_cnt = 0).  The library writes every
+   mask bit, coefficient row and list entry it covers, so stale contents past
+   seq_len / full_cnt are harmless. */
+
+/* Bytes of device workspace that lrkv_compress and lrkv_decode_attn need for
+   these sizes (0 for invalid sizes).  The workspace must be zero-filled once
+   after allocation; the kernels leave it zeroed where it needs to be, so it
+   can be reused by any later call with the same dims.  One workspace serves
+   one stream of calls: concurrent calls need their own. */
+LRKV_API size_t lrkv_workspace_size(const lrkv_dims* dims);
+
+/* Append new tokens to every sequence of the cache (prefill or a decode step).
+ *
+ * k_new, v_new: [B][t_new][Hkv][d] bf16, the new key and value rows.  Row b
+ *   contributes its first n_b tokens: n_b = t_new_b[b] when t_new_b (device
+ *   [B] int32, nullable) is given, else t_new (ragged prefill passes padded
+ *   rows plus t_new_b).  They go to positions seq_len[b] .. seq_len[b]+n_b-1;
+ *   seq_len[b] is advanced on the device.  Positions at or past T_cap are
+ *   dropped (LRKV_DEV_SEQ_OVERFLOW).
+ * tau: routing threshold on the relative reconstruction error (strict >).
+ * err_out: nullable device [B][Hkv][t_new] fp32; receives e_t for every token
+ *   written (entries of dropped or padding tokens are left untouched).
+ * ws: workspace of at least lrkv_workspace_size(dims) bytes (ws_bytes).
+ * Returns LRKV_OK when the work was enqueued.
+ */
+LRKV_API lrkv_status lrkv_compress(const lrkv_dims* dims, const lrkv_cache* cache,
+                                   const lrkv_bf16* k_new, const lrkv_bf16* v_new,
+                                   int32_t t_new, const int32_t* t_new_b, float tau,
+                                   float* err_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Single-token decode attention for every query head of every sequence.
+ *
+ * q:   [B][Hq][d] bf16, one query per head.
+ * out: [B][Hq][d] fp32, the attention output (0 for an empty sequence).
+ * Attends to positions 0..seq_len[b]-1 as the cache holds them on the
+ * device when the kernel runs (so an append issued earlier on the same
+ * stream is included).
+ * ws: workspace of at least lrkv_workspace_size(dims) bytes (ws_bytes).
+ */
+LRKV_API lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache,
+                                      const lrkv_bf16* q, float* out, void* ws,
+                                      size_t ws_bytes, void* stream);
+
+/* Static text for a status code. */
+LRKV_API const char* lrkv_status_str(lrkv_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LRKV_H */

@@ -1,0 +1,122 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/lrkv.h declares, sizes workspaces, and rejects bad arguments on the
+host before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import decode_attention_lrkv_b200 as L
+from decode_attention_lrkv_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lrkv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return L.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lrkv_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted(
+        ["lrkv_workspace_size", "lrkv_compress", "lrkv_decode_attn", "lrkv_status_str"])
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (lrkv_\w+)", out))
+    assert set(declared_functions()) <= exported
+    # nothing but the declared C ABI is exported
+    assert exported == set(declared_functions())
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert L.lrkv_status_str(code)
+    assert L.lrkv_status_str(0) == "ok"
+    assert "unknown" in L.lrkv_status_str(99)
+
+
+def _dims(**kw):
+    base = dict(B=2, Hq=32, Hkv=8, d=128, r_k=64, r_v=96, T_cap=8192, F_cap=1024)
+    base.update(kw)
+    return L.Dims(**base)
+
+
+def test_workspace_size(lib):
+    n = L.lrkv_workspace_size(_dims())
+    assert n > 0 and n % 256 == 0
+    assert L.lrkv_workspace_size(_dims(T_cap=16384)) > n
+    for bad in (dict(d=64), dict(r_k=40), dict(r_v=0), dict(r_k=144), dict(Hq=30),
+                dict(T_cap=100), dict(T_cap=0), dict(F_cap=-1), dict(B=0), dict(Hq=72, Hkv=8)):
+        assert L.lrkv_workspace_size(_dims(**bad)) == 0, bad
+    assert lib.lrkv_workspace_size(None) == 0
+
+
+class _FakeCache:
+    """Cache-shaped object with fake, never-dereferenced device addresses."""
+    def __init__(self, base=0x10000000, **override):
+        self.ptrs = {f: base + 0x1000000 * i for i, f in enumerate(L.LayerCache.FIELDS)}
+        self.ptrs.update(override)
+
+    def c(self):
+        return L._Cache(*[self.ptrs[f] for f in L.LayerCache.FIELDS])
+
+
+def _call_compress(lib, dims, cache, k=0x20000000, v=0x30000000, t_new=4, t_new_b=None,
+                   err=None, ws=0x40000000, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.lrkv_workspace_size(ctypes.byref(dims.c())) if dims else 1 << 30
+    return lib.lrkv_compress(ctypes.byref(dims.c()) if dims else None,
+                             ctypes.byref(cache.c()) if cache else None, k, v, t_new, t_new_b,
+                             0.25, err, ws, ws_bytes, None)
+
+
+def _call_decode(lib, dims, cache, q=0x20000000, out=0x30000000, ws=0x40000000, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.lrkv_workspace_size(ctypes.byref(dims.c())) if dims else 1 << 30
+    return lib.lrkv_decode_attn(ctypes.byref(dims.c()) if dims else None,
+                                ctypes.byref(cache.c()) if cache else None, q, out, ws, ws_bytes,
+                                None)
+
+
+def test_host_validation_rejects_before_launch(lib):
+    D = _dims()
+    C = _FakeCache()
+    INVALID, UNSUP, ALIGN = 1, 2, 3
+    assert _call_compress(lib, None, C) == INVALID
+    assert _call_compress(lib, D, None) == INVALID
+    assert _call_compress(lib, _dims(d=64), C, ws_bytes=1 << 30) == UNSUP
+    assert _call_compress(lib, _dims(Hq=33), C, ws_bytes=1 << 30) == INVALID
+    assert _call_compress(lib, D, C, k=None) == INVALID
+    assert _call_compress(lib, D, C, t_new=-1) == INVALID
+    assert _call_compress(lib, D, _FakeCache(seq_len=None)) == INVALID
+    assert _call_compress(lib, D, _FakeCache(coef_k=0x10000008)) == ALIGN
+    assert _call_compress(lib, D, C, v=0x30000004) == ALIGN
+    assert _call_compress(lib, D, C, t_new_b=0x50000002) == ALIGN
+    assert _call_compress(lib, D, C, ws=None) == INVALID
+    assert _call_compress(lib, D, C, ws_bytes=16) == INVALID
+    assert _call_compress(lib, D, C, ws=0x40000001) == ALIGN
+    assert _call_compress(lib, D, C, t_new=0) == 0          # nothing to append: no launch
+    assert _call_decode(lib, None, C) == INVALID
+    assert _call_decode(lib, D, C, q=None) == INVALID
+    assert _call_decode(lib, D, C, out=0x30000002) == ALIGN
+    assert _call_decode(lib, D, C, ws_bytes=1) == INVALID
+    assert _call_decode(lib, _dims(Hq=72), C, ws_bytes=1 << 30) == UNSUP
+    # F_cap = 0 lets the full-rank buffers be null; otherwise they are required
+    assert _call_compress(lib, _dims(F_cap=0), _FakeCache(full_k=None, full_v=None, full_idx=None),
+                          t_new=0) == 0
+    assert _call_compress(lib, D, _FakeCache(full_v=None)) == INVALID
