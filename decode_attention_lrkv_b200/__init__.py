@@ -10,6 +10,7 @@ Entry points (same names as the C ABI):
     lrkv_workspace_size(dims) -> int
     lrkv_compress(dims, cache, k_new, v_new, tau, t_new_b=None, err_out=None, ws=...)
     lrkv_decode_attn(dims, cache, q, out, ws=...)
+    lrkv_decode_attn_noalloc(dims, cache, q, out)   (scratch held by the library)
     lrkv_status_str(code) -> str
 plus ``LayerCache`` (allocates one layer's buffers with torch) and
 ``make_workspace``.
@@ -70,6 +71,8 @@ def load_library(path=None):
     lib.lrkv_decode_attn.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Cache), P, P, P,
                                      ctypes.c_size_t, P]
     lib.lrkv_decode_attn.restype = ctypes.c_int
+    lib.lrkv_decode_attn_noalloc.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Cache), P, P, P]
+    lib.lrkv_decode_attn_noalloc.restype = ctypes.c_int
     lib.lrkv_status_str.argtypes = [ctypes.c_int]
     lib.lrkv_status_str.restype = ctypes.c_char_p
     if path is None:
@@ -177,4 +180,14 @@ def lrkv_decode_attn(dims, cache, q, out, ws=None, stream=None, check=True):
                                 _ptr(ws), 0 if ws is None else ws.numel(), _stream_ptr(stream))
     if check and code != LRKV_OK:
         raise LrkvError(code, "lrkv_decode_attn")
+    return code
+
+
+def lrkv_decode_attn_noalloc(dims, cache, q, out, stream=None, check=True):
+    """lrkv_decode_attn with the library's own device scratch instead of a workspace."""
+    lib = load_library()
+    code = lib.lrkv_decode_attn_noalloc(ctypes.byref(dims.c()), ctypes.byref(cache.c()), _ptr(q),
+                                        _ptr(out), _stream_ptr(stream))
+    if check and code != LRKV_OK:
+        raise LrkvError(code, "lrkv_decode_attn_noalloc")
     return code

@@ -145,6 +145,39 @@ LRKV_API lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* c
                                       const lrkv_bf16* q, float* out, void* ws,
                                       size_t ws_bytes, void* stream);
 
+/* Device scratch built into the library for lrkv_decode_attn_noalloc, bytes. */
+#define LRKV_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* lrkv_decode_attn without a workspace: the same computation and result, with
+ * the split-K scratch taken from memory the library itself holds.  The paper
+ * has no counterpart; this is an interface addition.
+ *
+ * Who it is for: callers that may not allocate device memory at decode time --
+ * a plugin's enqueue hook in an inference engine that may only touch memory
+ * the engine handed it when it was built, a latency-critical decode loop that
+ * cannot afford cudaMalloc/cudaFree (they cost host time and can synchronise
+ * the whole device), or a plain C caller with no device allocator of its own.
+ *
+ * The scratch is one file-scope device array of LRKV_NOALLOC_SCRATCH_BYTES.
+ * It exists on every GPU that loads the library, from load until the process
+ * exits.  A call needs 256-byte-rounded B*Hkv*4 bytes of tickets plus the split
+ * partials (the decode part of lrkv_workspace_size for the same dims); when
+ * that exceeds the maximum the call returns LRKV_ERR_UNSUPPORTED and launches
+ * nothing.  The function calls no cudaMalloc, cudaFree or other allocating
+ * routine; it clears the tickets with cudaMemsetAsync on `stream`, then
+ * launches the decode kernel there.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress), once per device, with that device current: make
+ * that first call before any stream capture starts.
+ * All calls on one device share the array.  Calls whose executions overlap on
+ * the GPU (different streams, or host threads without ordering) race on it
+ * and give wrong results: order them, e.g. issue them on one stream.
+ * Arguments, layouts and synchronous errors are those of lrkv_decode_attn.
+ */
+LRKV_API lrkv_status lrkv_decode_attn_noalloc(const lrkv_dims* dims, const lrkv_cache* cache,
+                                              const lrkv_bf16* q, float* out, void* stream);
+
 /* Static text for a status code. */
 LRKV_API const char* lrkv_status_str(lrkv_status status);
 

@@ -1,0 +1,64 @@
+"""lrkv_decode_attn_noalloc: decode attention for callers that cannot allocate.
+
+Some callers may not allocate device memory on the decode path (an inference
+engine's plugin hook that only gets memory at build time, a latency-critical
+loop where cudaMalloc's cost and device synchronisation are unacceptable, a C
+caller without a device allocator).  This entry point takes its split-K
+scratch from a device array the library holds instead of a workspace.  Its
+output must match lrkv_decode_attn's, within the parity tolerance, call
+after call: the shared array keeps the previous call's contents, so each
+call has to start from cleared tickets.  This file is collected last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+import decode_attention_lrkv_b200 as L
+
+pytestmark = pytest.mark.gpu
+
+OUT_RTOL = 2e-3     # the parity bar used for every decode output
+
+
+def _rel(a, b):
+    a, b = a.double().cpu().numpy(), b.double().cpu().numpy()
+    return np.abs(a - b).max() / max(np.abs(b).max(), 1e-30)
+
+
+def test_noalloc_matches_workspace_decode_on_consecutive_calls():
+    dev = torch.device("cuda", 0)
+    w = synth.workload(1, T=3000, layers=1)
+    lay = synth.make_layer(w, 0, 77, device=dev)
+    D = L.Dims(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, r_k=w.r_k, r_v=w.r_v, T_cap=3008, F_cap=3008)
+    cache = L.LayerCache(D, lay["U_k"], lay["U_v"], device=dev)
+    ws = L.make_workspace(D, dev)
+    L.lrkv_compress(D, cache, lay["K"], lay["V"], w.tau, ws=ws)
+    qs = synth.decode_queries(w, 2, 77, 0, dev)
+    lib = L.load_library()
+    stream = torch.cuda.current_stream()
+    for i in range(2):                       # two calls in a row share the library's scratch
+        ref = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
+        L.lrkv_decode_attn(D, cache, qs[i], ref, ws=ws)
+        out = torch.full((w.B, w.Hq, w.d), float("nan"), dtype=torch.float32, device=dev)
+        code = lib.lrkv_decode_attn_noalloc(ctypes.byref(D.c()), ctypes.byref(cache.c()),
+                                            ctypes.c_void_p(qs[i].data_ptr()),
+                                            ctypes.c_void_p(out.data_ptr()),
+                                            ctypes.c_void_p(stream.cuda_stream))
+        assert code == L.LRKV_OK, L.lrkv_status_str(code)
+        torch.cuda.synchronize()
+        assert torch.isfinite(out).all()
+        assert _rel(out, ref) <= OUT_RTOL
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    dev = torch.device("cuda", 0)
+    big = L.Dims(B=64, Hq=64, Hkv=8, d=128, r_k=64, r_v=96, T_cap=65536, F_cap=32)
+    fake = L._Cache(*[0x10000000 + 0x100000 * i for i in range(11)])
+    lib = L.load_library()
+    code = lib.lrkv_decode_attn_noalloc(ctypes.byref(big.c()), ctypes.byref(fake),
+                                        ctypes.c_void_p(0x20000000), ctypes.c_void_p(0x30000000),
+                                        ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream))
+    assert code == 2          # LRKV_ERR_UNSUPPORTED: needs more than LRKV_NOALLOC_SCRATCH_BYTES
