@@ -44,7 +44,7 @@ from decode_attention_lrkv_b200 import accounting as A  # noqa: E402
 
 HBM_SPEC_GBS = 8000.0
 FALLBACK_PEAK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-COMPRESS_LAUNCHES = 2     # kernels one lrkv_compress call launches
+COMPRESS_LAUNCHES = 1     # kernels one decode-time (one-token) lrkv_compress call launches
 DECODE_LAUNCHES = 1       # kernels one lrkv_decode_attn call launches
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 

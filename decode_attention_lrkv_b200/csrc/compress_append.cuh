@@ -1,0 +1,212 @@
+// Write path for a few new tokens per sequence (decode-time appends): one
+// CTA per (kv head, batch row) projects, measures and routes the row's new
+// tokens in position order, all in one launch.
+//
+// OjaKV repository README, "Method Summary": the fixed per-head basis of
+// StaticPCA, and the hybrid policy of OjaKV that keeps tokens with a high
+// reconstruction error in full rank.  Per token x (key, then value):
+//   c = U^T x (fp32), stored as bf16 at the token's position;
+//   e = ||x - U c|| / ||x|| by direct reconstruction (0 when x = 0);
+//   routed iff max(e_k, e_v) > tau: the k and v rows go to the next slot of
+//   the full-rank list and the mask bit is set (kept compressed with
+//   FULL_OVERFLOW when the list is full).
+#pragma once
+
+#include "compress_simple.cuh"
+#include "lrkv_common.cuh"
+#include "ptx.cuh"
+
+namespace lrkv {
+
+constexpr int kAppendThreads = 256;    // two halves of 128: keys and values side by side
+constexpr int kAppendMaxTokens = 16;   // larger appends take the tiled path
+constexpr uint32_t kAppendWaitIters = 1u << 24;
+
+// Shared memory: U_k, U_v as stored (bf16 [d][r]) and the new tokens' key and
+// value rows (bf16 [kAppendMaxTokens][d] each), all filled by bulk copies; then
+// per half: x [d], partial c [4][d], c [d], reduction scratch; one mbarrier.
+inline size_t append_smem_bytes(int r_k, int r_v) {
+  return sizeof(uint16_t) * (size_t)kD * (r_k + r_v + 2 * kAppendMaxTokens) +
+         sizeof(float) * 2 * (6 * kD + 8) + 16;
+}
+
+// One tensor (the key for half 0, the value for half 1) of one token: x (bf16
+// [d] in shared memory) -> coefficients (bf16, global); returns the relative error
+// to every thread of the half.  All 256 threads call it together.
+__device__ __forceinline__ float append_project(const uint16_t* __restrict__ x_s,
+                                                const uint16_t* Us, int r,
+                                                lrkv_bf16* __restrict__ coef_g, float* ws) {
+  const int tid = threadIdx.x & 127;
+  const int warp = tid >> 5, lane = tid & 31;
+  float* xs = ws;                 // [d]
+  float* part = xs + kD;          // [4][d]
+  float* cs = part + 4 * kD;      // [d]
+  float* red = cs + kD;           // [8]
+  const float x = bf2f(x_s[tid]);
+  xs[tid] = x;
+  __syncthreads();
+  // c_j = sum_i U[i][j] x_i: warp w sums rows 32w..32w+31, lane owns columns lane + 32k
+  {
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint16_t* U = Us + warp * 32 * r;
+#pragma unroll 8
+    for (int ii = 0; ii < 32; ++ii) {
+      const float xi = xs[warp * 32 + ii];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (lane + 32 * k < r) a[k] = fmaf(bf2f(U[ii * r + lane + 32 * k]), xi, a[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (lane + 32 * k < r) part[warp * kD + lane + 32 * k] = a[k];
+  }
+  __syncthreads();
+  if (tid < r) {
+    const float c = (part[tid] + part[kD + tid]) + (part[2 * kD + tid] + part[3 * kD + tid]);
+    cs[tid] = c;
+    coef_g[tid] = f2bf(c);
+  }
+  __syncthreads();
+  // x_hat_i = sum_j U[i][j] c_j: thread i walks row i two columns at a time,
+  // starting at column pair (i mod r/2), so a warp's 32 rows hit 32 banks.
+  const int npair = r >> 1;
+  const uint32_t* row = reinterpret_cast<const uint32_t*>(Us) + tid * npair;
+  const float2* c2 = reinterpret_cast<const float2*>(cs);
+  float h0 = 0.f, h1 = 0.f;
+  int w = tid % npair;
+#pragma unroll 8
+  for (int k = 0; k < npair; ++k) {
+    const uint32_t u = row[w];
+    const float2 cc = c2[w];
+    h0 = fmaf(bf_lo(u), cc.x, h0);
+    h1 = fmaf(bf_hi(u), cc.y, h1);
+    w = (w + 1 == npair) ? 0 : w + 1;
+  }
+  const float dlt = x - (h0 + h1);
+  const float rs = warp_sum(dlt * dlt), ns = warp_sum(x * x);
+  if (lane == 0) red[warp] = rs, red[4 + warp] = ns;
+  __syncthreads();
+  const float rsum = (red[0] + red[1]) + (red[2] + red[3]);
+  const float nsum = (red[4] + red[5]) + (red[6] + red[7]);
+  return nsum > 0.f ? sqrtf(rsum / nsum) : 0.f;
+}
+
+// grid (Hkv, B), kAppendThreads threads
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p) {
+  extern __shared__ __align__(16) unsigned char sm_app[];
+  const lrkv_dims& D = p.D;
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int r_k = D.r_k, r_v = D.r_v;
+  uint16_t* Uks = reinterpret_cast<uint16_t*>(sm_app);
+  uint16_t* Uvs = Uks + kD * r_k;
+  uint16_t* Xks = Uvs + kD * r_v;                          // new key rows
+  uint16_t* Xvs = Xks + kD * kAppendMaxTokens;             // new value rows
+  float* ws0 = reinterpret_cast<float*>(Xvs + kD * kAppendMaxTokens);   // per-half scratch
+  const int half = tid >> 7;
+  float* ws = ws0 + half * (6 * kD + 8);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(ws0 + 2 * (6 * kD + 8));
+  __shared__ int s_cnt;
+  __shared__ bool s_last;
+  __shared__ float s_err[2];
+  __shared__ uint32_t s_mask[2];    // the (at most two) mask words the new positions touch
+
+  uint32_t st = 0;
+  const int n = new_tokens(p.t_new_b, b, p.t_new, &st);
+  const int start = min(max(p.C.seq_len[b], 0), D.T_cap);
+  int n_eff = D.T_cap - start;
+  if (n_eff > n) n_eff = n;
+  if (n_eff < 0) n_eff = 0;
+  const size_t bh = (size_t)b * D.Hkv + h;
+  uint32_t* mask_row = p.C.route_mask + bh * (D.T_cap / 32);
+
+  if (n_eff > 0) {
+    if (tid == 0) {
+      mbar_init(bar, 1);
+      fence_mbar_init();
+      const uint32_t bk = kD * r_k * 2, bv = kD * r_v * 2;
+      mbar_arrive_expect_tx(bar, bk + bv + n_eff * 4u * kD);
+      bulk_g2s(Uks, p.C.U_k + (size_t)h * kD * r_k, bk, bar);
+      bulk_g2s(Uvs, p.C.U_v + (size_t)h * kD * r_v, bv, bar);
+      for (int t = 0; t < n_eff; ++t) {
+        const size_t x = (((size_t)b * p.t_new + t) * D.Hkv + h) * kD;
+        bulk_g2s(Xks + t * kD, p.k_new + x, 2u * kD, bar);
+        bulk_g2s(Xvs + t * kD, p.v_new + x, 2u * kD, bar);
+      }
+      s_cnt = min(max(p.C.full_cnt[bh], 0), D.F_cap);
+      s_mask[0] = mask_row[start >> 5];
+      s_mask[1] = ((start + n_eff - 1) >> 5) != (start >> 5) ? mask_row[(start >> 5) + 1] : 0u;
+    }
+    __syncthreads();
+    if (!mbar_wait_bounded(bar, 0, kAppendWaitIters)) st |= LRKV_DEV_WAIT_TIMEOUT;
+    if (__syncthreads_or(st & LRKV_DEV_WAIT_TIMEOUT)) {
+      mbar_wait_bounded(bar, 0, kAppendWaitIters);   // one more bounded wait for the copies
+      st |= LRKV_DEV_WAIT_TIMEOUT;
+      if (tid == 0) atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
+      n_eff = 0;   // leave the cache untouched; the call's results are flagged invalid
+    }
+    bool overflow = false;
+    for (int t = 0; t < n_eff; ++t) {
+      const int pos = start + t;
+      const size_t row = bh * D.T_cap + pos;
+      // one call site for both halves: every __syncthreads inside is reached by all threads
+      const float eh = append_project(half == 0 ? Xks + t * kD : Xvs + t * kD,
+                                      half == 0 ? Uks : Uvs, half == 0 ? r_k : r_v,
+                                      half == 0 ? p.C.coef_k + row * r_k : p.C.coef_v + row * r_v,
+                                      ws);
+      if ((tid & 127) == 0) s_err[half] = eh;
+      __syncthreads();
+      const float e = fmaxf(s_err[0], s_err[1]);
+      const bool routed = e > p.tau;
+      const int slot = s_cnt;
+      const bool keep = routed && slot < D.F_cap;
+      if (routed && !keep) overflow = true;
+      if (keep) {
+        const int i = tid & 127;
+        if (half == 0) p.C.full_k[(bh * D.F_cap + slot) * kD + i] = Xks[t * kD + i];
+        else p.C.full_v[(bh * D.F_cap + slot) * kD + i] = Xvs[t * kD + i];
+      }
+      if (tid == 0) {
+        const uint32_t bit = 1u << (pos & 31);
+        uint32_t& mw = s_mask[(pos >> 5) - (start >> 5)];
+        mw = keep ? (mw | bit) : (mw & ~bit);
+        if (keep) {
+          p.C.full_idx[bh * D.F_cap + slot] = pos;
+          s_cnt = slot + 1;
+        }
+        if (p.err_out) p.err_out[bh * p.t_new + t] = e;
+      }
+      __syncthreads();
+    }
+    if (tid == 0) {
+      p.C.full_cnt[bh] = s_cnt;
+      mask_row[start >> 5] = s_mask[0];
+      if (((start + n_eff - 1) >> 5) != (start >> 5)) mask_row[(start >> 5) + 1] = s_mask[1];
+      if (overflow) st |= LRKV_DEV_FULL_OVERFLOW;
+    }
+  }
+  if (n_eff < n && !(st & LRKV_DEV_WAIT_TIMEOUT)) st |= LRKV_DEV_SEQ_OVERFLOW;
+  if (h != 0) st &= LRKV_DEV_FULL_OVERFLOW;     // per-sequence conditions: reported once
+  if (tid == 0 && st) atomicOr(p.C.dev_status, st);
+  // the last CTA advances every sequence's length (all CTAs have read them)
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    s_last = atomicAdd(p.ticket, 1) == (int)(gridDim.x * gridDim.y) - 1;
+  }
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    for (int bb = tid; bb < D.B; bb += kAppendThreads) {
+      uint32_t dummy = 0;
+      const int nb = new_tokens(p.t_new_b, bb, p.t_new, &dummy);
+      const int sb = min(max(p.C.seq_len[bb], 0), D.T_cap);
+      int ne = D.T_cap - sb;
+      if (ne > nb) ne = nb;
+      if (ne < 0) ne = 0;
+      p.C.seq_len[bb] = sb + ne;
+    }
+    if (tid == 0) *p.ticket = 0;
+  }
+}
+
+}  // namespace lrkv

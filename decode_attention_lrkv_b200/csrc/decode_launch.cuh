@@ -1,0 +1,85 @@
+// Decode dispatch shared by lrkv_decode_attn and lrkv_decode_attn_noalloc:
+// the tensor-core pipeline kernel for the shapes it is instantiated for, the
+// CUDA-core kernel for every other valid shape.
+#pragma once
+
+#include "decode_tc.cuh"
+#include "decode_simple.cuh"
+
+namespace lrkv {
+
+template <int G, int RK, int RV>
+inline lrkv_status launch_fast(const DecodeParams& p, dim3 grid, cudaStream_t s) {
+  using S = tc::Shape<G, RK, RV>;
+  auto kern = tc::decode_tc_kernel<G, RK, RV>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return LRKV_ERR_CUDA;
+  }
+  kern<<<grid, tc::kThreads, S::SMEM, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+}
+
+template <int G>
+inline lrkv_status launch_simple(const DecodeParams& p, dim3 grid, cudaStream_t s) {
+  const size_t smem = decode_simple_smem_bytes(G, p.n_chunk_max);
+  if (cudaFuncSetAttribute(decode_simple_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess) {
+    cudaGetLastError();
+    return LRKV_ERR_CUDA;
+  }
+  decode_simple_kernel<G><<<grid, kDecThreads, smem, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+}
+
+template <int G>
+inline lrkv_status launch_fast_g(const DecodeParams& p, dim3 grid, cudaStream_t s, bool* done) {
+  *done = true;
+  const int rk = p.D.r_k, rv = p.D.r_v;
+  if (rk == 32 && rv == 32) return launch_fast<G, 32, 32>(p, grid, s);
+  if (rk == 48 && rv == 64) return launch_fast<G, 48, 64>(p, grid, s);
+  if (rk == 48 && rv == 80) return launch_fast<G, 48, 80>(p, grid, s);
+  if (rk == 64 && rv == 64) return launch_fast<G, 64, 64>(p, grid, s);
+  if (rk == 64 && rv == 96) return launch_fast<G, 64, 96>(p, grid, s);
+  *done = false;
+  return LRKV_OK;
+}
+
+// Whether the pipeline kernel covers these sizes.
+inline bool fast_decode_supported(const lrkv_dims& D, int chunk, int n_chunk_max) {
+  const int g = D.Hq / D.Hkv;
+  if (g != 1 && g != 2 && g != 4) return false;
+  if (chunk > tc::kMaxChunk || chunk % 32) return false;
+  // the merge keeps a max and a sum per (split, head) in the staging area (>= 10 KiB)
+  if ((long long)n_chunk_max * g * 8 > 10 * 1024) return false;
+  const int rk = D.r_k, rv = D.r_v;
+  return (rk == 32 && rv == 32) || (rk == 48 && rv == 64) || (rk == 48 && rv == 80) ||
+         (rk == 64 && rv == 64) || (rk == 64 && rv == 96);
+}
+
+inline lrkv_status launch_decode(const DecodeParams& p, cudaStream_t s) {
+  const dim3 grid(p.n_chunk_max, p.D.Hkv, p.D.B);
+  const int g = p.D.Hq / p.D.Hkv;
+  if (fast_decode_supported(p.D, p.chunk, p.n_chunk_max)) {
+    bool done = false;
+    lrkv_status st = LRKV_OK;
+    if (g == 1) st = launch_fast_g<1>(p, grid, s, &done);
+    else if (g == 2) st = launch_fast_g<2>(p, grid, s, &done);
+    else st = launch_fast_g<4>(p, grid, s, &done);
+    if (done) return st;
+  }
+  switch (g) {
+    case 1: return launch_simple<1>(p, grid, s);
+    case 2: return launch_simple<2>(p, grid, s);
+    case 3: return launch_simple<3>(p, grid, s);
+    case 4: return launch_simple<4>(p, grid, s);
+    case 5: return launch_simple<5>(p, grid, s);
+    case 6: return launch_simple<6>(p, grid, s);
+    case 7: return launch_simple<7>(p, grid, s);
+    case 8: return launch_simple<8>(p, grid, s);
+    default: return LRKV_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace lrkv

@@ -3,8 +3,9 @@
 #include <cmath>
 #include <cstdint>
 
+#include "compress_append.cuh"
 #include "compress_simple.cuh"
-#include "decode_simple.cuh"
+#include "decode_launch.cuh"
 #include "lrkv.h"
 #include "lrkv_common.cuh"
 
@@ -57,16 +58,6 @@ lrkv_status launched() {
   return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
 }
 
-template <int G>
-lrkv_status launch_decode(const DecodeParams& p, dim3 grid, cudaStream_t s) {
-  const size_t smem = decode_simple_smem_bytes(G, p.n_chunk_max);
-  if (cudaFuncSetAttribute(decode_simple_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return launched(), LRKV_ERR_CUDA;
-  decode_simple_kernel<G><<<grid, kDecThreads, smem, s>>>(p);
-  return launched();
-}
-
 }  // namespace
 
 extern "C" {
@@ -102,6 +93,14 @@ lrkv_status lrkv_compress(const lrkv_dims* dims, const lrkv_cache* cache,
   p.err_out = err_out;
   p.flags = reinterpret_cast<uint8_t*>(w + L.flags);
   p.ticket = reinterpret_cast<int32_t*>(w + L.compress_ticket);
+  if (t_new <= kAppendMaxTokens) {  // decode-time appends: one fused launch
+    const size_t smem = append_smem_bytes(dims->r_k, dims->r_v);
+    if (cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return launched(), LRKV_ERR_CUDA;
+    append_kernel<<<dim3(dims->Hkv, dims->B), kAppendThreads, smem, s>>>(p);
+    return launched();
+  }
   const int tmax = t_new < dims->T_cap ? t_new : dims->T_cap;
   const size_t smem = proj_smem_bytes(dims->r_k > dims->r_v ? dims->r_k : dims->r_v);
   if (cudaFuncSetAttribute(project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -134,18 +133,7 @@ lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache, con
   p.partials = reinterpret_cast<float*>(w + L.partials);
   p.chunk = L.chunk;
   p.n_chunk_max = L.n_chunk_max;
-  const dim3 grid(L.n_chunk_max, dims->Hkv, dims->B);
-  switch (dims->Hq / dims->Hkv) {
-    case 1: return launch_decode<1>(p, grid, s);
-    case 2: return launch_decode<2>(p, grid, s);
-    case 3: return launch_decode<3>(p, grid, s);
-    case 4: return launch_decode<4>(p, grid, s);
-    case 5: return launch_decode<5>(p, grid, s);
-    case 6: return launch_decode<6>(p, grid, s);
-    case 7: return launch_decode<7>(p, grid, s);
-    case 8: return launch_decode<8>(p, grid, s);
-    default: return LRKV_ERR_UNSUPPORTED;
-  }
+  return launch_decode(p, s);
 }
 
 const char* lrkv_status_str(lrkv_status status) {

@@ -11,6 +11,7 @@ namespace lrkv {
 
 constexpr int kD = 128;            // head dimension handled by this build
 constexpr int kNumSMs = 148;       // B200; only used to size work splits
+constexpr int kMaxDecodeChunk = 8192;   // positions per decode split, at most
 constexpr float kLog2e = 1.4426950408889634f;
 
 // bf16 <-> fp32.  A bf16 value is the top half of the fp32 with the same
@@ -56,16 +57,30 @@ struct WsLayout {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Positions per decode split: aim for ~4 CTAs per SM over the whole grid,
-// between 256 and 4096 positions, a multiple of 32 (one mask word).
+// Positions per decode split.  One CTA per SM: choose the number of waves W
+// so that a split holds at most 2048 positions, then give every (batch row,
+// kv head) floor(W * SMs / rows) splits, so the grid is close to W full
+// waves.  At least 128 positions, a multiple of 32 (one mask word).
 inline int decode_chunk(const lrkv_dims& D) {
-  long long units = (long long)D.B * D.Hkv;
-  long long target = (long long)kNumSMs * 4;
-  long long ch = ((long long)D.T_cap * units + target - 1) / target;
-  ch = (ch + 31) / 32 * 32;
-  if (ch < 256) ch = 256;
-  if (ch > 4096) ch = 4096;
-  return (int)ch;
+  // Pick the split count n that minimises the modelled makespan
+  //   ceil(B*Hkv*n / SMs) * (chunk + overhead)
+  // with one CTA per SM resident at a time; `overhead` is a CTA's fixed cost
+  // (bases, q~, merge) expressed in streamed positions.
+  const long long bh = (long long)D.B * D.Hkv;
+  const long long overhead = 1024;
+  long long best_cost = -1, best = kMaxDecodeChunk;
+  const long long n_max = (D.T_cap + 127) / 128;
+  for (long long n = 1; n <= n_max && n <= 1024; ++n) {
+    long long ch = (D.T_cap + n - 1) / n;
+    ch = (ch + 31) / 32 * 32;
+    if (ch < 128) ch = 128;
+    if (ch > kMaxDecodeChunk) continue;
+    const long long splits = (D.T_cap + ch - 1) / ch;
+    const long long waves = (bh * splits + kNumSMs - 1) / kNumSMs;
+    const long long cost = waves * (ch + overhead);
+    if (best_cost < 0 || cost < best_cost) best_cost = cost, best = ch;
+  }
+  return (int)best;
 }
 
 inline WsLayout ws_layout(const lrkv_dims& D) {

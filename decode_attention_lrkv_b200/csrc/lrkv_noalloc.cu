@@ -11,7 +11,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "decode_simple.cuh"
+#include "decode_launch.cuh"
 #include "lrkv.h"
 #include "lrkv_common.cuh"
 
@@ -74,18 +74,6 @@ lrkv_status check_args(const lrkv_dims* D, const lrkv_cache* C, const void* q, c
   return LRKV_OK;
 }
 
-template <int G>
-lrkv_status launch(const DecodeParams& p, dim3 grid, cudaStream_t s) {
-  const size_t smem = decode_simple_smem_bytes(G, p.n_chunk_max);
-  if (cudaFuncSetAttribute(decode_simple_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess) {
-    cudaGetLastError();
-    return LRKV_ERR_CUDA;
-  }
-  decode_simple_kernel<G><<<grid, kDecThreads, smem, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
-}
-
 }  // namespace
 
 extern "C" LRKV_API lrkv_status lrkv_decode_attn_noalloc(const lrkv_dims* dims,
@@ -118,16 +106,5 @@ extern "C" LRKV_API lrkv_status lrkv_decode_attn_noalloc(const lrkv_dims* dims,
   p.partials = reinterpret_cast<float*>(base + ticket_bytes);
   p.chunk = L.chunk;
   p.n_chunk_max = L.n_chunk_max;
-  const dim3 grid(L.n_chunk_max, dims->Hkv, dims->B);
-  switch (dims->Hq / dims->Hkv) {
-    case 1: return launch<1>(p, grid, s);
-    case 2: return launch<2>(p, grid, s);
-    case 3: return launch<3>(p, grid, s);
-    case 4: return launch<4>(p, grid, s);
-    case 5: return launch<5>(p, grid, s);
-    case 6: return launch<6>(p, grid, s);
-    case 7: return launch<7>(p, grid, s);
-    case 8: return launch<8>(p, grid, s);
-    default: return LRKV_ERR_UNSUPPORTED;
-  }
+  return launch_decode(p, s);
 }

@@ -75,6 +75,8 @@ typedef enum {
 #define LRKV_DEV_SEQ_OVERFLOW 0x2u  /* seq_len + new tokens exceeded T_cap: the tokens past
                                        T_cap were dropped */
 #define LRKV_DEV_BAD_COUNT 0x4u     /* a t_new_b entry outside [0, t_new]: clamped into it */
+#define LRKV_DEV_WAIT_TIMEOUT 0x8u  /* a kernel gave up waiting for its own copies (bounded
+                                       wait): its outputs for that call are not valid */
 
 /* Problem sizes of one layer. */
 typedef struct {

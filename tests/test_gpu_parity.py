@@ -196,3 +196,18 @@ def test_canaries_past_buffers_untouched():
         assert (big[n:] == 0x5A5A).all(), f
     assert (ws_big[ws_n:] == 0x5A).all()
     assert int(cache.dev_status[0]) == L.DEV_FULL_OVERFLOW
+
+
+def test_small_multi_token_appends_with_ragged_counts():
+    """Appends of a few tokens (the fused one-launch path) with ragged counts and a
+    nearly full list, interleaved with decode."""
+    w = synth.workload(1, B=3, T=300, layers=1)
+    layer, D, cache, oc, ws = _setup(w, seed=21, T_cap=352, F_cap=40)
+    gc, band = _compress_both(D, cache, oc, layer["K"], layer["V"], w.tau, ws,
+                              t_new_b=[300, 150, 290])
+    extra = synth.decode_tokens(w, layer["Qk"], layer["Qv"], 7, 21, 0, DEV)
+    for counts in ([7, 0, 3], [1, 7, 7], [7, 7, 7]):
+        gc, band = _compress_both(D, cache, oc, extra[0], extra[1], w.tau, ws, t_new_b=counts,
+                                  band=band)
+        out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
+        assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
