@@ -52,7 +52,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=1)
@@ -94,13 +94,19 @@ def stored_traffic(kernel, workload_name):
 
 
 class Clocks:
-    """nvidia-smi samples during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples (every 20 ms) from before the warm-up to after the timed region.
+
+    Reported: the samples whose timestamps fall inside the timed region; when the
+    region is shorter than the sampling interval, the samples of warm-up plus timed
+    region (the GPU runs the same step throughout), marked as such."""
+    Q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, dev, enabled=True):
         self.p = None
+        self.t_start = self.t_end = None
         self.out = os.path.join("/tmp", f"lrkv_clocks_{os.getpid()}.csv")
         if not enabled:
             return
@@ -109,14 +115,30 @@ class Clocks:
             uuid = str(torch.cuda.get_device_properties(dev).uuid)
             sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
             self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                                       "-i", sel, "-lms", "100"], stdout=self.f,
+                                       "-i", sel, "-lms", "20"], stdout=self.f,
                                       stderr=subprocess.DEVNULL)
+            time.sleep(0.3)   # let the sampler come up before the warm-up starts
         except OSError:
             self.p = None
+
+    def mark_start(self):
+        self.t_start = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
+
+    @staticmethod
+    def _stamp(s):
+        import datetime
+        try:
+            return datetime.datetime.strptime(s, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def stop(self):
         if self.p is None:
             return None
+        time.sleep(0.05)
         self.p.terminate()
         try:
             self.p.wait(timeout=5)
@@ -128,16 +150,23 @@ class Clocks:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) >= 9:
-                    rows.append(parts)
+                    rows.append((self._stamp(parts[0]), parts))
         os.unlink(self.out)
-        if not rows:
+        window = "timed"
+        sel = [r for ts, r in rows if ts is not None and self.t_start is not None
+               and self.t_start <= ts <= self.t_end]
+        if not sel:
+            window = "warmup+timed"
+            sel = [r for ts, r in rows if ts is not None and self.t_start is not None
+                   and ts <= self.t_end and ts >= self.t_start - 2.0]
+        if not sel:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        sm = [float(r[1]) for r in sel if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in sel if r[2].replace(".", "").isdigit()]
+        reasons = sorted({self.NAMES[i] for r in sel for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(sel),
+                "window": window}
 
 
 # ---------------------------------------------------------------------------
@@ -223,20 +252,22 @@ def run_ours(args, rank, world, dev):
            for _ in range(w.layers)] for _ in range(steps_total)]
     graphs = [capture_step_graph(L, dims, ws, layers, w, s, out, ev[s]) for s in range(steps_total)]
     torch.cuda.synchronize()
+    clocks = Clocks(dev, enabled=not args.no_clocks)
     for s in range(W):
         graphs[s].replay()
     torch.cuda.synchronize()
     seq_before = layers[0]["cache"].seq_len.cpu().tolist()
-    clocks = Clocks(dev, enabled=not args.no_clocks)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark_start()
     t0.record()
     for s in range(W, steps_total):
         graphs[s].replay()
     t1.record()
     torch.cuda.synchronize()
+    clocks.mark_end()
     if world > 1:
         torch.distributed.barrier()
     clk = clocks.stop()
