@@ -174,21 +174,34 @@ class Clocks:
 # ---------------------------------------------------------------------------
 
 def build_layers(L, w, seed, steps_total, dev):
-    """Prefill every layer's cache through lrkv_compress; time each prefill."""
+    """Prefill every layer's cache through lrkv_compress; time each prefill.
+
+    Each timed prefill starts with a cold L2 (a 256 MB buffer is written first)
+    and behind a short device-side sleep, so that the host-side launch work of
+    the call overlaps the sleep and the events bracket device time only.  One
+    untimed prefill into a scratch cache first loads the kernels."""
     T_cap = synth.pad_to(w.T + steps_total + 1, 32)
     F_cap = T_cap
     dims = L.Dims(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, r_k=w.r_k, r_v=w.r_v, T_cap=T_cap, F_cap=F_cap)
     ws = L.make_workspace(dims, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     layers = []
     comp_ms = []
     lengths = None
     for li in range(w.layers):
         lay = synth.make_layer(w, li, seed, device=dev)
         lengths = lay["lengths"]
-        cache = L.LayerCache(dims, lay["U_k"], lay["U_v"], device=dev)
         t_new_b = (lengths.to(torch.int32).to(dev) if w.ragged_min else None)
+        if li == 0:
+            scratch = L.LayerCache(dims, lay["U_k"], lay["U_v"], device=dev)
+            L.lrkv_compress(dims, scratch, lay["K"], lay["V"], w.tau, t_new_b=t_new_b, ws=ws)
+            torch.cuda.synchronize()
+            del scratch
+        cache = L.LayerCache(dims, lay["U_k"], lay["U_v"], device=dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
+        flush.zero_()
+        torch.cuda._sleep(1_000_000)
         e0.record()
         L.lrkv_compress(dims, cache, lay["K"], lay["V"], w.tau, t_new_b=t_new_b, ws=ws)
         e1.record()
@@ -198,6 +211,7 @@ def build_layers(L, w, seed, steps_total, dev):
         qa = synth.decode_queries(w, steps_total, seed, li, dev)
         layers.append(dict(cache=cache, K_app=Ka, V_app=Va, q_app=qa))
         del lay
+    del flush
     return dims, ws, layers, comp_ms, lengths
 
 
@@ -297,6 +311,7 @@ def run_ours(args, rank, world, dev):
     n_tok = float(sum(int(x) for x in lengths))
     comp_tok_s = n_tok / (float(np.mean(comp_ms)) * 1e-3)
     comp_bytes = A.compress_bytes(w.Hkv, w.d, w.r_k, w.r_v, n_tok, n_tok * w.Hkv * routed_frac)
+    comp_tflops = A.compress_tc_flops(w.Hkv, w.d, w.r_k, w.r_v, n_tok) / (float(np.mean(comp_ms)) * 1e-3) / 1e12
 
     # --- end-to-end through host buffers --------------------------------------------------
     e2e = run_e2e(L, args, w, dims, ws, layers, dev, world, steps_total)
@@ -319,6 +334,11 @@ def run_ours(args, rank, world, dev):
         "compress": {"tok_per_s_per_layer": round(comp_tok_s, 1),
                      "us_per_layer": round(float(np.mean(comp_ms)) * 1e3, 2),
                      "gbs": round(comp_bytes / (float(np.mean(comp_ms)) * 1e-3) / 1e9, 2),
+                     "frac_of_measured_hbm": round(comp_bytes / (float(np.mean(comp_ms)) * 1e-3) / 1e9
+                                                   / pk.get("hbm_gbs", FALLBACK_PEAK["hbm_gbs"]), 4),
+                     "tensor_tflops_executed": round(comp_tflops, 1),
+                     "tensor_frac_of_measured_bf16": round(comp_tflops / pk.get("bf16_tflops",
+                                                                                FALLBACK_PEAK["bf16_tflops"]), 4),
                      "tokens_per_layer": n_tok},
         "roofline": {"kernel": "decode_attn", "bound": "hbm", "achieved": round(achieved, 2),
                      "peak": pk.get("hbm_gbs", FALLBACK_PEAK["hbm_gbs"]),

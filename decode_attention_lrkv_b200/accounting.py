@@ -59,3 +59,13 @@ def compress_bytes(Hkv, d, r_k, r_v, n_tokens, n_routed):
     """
     per_tok = Hkv * (2 * d * BF16 + (r_k + r_v) * BF16) + Hkv / 8.0
     return int(n_tokens * per_tok + n_routed * full_row_bytes(d) + Hkv * d * (r_k + r_v) * BF16)
+
+
+def compress_tc_flops(Hkv, d, r_k, r_v, n_tokens):
+    """Tensor-core flops the prefill projection executes per call.
+
+    Per (token, kv head) and tensor: c = U^T x (2 d r) and the residual
+    P x = (P_hi + P_lo) x with P = I - U U^T (2 * 2 d^2); the once-per-CTA
+    U U^T products are not counted.
+    """
+    return int(n_tokens * Hkv * (2 * d * (r_k + r_v) + 2 * 4 * d * d))

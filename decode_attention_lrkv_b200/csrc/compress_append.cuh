@@ -12,7 +12,7 @@
 //   FULL_OVERFLOW when the list is full).
 #pragma once
 
-#include "compress_simple.cuh"
+#include "compress_params.cuh"
 #include "lrkv_common.cuh"
 #include "ptx.cuh"
 

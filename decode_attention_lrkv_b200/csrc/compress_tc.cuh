@@ -1,0 +1,539 @@
+// Write path for prefill-sized appends on the 5th-generation tensor cores.
+//
+// OjaKV repository README, "Method Summary": a fixed per-head basis U
+// (StaticPCA) and the hybrid policy that keeps tokens whose reconstruction
+// error is high in full rank (OjaKV).  For every new row x (a key with U_k, a
+// value with U_v):
+//   c = U^T x                       (fp32 accumulation, stored as bf16 RNE)
+//   e = ||x - U c|| / ||x||         (0 when x = 0)
+// Since c = U^T x, the residual is x - U U^T x = P x with P = I - U U^T, the
+// same quantity computed in one product; U is bf16 and not exactly
+// orthonormal, so P is not a projector and no norm identity is used.
+//
+// Kernel 1, project_tc_kernel: one CTA per SM works on one (kv head, K or V)
+// stream of 128-token tiles.  Per CTA, P is formed once on the tensor cores
+// (U U^T) and split into bf16 high and low parts (P = P_hi + P_lo to 2^-17).
+// Per tile, TMA brings the 128 x 128 input rows (128-byte swizzle); one
+// thread issues
+//     D1 = X U        (M 128, N r, K 128)      -> coefficients
+//     D2 = X P_hi^T + X P_lo^T  (M 128, N 128) -> residual vectors
+// into tensor memory (double-buffered), and four epilogue warps (one token
+// row per thread) store bf16(c), sum the squared residual and the squared
+// input, and write e.  Three input stages and two accumulator buffers let
+// the loads, the MMAs and the epilogue of consecutive tiles overlap.
+//
+// Kernel 2, route_count_kernel: e_t = max(e_k, e_v); routed iff e_t > tau.
+// Per 128-token tile: err_out, the routed bits (warp ballots) and their count.
+//
+// Kernel 3, route_scatter_kernel: the list slot of a routed token is the
+// list length before the call + routed tokens of earlier tiles (a block sum
+// over the tile counts) + earlier routed tokens of its tile (ballot prefix),
+// so the list stays in position order.  Rows are copied warp-cooperatively;
+// mask words are updated with atomics where tiles share a word.  The last CTA
+// of each (b, kv head) sets full_cnt; the last CTA of the grid advances seq_len.
+#pragma once
+
+#include <cuda.h>
+
+#include "compress_params.cuh"
+#include "lrkv_common.cuh"
+#include "ptx.cuh"
+#include "tc_ptx.cuh"
+
+namespace lrkv {
+namespace ptc {
+
+constexpr int kTile = 128;                 // tokens per tile (MMA M)
+constexpr int kStages = 3;                 // input stages
+constexpr int kThreads = 192;              // warps 0-3 epilogue, 4 TMA, 5 MMA + TMEM
+constexpr int kStageBytes = kTile * kD * 2;          // two 64-column boxes
+constexpr int kBoxBytes = kStageBytes / 2;
+constexpr uint32_t kTmemCols = 512;                  // two buffers of [D1 | D2]
+constexpr uint32_t kWaitIters = 1u << 22;
+
+// shared memory (bytes); every operand region 1024-byte aligned
+constexpr int OFF_X = 0;
+constexpr int OFF_PHI = OFF_X + kStages * kStageBytes;      // B operand [N 128][K 128]
+constexpr int OFF_PLO = OFF_PHI + kD * kD * 2;
+constexpr int OFF_UT = OFF_PLO + kD * kD * 2;               // B operand U^T [N r][K 128]
+// rm = the larger rank of the launch (both tensors share one layout)
+__host__ __device__ inline constexpr int off_u(int rm) { return OFF_UT + rm * kD * 2; }  // U [128][K r]
+__host__ __device__ inline constexpr int off_bar(int rm) { return off_u(rm) + kD * rm * 2; }
+inline constexpr size_t smem_bytes(int rm) { return (size_t)off_bar(rm) + 128 + 1024; }
+
+struct Params {
+  CUtensorMap map_k;     // k_new viewed as [B*t_new][Hkv][d], box {64, 1, 128}
+  CUtensorMap map_v;
+  lrkv_dims D;
+  lrkv_cache C;
+  int t_new;
+  const int32_t* t_new_b;
+  float* errs;           // [2][B][Hkv][T_cap]
+  int tiles_per_b;       // ceil(min(t_new, T_cap) / 128)
+  int r_max;             // max(r_k, r_v): the shared-memory layout
+};
+
+// Byte offset of element (row n, column k) in a no-swizzle K-major operand:
+// 8x8 core matrices of 128 contiguous bytes, K-adjacent ones 128 B apart and
+// 8-row groups `sbo` bytes apart.
+__device__ __forceinline__ int core_off(int n, int k, int sbo) {
+  return (n >> 3) * sbo + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
+}
+
+// Tokens of row b in this call, and the position of the first one.
+__device__ __forceinline__ int eff_tokens(const Params& p, int b, int* start) {
+  uint32_t st = 0;
+  const int n = new_tokens(p.t_new_b, b, p.t_new, &st);
+  const int s0 = min(max(p.C.seq_len[b], 0), p.D.T_cap);
+  int ne = p.D.T_cap - s0;
+  if (ne > n) ne = n;
+  if (ne < 0) ne = 0;
+  *start = s0;
+  return ne;
+}
+
+// Bounded wait that also gives up once another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag) {
+  for (uint32_t i = 0; i < kWaitIters; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 63 && *abort_flag) return false;
+    if (i > 64) __nanosleep(32);
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+// grid (CTAs per group, 2 * Hkv): group = 2 h + tensor (0 keys, 1 values)
+__global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // the dynamic window is only guaranteed 16-byte aligned: round up to 1024
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const lrkv_dims& D = p.D;
+  const int group = blockIdx.y, tensor = group & 1, h = group >> 1;
+  const CUtensorMap* map = tensor == 0 ? &p.map_k : &p.map_v;
+  const int R = tensor == 0 ? D.r_k : D.r_v;
+  const int RM = p.r_max;
+  const lrkv_bf16* Ug = (tensor == 0 ? p.C.U_k : p.C.U_v) + (size_t)h * kD * R;
+  lrkv_bf16* coef = tensor == 0 ? p.C.coef_k : p.C.coef_v;
+  float* errs = p.errs + (size_t)tensor * D.B * D.Hkv * D.T_cap;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + off_bar(RM));
+  uint64_t* full = bars;                 // [kStages] TMA -> MMA
+  uint64_t* empty = bars + kStages;      // [kStages] epilogue -> TMA (128 arrivals)
+  uint64_t* dready = bars + 2 * kStages; // [2] MMA -> epilogue
+  uint64_t* tfree = dready + 2;          // [2] epilogue -> MMA (128 arrivals)
+  uint64_t* pready = tfree + 2;          // U U^T done
+  uint64_t* drain = pready + 1;          // final MMA drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  // this CTA's units: a contiguous range of the (b, tile) list of its group
+  const int n_units = D.B * p.tiles_per_b;
+  const int u_begin = (int)((long long)blockIdx.x * n_units / gridDim.x);
+  const int u_end = (int)((long long)(blockIdx.x + 1) * n_units / gridDim.x);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 128);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&dready[b], 1);
+      mbar_init(&tfree[b], 128);
+    }
+    mbar_init(pready, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tc5::tmem_alloc(tmem_slot, kTmemCols);
+    tc5::tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) tc5::prefetch_tensormap(map);
+  // U into two K-major no-swizzle operand layouts:
+  //   U   as [m = i][k = j]   (A and B of U U^T), 8-row groups 16 r bytes apart
+  //   U^T as [n = j][k = i]   (B of X U),         8-row groups 2048 bytes apart
+  {
+    unsigned char* su = sm + off_u(RM);
+    unsigned char* sut = sm + OFF_UT;
+    for (int idx = tid; idx < kD * R; idx += kThreads) {
+      const int i = idx / R, j = idx - (idx / R) * R;
+      const uint16_t u = Ug[idx];
+      *reinterpret_cast<uint16_t*>(su + core_off(i, j, 16 * R)) = u;
+      *reinterpret_cast<uint16_t*>(sut + core_off(j, i, 2048)) = u;
+    }
+  }
+  fence_proxy_async_smem();
+  tc5::fence_before_sync();
+  __syncthreads();
+  tc5::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  // ---- P = I - U U^T, split into bf16 high and low parts ----------------------------
+  if (warp == 5 && lane == 0) {
+    const uint32_t ub = smem_u32(sm + off_u(RM));
+    for (int j = 0; j < R / 16; ++j) {
+      const uint64_t d = tc5::smem_desc(ub + j * 256, 128, 16 * R, tc5::kSwizzleNone);
+      tc5::mma_bf16(tmem + 128, d, d, tc5::idesc_bf16_f32(128, 128), j > 0);
+    }
+    tc5::mma_commit(pready);
+  }
+  if (warp < 4) {
+    const int m = tid;   // row of U U^T = TMEM lane
+    if (!wait_or_abort(pready, 0, abort_flag)) {
+      atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
+    }
+    tc5::fence_after_sync();
+    unsigned char* phi = sm + OFF_PHI;
+    unsigned char* plo = sm + OFF_PLO;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kD; c0 += 16) {
+      float v[16];
+      tc5::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + 128 + c0, v);
+      tc5::tmem_wait_ld();
+      uint32_t hi[8], lo[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float a = (m == c0 + 2 * q ? 1.f : 0.f) - v[2 * q];
+        float b = (m == c0 + 2 * q + 1 ? 1.f : 0.f) - v[2 * q + 1];
+        const float ah = __bfloat162float(__float2bfloat16_rn(a));
+        const float bh = __bfloat162float(__float2bfloat16_rn(b));
+        hi[q] = pack_bf16(ah, bh);
+        lo[q] = pack_bf16(a - ah, b - bh);
+      }
+      // row m of P is row n = m of the B operand, columns c0..c0+15 = two core matrices
+      *reinterpret_cast<uint4*>(phi + core_off(m, c0, 2048)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(phi + core_off(m, c0 + 8, 2048)) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+      *reinterpret_cast<uint4*>(plo + core_off(m, c0, 2048)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(plo + core_off(m, c0 + 8, 2048)) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+    }
+  }
+  fence_proxy_async_smem();
+  tc5::fence_before_sync();
+  __syncthreads();
+  tc5::fence_after_sync();
+
+  // ---- pipeline over this CTA's tiles -------------------------------------------------
+  if (warp == 4) {
+    // TMA producer
+    if (lane == 0) {
+      int i = 0;
+      for (int u = u_begin; u < u_end && !*abort_flag; ++u) {
+        const int b = u / p.tiles_per_b, t0 = (u - b * p.tiles_per_b) * kTile;
+        int start;
+        if (t0 >= eff_tokens(p, b, &start)) continue;
+        const int s = i % kStages;
+        if (i >= kStages && !wait_or_abort(&empty[s], ((i / kStages) - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        unsigned char* dst = sm + OFF_X + s * kStageBytes;
+        const int z = b * p.t_new + t0;
+        tc5::tma_load_3d(dst, map, 0, h, z, &full[s]);
+        tc5::tma_load_3d(dst + kBoxBytes, map, 64, h, z, &full[s]);
+        ++i;
+      }
+      // leave no copy in flight: wait for the last fill of every stage
+      for (int k = (i > kStages ? i - kStages : 0); k < i; ++k)
+        mbar_wait_bounded(&full[k % kStages], (k / kStages) & 1, kWaitIters);
+    }
+  } else if (warp == 5) {
+    // MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc1 = tc5::idesc_bf16_f32(128, R);
+      const uint32_t idesc2 = tc5::idesc_bf16_f32(128, 128);
+      const uint32_t xbase = smem_u32(sm + OFF_X);
+      const uint32_t utb = smem_u32(sm + OFF_UT);
+      const uint32_t phb = smem_u32(sm + OFF_PHI);
+      const uint32_t plb = smem_u32(sm + OFF_PLO);
+      int i = 0;
+      for (int u = u_begin; u < u_end && !*abort_flag; ++u) {
+        const int b = u / p.tiles_per_b, t0 = (u - b * p.tiles_per_b) * kTile;
+        int start;
+        if (t0 >= eff_tokens(p, b, &start)) continue;
+        const int s = i % kStages, buf = i & 1;
+        if (!wait_or_abort(&full[s], (i / kStages) & 1, abort_flag)) break;
+        if (i >= 2 && !wait_or_abort(&tfree[buf], ((i >> 1) - 1) & 1, abort_flag)) break;
+        tc5::fence_after_sync();
+        const uint32_t d1 = tmem + buf * 256, d2 = d1 + 128;
+        const uint32_t xs = xbase + s * kStageBytes;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint64_t a = tc5::smem_desc(xs + (j >> 2) * kBoxBytes + (j & 3) * 32, 16, 1024,
+                                            tc5::kSwizzle128B);
+          tc5::mma_bf16(d1, a, tc5::smem_desc(utb + j * 256, 128, 2048, tc5::kSwizzleNone), idesc1,
+                        j > 0);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint64_t a = tc5::smem_desc(xs + (j >> 2) * kBoxBytes + (j & 3) * 32, 16, 1024,
+                                            tc5::kSwizzle128B);
+          tc5::mma_bf16(d2, a, tc5::smem_desc(phb + j * 256, 128, 2048, tc5::kSwizzleNone), idesc2,
+                        j > 0);
+          tc5::mma_bf16(d2, a, tc5::smem_desc(plb + j * 256, 128, 2048, tc5::kSwizzleNone), idesc2,
+                        1);
+        }
+        tc5::mma_commit(&dready[buf]);
+        ++i;
+      }
+      // every MMA done before the epilogue leaves and TMEM is freed
+      tc5::mma_commit(drain);
+      mbar_wait_bounded(drain, 0, kWaitIters);
+    }
+  } else {
+    // epilogue: thread m = row m of the tile = TMEM lane m
+    const int m = tid;
+    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    int i = 0;
+    for (int u = u_begin; u < u_end; ++u) {
+      const int b = u / p.tiles_per_b, t0 = (u - b * p.tiles_per_b) * kTile;
+      int start;
+      const int ne = eff_tokens(p, b, &start);
+      if (t0 >= ne) continue;
+      const int s = i % kStages, buf = i & 1;
+      if (!wait_or_abort(&dready[buf], (i >> 1) & 1, abort_flag)) break;
+      tc5::fence_after_sync();
+      const int t = t0 + m;
+      const bool valid = t < ne;
+      const size_t bh = (size_t)b * D.Hkv + h;
+      // coefficients
+      {
+        lrkv_bf16* crow = coef + (bh * D.T_cap + start + t) * R;
+#pragma unroll 1
+        for (int c0 = 0; c0 < R; c0 += 16) {
+          float v[16];
+          tc5::tmem_ld16(lane_base + buf * 256 + c0, v);
+          tc5::tmem_wait_ld();
+          if (valid) {
+            uint4 w0 = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                  pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+            uint4 w1 = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
+                                  pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
+            *reinterpret_cast<uint4*>(crow + c0) = w0;
+            *reinterpret_cast<uint4*>(crow + c0 + 8) = w1;
+          }
+        }
+      }
+      // squared residual
+      float rs = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kD; c0 += 16) {
+        float v[16];
+        tc5::tmem_ld16(lane_base + buf * 256 + 128 + c0, v);
+        tc5::tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) rs = fmaf(v[q], v[q], rs);
+      }
+      // squared input: row m of both 64-column boxes, every 16-byte chunk
+      // (the swizzle only permutes chunks within the row)
+      float xs = 0.f;
+      {
+        const unsigned char* xr = sm + OFF_X + s * kStageBytes + m * 128;
+#pragma unroll
+        for (int box = 0; box < 2; ++box) {
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const uint4 w = *reinterpret_cast<const uint4*>(xr + box * kBoxBytes + (((cc + m) & 7) << 4));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float a = bf_lo(ws[q]), c = bf_hi(ws[q]);
+              xs = fmaf(a, a, xs);
+              xs = fmaf(c, c, xs);
+            }
+          }
+        }
+      }
+      tc5::fence_before_sync();
+      mbar_arrive(&tfree[buf]);
+      mbar_arrive(&empty[s]);
+      if (valid) errs[bh * D.T_cap + t] = xs > 0.f ? sqrtf(rs / xs) : 0.f;
+      ++i;
+    }
+  }
+  if (*abort_flag && tid == 0) atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
+  tc5::fence_before_sync();
+  __syncthreads();
+  if (warp == 5) {
+    tc5::fence_after_sync();
+    tc5::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---- routing -------------------------------------------------------------------------
+
+struct RouteParams {
+  lrkv_dims D;
+  lrkv_cache C;
+  const lrkv_bf16* k_new;
+  const lrkv_bf16* v_new;
+  int t_new;
+  const int32_t* t_new_b;
+  float tau;
+  float* err_out;          // nullable [B][Hkv][t_new]
+  const float* errs;       // [2][B][Hkv][T_cap]
+  int32_t* tile_cnt;       // [B][Hkv][n_tiles]
+  uint32_t* tile_bits;     // [B][Hkv][n_tiles][4]
+  int n_tiles;
+  int32_t* bh_tickets;     // [B][Hkv], zero between calls
+  int32_t* ticket;         // [1], zero between calls
+};
+
+__device__ __forceinline__ int route_eff(const RouteParams& p, int b, int* start, uint32_t* st) {
+  const int n = new_tokens(p.t_new_b, b, p.t_new, st);
+  const int s0 = min(max(p.C.seq_len[b], 0), p.D.T_cap);
+  int ne = p.D.T_cap - s0;
+  if (ne > n) ne = n;
+  if (ne < 0) ne = 0;
+  *start = s0;
+  return ne;
+}
+
+// grid (tiles_per_b, Hkv, B), 128 threads
+__global__ void __launch_bounds__(128) route_count_kernel(RouteParams p) {
+  const lrkv_dims& D = p.D;
+  const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ int s_cnt[4];
+  uint32_t st = 0;
+  int start;
+  const int ne = route_eff(p, b, &start, &st);
+  const size_t bh = (size_t)b * D.Hkv + h;
+  const int t = tile * 128 + tid;
+  const bool valid = t < ne;
+  bool routed = false;
+  if (valid) {
+    const size_t i = bh * D.T_cap + t;
+    const float e = fmaxf(p.errs[i], p.errs[(size_t)D.B * D.Hkv * D.T_cap + i]);
+    routed = e > p.tau;
+    if (p.err_out) p.err_out[bh * p.t_new + t] = e;
+  }
+  const uint32_t bits = __ballot_sync(0xffffffffu, routed);
+  if (lane == 0) {
+    p.tile_bits[(bh * p.n_tiles + tile) * 4 + warp] = bits;
+    s_cnt[warp] = __popc(bits);
+  }
+  __syncthreads();
+  if (tid == 0) p.tile_cnt[bh * p.n_tiles + tile] = (s_cnt[0] + s_cnt[1]) + (s_cnt[2] + s_cnt[3]);
+}
+
+// grid (tiles_per_b, Hkv, B), 128 threads
+__global__ void __launch_bounds__(128) route_scatter_kernel(RouteParams p) {
+  const lrkv_dims& D = p.D;
+  const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ int s_red[4];
+  __shared__ int s_wcnt[4];
+  __shared__ bool s_last_bh, s_last;
+  uint32_t st = 0;
+  int start;
+  const int ne = route_eff(p, b, &start, &st);
+  const size_t bh = (size_t)b * D.Hkv + h;
+  const int32_t* cnt = p.tile_cnt + bh * p.n_tiles;
+  const int old = min(max(p.C.full_cnt[bh], 0), D.F_cap);
+  const int t0 = tile * 128;
+  bool overflow = false;
+  if (t0 < ne) {
+    // routed tokens of the earlier tiles of this (b, kv head)
+    int before = 0;
+    for (int i = tid; i < tile; i += 128) before += cnt[i];
+    before = (int)warp_sum((float)before);   // counts < 2^24: exact in fp32
+    if (lane == 0) s_red[warp] = before;
+    const uint32_t wbits = p.tile_bits[(bh * p.n_tiles + tile) * 4 + warp];
+    if (lane == 0) s_wcnt[warp] = __popc(wbits);
+    __syncthreads();
+    const int base = old + (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
+    int wbefore = 0;
+    for (int w = 0; w < warp; ++w) wbefore += s_wcnt[w];
+    const int t = t0 + tid;
+    const bool valid = t < ne;
+    const bool routed = (wbits >> lane) & 1u;
+    const int slot = base + wbefore + __popc(wbits & ((1u << lane) - 1u));
+    const bool keep = routed && slot < D.F_cap;
+    overflow = routed && !keep;
+    const int pos = start + t;
+    if (keep) p.C.full_idx[bh * D.F_cap + slot] = pos;
+    // mask words: this warp's 32 positions span at most two words
+    const uint32_t keep_b = __ballot_sync(0xffffffffu, keep);
+    const uint32_t valid_b = __ballot_sync(0xffffffffu, valid);
+    if (lane == 0 && valid_b) {
+      uint32_t* mrow = p.C.route_mask + bh * (D.T_cap / 32);
+      const int p0 = start + t0 + warp * 32;
+      const int w0 = p0 >> 5, sh = p0 & 31;
+      const uint32_t r0 = valid_b << sh, k0 = keep_b << sh;
+      if (r0) {
+        if (r0 == 0xffffffffu) mrow[w0] = k0;
+        else {
+          atomicAnd(&mrow[w0], ~r0);
+          if (k0) atomicOr(&mrow[w0], k0);
+        }
+      }
+      if (sh) {
+        const uint32_t r1 = valid_b >> (32 - sh), k1 = keep_b >> (32 - sh);
+        if (r1) {
+          atomicAnd(&mrow[w0 + 1], ~r1);
+          if (k1) atomicOr(&mrow[w0 + 1], k1);
+        }
+      }
+    }
+    // copy the kept rows, one row per warp pass (32 lanes x 8 bytes)
+    uint32_t todo = keep_b;
+    const int wslot0 = base + wbefore;
+    while (todo) {
+      const int src = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int ts = t0 + warp * 32 + src;
+      const int sl = wslot0 + __popc(wbits & ((1u << src) - 1u));
+      const size_t x = (((size_t)b * p.t_new + ts) * D.Hkv + h) * kD;
+      const uint2* ks = reinterpret_cast<const uint2*>(p.k_new + x);
+      const uint2* vs = reinterpret_cast<const uint2*>(p.v_new + x);
+      reinterpret_cast<uint2*>(p.C.full_k + (bh * D.F_cap + sl) * kD)[lane] = ks[lane];
+      reinterpret_cast<uint2*>(p.C.full_v + (bh * D.F_cap + sl) * kD)[lane] = vs[lane];
+    }
+  }
+  if (__syncthreads_or(overflow)) st |= LRKV_DEV_FULL_OVERFLOW;
+  if (tile == 0 && h == 0) {
+    uint32_t dummy = 0;
+    const int n = new_tokens(p.t_new_b, b, p.t_new, &dummy);
+    if (ne < n) st |= LRKV_DEV_SEQ_OVERFLOW;
+  } else {
+    st &= LRKV_DEV_FULL_OVERFLOW;   // per-sequence conditions: reported once
+  }
+  if (tid == 0 && st) atomicOr(p.C.dev_status, st);
+  // the last CTA of this (b, kv head) sets its list length
+  __syncthreads();
+  if (tid == 0) s_last_bh = atom_add_acq_rel_gpu(&p.bh_tickets[bh], 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (s_last_bh) {
+    int tot = 0;
+    const int nt = (ne + 127) / 128;
+    for (int i = tid; i < nt; i += 128) tot += cnt[i];
+    tot = (int)warp_sum((float)tot);
+    if (lane == 0) s_red[warp] = tot;
+    __syncthreads();
+    if (tid == 0) {
+      const int total = (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
+      p.C.full_cnt[bh] = min(old + total, D.F_cap);
+      p.bh_tickets[bh] = 0;
+      s_last = atom_add_acq_rel_gpu(p.ticket, 1) == (int)(gridDim.y * gridDim.z) - 1;
+    }
+    __syncthreads();
+    if (s_last) {   // every (b, kv head) done: all seq_len reads are behind us
+      for (int bb = tid; bb < D.B; bb += 128) {
+        uint32_t dummy = 0;
+        const int nb = new_tokens(p.t_new_b, bb, p.t_new, &dummy);
+        const int sb = min(max(p.C.seq_len[bb], 0), D.T_cap);
+        int e2 = D.T_cap - sb;
+        if (e2 > nb) e2 = nb;
+        if (e2 < 0) e2 = 0;
+        p.C.seq_len[bb] = sb + e2;
+      }
+      if (tid == 0) *p.ticket = 0;
+    }
+  }
+}
+
+}  // namespace ptc
+}  // namespace lrkv

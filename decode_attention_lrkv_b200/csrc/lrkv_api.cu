@@ -3,8 +3,11 @@
 #include <cmath>
 #include <cstdint>
 
+#include <cuda.h>
+
 #include "compress_append.cuh"
-#include "compress_simple.cuh"
+#include "compress_params.cuh"
+#include "compress_tc.cuh"
 #include "decode_launch.cuh"
 #include "lrkv.h"
 #include "lrkv_common.cuh"
@@ -58,6 +61,87 @@ lrkv_status launched() {
   return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// New key or value rows [B][t_new][Hkv][d] as a 3-d tensor (d, Hkv, B * t_new),
+// boxes of 64 columns x 1 head x 128 tokens, 128-byte swizzle.
+bool rows_map(CUtensorMap* map, const lrkv_bf16* base, const lrkv_dims& D, int t_new) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)D.Hkv, (cuuint64_t)D.B * t_new};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)D.Hkv * kD * 2};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)ptc::kTile};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<lrkv_bf16*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Prefill-sized compress: tensor-core projection, then the two routing passes.
+lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16* k_new,
+                        const lrkv_bf16* v_new, int t_new, const int32_t* t_new_b, float tau,
+                        float* err_out, char* w, const WsLayout& L, cudaStream_t s) {
+  ptc::Params pp;
+  if (!rows_map(&pp.map_k, k_new, D, t_new) || !rows_map(&pp.map_v, v_new, D, t_new))
+    return LRKV_ERR_CUDA;
+  const int tmax = t_new < D.T_cap ? t_new : D.T_cap;
+  pp.D = D;
+  pp.C = C;
+  pp.t_new = t_new;
+  pp.t_new_b = t_new_b;
+  pp.errs = reinterpret_cast<float*>(w + L.errs);
+  pp.tiles_per_b = (tmax + ptc::kTile - 1) / ptc::kTile;
+  pp.r_max = D.r_k > D.r_v ? D.r_k : D.r_v;
+  const int groups = 2 * D.Hkv;
+  const int n_units = D.B * pp.tiles_per_b;
+  int per_group = kNumSMs / groups;
+  if (per_group < 1) per_group = 1;
+  if (per_group > n_units) per_group = n_units;
+  const size_t smem = ptc::smem_bytes(pp.r_max);
+  if (cudaFuncSetAttribute(ptc::project_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return launched(), LRKV_ERR_CUDA;
+  ptc::project_tc_kernel<<<dim3(per_group, groups), ptc::kThreads, smem, s>>>(pp);
+  lrkv_status st = launched();
+  if (st != LRKV_OK) return st;
+  ptc::RouteParams rp;
+  rp.D = D;
+  rp.C = C;
+  rp.k_new = k_new;
+  rp.v_new = v_new;
+  rp.t_new = t_new;
+  rp.t_new_b = t_new_b;
+  rp.tau = tau;
+  rp.err_out = err_out;
+  rp.errs = pp.errs;
+  rp.tile_cnt = reinterpret_cast<int32_t*>(w + L.tile_cnt);
+  rp.tile_bits = reinterpret_cast<uint32_t*>(w + L.tile_bits);
+  rp.n_tiles = L.n_tiles;
+  rp.bh_tickets = reinterpret_cast<int32_t*>(w + L.decode_tickets);
+  rp.ticket = reinterpret_cast<int32_t*>(w + L.compress_ticket);
+  const dim3 grid(pp.tiles_per_b, D.Hkv, D.B);
+  ptc::route_count_kernel<<<grid, 128, 0, s>>>(rp);
+  if ((st = launched()) != LRKV_OK) return st;
+  ptc::route_scatter_kernel<<<grid, 128, 0, s>>>(rp);
+  return launched();
+}
+
 }  // namespace
 
 extern "C" {
@@ -91,7 +175,6 @@ lrkv_status lrkv_compress(const lrkv_dims* dims, const lrkv_cache* cache,
   p.t_new_b = t_new_b;
   p.tau = tau;
   p.err_out = err_out;
-  p.flags = reinterpret_cast<uint8_t*>(w + L.flags);
   p.ticket = reinterpret_cast<int32_t*>(w + L.compress_ticket);
   if (t_new <= kAppendMaxTokens) {  // decode-time appends: one fused launch
     const size_t smem = append_smem_bytes(dims->r_k, dims->r_v);
@@ -101,16 +184,7 @@ lrkv_status lrkv_compress(const lrkv_dims* dims, const lrkv_cache* cache,
     append_kernel<<<dim3(dims->Hkv, dims->B), kAppendThreads, smem, s>>>(p);
     return launched();
   }
-  const int tmax = t_new < dims->T_cap ? t_new : dims->T_cap;
-  const size_t smem = proj_smem_bytes(dims->r_k > dims->r_v ? dims->r_k : dims->r_v);
-  if (cudaFuncSetAttribute(project_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return launched(), LRKV_ERR_CUDA;
-  project_kernel<<<dim3((tmax + kProjTok - 1) / kProjTok, dims->Hkv, dims->B), kProjThreads, smem,
-                   s>>>(p);
-  if ((st = launched()) != LRKV_OK) return st;
-  compact_kernel<<<dim3(dims->Hkv, dims->B), kCompactThreads, 0, s>>>(p);
-  return launched();
+  return compress_tc(*dims, *cache, k_new, v_new, t_new, t_new_b, tau, err_out, w, L, s);
 }
 
 lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache, const lrkv_bf16* q,

@@ -47,7 +47,10 @@ __device__ __forceinline__ int new_tokens(const int32_t* t_new_b, int b, int t_n
 struct WsLayout {
   size_t decode_tickets;   // int32 [B][Hkv], zero between calls
   size_t compress_ticket;  // int32 [1], zero between calls
-  size_t flags;            // uint8 [B][Hkv][T_cap] routing flags of a compress call
+  size_t errs;             // float [2][B][Hkv][T_cap] e_k, e_v of a prefill compress call
+  size_t tile_cnt;         // int32 [B][Hkv][n_tiles] routed tokens per 128-token tile
+  size_t tile_bits;        // uint32 [B][Hkv][n_tiles][4] routed bits per tile
+  int n_tiles;             // ceil(T_cap / 128)
   size_t partials;         // float [B][Hkv][n_chunk_max][g][2 + r_v + d]
   size_t total;
   int chunk;               // decode: positions per split
@@ -57,15 +60,12 @@ struct WsLayout {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Positions per decode split.  One CTA per SM: choose the number of waves W
-// so that a split holds at most 2048 positions, then give every (batch row,
-// kv head) floor(W * SMs / rows) splits, so the grid is close to W full
-// waves.  At least 128 positions, a multiple of 32 (one mask word).
+// Positions per decode split: at least 128, a multiple of 32 (one mask word),
+// at most kMaxDecodeChunk.  The split count n minimises the modelled makespan
+//   ceil(B*Hkv*n / SMs) * (chunk + overhead)
+// with one CTA per SM resident at a time; `overhead` is a CTA's fixed cost
+// (bases, q~, merge) expressed in streamed positions.
 inline int decode_chunk(const lrkv_dims& D) {
-  // Pick the split count n that minimises the modelled makespan
-  //   ceil(B*Hkv*n / SMs) * (chunk + overhead)
-  // with one CTA per SM resident at a time; `overhead` is a CTA's fixed cost
-  // (bases, q~, merge) expressed in streamed positions.
   const long long bh = (long long)D.B * D.Hkv;
   const long long overhead = 1024;
   long long best_cost = -1, best = kMaxDecodeChunk;
@@ -90,8 +90,13 @@ inline WsLayout ws_layout(const lrkv_dims& D) {
   off = align_up(off + sizeof(int32_t) * (size_t)D.B * D.Hkv, 256);
   L.compress_ticket = off;
   off = align_up(off + sizeof(int32_t), 256);
-  L.flags = off;
-  off = align_up(off + (size_t)D.B * D.Hkv * D.T_cap, 256);
+  L.n_tiles = (D.T_cap + 127) / 128;
+  L.errs = off;
+  off = align_up(off + sizeof(float) * 2 * (size_t)D.B * D.Hkv * D.T_cap, 256);
+  L.tile_cnt = off;
+  off = align_up(off + sizeof(int32_t) * (size_t)D.B * D.Hkv * L.n_tiles, 256);
+  L.tile_bits = off;
+  off = align_up(off + sizeof(uint32_t) * 4 * (size_t)D.B * D.Hkv * L.n_tiles, 256);
   L.chunk = decode_chunk(D);
   L.n_chunk_max = (D.T_cap + L.chunk - 1) / L.chunk;
   L.partial_floats = 2 + D.r_v + D.d;

@@ -211,3 +211,19 @@ def test_small_multi_token_appends_with_ragged_counts():
                                   band=band)
         out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
         assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
+
+
+def test_prefill_in_two_parts_unaligned_start():
+    """Two prefill calls, the second starting mid mask word, with several
+    128-token tiles per projection CTA (stage and accumulator buffers reused)."""
+    w = synth.workload(1, B=2, T=3000, layers=1)
+    layer, D, cache, oc, ws = _setup(w, seed=9, T_cap=3008)
+    K, V = layer["K"], layer["V"]
+    cut = 1237
+    gc, band = _compress_both(D, cache, oc, K[:, :cut].contiguous(), V[:, :cut].contiguous(),
+                              w.tau, ws, t_new_b=[cut, 1000])
+    gc, band = _compress_both(D, cache, oc, K[:, cut:].contiguous(), V[:, cut:].contiguous(),
+                              w.tau, ws, t_new_b=[3000 - cut, 1500], band=band)
+    assert list(gc.seq_len) == [3000, 2500]
+    out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
+    assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
