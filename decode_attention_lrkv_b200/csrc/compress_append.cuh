@@ -110,6 +110,18 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
   __shared__ float s_err[2];
   __shared__ uint32_t s_mask[2];    // the (at most two) mask words the new positions touch
 
+  // bases first: they do not depend on the preceding kernel of the stream
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    const uint32_t bk = kD * r_k * 2, bv = kD * r_v * 2;
+    mbar_expect_tx(bar, bk + bv);
+    bulk_g2s(Uks, p.C.U_k + (size_t)h * kD * r_k, bk, bar);
+    bulk_g2s(Uvs, p.C.U_v + (size_t)h * kD * r_v, bv, bar);
+  }
+  griddep_launch_dependents();
+  griddep_wait();   // the new rows and the cache state come from earlier kernels
+
   uint32_t st = 0;
   const int n = new_tokens(p.t_new_b, b, p.t_new, &st);
   const int start = min(max(p.C.seq_len[b], 0), D.T_cap);
@@ -119,31 +131,29 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
   const size_t bh = (size_t)b * D.Hkv + h;
   uint32_t* mask_row = p.C.route_mask + bh * (D.T_cap / 32);
 
-  if (n_eff > 0) {
-    if (tid == 0) {
-      mbar_init(bar, 1);
-      fence_mbar_init();
-      const uint32_t bk = kD * r_k * 2, bv = kD * r_v * 2;
-      mbar_arrive_expect_tx(bar, bk + bv + n_eff * 4u * kD);
-      bulk_g2s(Uks, p.C.U_k + (size_t)h * kD * r_k, bk, bar);
-      bulk_g2s(Uvs, p.C.U_v + (size_t)h * kD * r_v, bv, bar);
-      for (int t = 0; t < n_eff; ++t) {
-        const size_t x = (((size_t)b * p.t_new + t) * D.Hkv + h) * kD;
-        bulk_g2s(Xks + t * kD, p.k_new + x, 2u * kD, bar);
-        bulk_g2s(Xvs + t * kD, p.v_new + x, 2u * kD, bar);
-      }
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar, n_eff * 4u * kD);   // the arrival that closes the phase
+    for (int t = 0; t < n_eff; ++t) {
+      const size_t x = (((size_t)b * p.t_new + t) * D.Hkv + h) * kD;
+      bulk_g2s(Xks + t * kD, p.k_new + x, 2u * kD, bar);
+      bulk_g2s(Xvs + t * kD, p.v_new + x, 2u * kD, bar);
+    }
+    if (n_eff > 0) {
       s_cnt = min(max(p.C.full_cnt[bh], 0), D.F_cap);
       s_mask[0] = mask_row[start >> 5];
       s_mask[1] = ((start + n_eff - 1) >> 5) != (start >> 5) ? mask_row[(start >> 5) + 1] : 0u;
     }
-    __syncthreads();
-    if (!mbar_wait_bounded(bar, 0, kAppendWaitIters)) st |= LRKV_DEV_WAIT_TIMEOUT;
-    if (__syncthreads_or(st & LRKV_DEV_WAIT_TIMEOUT)) {
-      mbar_wait_bounded(bar, 0, kAppendWaitIters);   // one more bounded wait for the copies
-      st |= LRKV_DEV_WAIT_TIMEOUT;
-      if (tid == 0) atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
-      n_eff = 0;   // leave the cache untouched; the call's results are flagged invalid
-    }
+  }
+  __syncthreads();
+  // every copy (bases included) lands before anything else, also when there is no token
+  if (!mbar_wait_bounded(bar, 0, kAppendWaitIters)) st |= LRKV_DEV_WAIT_TIMEOUT;
+  if (__syncthreads_or(st & LRKV_DEV_WAIT_TIMEOUT)) {
+    mbar_wait_bounded(bar, 0, kAppendWaitIters);   // one more bounded wait for the copies
+    st |= LRKV_DEV_WAIT_TIMEOUT;
+    if (tid == 0) atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
+    n_eff = 0;   // leave the cache untouched; the call's results are flagged invalid
+  }
+  if (n_eff > 0) {
     bool overflow = false;
     for (int t = 0; t < n_eff; ++t) {
       const int pos = start + t;

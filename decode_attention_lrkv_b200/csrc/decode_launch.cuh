@@ -1,24 +1,24 @@
 // Decode dispatch shared by lrkv_decode_attn and lrkv_decode_attn_noalloc:
-// the tensor-core pipeline kernel for the shapes it is instantiated for, the
+// the tensor-core streaming kernel for the shapes it is instantiated for, the
 // CUDA-core kernel for every other valid shape.
 #pragma once
 
-#include "decode_tc.cuh"
 #include "decode_simple.cuh"
+#include "decode_stream.cuh"
+#include "launch_util.cuh"
 
 namespace lrkv {
 
 template <int G, int RK, int RV>
-inline lrkv_status launch_fast(const DecodeParams& p, dim3 grid, cudaStream_t s) {
-  using S = tc::Shape<G, RK, RV>;
-  auto kern = tc::decode_tc_kernel<G, RK, RV>;
+inline lrkv_status launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t s) {
+  using S = ds::Shape<G, RK, RV>;
+  auto kern = ds::decode_stream_kernel<G, RK, RV>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM) !=
       cudaSuccess) {
     cudaGetLastError();
     return LRKV_ERR_CUDA;
   }
-  kern<<<grid, tc::kThreads, S::SMEM, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+  return launch_pdl(kern, grid, dim3(ds::kThreads), S::SMEM, s, p);
 }
 
 template <int G>
@@ -34,25 +34,23 @@ inline lrkv_status launch_simple(const DecodeParams& p, dim3 grid, cudaStream_t 
 }
 
 template <int G>
-inline lrkv_status launch_fast_g(const DecodeParams& p, dim3 grid, cudaStream_t s, bool* done) {
+inline lrkv_status launch_stream_g(const DecodeParams& p, dim3 grid, cudaStream_t s, bool* done) {
   *done = true;
   const int rk = p.D.r_k, rv = p.D.r_v;
-  if (rk == 32 && rv == 32) return launch_fast<G, 32, 32>(p, grid, s);
-  if (rk == 48 && rv == 64) return launch_fast<G, 48, 64>(p, grid, s);
-  if (rk == 48 && rv == 80) return launch_fast<G, 48, 80>(p, grid, s);
-  if (rk == 64 && rv == 64) return launch_fast<G, 64, 64>(p, grid, s);
-  if (rk == 64 && rv == 96) return launch_fast<G, 64, 96>(p, grid, s);
+  if (rk == 32 && rv == 32) return launch_stream<G, 32, 32>(p, grid, s);
+  if (rk == 48 && rv == 64) return launch_stream<G, 48, 64>(p, grid, s);
+  if (rk == 48 && rv == 80) return launch_stream<G, 48, 80>(p, grid, s);
+  if (rk == 64 && rv == 64) return launch_stream<G, 64, 64>(p, grid, s);
+  if (rk == 64 && rv == 96) return launch_stream<G, 64, 96>(p, grid, s);
   *done = false;
   return LRKV_OK;
 }
 
-// Whether the pipeline kernel covers these sizes.
-inline bool fast_decode_supported(const lrkv_dims& D, int chunk, int n_chunk_max) {
+// Whether the streaming kernel covers these sizes.
+inline bool stream_decode_supported(const lrkv_dims& D, int chunk) {
   const int g = D.Hq / D.Hkv;
   if (g != 1 && g != 2 && g != 4) return false;
-  if (chunk > tc::kMaxChunk || chunk % 32) return false;
-  // the merge keeps a max and a sum per (split, head) in the staging area (>= 10 KiB)
-  if ((long long)n_chunk_max * g * 8 > 10 * 1024) return false;
+  if (chunk > ds::kMaxChunk || chunk % 32) return false;
   const int rk = D.r_k, rv = D.r_v;
   return (rk == 32 && rv == 32) || (rk == 48 && rv == 64) || (rk == 48 && rv == 80) ||
          (rk == 64 && rv == 64) || (rk == 64 && rv == 96);
@@ -61,12 +59,12 @@ inline bool fast_decode_supported(const lrkv_dims& D, int chunk, int n_chunk_max
 inline lrkv_status launch_decode(const DecodeParams& p, cudaStream_t s) {
   const dim3 grid(p.n_chunk_max, p.D.Hkv, p.D.B);
   const int g = p.D.Hq / p.D.Hkv;
-  if (fast_decode_supported(p.D, p.chunk, p.n_chunk_max)) {
+  if (stream_decode_supported(p.D, p.chunk)) {
     bool done = false;
     lrkv_status st = LRKV_OK;
-    if (g == 1) st = launch_fast_g<1>(p, grid, s, &done);
-    else if (g == 2) st = launch_fast_g<2>(p, grid, s, &done);
-    else st = launch_fast_g<4>(p, grid, s, &done);
+    if (g == 1) st = launch_stream_g<1>(p, grid, s, &done);
+    else if (g == 2) st = launch_stream_g<2>(p, grid, s, &done);
+    else st = launch_stream_g<4>(p, grid, s, &done);
     if (done) return st;
   }
   switch (g) {

@@ -1,0 +1,570 @@
+// Read path, B200 version: split-K decode attention over the compressed
+// cache, logits and value sums on the tensor cores.
+//
+// Coefficient-space form of the StaticPCA read path (OjaKV repository
+// README, "Method Summary > StaticPCA": keys and values reconstructed on the
+// fly for standard attention).  With q~ = U_k^T q, a compressed token's logit
+// is q~ . c_k / sqrt(d) and its value contribution is accumulated in r_v
+// space, lifted by U_v once per split; full-rank tokens ("Method Summary >
+// OjaKV", hybrid storage) use their stored rows.  One softmax covers both.
+//
+// Why mma.sync: per kv head the work is [tokens x r] x [r x g] and
+// [r x tokens] x [tokens x g] with g <= 4 query heads.  On CUDA cores that is
+// tens of instructions per token and the kernel is issue-bound far below the
+// HBM roof; as m16n8k16 MMAs it is a handful.  Tokens are the M dimension and
+// the query heads the N dimension: q~ and the probabilities p are fp32, so
+// each is split into a bf16 high part (columns 0..3) and low part (columns
+// 4..7) and the two columns of a head are summed afterwards -- fp32-level
+// accuracy.  tcgen05 wants M >= 64 per instruction and a single issuing
+// thread; here N is 8 and the contraction per tile is tiny, so the
+// warp-level MMA keeps the whole per-token chain inside one warp.
+//
+// Work split.  Grid (splits, Hkv, B), one CTA of 8 warps per SM (255
+// registers per thread).  A CTA takes positions [c*chunk, (c+1)*chunk) of one
+// (batch row, kv head) and an equal share of its full-rank list.  Each warp
+// streams its own tiles through a 2-stage cp.async ring:
+//   - a compressed tile is 32 consecutive positions, copied in place with
+//     16-byte pieces, consecutive lanes on consecutive bytes; a routed
+//     position (mask bit set) or one past the end is zero-filled instead of
+//     read, and its logit is -inf;
+//   - a full-rank tile is 16 list rows (keys, then values).
+// Rows land in padded shared-memory rows (stride 2r+16 bytes) so ldmatrix is
+// conflict-free.  At the end each warp leaves its partial softmax state in its
+// own ring slots, the CTA merges its warps, lifts by U_v (MMA), writes one
+// record (m, l, o[d]) per query head, and the last CTA of the (batch row, kv
+// head) merges all records (atomic ticket, no waiting).
+//
+// Programmatic dependent launch: the bases and q are loaded before waiting on
+// the preceding kernel of the stream (an append to the same cache); every
+// read of cache state comes after the wait.
+#pragma once
+
+#include <type_traits>
+
+#include "decode_simple.cuh"
+#include "lrkv_common.cuh"
+#include "ptx.cuh"
+
+namespace lrkv {
+namespace ds {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kStages = 2;
+constexpr int kTileC = 32;                       // positions per compressed tile (one mask word)
+constexpr int kTileF = 16;                       // rows per full-rank tile
+constexpr int kMaxChunk = kMaxDecodeChunk;       // positions per split (mask words in smem)
+constexpr int kRecFloats = 4 + kD;               // m, l, (pad), o[d]: 16-byte multiple
+constexpr uint32_t kWaitIters = 1u << 24;        // bounded mbarrier polls (seconds)
+constexpr unsigned kFull = 0xffffffffu;
+
+constexpr int al16(int x) { return (x + 15) & ~15; }
+constexpr int al128(int x) { return (x + 127) & ~127; }
+constexpr int imax(int a, int b) { return a > b ? a : b; }
+
+template <int G, int RK, int RV>
+struct Shape {
+  static_assert(G == 1 || G == 2 || G == 4, "1, 2 or 4 query heads per kv head");
+  static_assert(RK % 16 == 0 && RV % 16 == 0 && RK <= kD && RV <= kD, "ranks");
+  static constexpr int KP = RK / 8, VP = RV / 8;   // 16-byte pieces per row
+  static constexpr int KS = 2 * RK + 16;           // padded row strides (bytes): odd multiples of 16
+  static constexpr int VS = 2 * RV + 16;
+  static constexpr int FS = 2 * kD + 16;
+  static constexpr int SLOT_C = kTileC * (KS + VS);
+  static constexpr int SLOT_F = kTileF * 2 * FS;
+  static constexpr int SLOT = al128(imax(SLOT_C, SLOT_F));
+  static constexpr int OFF_UK = kWarps * kStages * SLOT;      // U_k rows [d][KS]
+  static constexpr int OFF_UV = al128(OFF_UK + kD * KS);      // U_v rows [d][VS]
+  static constexpr int OFF_MASK = al128(OFF_UV + kD * VS);
+  static constexpr int OFF_BAR = al16(OFF_MASK + (kMaxChunk / 32) * 4);   // merge, bases mbarriers
+  static constexpr int SMEM = OFF_BAR + 16;
+  static_assert(SMEM <= 227 * 1024, "shared memory of one CTA");
+  // per-warp partial state in the warp's own ring slots (floats)
+  static constexpr int W_PC = 0;                    // [G][RV]
+  static constexpr int W_PF = W_PC + G * RV;        // [G][d]
+  static constexpr int W_M = W_PF + G * kD;         // [G]
+  static constexpr int W_L = W_M + G;               // [G]
+  static_assert((W_L + G) * 4 <= kStages * SLOT, "partials fit in a warp's slots");
+  // CTA merge in the U_k area (free once every warp has its q~)
+  static constexpr int C_CC = 0;                    // [G][RV] merged acc_c
+  static constexpr int C_CF = C_CC + G * RV;        // [G][d] merged acc_f
+  static constexpr int C_M = C_CF + G * kD;         // [G] max, [G] sum
+  static constexpr int C_WE = C_M + 2 * G;          // [warps][G] warp weights
+  static_assert((C_WE + kWarps * G) * 4 <= kD * KS, "merge scratch fits in the U_k area");
+};
+
+template <int G, int RK, int RV>
+__global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams p) {
+  using S = Shape<G, RK, RV>;
+  constexpr int KST = RK / 16;                   // k-steps of the compressed logits
+  constexpr int MVT = RV / 16;                   // m-tiles of the compressed value sum
+  constexpr int KP = S::KP, VP = S::VP;
+  extern __shared__ __align__(128) unsigned char sm[];
+  const lrkv_dims& D = p.D;
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;         // MMA fragment coordinates
+  const bool lo_col = t >= 2;                    // columns 4..7 hold the bf16 low parts
+  const int ha = 2 * (t & 1);                    // heads ha, ha + 1 of this lane's two columns
+  const int lm = lane >> 3, lr = lane & 7;       // ldmatrix address roles
+  const size_t bh = (size_t)b * D.Hkv + h;
+
+  unsigned char* uk = sm + S::OFF_UK;
+  unsigned char* uv = sm + S::OFF_UV;
+  uint32_t* maskw = reinterpret_cast<uint32_t*>(sm + S::OFF_MASK);
+  uint64_t* merge_bar = reinterpret_cast<uint64_t*>(sm + S::OFF_BAR);
+  uint64_t* base_bar = merge_bar + 1;
+  unsigned char* ring = sm + (size_t)warp * kStages * S::SLOT;
+  __shared__ int s_last;
+
+  // ---- prologue, independent of the preceding kernel: bases and q ------------------
+  if (tid == 0) {
+    mbar_init(merge_bar, 1);
+    mbar_init(base_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) {  // both bases into padded rows, one bulk copy per row
+    const lrkv_bf16* Uk = p.C.U_k + (size_t)h * kD * RK;
+    const lrkv_bf16* Uv = p.C.U_v + (size_t)h * kD * RV;
+    if (lane == 0) mbar_arrive_expect_tx(base_bar, kD * 2u * (RK + RV));
+    __syncwarp();
+    for (int r = lane; r < kD; r += 32) {
+      bulk_g2s(uk + r * S::KS, Uk + (size_t)r * RK, 2u * RK, base_bar);
+      bulk_g2s(uv + r * S::VS, Uv + (size_t)r * RV, 2u * RV, base_bar);
+    }
+  }
+  // q as fragments over k = d: the B operand of the full-rank logits (column
+  // n = head n < G; q is bf16, hence exact, so no low-part columns) and, the
+  // same bytes, the A operand (rows = heads) of q~ = U_k^T q
+  uint32_t qf0[8], qf1[8];
+  {
+    const lrkv_bf16* qrow = p.q + ((size_t)b * D.Hq + (size_t)h * G + (g < G ? g : 0)) * kD;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qf0[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
+      qf1[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
+    }
+  }
+  const float scale = kLog2e * rsqrtf((float)kD);
+
+  // ---- cache state: after the preceding kernel (an append) has completed ------------
+  griddep_wait();
+  int T = p.C.seq_len[b];
+  T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
+  const int n_chunks = T > 0 ? (T + p.chunk - 1) / p.chunk : 1;
+  if (c >= n_chunks) {   // no work: let the bases land before leaving
+    mbar_wait_bounded(base_bar, 0, kWaitIters);
+    return;
+  }
+  const int c0 = c * p.chunk;
+  const int c1 = min(T, c0 + p.chunk);
+  const int n_pos = c1 > c0 ? c1 - c0 : 0;
+  const int F = min(max(p.C.full_cnt[bh], 0), D.F_cap);
+  const int share = (F + n_chunks - 1) / n_chunks;
+  const int f0 = min(F, c * share), f1 = min(F, f0 + share);
+  const int n_full = f1 - f0;
+  const lrkv_bf16* ck = p.C.coef_k + bh * D.T_cap * RK + (size_t)c0 * RK;
+  const lrkv_bf16* cv = p.C.coef_v + bh * D.T_cap * RV + (size_t)c0 * RV;
+  const lrkv_bf16* fk = p.C.full_k + (bh * D.F_cap + f0) * kD;
+  const lrkv_bf16* fv = p.C.full_v + (bh * D.F_cap + f0) * kD;
+  {
+    const int n_words = (n_pos + 31) / 32;
+    const uint32_t* mask_g = p.C.route_mask + bh * (D.T_cap / 32) + c0 / 32;
+    for (int i = tid; i < n_words; i += kThreads) maskw[i] = mask_g[i];
+  }
+  __syncthreads();
+
+  // this warp's tiles: full-rank ones first (they need only q), then compressed ones
+  const int n_ct = (n_pos + kTileC - 1) / kTileC;
+  const int n_ft = (n_full + kTileF - 1) / kTileF;
+  const int nct_w = n_ct > warp ? (n_ct - warp + kWarps - 1) / kWarps : 0;
+  const int nft_w = n_ft > warp ? (n_ft - warp + kWarps - 1) / kWarps : 0;
+  const int n_tiles = nct_w + nft_w;
+  // tile i of this warp: i < nft_w -> full-rank tile warp + kWarps*i, else
+  // compressed tile warp + kWarps*(i - nft_w)
+
+  // positions of compressed tile k that are read: unmasked and before the end
+  auto tile_bits = [&](int k) -> uint32_t {
+    const int nv = n_pos - k * kTileC;
+    const uint32_t valid = nv >= 32 ? kFull : ((1u << nv) - 1u);
+    return ~maskw[k] & valid;
+  };
+  auto issue = [&](int i) {
+    unsigned char* slot = ring + (i % kStages) * S::SLOT;
+    if (i >= nft_w) {
+      const int k = warp + kWarps * (i - nft_w);
+      const uint32_t bits = tile_bits(k);
+      const unsigned char* src_k = reinterpret_cast<const unsigned char*>(ck + (size_t)k * kTileC * RK);
+      const unsigned char* src_v = reinterpret_cast<const unsigned char*>(cv + (size_t)k * kTileC * RV);
+#pragma unroll
+      for (int j = 0; j < KP; ++j) {   // piece q = lane + 32 j of the tile's key rows
+        const int q = lane + 32 * j, r = q / KP, sg = q - r * KP;
+        const bool on = (bits >> r) & 1u;
+        cp_async16_zfill(slot + r * S::KS + sg * 16, on ? src_k + q * 16 : src_k, on ? 16u : 0u);
+      }
+      unsigned char* vslot = slot + kTileC * S::KS;
+#pragma unroll
+      for (int j = 0; j < VP; ++j) {
+        const int q = lane + 32 * j, r = q / VP, sg = q - r * VP;
+        const bool on = (bits >> r) & 1u;
+        cp_async16_zfill(vslot + r * S::VS + sg * 16, on ? src_v + q * 16 : src_v, on ? 16u : 0u);
+      }
+    } else {
+      const int k = warp + kWarps * i;
+      const int r0 = k * kTileF;
+      const int n = min(kTileF, n_full - r0);
+      const unsigned char* src_k = reinterpret_cast<const unsigned char*>(fk + (size_t)r0 * kD);
+      const unsigned char* src_v = reinterpret_cast<const unsigned char*>(fv + (size_t)r0 * kD);
+      const int sg = lane & 15;
+#pragma unroll
+      for (int j = 0; j < kTileF / 2; ++j) {
+        const int r = (lane >> 4) + 2 * j;
+        const bool on = r < n;
+        const int off = r * kD * 2 + sg * 16;
+        cp_async16_zfill(slot + r * S::FS + sg * 16, on ? src_k + off : src_k, on ? 16u : 0u);
+        cp_async16_zfill(slot + (kTileF + r) * S::FS + sg * 16, on ? src_v + off : src_v,
+                         on ? 16u : 0u);
+      }
+    }
+  };
+#pragma unroll
+  for (int s = 0; s < kStages - 1; ++s) {
+    if (s < n_tiles) issue(s);
+    cp_async_commit();
+  }
+
+  // q~ = U_k^T q as this warp's B fragments over k = r_k (column n < 4 = bf16
+  // high part of head n, n >= 4 = low part of head n - 4), on the tensor cores,
+  // while the first tiles are in flight
+  bool bases_ok = true;
+  uint32_t qb0[KST], qb1[KST];
+  if (nct_w > 0) {
+    bases_ok = mbar_wait_bounded(base_bar, 0, kWaitIters);
+#pragma unroll
+    for (int ks2 = 0; ks2 < KST; ++ks2) {      // columns [16 ks2, 16 ks2 + 16) of q~
+      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(b0, b1, b2, b3, uk + (ks * 16 + (lm & 1) * 8 + lr) * S::KS + (16 * ks2 + (lm >> 1) * 8) * 2);
+        mma_16816(a0, qf0[ks], 0u, qf1[ks], 0u, b0, b1);
+        mma_16816(a1, qf0[ks], 0u, qf1[ks], 0u, b2, b3);
+      }
+      // lane (g, t) holds q~[head g][16 ks2 + 2t (+1)] in a0 and [+8] in a1 (rows g < 4);
+      // the low-part columns n = g >= 4 take head g - 4 from lane ^ 16
+      float x0 = __shfl_xor_sync(kFull, a0[0], 16), x1 = __shfl_xor_sync(kFull, a0[1], 16);
+      float y0 = __shfl_xor_sync(kFull, a1[0], 16), y1 = __shfl_xor_sync(kFull, a1[1], 16);
+      const bool lo_n = g >= 4;
+      if (!lo_n) x0 = a0[0], x1 = a0[1], y0 = a1[0], y1 = a1[1];
+      const bool live = (g & 3) < G;
+      qb0[ks2] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
+      qb1[ks2] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
+    }
+  }
+
+  // ---- stream the tiles ------------------------------------------------------------
+  // lane state: running max and sum of heads ha, hb; accumulators O^T (rows =
+  // value columns, columns = head parts) for the compressed and full-rank sums
+  float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+  float oc[MVT][4], of[8][4];
+#pragma unroll
+  for (int mt = 0; mt < MVT; ++mt) oc[mt][0] = oc[mt][1] = oc[mt][2] = oc[mt][3] = 0.f;
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) of[mt][0] = of[mt][1] = of[mt][2] = of[mt][3] = 0.f;
+
+  // Online softmax over NB 16-row blocks: s[nb] = {head ha at row g, hb at g,
+  // ha at g+8, hb at g+8} (-inf = no token).  Rescales this lane's accumulator
+  // columns when a max grows, and returns the probabilities packed as the
+  // P^T B fragments (bf16 high or low part by column) of each block.
+  auto softmax_pack = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag) {
+    constexpr int NB = decltype(nb_tag)::value;
+    float xa = -INFINITY, xb = -INFINITY;
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      xa = fmaxf(xa, fmaxf(s[nb][0], s[nb][2]));
+      xb = fmaxf(xb, fmaxf(s[nb][1], s[nb][3]));
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      xa = fmaxf(xa, __shfl_xor_sync(kFull, xa, o));
+      xb = fmaxf(xb, __shfl_xor_sync(kFull, xb, o));
+    }
+    if (xa > ma || xb > mb) {
+      const float na = fmaxf(ma, xa), nbm = fmaxf(mb, xb);
+      const float sa = ma == -INFINITY ? 0.f : exp2f(ma - na);
+      const float sb = mb == -INFINITY ? 0.f : exp2f(mb - nbm);
+      la *= sa;
+      lb *= sb;
+#pragma unroll
+      for (int mt = 0; mt < MVT; ++mt) oc[mt][0] *= sa, oc[mt][2] *= sa, oc[mt][1] *= sb, oc[mt][3] *= sb;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) of[mt][0] *= sa, of[mt][2] *= sa, of[mt][1] *= sb, of[mt][3] *= sb;
+      ma = na;
+      mb = nbm;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const float p0 = s[nb][0] == -INFINITY ? 0.f : exp2f(s[nb][0] - ma);
+      const float p1 = s[nb][1] == -INFINITY ? 0.f : exp2f(s[nb][1] - mb);
+      const float p2 = s[nb][2] == -INFINITY ? 0.f : exp2f(s[nb][2] - ma);
+      const float p3 = s[nb][3] == -INFINITY ? 0.f : exp2f(s[nb][3] - mb);
+      la += p0 + p2;
+      lb += p1 + p3;
+      pb0[nb] = movmatrix_t(pack_bf16(bf16_part(p0, lo_col), bf16_part(p1, lo_col)));
+      pb1[nb] = movmatrix_t(pack_bf16(bf16_part(p2, lo_col), bf16_part(p3, lo_col)));
+    }
+  };
+
+  for (int i = 0; i < n_tiles; ++i) {
+    if (i + kStages - 1 < n_tiles) issue(i + kStages - 1);
+    cp_async_commit();
+    cp_async_wait<kStages - 1>();
+    __syncwarp();
+    const unsigned char* slot = ring + (i % kStages) * S::SLOT;
+    if (i >= nft_w) {
+      // compressed tile: S^T[token][head part] = C_k q~^T, then O^T += C_v^T P^T
+      const uint32_t bits = tile_bits(warp + kWarps * (i - nft_w));
+      float st[2][4];
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb) {
+        st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KST; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(a0, a1, a2, a3,
+                  slot + (16 * nb + (lm & 1) * 8 + lr) * S::KS + (ks * 16 + (lm >> 1) * 8) * 2);
+          mma_16816(st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
+        }
+      }
+      float s[2][4];
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const float v = st[nb][x] + __shfl_xor_sync(kFull, st[nb][x], 2);   // high + low part
+          s[nb][x] = (bits >> (16 * nb + g + (x >> 1) * 8)) & 1u ? v : -INFINITY;
+        }
+      uint32_t pb0[2], pb1[2];
+      softmax_pack(s, pb0, pb1, std::integral_constant<int, 2>{});
+      const unsigned char* vrows = slot + kTileC * S::KS;
+#pragma unroll
+      for (int mt = 0; mt < MVT; ++mt)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(a0, a1, a2, a3,
+                    vrows + (16 * nb + (lm >> 1) * 8 + lr) * S::VS + (mt * 16 + (lm & 1) * 8) * 2);
+          mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
+        }
+    } else {
+      // full-rank tile: 16 list rows
+      const int k = warp + kWarps * i;
+      const int nrows = min(kTileF, n_full - k * kTileF);
+      float st[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(a0, a1, a2, a3, slot + ((lm & 1) * 8 + lr) * S::FS + (ks * 16 + (lm >> 1) * 8) * 2);
+        mma_16816(st, a0, a1, a2, a3, qf0[ks], qf1[ks]);
+      }
+      float s[1][4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const float v = (st[x] + __shfl_xor_sync(kFull, st[x], 2)) * scale;   // low-part columns are 0
+        s[0][x] = g + (x >> 1) * 8 < nrows ? v : -INFINITY;
+      }
+      uint32_t pb0[1], pb1[1];
+      softmax_pack(s, pb0, pb1, std::integral_constant<int, 1>{});
+      const unsigned char* vrows = slot + kTileF * S::FS;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(a0, a1, a2, a3, vrows + ((lm >> 1) * 8 + lr) * S::FS + (mt * 16 + (lm & 1) * 8) * 2);
+        mma_16816(of[mt], a0, a1, a2, a3, pb0[0], pb1[0]);
+      }
+    }
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+  griddep_launch_dependents();
+
+  // ---- this warp's partial state into its own ring slots --------------------------
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    la += __shfl_xor_sync(kFull, la, o);
+    lb += __shfl_xor_sync(kFull, lb, o);
+  }
+#pragma unroll
+  for (int mt = 0; mt < MVT; ++mt)
+#pragma unroll
+    for (int x = 0; x < 4; ++x) oc[mt][x] += __shfl_xor_sync(kFull, oc[mt][x], 2);
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+    for (int x = 0; x < 4; ++x) of[mt][x] += __shfl_xor_sync(kFull, of[mt][x], 2);
+  {
+    float* W = reinterpret_cast<float*>(ring);
+    if (t < 2) {
+      // lane (g, t<2): heads ha, hb; value columns mt*16 + g and mt*16 + g + 8
+#pragma unroll
+      for (int hx = 0; hx < 2; ++hx) {
+        const int hd = ha + hx;
+        if (hd < G) {
+          float* pc = W + S::W_PC + hd * RV;
+          float* pf = W + S::W_PF + hd * kD;
+#pragma unroll
+          for (int mt = 0; mt < MVT; ++mt) pc[mt * 16 + g] = oc[mt][hx], pc[mt * 16 + g + 8] = oc[mt][2 + hx];
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) pf[mt * 16 + g] = of[mt][hx], pf[mt * 16 + g + 8] = of[mt][2 + hx];
+          if (g == 0) {
+            W[S::W_M + hd] = hx == 0 ? ma : mb;
+            W[S::W_L + hd] = hx == 0 ? la : lb;
+          }
+        }
+      }
+    }
+  }
+  // the merge scratch reuses the U_k area: its bulk copy must have landed
+  if (!mbar_wait_bounded(base_bar, 0, kWaitIters)) bases_ok = false;
+  __syncthreads();   // every warp's partials written; every warp is past its q~
+
+  // ---- merge the warps (scratch in the U_k area) ------------------------------------
+  float* Cm = reinterpret_cast<float*>(uk);
+  auto wpart = [&](int w) { return reinterpret_cast<const float*>(sm + (size_t)w * kStages * S::SLOT); };
+  if (tid < G) {
+    float M = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wpart(w)[S::W_M + tid]);
+    float Ls = 0.f;
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = wpart(w)[S::W_M + tid];
+      const float e = mw == -INFINITY ? 0.f : exp2f(mw - M);
+      Cm[S::C_WE + w * G + tid] = e;
+      Ls = fmaf(wpart(w)[S::W_L + tid], e, Ls);
+    }
+    Cm[S::C_M + tid] = M;
+    Cm[S::C_M + G + tid] = Ls;
+  }
+  __syncthreads();
+  for (int o = tid; o < G * RV; o += kThreads) {
+    const int gi = o / RV;
+    float x = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[S::W_PC + o], Cm[S::C_WE + w * G + gi], x);
+    Cm[S::C_CC + o] = x;
+  }
+  for (int o = tid; o < G * kD; o += kThreads) {
+    const int gi = o / kD;
+    float x = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[S::W_PF + o], Cm[S::C_WE + w * G + gi], x);
+    Cm[S::C_CF + o] = x;
+  }
+  __syncthreads();
+
+  // ---- lift by U_v on the tensor cores, write this split's record ------------------
+  if (!bases_ok && lane == 0) atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
+  {
+    // A = merged acc_c split into hi (rows 0..3) / lo (rows 4..7) parts over
+    // k = r_v; B = U_v rows (n = output column); warp w owns the 8-column
+    // blocks w and w + 8
+    const int hh = g & 3;
+    const bool lo_row = g >= 4;
+    float* rec0 = p.partials + (bh * p.n_chunk_max + c) * G * (size_t)kRecFloats;
+#pragma unroll
+    for (int nbk = 0; nbk < 2; ++nbk) {
+      const int n0 = 8 * (warp + kWarps * nbk);
+      float l0[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < RV / 16; ++ks) {
+        uint32_t a0 = 0u, a2 = 0u;
+        if (hh < G) {
+          const float* row = Cm + S::C_CC + hh * RV + ks * 16 + 2 * t;
+          a0 = pack_bf16(bf16_part(row[0], lo_row), bf16_part(row[1], lo_row));
+          a2 = pack_bf16(bf16_part(row[8], lo_row), bf16_part(row[9], lo_row));
+        }
+        uint32_t b0, b1, b2, b3;   // (cols n0.., k lo), (cols n0.., k hi), repeated
+        ldsm_x4(b0, b1, b2, b3, uv + (n0 + lr) * S::VS + (ks * 16 + (lm & 1) * 8) * 2);
+        mma_16816(l0, a0, 0u, a2, 0u, b0, b1);
+      }
+#pragma unroll
+      for (int x = 0; x < 2; ++x) l0[x] += __shfl_xor_sync(kFull, l0[x], 16);
+      if (g < G) {
+        const int i0 = n0 + 2 * t;
+        const float* cf = Cm + S::C_CF + g * kD;
+        float* o = rec0 + g * kRecFloats + 4;
+        o[i0] = l0[0] + cf[i0];
+        o[i0 + 1] = l0[1] + cf[i0 + 1];
+      }
+    }
+    if (tid < G) {
+      rec0[tid * kRecFloats] = Cm[S::C_M + tid];
+      rec0[tid * kRecFloats + 1] = Cm[S::C_M + G + tid];
+    }
+  }
+
+  // ---- the last split of this (batch row, kv head) merges every record ------------
+  fence_proxy_async_smem();   // the ring is about to be refilled by bulk copies
+  __syncthreads();
+  if (tid == 0) s_last = atom_add_acq_rel_gpu(p.tickets + bh, 1) == n_chunks - 1;
+  __syncthreads();
+  if (!s_last) return;
+  // one pass: records streamed by bulk copy into the (idle) ring, merged with a
+  // running max per head
+  const float* recs = p.partials + bh * p.n_chunk_max * G * (size_t)kRecFloats;
+  constexpr int kRecBytes = G * kRecFloats * 4;
+  constexpr int per_batch = (kWarps * kStages * S::SLOT) / kRecBytes;
+  float* stage = reinterpret_cast<float*>(sm);
+  constexpr int NO = (G * kD + kThreads - 1) / kThreads;
+  float acc_o[NO], m_o[NO], l_o[NO];
+#pragma unroll
+  for (int u = 0; u < NO; ++u) acc_o[u] = 0.f, m_o[u] = -INFINITY, l_o[u] = 0.f;
+  int batch = 0;
+  for (int cb = 0; cb < n_chunks; cb += per_batch, ++batch) {
+    const int nb = min(per_batch, n_chunks - cb);
+    if (tid == 0) {
+      fence_proxy_async_smem();
+      fence_proxy_async_global();
+      mbar_arrive_expect_tx(merge_bar, nb * kRecBytes);
+      bulk_g2s(stage, recs + (size_t)cb * G * kRecFloats, nb * kRecBytes, merge_bar);
+    }
+    const bool timed_out = !mbar_wait_bounded(merge_bar, batch & 1, kWaitIters);
+    if (__syncthreads_or(timed_out)) {
+      if (tid == 0) atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
+      break;
+    }
+#pragma unroll
+    for (int u = 0; u < NO; ++u) {
+      const int o = tid + u * kThreads;
+      if (o < G * kD) {
+        const int gi = o / kD, ii = o % kD;
+        float mx = m_o[u];
+        for (int k2 = 0; k2 < nb; ++k2) mx = fmaxf(mx, stage[(k2 * G + gi) * kRecFloats]);
+        const float sc = m_o[u] == -INFINITY ? 0.f : exp2f(m_o[u] - mx);
+        float x = acc_o[u] * sc, l = l_o[u] * sc;
+        for (int k2 = 0; k2 < nb; ++k2) {
+          const float* rc = stage + (k2 * G + gi) * kRecFloats;
+          const float w = rc[0] == -INFINITY ? 0.f : exp2f(rc[0] - mx);
+          x = fmaf(w, rc[4 + ii], x);
+          l = fmaf(w, rc[1], l);
+        }
+        acc_o[u] = x, l_o[u] = l, m_o[u] = mx;
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int u = 0; u < NO; ++u) {
+    const int o = tid + u * kThreads;
+    if (o < G * kD) {
+      const int gi = o / kD, ii = o % kD;
+      p.out[((size_t)b * D.Hq + (size_t)h * G + gi) * kD + ii] = l_o[u] > 0.f ? acc_o[u] / l_o[u] : 0.f;
+    }
+  }
+  if (tid == 0) p.tickets[bh] = 0;
+}
+
+}  // namespace ds
+}  // namespace lrkv

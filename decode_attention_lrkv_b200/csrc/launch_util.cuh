@@ -1,0 +1,32 @@
+// Kernel launch with programmatic dependent launch enabled: the kernel may
+// start while the preceding kernel of the stream finishes; it must execute
+// griddepcontrol.wait before touching anything that kernel writes.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "lrkv.h"
+
+namespace lrkv {
+
+template <typename Params>
+inline lrkv_status launch_pdl(void (*kern)(Params), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, const Params& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
+    cudaGetLastError();
+    return LRKV_ERR_CUDA;
+  }
+  return LRKV_OK;
+}
+
+}  // namespace lrkv

@@ -9,6 +9,7 @@
 #include "compress_params.cuh"
 #include "compress_tc.cuh"
 #include "decode_launch.cuh"
+#include "launch_util.cuh"
 #include "lrkv.h"
 #include "lrkv_common.cuh"
 
@@ -181,8 +182,7 @@ lrkv_status lrkv_compress(const lrkv_dims* dims, const lrkv_cache* cache,
     if (cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return launched(), LRKV_ERR_CUDA;
-    append_kernel<<<dim3(dims->Hkv, dims->B), kAppendThreads, smem, s>>>(p);
-    return launched();
+    return launch_pdl(append_kernel, dim3(dims->Hkv, dims->B), dim3(kAppendThreads), smem, s, p);
   }
   return compress_tc(*dims, *cache, k_new, v_new, t_new, t_new_b, tau, err_out, w, L, s);
 }
