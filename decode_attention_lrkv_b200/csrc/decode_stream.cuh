@@ -29,14 +29,15 @@
 //     read, and its logit is -inf;
 //   - a full-rank tile is 16 list rows (keys, then values).
 // Rows land in padded shared-memory rows (stride 2r+16 bytes) so ldmatrix is
-// conflict-free.  At the end each warp leaves its partial softmax state in its
-// own ring slots, the CTA merges its warps, lifts by U_v (MMA), writes one
-// record (m, l, o[d]) per query head, and the last CTA of the (batch row, kv
-// head) merges all records (atomic ticket, no waiting).
+// conflict-free.  Three ring stages where shared memory allows, else two.
+// At the end each warp leaves its partial softmax state in its own slot, the
+// CTA merges its warps and writes one record (m, l, acc_c[r_v], acc_f[d]) per
+// query head, and the last CTA of the (batch row, kv head) merges all records
+// (atomic ticket, no waiting) and lifts once: o = (U_v acc_c + acc_f) / l.
 //
-// Programmatic dependent launch: the bases and q are loaded before waiting on
-// the preceding kernel of the stream (an append to the same cache); every
-// read of cache state comes after the wait.
+// Programmatic dependent launch: U_k and q are loaded and q~ is formed before
+// waiting on the preceding kernel of the stream (an append to the same
+// cache); every read of cache state comes after the wait.
 #pragma once
 
 #include <type_traits>
@@ -50,12 +51,9 @@ namespace ds {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 2;
 constexpr int kTileC = 32;                       // positions per compressed tile (one mask word)
 constexpr int kTileF = 16;                       // rows per full-rank tile
 constexpr int kMaxChunk = kMaxDecodeChunk;       // positions per split (mask words in smem)
-constexpr int kRecFloats = 4 + kD;               // m, l, (pad), o[d]: 16-byte multiple
-constexpr uint32_t kWaitIters = 1u << 24;        // bounded mbarrier polls (seconds)
 constexpr unsigned kFull = 0xffffffffu;
 
 constexpr int al16(int x) { return (x + 15) & ~15; }
@@ -73,24 +71,30 @@ struct Shape {
   static constexpr int SLOT_C = kTileC * (KS + VS);
   static constexpr int SLOT_F = kTileF * 2 * FS;
   static constexpr int SLOT = al128(imax(SLOT_C, SLOT_F));
-  static constexpr int OFF_UK = kWarps * kStages * SLOT;      // U_k rows [d][KS]
-  static constexpr int OFF_UV = al128(OFF_UK + kD * KS);      // U_v rows [d][VS]
-  static constexpr int OFF_MASK = al128(OFF_UV + kD * VS);
-  static constexpr int OFF_BAR = al16(OFF_MASK + (kMaxChunk / 32) * 4);   // merge, bases mbarriers
-  static constexpr int SMEM = OFF_BAR + 16;
+  static constexpr int FIXED = (kMaxChunk / 32) * 4;               // mask words
+  static constexpr int STAGES = kWarps * 3 * SLOT + FIXED <= 227 * 1024 ? 3 : 2;
+  static constexpr int RING = kWarps * STAGES * SLOT;             // [stage][warp][SLOT]
+  static constexpr int OFF_MASK = RING;
+  static constexpr int SMEM = OFF_MASK + (kMaxChunk / 32) * 4;
   static_assert(SMEM <= 227 * 1024, "shared memory of one CTA");
-  // per-warp partial state in the warp's own ring slots (floats)
+  // U_k rows [d][KS] live in the last stage until every warp has its q~
+  static constexpr int OFF_UK = (STAGES - 1) * kWarps * SLOT;
+  static_assert(kD * KS <= kWarps * SLOT, "U_k fits in one stage");
+  // per-warp partial state in the warp's stage-0 slot (floats)
   static constexpr int W_PC = 0;                    // [G][RV]
   static constexpr int W_PF = W_PC + G * RV;        // [G][d]
   static constexpr int W_M = W_PF + G * kD;         // [G]
   static constexpr int W_L = W_M + G;               // [G]
-  static_assert((W_L + G) * 4 <= kStages * SLOT, "partials fit in a warp's slots");
-  // CTA merge in the U_k area (free once every warp has its q~)
-  static constexpr int C_CC = 0;                    // [G][RV] merged acc_c
-  static constexpr int C_CF = C_CC + G * RV;        // [G][d] merged acc_f
-  static constexpr int C_M = C_CF + G * kD;         // [G] max, [G] sum
-  static constexpr int C_WE = C_M + 2 * G;          // [warps][G] warp weights
-  static_assert((C_WE + kWarps * G) * 4 <= kD * KS, "merge scratch fits in the U_k area");
+  static_assert((W_L + G) * 4 <= SLOT, "partials fit in a slot");
+  static constexpr int REC = 4 + RV + kD;           // record floats per query head
+  // final merge: U_v rows [d][VS] at the end of the ring, records staged before it
+  static constexpr int OFF_UV = (RING - kD * VS) & ~127;
+  static constexpr int STAGE_BYTES = OFF_UV;
+  // merged sums of the final merge, after the staged records' batch area (floats)
+  static constexpr int M_CC = 0;                    // [G][RV]
+  static constexpr int M_CF = M_CC + G * RV;        // [G][d]
+  static constexpr int M_L = M_CF + G * kD;         // [G]
+  static constexpr int MERGE_FLOATS = M_L + G;
 };
 
 template <int G, int RK, int RV>
@@ -99,6 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   constexpr int KST = RK / 16;                   // k-steps of the compressed logits
   constexpr int MVT = RV / 16;                   // m-tiles of the compressed value sum
   constexpr int KP = S::KP, VP = S::VP;
+  constexpr int NST = S::STAGES;
   extern __shared__ __align__(128) unsigned char sm[];
   const lrkv_dims& D = p.D;
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -110,29 +115,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   const size_t bh = (size_t)b * D.Hkv + h;
 
   unsigned char* uk = sm + S::OFF_UK;
-  unsigned char* uv = sm + S::OFF_UV;
   uint32_t* maskw = reinterpret_cast<uint32_t*>(sm + S::OFF_MASK);
-  uint64_t* merge_bar = reinterpret_cast<uint64_t*>(sm + S::OFF_BAR);
-  uint64_t* base_bar = merge_bar + 1;
-  unsigned char* ring = sm + (size_t)warp * kStages * S::SLOT;
+  auto slot_of = [&](int stage, int w) { return sm + (size_t)(stage * kWarps + w) * S::SLOT; };
   __shared__ int s_last;
 
-  // ---- prologue, independent of the preceding kernel: bases and q ------------------
-  if (tid == 0) {
-    mbar_init(merge_bar, 1);
-    mbar_init(base_bar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (warp == 0) {  // both bases into padded rows, one bulk copy per row
-    const lrkv_bf16* Uk = p.C.U_k + (size_t)h * kD * RK;
-    const lrkv_bf16* Uv = p.C.U_v + (size_t)h * kD * RV;
-    if (lane == 0) mbar_arrive_expect_tx(base_bar, kD * 2u * (RK + RV));
-    __syncwarp();
-    for (int r = lane; r < kD; r += 32) {
-      bulk_g2s(uk + r * S::KS, Uk + (size_t)r * RK, 2u * RK, base_bar);
-      bulk_g2s(uv + r * S::VS, Uv + (size_t)r * RV, 2u * RV, base_bar);
+  // ---- prologue, independent of the preceding kernel: U_k, q and q~ ----------------
+  {  // U_k into padded rows, 16-byte pieces over every thread
+    const unsigned char* Uk = reinterpret_cast<const unsigned char*>(p.C.U_k + (size_t)h * kD * RK);
+    for (int q = tid; q < kD * KP; q += kThreads) {
+      const int r = q / KP, sg = q - r * KP;
+      cp_async16(uk + r * S::KS + sg * 16, Uk + q * 16);
     }
+    cp_async_commit();
   }
   // q as fragments over k = d: the B operand of the full-rank logits (column
   // n = head n < G; q is bf16, hence exact, so no low-part columns) and, the
@@ -147,16 +141,38 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     }
   }
   const float scale = kLog2e * rsqrtf((float)kD);
+  // q~ = U_k^T q as this warp's B fragments over k = r_k (column n < 4 = bf16
+  // high part of head n, n >= 4 = low part of head n - 4), on the tensor cores
+  uint32_t qb0[KST], qb1[KST];
+  cp_async_wait<0>();
+  __syncthreads();
+#pragma unroll
+  for (int ks2 = 0; ks2 < KST; ++ks2) {        // columns [16 ks2, 16 ks2 + 16) of q~
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(b0, b1, b2, b3, uk + (ks * 16 + (lm & 1) * 8 + lr) * S::KS + (16 * ks2 + (lm >> 1) * 8) * 2);
+      mma_16816(a0, qf0[ks], 0u, qf1[ks], 0u, b0, b1);
+      mma_16816(a1, qf0[ks], 0u, qf1[ks], 0u, b2, b3);
+    }
+    // lane (g, t) holds q~[head g][16 ks2 + 2t (+1)] in a0 and [+8] in a1 (rows g < 4);
+    // the low-part columns n = g >= 4 take head g - 4 from lane ^ 16
+    float x0 = __shfl_xor_sync(kFull, a0[0], 16), x1 = __shfl_xor_sync(kFull, a0[1], 16);
+    float y0 = __shfl_xor_sync(kFull, a1[0], 16), y1 = __shfl_xor_sync(kFull, a1[1], 16);
+    const bool lo_n = g >= 4;
+    if (!lo_n) x0 = a0[0], x1 = a0[1], y0 = a1[0], y1 = a1[1];
+    const bool live = (g & 3) < G;
+    qb0[ks2] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
+    qb1[ks2] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
+  }
 
   // ---- cache state: after the preceding kernel (an append) has completed ------------
   griddep_wait();
   int T = p.C.seq_len[b];
   T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
   const int n_chunks = T > 0 ? (T + p.chunk - 1) / p.chunk : 1;
-  if (c >= n_chunks) {   // no work: let the bases land before leaving
-    mbar_wait_bounded(base_bar, 0, kWaitIters);
-    return;
-  }
+  if (c >= n_chunks) return;
   const int c0 = c * p.chunk;
   const int c1 = min(T, c0 + p.chunk);
   const int n_pos = c1 > c0 ? c1 - c0 : 0;
@@ -173,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     const uint32_t* mask_g = p.C.route_mask + bh * (D.T_cap / 32) + c0 / 32;
     for (int i = tid; i < n_words; i += kThreads) maskw[i] = mask_g[i];
   }
-  __syncthreads();
+  __syncthreads();   // mask words in; every warp is done with U_k (the last stage is free)
 
   // this warp's tiles: full-rank ones first (they need only q), then compressed ones
   const int n_ct = (n_pos + kTileC - 1) / kTileC;
@@ -191,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     return ~maskw[k] & valid;
   };
   auto issue = [&](int i) {
-    unsigned char* slot = ring + (i % kStages) * S::SLOT;
+    unsigned char* slot = slot_of(i % NST, warp);
     if (i >= nft_w) {
       const int k = warp + kWarps * (i - nft_w);
       const uint32_t bits = tile_bits(k);
@@ -229,38 +245,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     }
   };
 #pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
+  for (int s = 0; s < NST - 1; ++s) {
     if (s < n_tiles) issue(s);
     cp_async_commit();
-  }
-
-  // q~ = U_k^T q as this warp's B fragments over k = r_k (column n < 4 = bf16
-  // high part of head n, n >= 4 = low part of head n - 4), on the tensor cores,
-  // while the first tiles are in flight
-  bool bases_ok = true;
-  uint32_t qb0[KST], qb1[KST];
-  if (nct_w > 0) {
-    bases_ok = mbar_wait_bounded(base_bar, 0, kWaitIters);
-#pragma unroll
-    for (int ks2 = 0; ks2 < KST; ++ks2) {      // columns [16 ks2, 16 ks2 + 16) of q~
-      float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(b0, b1, b2, b3, uk + (ks * 16 + (lm & 1) * 8 + lr) * S::KS + (16 * ks2 + (lm >> 1) * 8) * 2);
-        mma_16816(a0, qf0[ks], 0u, qf1[ks], 0u, b0, b1);
-        mma_16816(a1, qf0[ks], 0u, qf1[ks], 0u, b2, b3);
-      }
-      // lane (g, t) holds q~[head g][16 ks2 + 2t (+1)] in a0 and [+8] in a1 (rows g < 4);
-      // the low-part columns n = g >= 4 take head g - 4 from lane ^ 16
-      float x0 = __shfl_xor_sync(kFull, a0[0], 16), x1 = __shfl_xor_sync(kFull, a0[1], 16);
-      float y0 = __shfl_xor_sync(kFull, a1[0], 16), y1 = __shfl_xor_sync(kFull, a1[1], 16);
-      const bool lo_n = g >= 4;
-      if (!lo_n) x0 = a0[0], x1 = a0[1], y0 = a1[0], y1 = a1[1];
-      const bool live = (g & 3) < G;
-      qb0[ks2] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
-      qb1[ks2] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
-    }
   }
 
   // ---- stream the tiles ------------------------------------------------------------
@@ -318,11 +305,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   };
 
   for (int i = 0; i < n_tiles; ++i) {
-    if (i + kStages - 1 < n_tiles) issue(i + kStages - 1);
+    if (i + NST - 1 < n_tiles) issue(i + NST - 1);
     cp_async_commit();
-    cp_async_wait<kStages - 1>();
+    cp_async_wait<NST - 1>();
     __syncwarp();
-    const unsigned char* slot = ring + (i % kStages) * S::SLOT;
+    const unsigned char* slot = slot_of(i % NST, warp);
     if (i >= nft_w) {
       // compressed tile: S^T[token][head part] = C_k q~^T, then O^T += C_v^T P^T
       const uint32_t bits = tile_bits(warp + kWarps * (i - nft_w));
@@ -391,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   __syncwarp();
   griddep_launch_dependents();
 
-  // ---- this warp's partial state into its own ring slots --------------------------
+  // ---- this warp's partial state into its stage-0 slot -------------------------------
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     la += __shfl_xor_sync(kFull, la, o);
@@ -406,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
 #pragma unroll
     for (int x = 0; x < 4; ++x) of[mt][x] += __shfl_xor_sync(kFull, of[mt][x], 2);
   {
-    float* W = reinterpret_cast<float*>(ring);
+    float* W = reinterpret_cast<float*>(slot_of(0, warp));
     if (t < 2) {
       // lane (g, t<2): heads ha, hb; value columns mt*16 + g and mt*16 + g + 8
 #pragma unroll
@@ -427,13 +414,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
       }
     }
   }
-  // the merge scratch reuses the U_k area: its bulk copy must have landed
-  if (!mbar_wait_bounded(base_bar, 0, kWaitIters)) bases_ok = false;
-  __syncthreads();   // every warp's partials written; every warp is past its q~
+  __syncthreads();
 
-  // ---- merge the warps (scratch in the U_k area) ------------------------------------
-  float* Cm = reinterpret_cast<float*>(uk);
-  auto wpart = [&](int w) { return reinterpret_cast<const float*>(sm + (size_t)w * kStages * S::SLOT); };
+  // ---- merge the warps into this split's record --------------------------------------
+  auto wpart = [&](int w) { return reinterpret_cast<const float*>(slot_of(0, w)); };
+  __shared__ float s_we[kWarps][G];
+  float* rec0 = p.partials + (bh * p.n_chunk_max + c) * G * (size_t)S::REC;
   if (tid < G) {
     float M = -INFINITY;
     for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wpart(w)[S::W_M + tid]);
@@ -441,38 +427,109 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     for (int w = 0; w < kWarps; ++w) {
       const float mw = wpart(w)[S::W_M + tid];
       const float e = mw == -INFINITY ? 0.f : exp2f(mw - M);
-      Cm[S::C_WE + w * G + tid] = e;
+      s_we[w][tid] = e;
       Ls = fmaf(wpart(w)[S::W_L + tid], e, Ls);
     }
-    Cm[S::C_M + tid] = M;
-    Cm[S::C_M + G + tid] = Ls;
+    rec0[tid * S::REC] = M;
+    rec0[tid * S::REC + 1] = Ls;
   }
   __syncthreads();
-  for (int o = tid; o < G * RV; o += kThreads) {
-    const int gi = o / RV;
+  for (int o = tid; o < G * (RV + kD); o += kThreads) {
+    const int gi = o / (RV + kD), j = o - gi * (RV + kD);
+    const int src = j < RV ? S::W_PC + gi * RV + j : S::W_PF + gi * kD + (j - RV);
     float x = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[S::W_PC + o], Cm[S::C_WE + w * G + gi], x);
-    Cm[S::C_CC + o] = x;
+    for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[src], s_we[w][gi], x);
+    rec0[gi * S::REC + 4 + j] = x;
   }
-  for (int o = tid; o < G * kD; o += kThreads) {
-    const int gi = o / kD;
-    float x = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[S::W_PF + o], Cm[S::C_WE + w * G + gi], x);
-    Cm[S::C_CF + o] = x;
-  }
-  __syncthreads();
 
-  // ---- lift by U_v on the tensor cores, write this split's record ------------------
-  if (!bases_ok && lane == 0) atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
+  // ---- the last split of this (batch row, kv head) merges every record ------------
+  __syncthreads();
+  if (tid == 0) s_last = atom_add_acq_rel_gpu(p.tickets + bh, 1) == n_chunks - 1;
+  __syncthreads();
+  if (!s_last) return;
+  // U_v for the lift, then the records in batches through the ring, merged
+  // with a running max per (head, element); all loads are 16-byte cp.async
+  // pieces over every thread
+  unsigned char* uv = sm + S::OFF_UV;
   {
-    // A = merged acc_c split into hi (rows 0..3) / lo (rows 4..7) parts over
-    // k = r_v; B = U_v rows (n = output column); warp w owns the 8-column
-    // blocks w and w + 8
+    const unsigned char* Uv = reinterpret_cast<const unsigned char*>(p.C.U_v + (size_t)h * kD * RV);
+    for (int q = tid; q < kD * VP; q += kThreads) {
+      const int r = q / VP, sg = q - r * VP;
+      cp_async16(uv + r * S::VS + sg * 16, Uv + q * 16);
+    }
+    cp_async_commit();
+  }
+  const float* recs = p.partials + bh * p.n_chunk_max * G * (size_t)S::REC;
+  constexpr int kRecBytes = G * S::REC * 4;
+  constexpr int per_batch = (S::STAGE_BYTES - S::MERGE_FLOATS * 4) / kRecBytes;
+  static_assert(per_batch >= 1, "one record batch fits");
+  float* stage = reinterpret_cast<float*>(sm);
+  float* merged = stage + per_batch * G * S::REC;   // [G][RV], [G][d], [G]
+  __shared__ float s_w[per_batch < 64 ? per_batch : 64][G];   // weights of one batch
+  __shared__ float s_run[2][G];                               // [1]: old-sum scale of a batch
+  constexpr int kWB = per_batch < 64 ? per_batch : 64;        // records per batch
+  constexpr int NE = G * (RV + kD);
+  constexpr int NO = (NE + kThreads - 1) / kThreads;
+  float acc_o[NO];
+#pragma unroll
+  for (int u = 0; u < NO; ++u) acc_o[u] = 0.f;
+  float run_m = -INFINITY, run_l = 0.f;           // threads < G: head tid
+  for (int cb = 0; cb < n_chunks; cb += kWB) {
+    const int nb = min(kWB, n_chunks - cb);
+    {
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(recs + (size_t)cb * G * S::REC);
+      unsigned char* dst = reinterpret_cast<unsigned char*>(stage);
+      for (int q = tid; q < nb * kRecBytes / 16; q += kThreads) cp_async16(dst + q * 16, src + q * 16);
+      cp_async_commit();
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    // per (record, head) weights against the new running max
+    if (tid < G) {
+      float mx = run_m;
+      for (int k = 0; k < nb; ++k) mx = fmaxf(mx, stage[(k * G + tid) * S::REC]);
+      const float sc = run_m == -INFINITY ? 0.f : exp2f(run_m - mx);
+      float l = run_l * sc;
+      for (int k = 0; k < nb; ++k) {
+        const float* rc = stage + (k * G + tid) * S::REC;
+        const float w = rc[0] == -INFINITY ? 0.f : exp2f(rc[0] - mx);
+        s_w[k][tid] = w;
+        l = fmaf(w, rc[1], l);
+      }
+      s_run[1][tid] = sc;
+      run_m = mx;
+      run_l = l;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < NO; ++u) {
+      const int o = tid + u * kThreads;
+      if (o < NE) {
+        const int gi = o / (RV + kD), j = o - gi * (RV + kD);
+        float x = acc_o[u] * s_run[1][gi];
+        for (int k = 0; k < nb; ++k) x = fmaf(s_w[k][gi], stage[(k * G + gi) * S::REC + 4 + j], x);
+        acc_o[u] = x;
+      }
+    }
+    __syncthreads();
+  }
+  if (tid < G) merged[S::M_L + tid] = run_l;
+#pragma unroll
+  for (int u = 0; u < NO; ++u) {
+    const int o = tid + u * kThreads;
+    if (o < NE) {
+      const int gi = o / (RV + kD), j = o - gi * (RV + kD);
+      merged[j < RV ? S::M_CC + gi * RV + j : S::M_CF + gi * kD + (j - RV)] = acc_o[u];
+    }
+  }
+  __syncthreads();
+  // lift on the tensor cores: A = merged acc_c split into hi (rows 0..3) / lo
+  // (rows 4..7) parts over k = r_v; B = U_v rows (n = output column); warp w
+  // owns the 8-column blocks w and w + 8
+  {
     const int hh = g & 3;
     const bool lo_row = g >= 4;
-    float* rec0 = p.partials + (bh * p.n_chunk_max + c) * G * (size_t)kRecFloats;
 #pragma unroll
     for (int nbk = 0; nbk < 2; ++nbk) {
       const int n0 = 8 * (warp + kWarps * nbk);
@@ -481,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
       for (int ks = 0; ks < RV / 16; ++ks) {
         uint32_t a0 = 0u, a2 = 0u;
         if (hh < G) {
-          const float* row = Cm + S::C_CC + hh * RV + ks * 16 + 2 * t;
+          const float* row = merged + S::M_CC + hh * RV + ks * 16 + 2 * t;
           a0 = pack_bf16(bf16_part(row[0], lo_row), bf16_part(row[1], lo_row));
           a2 = pack_bf16(bf16_part(row[8], lo_row), bf16_part(row[9], lo_row));
         }
@@ -492,75 +549,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
 #pragma unroll
       for (int x = 0; x < 2; ++x) l0[x] += __shfl_xor_sync(kFull, l0[x], 16);
       if (g < G) {
+        const float L = merged[S::M_L + g];
+        const float inv = L > 0.f ? 1.f / L : 0.f;
         const int i0 = n0 + 2 * t;
-        const float* cf = Cm + S::C_CF + g * kD;
-        float* o = rec0 + g * kRecFloats + 4;
-        o[i0] = l0[0] + cf[i0];
-        o[i0 + 1] = l0[1] + cf[i0 + 1];
+        const float* cf = merged + S::M_CF + g * kD;
+        float* o = p.out + ((size_t)b * D.Hq + (size_t)h * G + g) * kD;
+        o[i0] = (l0[0] + cf[i0]) * inv;
+        o[i0 + 1] = (l0[1] + cf[i0 + 1]) * inv;
       }
-    }
-    if (tid < G) {
-      rec0[tid * kRecFloats] = Cm[S::C_M + tid];
-      rec0[tid * kRecFloats + 1] = Cm[S::C_M + G + tid];
-    }
-  }
-
-  // ---- the last split of this (batch row, kv head) merges every record ------------
-  fence_proxy_async_smem();   // the ring is about to be refilled by bulk copies
-  __syncthreads();
-  if (tid == 0) s_last = atom_add_acq_rel_gpu(p.tickets + bh, 1) == n_chunks - 1;
-  __syncthreads();
-  if (!s_last) return;
-  // one pass: records streamed by bulk copy into the (idle) ring, merged with a
-  // running max per head
-  const float* recs = p.partials + bh * p.n_chunk_max * G * (size_t)kRecFloats;
-  constexpr int kRecBytes = G * kRecFloats * 4;
-  constexpr int per_batch = (kWarps * kStages * S::SLOT) / kRecBytes;
-  float* stage = reinterpret_cast<float*>(sm);
-  constexpr int NO = (G * kD + kThreads - 1) / kThreads;
-  float acc_o[NO], m_o[NO], l_o[NO];
-#pragma unroll
-  for (int u = 0; u < NO; ++u) acc_o[u] = 0.f, m_o[u] = -INFINITY, l_o[u] = 0.f;
-  int batch = 0;
-  for (int cb = 0; cb < n_chunks; cb += per_batch, ++batch) {
-    const int nb = min(per_batch, n_chunks - cb);
-    if (tid == 0) {
-      fence_proxy_async_smem();
-      fence_proxy_async_global();
-      mbar_arrive_expect_tx(merge_bar, nb * kRecBytes);
-      bulk_g2s(stage, recs + (size_t)cb * G * kRecFloats, nb * kRecBytes, merge_bar);
-    }
-    const bool timed_out = !mbar_wait_bounded(merge_bar, batch & 1, kWaitIters);
-    if (__syncthreads_or(timed_out)) {
-      if (tid == 0) atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
-      break;
-    }
-#pragma unroll
-    for (int u = 0; u < NO; ++u) {
-      const int o = tid + u * kThreads;
-      if (o < G * kD) {
-        const int gi = o / kD, ii = o % kD;
-        float mx = m_o[u];
-        for (int k2 = 0; k2 < nb; ++k2) mx = fmaxf(mx, stage[(k2 * G + gi) * kRecFloats]);
-        const float sc = m_o[u] == -INFINITY ? 0.f : exp2f(m_o[u] - mx);
-        float x = acc_o[u] * sc, l = l_o[u] * sc;
-        for (int k2 = 0; k2 < nb; ++k2) {
-          const float* rc = stage + (k2 * G + gi) * kRecFloats;
-          const float w = rc[0] == -INFINITY ? 0.f : exp2f(rc[0] - mx);
-          x = fmaf(w, rc[4 + ii], x);
-          l = fmaf(w, rc[1], l);
-        }
-        acc_o[u] = x, l_o[u] = l, m_o[u] = mx;
-      }
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int u = 0; u < NO; ++u) {
-    const int o = tid + u * kThreads;
-    if (o < G * kD) {
-      const int gi = o / kD, ii = o % kD;
-      p.out[((size_t)b * D.Hq + (size_t)h * G + gi) * kD + ii] = l_o[u] > 0.f ? acc_o[u] / l_o[u] : 0.f;
     }
   }
   if (tid == 0) p.tickets[bh] = 0;

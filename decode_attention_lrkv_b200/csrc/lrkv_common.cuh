@@ -51,7 +51,7 @@ struct WsLayout {
   size_t tile_cnt;         // int32 [B][Hkv][n_tiles] routed tokens per 128-token tile
   size_t tile_bits;        // uint32 [B][Hkv][n_tiles][4] routed bits per tile
   int n_tiles;             // ceil(T_cap / 128)
-  size_t partials;         // float [B][Hkv][n_chunk_max][g][2 + r_v + d]
+  size_t partials;         // float [B][Hkv][n_chunk_max][g][4 + r_v + d]
   size_t total;
   int chunk;               // decode: positions per split
   int n_chunk_max;         // decode: splits per (b, kv head)
@@ -99,7 +99,7 @@ inline WsLayout ws_layout(const lrkv_dims& D) {
   off = align_up(off + sizeof(uint32_t) * 4 * (size_t)D.B * D.Hkv * L.n_tiles, 256);
   L.chunk = decode_chunk(D);
   L.n_chunk_max = (D.T_cap + L.chunk - 1) / L.chunk;
-  L.partial_floats = 2 + D.r_v + D.d;
+  L.partial_floats = 4 + D.r_v + D.d;   // m, l, pad, pad, acc_c[r_v], acc_f[d]
   L.partials = off;
   int g = D.Hkv > 0 ? D.Hq / D.Hkv : 0;
   off = align_up(off + sizeof(float) * (size_t)D.B * D.Hkv * L.n_chunk_max * g *
