@@ -57,10 +57,21 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=1)
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (testing)")
+    ap.add_argument("--context", type=int, default=0,
+                    help="override the context length (small profiling cases)")
     ap.add_argument("--seed", type=int, default=1234)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     return ap.parse_args()
+
+
+def workload_of(args):
+    over = {}
+    if args.layers:
+        over["layers"] = args.layers
+    if args.context:
+        over["T"] = args.context
+    return synth.workload(args.workload, **over)
 
 
 def peaks():
@@ -170,6 +181,33 @@ class Clocks:
 
 
 # ---------------------------------------------------------------------------
+# ranks: one process per GPU; each runs its own independent sequences
+# ---------------------------------------------------------------------------
+
+def rank_seed(seed, rank):
+    """Seed of a rank's synthetic inputs: every rank draws different sequences."""
+    return seed + 7919 * rank
+
+
+def max_over_ranks(x, dev, world):
+    """The largest value over the ranks (the slowest rank's time); every rank calls it."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=dev, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x, dev, world):
+    """The sum over the ranks (the whole job's bytes); every rank calls it."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=dev, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
@@ -226,12 +264,12 @@ def capture_step_graph(L, dims, ws, layers, w, s, out, dec_events, host=None):
     stream.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(stream):
         with torch.cuda.graph(g, stream=stream):
+            if host is not None:   # the step's inputs for every layer: one copy per tensor
+                hin, hout, stage = host
+                for name in ("k", "v", "q"):
+                    stage[name].copy_(hin[name][s], non_blocking=True)
             for li, lay in enumerate(layers):
                 if host is not None:
-                    hin, hout, stage = host
-                    stage["k"][li].copy_(hin["k"][s, li], non_blocking=True)
-                    stage["v"][li].copy_(hin["v"][s, li], non_blocking=True)
-                    stage["q"][li].copy_(hin["q"][s, li], non_blocking=True)
                     k, v, q = stage["k"][li], stage["v"][li], stage["q"][li]
                 else:
                     k = lay["K_app"][:, s:s + 1]
@@ -243,8 +281,8 @@ def capture_step_graph(L, dims, ws, layers, w, s, out, dec_events, host=None):
                 L.lrkv_decode_attn(dims, lay["cache"], q, out[li], ws=ws, stream=stream)
                 if dec_events is not None:
                     dec_events[li][1].record(stream)
-                if host is not None:
-                    hout[s, li].copy_(out[li], non_blocking=True)
+            if host is not None:   # the step's result for every layer: one copy back
+                hout[s].copy_(out, non_blocking=True)
     torch.cuda.current_stream().wait_stream(stream)
     return g
 
@@ -252,12 +290,10 @@ def capture_step_graph(L, dims, ws, layers, w, s, out, dec_events, host=None):
 def run_ours(args, rank, world, dev):
     import decode_attention_lrkv_b200 as L
     L.load_library()
-    w = synth.workload(args.workload)
-    if args.layers:
-        w = synth.workload(args.workload, layers=args.layers)
+    w = workload_of(args)
     K, W = args.steps, args.warmup
     steps_total = W + K
-    seed = args.seed + 7919 * rank
+    seed = rank_seed(args.seed, rank)
     dims, ws, layers, comp_ms, lengths = build_layers(L, w, seed, 3 * steps_total, dev)
     out = torch.empty(w.layers, w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
 
@@ -290,10 +326,7 @@ def run_ours(args, rank, world, dev):
         g.reset()
     del graphs
     full_cnt = [lay["cache"].full_cnt.cpu().numpy() for lay in layers]
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev, world)
 
     # --- the decode kernel's own launch duration: the same steps again, with
     # CUDA events recorded on the launching stream around every decode ----------------
@@ -322,7 +355,7 @@ def run_ours(args, rank, world, dev):
     app_bytes = A.compress_bytes(w.Hkv, w.d, w.r_k, w.r_v, w.B, w.B * w.Hkv * routed_frac)
     step_bytes = sum(dec_bytes) + w.layers * app_bytes
     ms_step = ms / K
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    value = sum_over_ranks(step_bytes, dev, world) / (ms_step * 1e-3) / 1e9
     dec_launch_ms = float(np.mean(dec_ms))
     T_mid_k = [int(x) + (K + 1) / 2.0 for x in seq_k]
     dec_bytes_launch = float(np.mean([A.decode_bytes(w.B, w.Hq, w.Hkv, w.d, w.r_k, w.r_v, T_mid_k, fc)
@@ -408,11 +441,7 @@ def run_e2e(L, args, w, dims, ws, layers, dev, world, steps_total):
         graphs[s].replay()
     t1.record()
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), dev, world)
     for g in graphs:
         g.reset()
     T_now = [int(x) for x in layers[0]["cache"].seq_len.cpu()]
@@ -422,7 +451,8 @@ def run_e2e(L, args, w, dims, ws, layers, dev, world, steps_total):
     step_bytes += w.layers * A.compress_bytes(w.Hkv, w.d, w.r_k, w.r_v, w.B, 0)
     h2d = sum(t[0].numel() * t[0].element_size() for t in hin.values())
     d2h = hout[0].numel() * hout[0].element_size()
-    return {"value": round(world * step_bytes / (ms / K * 1e-3) / 1e9, 2), "unit": "GB/s",
+    job_bytes = sum_over_ranks(step_bytes, dev, world)
+    return {"value": round(job_bytes / (ms / K * 1e-3) / 1e9, 2), "unit": "GB/s",
             "us_per_step": round(ms / K * 1e3, 2), "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h)}
 
@@ -475,29 +505,25 @@ class OracleLayer:
         return nbytes, dt
 
 
-def oracle_sample(w, seed, wall_budget_s=40.0, max_layers=8):
-    """The oracle on whole layers of the workload until ~wall_budget_s of wall time.
+def oracle_sample(w, seed, timed_budget_s=12.0, max_steps=3000):
+    """The oracle on decode steps of layer 0 of the workload until ~timed_budget_s.
 
-    Returns (GB/s of algorithmic decode-step bytes, compress tokens/s, layers, timed s).
+    Setup (the layer's prefill through the oracle) is untimed but its tokens/s
+    is reported.  Returns (GB/s of algorithmic decode-step bytes, compress
+    tokens/s, steps, timed s).
     """
-    t_wall = time.perf_counter()
-    nbytes = secs = comp_s = comp_tok = 0.0
+    ol = OracleLayer(w, 0, seed, max_steps)
+    nbytes = secs = 0.0
     n = 0
-    for li in range(min(w.layers, max_layers)):
-        ol = OracleLayer(w, li, seed, 1)
+    while n < max_steps and secs < timed_budget_s:
         b, dt = ol.step()
         nbytes, secs = nbytes + b, secs + dt
-        comp_s, comp_tok = comp_s + ol.prefill_s, comp_tok + ol.prefill_tokens
         n += 1
-        if time.perf_counter() - t_wall > wall_budget_s:
-            break
-    return nbytes / secs / 1e9, comp_tok / comp_s, n, secs
+    return nbytes / secs / 1e9, ol.prefill_tokens / ol.prefill_s, n, secs
 
 
 def run_reference(args):
-    w = synth.workload(args.workload)
-    if args.layers:
-        w = synth.workload(args.workload, layers=args.layers)
+    w = workload_of(args)
     # setup (untimed): the oracle prefills one layer; each step is one oracle decode
     # step over that layer -- a bounded sample of the workload's step
     ol = OracleLayer(w, 0, args.seed, args.warmup + args.steps)
@@ -547,9 +573,9 @@ def main():
         result["cpu_baseline"] = {
             "value": round(v, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
             "compress_tok_per_s_per_layer": round(ctok, 1),
-            "sample": f"{n} of {w.layers} layers of {w.name}: fp64 oracle, one decode step "
-                      f"(append + attend) per layer, {secs:.2f} s timed; prefill compress timed "
-                      f"separately"}
+            "sample": f"{n} decode steps (append + attend) of layer 0 of {w.name} "
+                      f"(1 of {w.layers} layers, B={w.B}, T={w.T}): fp64 oracle, {secs:.1f} s "
+                      f"timed; the layer's prefill through the oracle timed separately"}
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

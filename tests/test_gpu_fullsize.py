@@ -1,0 +1,129 @@
+"""CUDA library vs the fp64 oracle at the benchmark's full sizes.
+
+One layer of each benchmark workload at its full context (Llama-3.1-8B
+geometry at 8K and 32K, the batch-16 ragged 8K-16K case and the LLaMA-7B MHA
+case at 131072), with the cache capacity bench.py uses, so the kernels run in
+the launch configuration bench.py times: a prefill through lrkv_compress,
+three one-token appends, then one decode.  The oracle cannot redo whole
+layers in seconds, so sampled (batch row, kv head) pairs are recomputed one
+by one and compared element by element:
+  - every coefficient of the head: 1 bf16 ulp + the fp32 accumulation bound;
+  - the routed set: identical except tokens within 1e-4 of tau;
+  - the full-rank list: ascending positions, rows bit-exact, length;
+  - decode output of the head's query heads: ||o - o_ref||_inf / ||o_ref||_inf
+    <= 2e-3, the oracle attending over the GPU-written cache.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+import decode_attention_lrkv_b200 as L
+from tests import lrkv_testutil as U
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+# bench.py's cache capacity: the context plus three passes of its default
+# 100 timed + 5 warm-up decode steps, plus one
+BENCH_EXTRA = 3 * (100 + 5) + 1
+N_APPEND = 3
+
+
+def _oracle_head(D, U_k1, U_v1, K, V, tau, n_b, appends):
+    """The oracle's cache for one (batch row, kv head), built call by call.
+
+    U_k1, U_v1: [1, d, r]; K, V and the appended rows: [1, t, 1, d]."""
+    od = O.Dims(B=1, Hq=D.Hq // D.Hkv, Hkv=1, d=D.d, r_k=D.r_k, r_v=D.r_v, T_cap=D.T_cap,
+                F_cap=D.F_cap)
+    oc = O.Cache.empty(od, U_k1, U_v1)
+    e_all = []
+    e, _, _ = O.compress(oc, K, V, tau, t_new_b=[n_b])
+    e_all.append(e[0, 0, :n_b])
+    for Ka, Va in appends:
+        e, _, _ = O.compress(oc, Ka, Va, tau)
+        e_all.append(e[0, 0])
+    return oc, np.concatenate(e_all)
+
+
+def _gpu_head(D, cache, b, h):
+    """The GPU cache's (b, h) slice as a one-head oracle cache."""
+    od = O.Dims(B=1, Hq=D.Hq // D.Hkv, Hkv=1, d=D.d, r_k=D.r_k, r_v=D.r_v, T_cap=D.T_cap,
+                F_cap=D.F_cap)
+    c = O.Cache.empty(od, U.f64(cache.U_k[h:h + 1]), U.f64(cache.U_v[h:h + 1]))
+    c.coef_k[0, 0] = U.f64(cache.coef_k[b, h])
+    c.coef_v[0, 0] = U.f64(cache.coef_v[b, h])
+    c.route_mask[0, 0] = cache.route_mask[b, h].cpu().numpy().view(np.uint32)
+    c.full_idx[0, 0] = cache.full_idx[b, h].cpu().numpy()
+    c.full_k[0, 0] = U.f64(cache.full_k[b, h])
+    c.full_v[0, 0] = U.f64(cache.full_v[b, h])
+    c.full_cnt[0, 0] = int(cache.full_cnt[b, h])
+    c.seq_len[0] = int(cache.seq_len[b])
+    return c
+
+
+WORKLOADS = [(i, synth.workload(i, layers=1)) for i in (1, 2, 3, 4)]
+
+
+@pytest.mark.parametrize("wi,w", WORKLOADS, ids=[w.name for _, w in WORKLOADS])
+def test_full_size_sampled_heads(wi, w):
+    seed = 31 + wi
+    layer = synth.make_layer(w, 0, seed, device=DEV)
+    T_cap = synth.pad_to(w.T + BENCH_EXTRA, 32)
+    D = U.dims_of(w, T_cap)
+    cache = L.LayerCache(D, layer["U_k"], layer["U_v"], device=DEV)
+    ws = L.make_workspace(D, DEV)
+    lengths = layer["lengths"].tolist()
+    t_new_b = torch.tensor(lengths, dtype=torch.int32, device=DEV) if w.ragged_min else None
+    L.lrkv_compress(D, cache, layer["K"], layer["V"], w.tau, t_new_b=t_new_b, ws=ws)
+    Ka, Va = synth.decode_tokens(w, layer["Qk"], layer["Qv"], N_APPEND, seed, 0, DEV)
+    appends = []
+    for s in range(N_APPEND):
+        k, v = Ka[:, s:s + 1].contiguous(), Va[:, s:s + 1].contiguous()
+        L.lrkv_compress(D, cache, k, v, w.tau, ws=ws)
+        appends.append((U.f64(k), U.f64(v)))
+    out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
+    torch.cuda.synchronize()
+    assert int(cache.dev_status[0]) == 0
+    assert cache.seq_len.tolist() == [n + N_APPEND for n in lengths]
+
+    rng = np.random.default_rng(seed)
+    picks = {(0, 0), (w.B - 1, w.Hkv - 1),
+             (int(rng.integers(w.B)), int(rng.integers(w.Hkv)))}
+    U_k, U_v = U.f64(layer["U_k"]), U.f64(layer["U_v"])
+    g = w.Hq // w.Hkv
+    q = U.f64(layer["q"])
+    for b, h in sorted(picks):
+        Kh = U.f64(layer["K"][b:b + 1, :, h:h + 1])
+        Vh = U.f64(layer["V"][b:b + 1, :, h:h + 1])
+        app_h = [(a[b:b + 1, :, h:h + 1], v[b:b + 1, :, h:h + 1]) for a, v in appends]
+        oc, e_ref = _oracle_head(D, U_k[h:h + 1], U_v[h:h + 1], Kh, Vh, w.tau, lengths[b], app_h)
+        gc = _gpu_head(D, cache, b, h)
+        T = int(oc.seq_len[0])
+        assert int(gc.seq_len[0]) == T
+        # coefficients of every position: 1 ulp + the fp32 accumulation bound
+        X_k = np.concatenate([Kh[0, :lengths[b], 0]] + [a[0, :, 0] for a, _ in app_h])
+        X_v = np.concatenate([Vh[0, :lengths[b], 0]] + [v[0, :, 0] for _, v in app_h])
+        for got, want, X, Ub in ((gc.coef_k[0, 0, :T], oc.coef_k[0, 0, :T], X_k, U_k[h]),
+                                 (gc.coef_v[0, 0, :T], oc.coef_v[0, 0, :T], X_v, U_v[h])):
+            tol = O.bf16_ulp(np.maximum(np.abs(got), np.abs(want)))
+            tol = tol + U.COEF_ABS_SAFETY * U.GAMMA_128 * (np.abs(X) @ np.abs(Ub))
+            bad = np.abs(got - want) > tol
+            assert not bad.any(), f"(b={b},h={h}) {bad.sum()} coefficients off the bound"
+        # routed sets: identical outside the band around tau
+        band = set(np.flatnonzero(np.abs(e_ref - w.tau) < U.BAND).tolist())
+        rg, ro = set(U.routed_positions(gc, 0, 0)), set(U.routed_positions(oc, 0, 0))
+        assert (rg ^ ro) <= band, f"(b={b},h={h}) routed sets differ: {sorted(rg ^ ro)[:10]}"
+        # the list: ascending, matching the mask, rows exact
+        n = int(gc.full_cnt[0, 0])
+        assert n == len(rg)
+        idx = gc.full_idx[0, 0, :n]
+        assert np.array_equal(idx, np.array(sorted(rg), dtype=idx.dtype))
+        src_k = np.concatenate([Kh[0, :lengths[b], 0]] + [a[0, :, 0] for a, _ in app_h])
+        src_v = np.concatenate([Vh[0, :lengths[b], 0]] + [v[0, :, 0] for _, v in app_h])
+        assert np.array_equal(gc.full_k[0, 0, :n], src_k[idx])
+        assert np.array_equal(gc.full_v[0, 0, :n], src_v[idx])
+        # decode over the GPU-written cache
+        ref = O.decode_attn(gc, q[b:b + 1, h * g:(h + 1) * g])
+        assert U.out_rel_err(out[b, h * g:(h + 1) * g], ref[0]) <= U.OUT_RTOL, (b, h)
