@@ -13,22 +13,14 @@ template <int G, int RK, int RV>
 inline lrkv_status launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t s) {
   using S = ds::Shape<G, RK, RV>;
   auto kern = ds::decode_stream_kernel<G, RK, RV>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    return LRKV_ERR_CUDA;
-  }
+  if (!set_smem(kern, S::SMEM)) return LRKV_ERR_CUDA;
   return launch_pdl(kern, grid, dim3(ds::kThreads), S::SMEM, s, p);
 }
 
 template <int G>
 inline lrkv_status launch_simple(const DecodeParams& p, dim3 grid, cudaStream_t s) {
   const size_t smem = decode_simple_smem_bytes(G, p.n_chunk_max);
-  if (cudaFuncSetAttribute(decode_simple_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess) {
-    cudaGetLastError();
-    return LRKV_ERR_CUDA;
-  }
+  if (!set_smem(decode_simple_kernel<G>, smem)) return LRKV_ERR_CUDA;
   decode_simple_kernel<G><<<grid, kDecThreads, smem, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
 }

@@ -169,14 +169,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
 
   // ---- cache state: after the preceding kernel (an append) has completed ------------
   griddep_wait();
+  // the split's mask words (at most one per thread; words past the sequence end
+  // are never used), the sequence length and the list length, all loaded at once
+  static_assert(kMaxChunk / 32 <= kThreads, "one mask word per thread");
+  const int c0 = c * p.chunk;
+  const int wi = c0 / 32 + tid;
+  const bool has_w = tid < p.chunk / 32 && wi < D.T_cap / 32;
+  const uint32_t mw = has_w ? p.C.route_mask[bh * (D.T_cap / 32) + wi] : 0u;
   int T = p.C.seq_len[b];
+  const int F_raw = p.C.full_cnt[bh];
+  if (has_w) maskw[tid] = mw;
   T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
   const int n_chunks = T > 0 ? (T + p.chunk - 1) / p.chunk : 1;
   if (c >= n_chunks) return;
-  const int c0 = c * p.chunk;
   const int c1 = min(T, c0 + p.chunk);
   const int n_pos = c1 > c0 ? c1 - c0 : 0;
-  const int F = min(max(p.C.full_cnt[bh], 0), D.F_cap);
+  const int F = min(max(F_raw, 0), D.F_cap);
   const int share = (F + n_chunks - 1) / n_chunks;
   const int f0 = min(F, c * share), f1 = min(F, f0 + share);
   const int n_full = f1 - f0;
@@ -184,11 +192,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   const lrkv_bf16* cv = p.C.coef_v + bh * D.T_cap * RV + (size_t)c0 * RV;
   const lrkv_bf16* fk = p.C.full_k + (bh * D.F_cap + f0) * kD;
   const lrkv_bf16* fv = p.C.full_v + (bh * D.F_cap + f0) * kD;
-  {
-    const int n_words = (n_pos + 31) / 32;
-    const uint32_t* mask_g = p.C.route_mask + bh * (D.T_cap / 32) + c0 / 32;
-    for (int i = tid; i < n_words; i += kThreads) maskw[i] = mask_g[i];
-  }
   __syncthreads();   // mask words in; every warp is done with U_k (the last stage is free)
 
   // this warp's tiles: full-rank ones first (they need only q), then compressed ones
@@ -272,23 +275,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
       xa = fmaxf(xa, fmaxf(s[nb][0], s[nb][2]));
       xb = fmaxf(xb, fmaxf(s[nb][1], s[nb][3]));
     }
+    // the running maxima only grow: the warp-wide reduction is needed only when
+    // some lane holds a score above them (rare after the first tiles)
+    if (__any_sync(kFull, xa > ma || xb > mb)) {
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      xa = fmaxf(xa, __shfl_xor_sync(kFull, xa, o));
-      xb = fmaxf(xb, __shfl_xor_sync(kFull, xb, o));
-    }
-    if (xa > ma || xb > mb) {
-      const float na = fmaxf(ma, xa), nbm = fmaxf(mb, xb);
-      const float sa = ma == -INFINITY ? 0.f : exp2f(ma - na);
-      const float sb = mb == -INFINITY ? 0.f : exp2f(mb - nbm);
-      la *= sa;
-      lb *= sb;
+      for (int o = 4; o < 32; o <<= 1) {
+        xa = fmaxf(xa, __shfl_xor_sync(kFull, xa, o));
+        xb = fmaxf(xb, __shfl_xor_sync(kFull, xb, o));
+      }
+      if (xa > ma || xb > mb) {
+        const float na = fmaxf(ma, xa), nbm = fmaxf(mb, xb);
+        const float sa = ma == -INFINITY ? 0.f : exp2f(ma - na);
+        const float sb = mb == -INFINITY ? 0.f : exp2f(mb - nbm);
+        la *= sa;
+        lb *= sb;
 #pragma unroll
-      for (int mt = 0; mt < MVT; ++mt) oc[mt][0] *= sa, oc[mt][2] *= sa, oc[mt][1] *= sb, oc[mt][3] *= sb;
+        for (int mt = 0; mt < MVT; ++mt) oc[mt][0] *= sa, oc[mt][2] *= sa, oc[mt][1] *= sb, oc[mt][3] *= sb;
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) of[mt][0] *= sa, of[mt][2] *= sa, of[mt][1] *= sb, of[mt][3] *= sb;
-      ma = na;
-      mb = nbm;
+        for (int mt = 0; mt < 8; ++mt) of[mt][0] *= sa, of[mt][2] *= sa, of[mt][1] *= sb, of[mt][3] *= sb;
+        ma = na;
+        mb = nbm;
+      }
     }
     __syncwarp();
 #pragma unroll
@@ -299,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
       const float p3 = s[nb][3] == -INFINITY ? 0.f : exp2f(s[nb][3] - mb);
       la += p0 + p2;
       lb += p1 + p3;
-      pb0[nb] = movmatrix_t(pack_bf16(bf16_part(p0, lo_col), bf16_part(p1, lo_col)));
-      pb1[nb] = movmatrix_t(pack_bf16(bf16_part(p2, lo_col), bf16_part(p3, lo_col)));
+      pb0[nb] = movmatrix_t(split_bf16x2(p0, p1, lo_col));
+      pb1[nb] = movmatrix_t(split_bf16x2(p2, p3, lo_col));
     }
   };
 
@@ -474,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   float acc_o[NO];
 #pragma unroll
   for (int u = 0; u < NO; ++u) acc_o[u] = 0.f;
-  float run_m = -INFINITY, run_l = 0.f;           // threads < G: head tid
+  float run_m = -INFINITY, run_l = 0.f;           // warps < G: head = warp
   for (int cb = 0; cb < n_chunks; cb += kWB) {
     const int nb = min(kWB, n_chunks - cb);
     {
@@ -485,21 +492,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
       cp_async_wait<0>();
     }
     __syncthreads();
-    // per (record, head) weights against the new running max
-    if (tid < G) {
+    // per (record, head) weights against the new running max: warp gi < G, lanes over records
+    if (warp < G) {
+      const int gi = warp;
       float mx = run_m;
-      for (int k = 0; k < nb; ++k) mx = fmaxf(mx, stage[(k * G + tid) * S::REC]);
-      const float sc = run_m == -INFINITY ? 0.f : exp2f(run_m - mx);
-      float l = run_l * sc;
-      for (int k = 0; k < nb; ++k) {
-        const float* rc = stage + (k * G + tid) * S::REC;
+      for (int k = lane; k < nb; k += 32) mx = fmaxf(mx, stage[(k * G + gi) * S::REC]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+      float l = 0.f;
+      for (int k = lane; k < nb; k += 32) {
+        const float* rc = stage + (k * G + gi) * S::REC;
         const float w = rc[0] == -INFINITY ? 0.f : exp2f(rc[0] - mx);
-        s_w[k][tid] = w;
+        s_w[k][gi] = w;
         l = fmaf(w, rc[1], l);
       }
-      s_run[1][tid] = sc;
+      l = warp_sum(l);
+      const float sc = run_m == -INFINITY ? 0.f : exp2f(run_m - mx);
+      if (lane == 0) s_run[1][gi] = sc;
+      run_l = fmaf(run_l, sc, l);
       run_m = mx;
-      run_l = l;
     }
     __syncthreads();
 #pragma unroll
@@ -507,14 +518,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
       const int o = tid + u * kThreads;
       if (o < NE) {
         const int gi = o / (RV + kD), j = o - gi * (RV + kD);
-        float x = acc_o[u] * s_run[1][gi];
-        for (int k = 0; k < nb; ++k) x = fmaf(s_w[k][gi], stage[(k * G + gi) * S::REC + 4 + j], x);
-        acc_o[u] = x;
+        const float* col = stage + gi * S::REC + 4 + j;
+        constexpr int kStride = G * S::REC;
+        float x0 = acc_o[u] * s_run[1][gi], x1 = 0.f, x2 = 0.f, x3 = 0.f;
+        int k = 0;
+        for (; k + 4 <= nb; k += 4) {
+          x0 = fmaf(s_w[k][gi], col[k * kStride], x0);
+          x1 = fmaf(s_w[k + 1][gi], col[(k + 1) * kStride], x1);
+          x2 = fmaf(s_w[k + 2][gi], col[(k + 2) * kStride], x2);
+          x3 = fmaf(s_w[k + 3][gi], col[(k + 3) * kStride], x3);
+        }
+        for (; k < nb; ++k) x0 = fmaf(s_w[k][gi], col[k * kStride], x0);
+        acc_o[u] = (x0 + x1) + (x2 + x3);
       }
     }
     __syncthreads();
   }
-  if (tid < G) merged[S::M_L + tid] = run_l;
+  if (warp < G && lane == 0) merged[S::M_L + warp] = run_l;
 #pragma unroll
   for (int u = 0; u < NO; ++u) {
     const int o = tid + u * kThreads;

@@ -9,6 +9,21 @@
 
 namespace lrkv {
 
+// Dynamic shared memory limit plus the largest shared-memory carveout: every
+// kernel of the library runs with the same L1/shared split, so an SM never
+// has to drain to reconfigure between consecutive kernels of a step.
+template <typename Kernel>
+inline bool set_smem(Kernel kern, size_t smem) {
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return true;
+}
+
 template <typename Params>
 inline lrkv_status launch_pdl(void (*kern)(Params), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t s, const Params& p) {

@@ -115,9 +115,9 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
   if (per_group < 1) per_group = 1;
   if (per_group > n_units) per_group = n_units;
   const size_t smem = ptc::smem_bytes(pp.r_max);
-  if (cudaFuncSetAttribute(ptc::project_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return launched(), LRKV_ERR_CUDA;
+  if (!set_smem(ptc::project_tc_kernel, smem) || !set_smem(ptc::route_count_kernel, 0) ||
+      !set_smem(ptc::route_scatter_kernel, 0))
+    return LRKV_ERR_CUDA;
   ptc::project_tc_kernel<<<dim3(per_group, groups), ptc::kThreads, smem, s>>>(pp);
   lrkv_status st = launched();
   if (st != LRKV_OK) return st;
@@ -179,9 +179,7 @@ lrkv_status lrkv_compress(const lrkv_dims* dims, const lrkv_cache* cache,
   p.ticket = reinterpret_cast<int32_t*>(w + L.compress_ticket);
   if (t_new <= kAppendMaxTokens) {  // decode-time appends: one fused launch
     const size_t smem = append_smem_bytes(dims->r_k, dims->r_v);
-    if (cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return launched(), LRKV_ERR_CUDA;
+    if (!set_smem(append_kernel, smem)) return LRKV_ERR_CUDA;
     return launch_pdl(append_kernel, dim3(dims->Hkv, dims->B), dim3(kAppendThreads), smem, s, p);
   }
   return compress_tc(*dims, *cache, k_new, v_new, t_new, t_new_b, tau, err_out, w, L, s);

@@ -163,6 +163,19 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
   return l | (h << 16);
 }
+// Two floats -> bf16x2 in one conversion (round to nearest even), `lo` in the low half.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+// The bf16x2 high parts (lo_part false) or low parts (true) of the pair (a, b):
+// x = hi + lo with hi = bf16(x), lo = bf16(x - hi); a in the low half.
+__device__ __forceinline__ uint32_t split_bf16x2(float a, float b, bool lo_part) {
+  const uint32_t h = cvt_bf16x2(a, b);
+  const uint32_t l = cvt_bf16x2(a - __uint_as_float(h << 16), b - __uint_as_float(h & 0xffff0000u));
+  return lo_part ? l : h;
+}
 // x = hi + lo with hi = bf16(x), lo = bf16(x - hi): the part selected by `lo_part`.
 __device__ __forceinline__ float bf16_part(float x, bool lo_part) {
   const float h = __bfloat162float(__float2bfloat16_rn(x));
