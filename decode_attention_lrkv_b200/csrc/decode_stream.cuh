@@ -109,8 +109,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;         // MMA fragment coordinates
-  const bool lo_col = t >= 2;                    // columns 4..7 hold the bf16 low parts
-  const int ha = 2 * (t & 1);                    // heads ha, ha + 1 of this lane's two columns
+  // N columns of the token-side MMAs: column 2h = bf16 high part of query head
+  // h, column 2h + 1 = its low part.  A lane's accumulator fragment (columns
+  // 2t, 2t + 1) therefore holds both parts of head t: one head per lane.
+  const bool live_t = t < G;                     // this lane's head exists
   const int lm = lane >> 3, lr = lane & 7;       // ldmatrix address roles
   const size_t bh = (size_t)b * D.Hkv + h;
 
@@ -129,15 +131,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     cp_async_commit();
   }
   // q as fragments over k = d: the B operand of the full-rank logits (column
-  // n = head n < G; q is bf16, hence exact, so no low-part columns) and, the
-  // same bytes, the A operand (rows = heads) of q~ = U_k^T q
+  // n = 2h holds head h; q is bf16, hence exact, so the low-part columns are 0)
+  // and the A operand (rows = heads) of q~ = U_k^T q
   uint32_t qf0[8], qf1[8];
   {
-    const lrkv_bf16* qrow = p.q + ((size_t)b * D.Hq + (size_t)h * G + (g < G ? g : 0)) * kD;
+    const int hq = g >> 1;                                    // B column g: head g / 2
+    const bool on = (g & 1) == 0 && hq < G;
+    const lrkv_bf16* qrow = p.q + ((size_t)b * D.Hq + (size_t)h * G + (hq < G ? hq : 0)) * kD;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      qf0[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
-      qf1[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
+      qf0[ks] = on ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
+      qf1[ks] = on ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
     }
   }
   const float scale = kLog2e * rsqrtf((float)kD);
@@ -146,6 +150,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   uint32_t qb0[KST], qb1[KST];
   cp_async_wait<0>();
   __syncthreads();
+  uint32_t qa0[8], qa1[8];   // q as the A operand: row m = head m < G
+  {
+    const lrkv_bf16* qrow = p.q + ((size_t)b * D.Hq + (size_t)h * G + (g < G ? g : 0)) * kD;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qa0[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
+      qa1[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
+    }
+  }
 #pragma unroll
   for (int ks2 = 0; ks2 < KST; ++ks2) {        // columns [16 ks2, 16 ks2 + 16) of q~
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -153,16 +166,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     for (int ks = 0; ks < 8; ++ks) {
       uint32_t b0, b1, b2, b3;
       ldsm_x4_t(b0, b1, b2, b3, uk + (ks * 16 + (lm & 1) * 8 + lr) * S::KS + (16 * ks2 + (lm >> 1) * 8) * 2);
-      mma_16816(a0, qf0[ks], 0u, qf1[ks], 0u, b0, b1);
-      mma_16816(a1, qf0[ks], 0u, qf1[ks], 0u, b2, b3);
+      mma_16816(a0, qa0[ks], 0u, qa1[ks], 0u, b0, b1);
+      mma_16816(a1, qa0[ks], 0u, qa1[ks], 0u, b2, b3);
     }
-    // lane (g, t) holds q~[head g][16 ks2 + 2t (+1)] in a0 and [+8] in a1 (rows g < 4);
-    // the low-part columns n = g >= 4 take head g - 4 from lane ^ 16
-    float x0 = __shfl_xor_sync(kFull, a0[0], 16), x1 = __shfl_xor_sync(kFull, a0[1], 16);
-    float y0 = __shfl_xor_sync(kFull, a1[0], 16), y1 = __shfl_xor_sync(kFull, a1[1], 16);
-    const bool lo_n = g >= 4;
-    if (!lo_n) x0 = a0[0], x1 = a0[1], y0 = a1[0], y1 = a1[1];
-    const bool live = (g & 3) < G;
+    // lane (m, t) holds q~[head m][16 ks2 + 2t (+1)] in a0 and [+8] in a1 (rows m < 4).
+    // B column g = 2h + part takes head h from lane 4h + t.
+    const int src = ((g >> 1) << 2) | t;
+    const float x0 = __shfl_sync(kFull, a0[0], src), x1 = __shfl_sync(kFull, a0[1], src);
+    const float y0 = __shfl_sync(kFull, a1[0], src), y1 = __shfl_sync(kFull, a1[1], src);
+    const bool lo_n = g & 1;
+    const bool live = (g >> 1) < G;
     qb0[ks2] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
     qb1[ks2] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
   }
@@ -254,60 +267,51 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   }
 
   // ---- stream the tiles ------------------------------------------------------------
-  // lane state: running max and sum of heads ha, hb; accumulators O^T (rows =
-  // value columns, columns = head parts) for the compressed and full-rank sums
-  float ma = -INFINITY, mb = -INFINITY, la = 0.f, lb = 0.f;
+  // lane state: running max and sum of head t; accumulators O^T (rows = value
+  // columns, columns = head parts: all four fragment entries are head t) for
+  // the compressed and full-rank sums
+  float m_run = -INFINITY, l_run = 0.f;
   float oc[MVT][4], of[8][4];
 #pragma unroll
   for (int mt = 0; mt < MVT; ++mt) oc[mt][0] = oc[mt][1] = oc[mt][2] = oc[mt][3] = 0.f;
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt) of[mt][0] = of[mt][1] = of[mt][2] = of[mt][3] = 0.f;
 
-  // Online softmax over NB 16-row blocks: s[nb] = {head ha at row g, hb at g,
-  // ha at g+8, hb at g+8} (-inf = no token).  Rescales this lane's accumulator
-  // columns when a max grows, and returns the probabilities packed as the
-  // P^T B fragments (bf16 high or low part by column) of each block.
+  // Online softmax over NB 16-row blocks: s[nb] = {row g, row g + 8} of head t
+  // (-inf = no token).  Rescales this lane's accumulators when the max grows,
+  // and returns the probabilities packed as the P^T B fragments of each block
+  // (column 2t = bf16 high part, 2t + 1 = low part).
   auto softmax_pack = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag) {
     constexpr int NB = decltype(nb_tag)::value;
-    float xa = -INFINITY, xb = -INFINITY;
+    float x = -INFINITY;
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      xa = fmaxf(xa, fmaxf(s[nb][0], s[nb][2]));
-      xb = fmaxf(xb, fmaxf(s[nb][1], s[nb][3]));
-    }
-    // the running maxima only grow: the warp-wide reduction is needed only when
-    // some lane holds a score above them (rare after the first tiles)
-    if (__any_sync(kFull, xa > ma || xb > mb)) {
+    for (int nb = 0; nb < NB; ++nb) x = fmaxf(x, fmaxf(s[nb][0], s[nb][1]));
+    // the running max only grows: the reduction over the rows is needed only
+    // when some lane holds a score above it (rare after the first tiles)
+    if (__any_sync(kFull, x > m_run)) {
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        xa = fmaxf(xa, __shfl_xor_sync(kFull, xa, o));
-        xb = fmaxf(xb, __shfl_xor_sync(kFull, xb, o));
-      }
-      if (xa > ma || xb > mb) {
-        const float na = fmaxf(ma, xa), nbm = fmaxf(mb, xb);
-        const float sa = ma == -INFINITY ? 0.f : exp2f(ma - na);
-        const float sb = mb == -INFINITY ? 0.f : exp2f(mb - nbm);
-        la *= sa;
-        lb *= sb;
+      for (int o = 4; o < 32; o <<= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
+      if (x > m_run) {
+        const float sc = m_run == -INFINITY ? 0.f : exp2f(m_run - x);
+        l_run *= sc;
 #pragma unroll
-        for (int mt = 0; mt < MVT; ++mt) oc[mt][0] *= sa, oc[mt][2] *= sa, oc[mt][1] *= sb, oc[mt][3] *= sb;
+        for (int mt = 0; mt < MVT; ++mt) oc[mt][0] *= sc, oc[mt][1] *= sc, oc[mt][2] *= sc, oc[mt][3] *= sc;
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) of[mt][0] *= sa, of[mt][2] *= sa, of[mt][1] *= sb, of[mt][3] *= sb;
-        ma = na;
-        mb = nbm;
+        for (int mt = 0; mt < 8; ++mt) of[mt][0] *= sc, of[mt][1] *= sc, of[mt][2] *= sc, of[mt][3] *= sc;
+        m_run = x;
       }
     }
     __syncwarp();
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
-      const float p0 = s[nb][0] == -INFINITY ? 0.f : exp2f(s[nb][0] - ma);
-      const float p1 = s[nb][1] == -INFINITY ? 0.f : exp2f(s[nb][1] - mb);
-      const float p2 = s[nb][2] == -INFINITY ? 0.f : exp2f(s[nb][2] - ma);
-      const float p3 = s[nb][3] == -INFINITY ? 0.f : exp2f(s[nb][3] - mb);
-      la += p0 + p2;
-      lb += p1 + p3;
-      pb0[nb] = movmatrix_t(split_bf16x2(p0, p1, lo_col));
-      pb1[nb] = movmatrix_t(split_bf16x2(p2, p3, lo_col));
+      const float p0 = s[nb][0] == -INFINITY ? 0.f : exp2f(s[nb][0] - m_run);
+      const float p1 = s[nb][1] == -INFINITY ? 0.f : exp2f(s[nb][1] - m_run);
+      l_run += p0 + p1;
+      // (high part, low part) of p: bf16(p) and bf16(p - bf16(p))
+      const float h0 = __uint_as_float(cvt_bf16x2(p0, p0) << 16);
+      const float h1 = __uint_as_float(cvt_bf16x2(p1, p1) << 16);
+      pb0[nb] = movmatrix_t(cvt_bf16x2(p0, p0 - h0));
+      pb1[nb] = movmatrix_t(cvt_bf16x2(p1, p1 - h1));
     }
   };
 
@@ -332,13 +336,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
           mma_16816(st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
         }
       }
-      float s[2][4];
+      float s[2][2];
 #pragma unroll
       for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const float v = st[nb][x] + __shfl_xor_sync(kFull, st[nb][x], 2);   // high + low part
-          s[nb][x] = (bits >> (16 * nb + g + (x >> 1) * 8)) & 1u ? v : -INFINITY;
+        for (int x = 0; x < 2; ++x) {   // rows g, g + 8: high + low part of head t
+          const float v = st[nb][2 * x] + st[nb][2 * x + 1];
+          s[nb][x] = live_t && ((bits >> (16 * nb + g + x * 8)) & 1u) ? v : -INFINITY;
         }
       uint32_t pb0[2], pb1[2];
       softmax_pack(s, pb0, pb1, std::integral_constant<int, 2>{});
@@ -363,11 +367,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
         ldsm_x4(a0, a1, a2, a3, slot + ((lm & 1) * 8 + lr) * S::FS + (ks * 16 + (lm >> 1) * 8) * 2);
         mma_16816(st, a0, a1, a2, a3, qf0[ks], qf1[ks]);
       }
-      float s[1][4];
+      float s[1][2];
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const float v = (st[x] + __shfl_xor_sync(kFull, st[x], 2)) * scale;   // low-part columns are 0
-        s[0][x] = g + (x >> 1) * 8 < nrows ? v : -INFINITY;
+      for (int x = 0; x < 2; ++x) {   // rows g, g + 8 (the low-part column is 0 for q)
+        const float v = (st[2 * x] + st[2 * x + 1]) * scale;
+        s[0][x] = live_t && g + x * 8 < nrows ? v : -INFINITY;
       }
       uint32_t pb0[1], pb1[1];
       softmax_pack(s, pb0, pb1, std::integral_constant<int, 1>{});
@@ -387,37 +391,26 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
 
   // ---- this warp's partial state into its stage-0 slot -------------------------------
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    la += __shfl_xor_sync(kFull, la, o);
-    lb += __shfl_xor_sync(kFull, lb, o);
-  }
-#pragma unroll
-  for (int mt = 0; mt < MVT; ++mt)
-#pragma unroll
-    for (int x = 0; x < 4; ++x) oc[mt][x] += __shfl_xor_sync(kFull, oc[mt][x], 2);
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-    for (int x = 0; x < 4; ++x) of[mt][x] += __shfl_xor_sync(kFull, of[mt][x], 2);
+  for (int o = 4; o < 32; o <<= 1) l_run += __shfl_xor_sync(kFull, l_run, o);
   {
     float* W = reinterpret_cast<float*>(slot_of(0, warp));
-    if (t < 2) {
-      // lane (g, t<2): heads ha, hb; value columns mt*16 + g and mt*16 + g + 8
+    if (live_t) {
+      // lane (g, t): head t, value columns mt*16 + g and mt*16 + g + 8, high + low part
+      float* pc = W + S::W_PC + t * RV;
+      float* pf = W + S::W_PF + t * kD;
 #pragma unroll
-      for (int hx = 0; hx < 2; ++hx) {
-        const int hd = ha + hx;
-        if (hd < G) {
-          float* pc = W + S::W_PC + hd * RV;
-          float* pf = W + S::W_PF + hd * kD;
+      for (int mt = 0; mt < MVT; ++mt) {
+        pc[mt * 16 + g] = oc[mt][0] + oc[mt][1];
+        pc[mt * 16 + g + 8] = oc[mt][2] + oc[mt][3];
+      }
 #pragma unroll
-          for (int mt = 0; mt < MVT; ++mt) pc[mt * 16 + g] = oc[mt][hx], pc[mt * 16 + g + 8] = oc[mt][2 + hx];
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) pf[mt * 16 + g] = of[mt][hx], pf[mt * 16 + g + 8] = of[mt][2 + hx];
-          if (g == 0) {
-            W[S::W_M + hd] = hx == 0 ? ma : mb;
-            W[S::W_L + hd] = hx == 0 ? la : lb;
-          }
-        }
+      for (int mt = 0; mt < 8; ++mt) {
+        pf[mt * 16 + g] = of[mt][0] + of[mt][1];
+        pf[mt * 16 + g + 8] = of[mt][2] + of[mt][3];
+      }
+      if (g == 0) {
+        W[S::W_M + t] = m_run;
+        W[S::W_L + t] = l_run;
       }
     }
   }
