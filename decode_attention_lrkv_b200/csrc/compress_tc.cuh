@@ -44,22 +44,40 @@ namespace lrkv {
 namespace ptc {
 
 constexpr int kTile = 128;                 // tokens per tile (MMA M)
-constexpr int kStages = 3;                 // input stages
-constexpr int kThreads = 192;              // warps 0-3 epilogue, 4 TMA, 5 MMA + TMEM
+constexpr int kMaxStages = 3;              // input stages (2 when shared memory is short)
+constexpr int kThreads = 320;              // warps 0-7 epilogue, 8 TMA, 9 MMA + TMEM
+constexpr int kEpi = 256;                  // epilogue threads: two per token row
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
 constexpr int kStageBytes = kTile * kD * 2;          // two 64-column boxes
 constexpr int kBoxBytes = kStageBytes / 2;
 constexpr uint32_t kTmemCols = 512;                  // two buffers of [D1 | D2]
 constexpr uint32_t kWaitIters = 1u << 22;
+constexpr size_t kSmemLimit = 227 * 1024;
 
-// shared memory (bytes); every operand region 1024-byte aligned
-constexpr int OFF_X = 0;
-constexpr int OFF_PHI = OFF_X + kStages * kStageBytes;      // B operand [N 128][K 128]
-constexpr int OFF_PLO = OFF_PHI + kD * kD * 2;
-constexpr int OFF_UT = OFF_PLO + kD * kD * 2;               // B operand U^T [N r][K 128]
-// rm = the larger rank of the launch (both tensors share one layout)
-__host__ __device__ inline constexpr int off_u(int rm) { return OFF_UT + rm * kD * 2; }  // U [128][K r]
-__host__ __device__ inline constexpr int off_bar(int rm) { return off_u(rm) + kD * rm * 2; }
-inline constexpr size_t smem_bytes(int rm) { return (size_t)off_bar(rm) + 128 + 1024; }
+// Shared memory (bytes) for rank rm (the larger rank of the launch: both
+// tensors share one layout) and ns input stages; operand regions 1024-aligned.
+//   X stages [ns][128][128] (128-byte swizzle), P_hi, P_lo [128][128],
+//   U^T [rm][128], mbarriers, group B's per-row sums [2][128].
+// U [128][rm] for U U^T is needed only before the first tile: it borrows the
+// last input stage.
+struct Layout {
+  int x, phi, plo, ut, u, bar, part;
+  size_t bytes;
+  __host__ __device__ Layout(int rm, int ns) {
+    x = 0;
+    phi = ns * kStageBytes;
+    plo = phi + kD * kD * 2;
+    ut = plo + kD * kD * 2;
+    u = (ns - 1) * kStageBytes;
+    bar = ut + rm * kD * 2;
+    part = bar + 128;
+    bytes = (size_t)part + 2 * kTile * 8 + 1024;   // + slack to align the base to 1024
+  }
+};
+static_assert(kD * 128 * 2 <= kStageBytes, "U fits in one input stage");
+inline int stages_for(int rm) {
+  return Layout(rm, kMaxStages).bytes <= kSmemLimit ? kMaxStages : kMaxStages - 1;
+}
 
 struct Params {
   CUtensorMap map_k;     // k_new viewed as [B*t_new][Hkv][d], box {64, 1, 128}
@@ -71,6 +89,7 @@ struct Params {
   float* errs;           // [2][B][Hkv][T_cap]
   int tiles_per_b;       // ceil(min(t_new, T_cap) / 128)
   int r_max;             // max(r_k, r_v): the shared-memory layout
+  int n_stages;          // input stages: stages_for(r_max)
 };
 
 // Byte offset of element (row n, column k) in a no-swizzle K-major operand:
@@ -115,15 +134,16 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   const int group = blockIdx.y, tensor = group & 1, h = group >> 1;
   const CUtensorMap* map = tensor == 0 ? &p.map_k : &p.map_v;
   const int R = tensor == 0 ? D.r_k : D.r_v;
-  const int RM = p.r_max;
+  const int NS = p.n_stages;
+  const Layout Lo(p.r_max, NS);
   const lrkv_bf16* Ug = (tensor == 0 ? p.C.U_k : p.C.U_v) + (size_t)h * kD * R;
   lrkv_bf16* coef = tensor == 0 ? p.C.coef_k : p.C.coef_v;
   float* errs = p.errs + (size_t)tensor * D.B * D.Hkv * D.T_cap;
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + off_bar(RM));
-  uint64_t* full = bars;                 // [kStages] TMA -> MMA
-  uint64_t* empty = bars + kStages;      // [kStages] epilogue -> TMA (128 arrivals)
-  uint64_t* dready = bars + 2 * kStages; // [2] MMA -> epilogue
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lo.bar);
+  uint64_t* full = bars;                 // [NS] TMA -> MMA
+  uint64_t* empty = bars + kMaxStages;   // [NS] epilogue -> TMA (kEpi arrivals)
+  uint64_t* dready = bars + 2 * kMaxStages;  // [2] MMA -> epilogue
   uint64_t* tfree = dready + 2;          // [2] epilogue -> MMA (128 arrivals)
   uint64_t* pready = tfree + 2;          // U U^T done
   uint64_t* drain = pready + 1;          // final MMA drain
@@ -136,30 +156,30 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   const int u_end = (int)((long long)(blockIdx.x + 1) * n_units / gridDim.x);
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 128);
+      mbar_init(&empty[s], kEpi);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&dready[b], 1);
-      mbar_init(&tfree[b], 128);
+      mbar_init(&tfree[b], kEpi);
     }
     mbar_init(pready, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc5::tmem_alloc(tmem_slot, kTmemCols);
     tc5::tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) tc5::prefetch_tensormap(map);
+  if (warp == kTmaWarp && lane == 0) tc5::prefetch_tensormap(map);
   // U into two K-major no-swizzle operand layouts:
   //   U   as [m = i][k = j]   (A and B of U U^T), 8-row groups 16 r bytes apart
   //   U^T as [n = j][k = i]   (B of X U),         8-row groups 2048 bytes apart
   {
-    unsigned char* su = sm + off_u(RM);
-    unsigned char* sut = sm + OFF_UT;
+    unsigned char* su = sm + Lo.u;
+    unsigned char* sut = sm + Lo.ut;
     for (int idx = tid; idx < kD * R; idx += kThreads) {
       const int i = idx / R, j = idx - (idx / R) * R;
       const uint16_t u = Ug[idx];
@@ -174,26 +194,28 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   const uint32_t tmem = *tmem_slot;
 
   // ---- P = I - U U^T, split into bf16 high and low parts ----------------------------
-  if (warp == 5 && lane == 0) {
-    const uint32_t ub = smem_u32(sm + off_u(RM));
+  if (warp == kMmaWarp && lane == 0) {
+    const uint32_t ub = smem_u32(sm + Lo.u);
     for (int j = 0; j < R / 16; ++j) {
       const uint64_t d = tc5::smem_desc(ub + j * 256, 128, 16 * R, tc5::kSwizzleNone);
       tc5::mma_bf16(tmem + 128, d, d, tc5::idesc_bf16_f32(128, 128), j > 0);
     }
     tc5::mma_commit(pready);
   }
-  if (warp < 4) {
-    const int m = tid;   // row of U U^T = TMEM lane
+  if (warp < 8) {
+    // row m of U U^T = TMEM lane m; warps w and w + 4 share the rows, columns split
+    const int m = (warp & 3) * 32 + lane;
+    const int cbeg = (warp >> 2) * 64;
     if (!wait_or_abort(pready, 0, abort_flag)) {
       atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
     }
     tc5::fence_after_sync();
-    unsigned char* phi = sm + OFF_PHI;
-    unsigned char* plo = sm + OFF_PLO;
+    unsigned char* phi = sm + Lo.phi;
+    unsigned char* plo = sm + Lo.plo;
 #pragma unroll 1
-    for (int c0 = 0; c0 < kD; c0 += 16) {
+    for (int c0 = cbeg; c0 < cbeg + 64; c0 += 16) {
       float v[16];
-      tc5::tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + 128 + c0, v);
+      tc5::tmem_ld16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + 128 + c0, v);
       tc5::tmem_wait_ld();
       uint32_t hi[8], lo[8];
 #pragma unroll
@@ -218,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   tc5::fence_after_sync();
 
   // ---- pipeline over this CTA's tiles -------------------------------------------------
-  if (warp == 4) {
+  if (warp == kTmaWarp) {
     // TMA producer
     if (lane == 0) {
       int i = 0;
@@ -226,35 +248,35 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
         const int b = u / p.tiles_per_b, t0 = (u - b * p.tiles_per_b) * kTile;
         int start;
         if (t0 >= eff_tokens(p, b, &start)) continue;
-        const int s = i % kStages;
-        if (i >= kStages && !wait_or_abort(&empty[s], ((i / kStages) - 1) & 1, abort_flag)) break;
+        const int s = i % NS;
+        if (i >= NS && !wait_or_abort(&empty[s], ((i / NS) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
-        unsigned char* dst = sm + OFF_X + s * kStageBytes;
+        unsigned char* dst = sm + Lo.x + s * kStageBytes;
         const int z = b * p.t_new + t0;
         tc5::tma_load_3d(dst, map, 0, h, z, &full[s]);
         tc5::tma_load_3d(dst + kBoxBytes, map, 64, h, z, &full[s]);
         ++i;
       }
       // leave no copy in flight: wait for the last fill of every stage
-      for (int k = (i > kStages ? i - kStages : 0); k < i; ++k)
-        mbar_wait_bounded(&full[k % kStages], (k / kStages) & 1, kWaitIters);
+      for (int k = (i > NS ? i - NS : 0); k < i; ++k)
+        mbar_wait_bounded(&full[k % NS], (k / NS) & 1, kWaitIters);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // MMA issuer
     if (lane == 0) {
       const uint32_t idesc1 = tc5::idesc_bf16_f32(128, R);
       const uint32_t idesc2 = tc5::idesc_bf16_f32(128, 128);
-      const uint32_t xbase = smem_u32(sm + OFF_X);
-      const uint32_t utb = smem_u32(sm + OFF_UT);
-      const uint32_t phb = smem_u32(sm + OFF_PHI);
-      const uint32_t plb = smem_u32(sm + OFF_PLO);
+      const uint32_t xbase = smem_u32(sm + Lo.x);
+      const uint32_t utb = smem_u32(sm + Lo.ut);
+      const uint32_t phb = smem_u32(sm + Lo.phi);
+      const uint32_t plb = smem_u32(sm + Lo.plo);
       int i = 0;
       for (int u = u_begin; u < u_end && !*abort_flag; ++u) {
         const int b = u / p.tiles_per_b, t0 = (u - b * p.tiles_per_b) * kTile;
         int start;
         if (t0 >= eff_tokens(p, b, &start)) continue;
-        const int s = i % kStages, buf = i & 1;
-        if (!wait_or_abort(&full[s], (i / kStages) & 1, abort_flag)) break;
+        const int s = i % NS, buf = i & 1;
+        if (!wait_or_abort(&full[s], (i / NS) & 1, abort_flag)) break;
         if (i >= 2 && !wait_or_abort(&tfree[buf], ((i >> 1) - 1) & 1, abort_flag)) break;
         tc5::fence_after_sync();
         const uint32_t d1 = tmem + buf * 256, d2 = d1 + 128;
@@ -283,54 +305,72 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
       mbar_wait_bounded(drain, 0, kWaitIters);
     }
   } else {
-    // epilogue: thread m = row m of the tile = TMEM lane m
-    const int m = tid;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    // epilogue: two threads per token row m = TMEM lane m.  Group A (warps 0-3)
+    // stores the coefficients and sums the squared residual of columns 0-63;
+    // group B (warps 4-7) sums columns 64-127 and the squared input, and hands
+    // its sums to A through shared memory (double-buffered by tile parity).
+    const int m = (warp & 3) * 32 + lane;
+    const bool grp_a = warp < 4;
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    float2* part = reinterpret_cast<float2*>(sm + Lo.part);   // [2][128]
     int i = 0;
     for (int u = u_begin; u < u_end; ++u) {
       const int b = u / p.tiles_per_b, t0 = (u - b * p.tiles_per_b) * kTile;
       int start;
       const int ne = eff_tokens(p, b, &start);
       if (t0 >= ne) continue;
-      const int s = i % kStages, buf = i & 1;
-      if (!wait_or_abort(&dready[buf], (i >> 1) & 1, abort_flag)) break;
+      const int s = i % NS, buf = i & 1;
+      // every epilogue thread stops together, so the named barriers below
+      // always see all of them
+      const bool ok = wait_or_abort(&dready[buf], (i >> 1) & 1, abort_flag);
+      if (!tc5::named_bar_and(1, kEpi, ok)) break;
       tc5::fence_after_sync();
       const int t = t0 + m;
       const bool valid = t < ne;
       const size_t bh = (size_t)b * D.Hkv + h;
-      // coefficients
-      {
+      const uint32_t d1 = lane_base + buf * 256, d2 = d1 + 128;
+      float rs = 0.f, xs = 0.f;
+      if (grp_a) {
+        // coefficients, 64 columns per batch of loads
         lrkv_bf16* crow = coef + (bh * D.T_cap + start + t) * R;
 #pragma unroll 1
-        for (int c0 = 0; c0 < R; c0 += 16) {
-          float v[16];
-          tc5::tmem_ld16(lane_base + buf * 256 + c0, v);
+        for (int c0 = 0; c0 < R; c0 += 64) {
+          float v[4][16];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (c0 + 16 * q < R) tc5::tmem_ld16(d1 + c0 + 16 * q, v[q]);
           tc5::tmem_wait_ld();
-          if (valid) {
-            uint4 w0 = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
-                                  pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-            uint4 w1 = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
-                                  pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
-            *reinterpret_cast<uint4*>(crow + c0) = w0;
-            *reinterpret_cast<uint4*>(crow + c0 + 8) = w1;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (valid && c0 + 16 * q < R) {
+              const float* w = v[q];
+              *reinterpret_cast<uint4*>(crow + c0 + 16 * q) =
+                  make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]),
+                             pack_bf16(w[6], w[7]));
+              *reinterpret_cast<uint4*>(crow + c0 + 16 * q + 8) =
+                  make_uint4(pack_bf16(w[8], w[9]), pack_bf16(w[10], w[11]),
+                             pack_bf16(w[12], w[13]), pack_bf16(w[14], w[15]));
+            }
           }
         }
       }
-      // squared residual
-      float rs = 0.f;
-#pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 16) {
-        float v[16];
-        tc5::tmem_ld16(lane_base + buf * 256 + 128 + c0, v);
-        tc5::tmem_wait_ld();
+      {  // squared residual of this group's 64 columns
+        float v[4][16];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) rs = fmaf(v[q], v[q], rs);
+        for (int q = 0; q < 4; ++q) tc5::tmem_ld16(d2 + (grp_a ? 0 : 64) + 16 * q, v[q]);
+        tc5::tmem_wait_ld();
+        float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int k = 0; k < 16; k += 2) r0 = fmaf(v[q][k], v[q][k], r0), r1 = fmaf(v[q][k + 1], v[q][k + 1], r1);
+        rs = r0 + r1;
       }
-      // squared input: row m of both 64-column boxes, every 16-byte chunk
-      // (the swizzle only permutes chunks within the row)
-      float xs = 0.f;
-      {
-        const unsigned char* xr = sm + OFF_X + s * kStageBytes + m * 128;
+      if (!grp_a) {
+        // squared input: row m of both 64-column boxes, every 16-byte chunk
+        // (the swizzle only permutes chunks within the row)
+        const unsigned char* xr = sm + Lo.x + s * kStageBytes + m * 128;
+        float x0 = 0.f, x1 = 0.f;
 #pragma unroll
         for (int box = 0; box < 2; ++box) {
 #pragma unroll
@@ -340,23 +380,30 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const float a = bf_lo(ws[q]), c = bf_hi(ws[q]);
-              xs = fmaf(a, a, xs);
-              xs = fmaf(c, c, xs);
+              x0 = fmaf(a, a, x0);
+              x1 = fmaf(c, c, x1);
             }
           }
         }
+        xs = x0 + x1;
+        part[(i & 1) * kTile + m] = make_float2(rs, xs);
       }
       tc5::fence_before_sync();
       mbar_arrive(&tfree[buf]);
       mbar_arrive(&empty[s]);
-      if (valid) errs[bh * D.T_cap + t] = xs > 0.f ? sqrtf(rs / xs) : 0.f;
+      tc5::named_bar_sync(1, kEpi);   // group B's sums are in
+      if (grp_a && valid) {
+        const float2 pb = part[(i & 1) * kTile + m];
+        const float rsum = rs + pb.x;
+        errs[bh * D.T_cap + t] = pb.y > 0.f ? sqrtf(rsum / pb.y) : 0.f;
+      }
       ++i;
     }
   }
   if (*abort_flag && tid == 0) atomicOr(p.C.dev_status, LRKV_DEV_WAIT_TIMEOUT);
   tc5::fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc5::fence_after_sync();
     tc5::tmem_dealloc(tmem, kTmemCols);
   }

@@ -109,12 +109,13 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
   pp.errs = reinterpret_cast<float*>(w + L.errs);
   pp.tiles_per_b = (tmax + ptc::kTile - 1) / ptc::kTile;
   pp.r_max = D.r_k > D.r_v ? D.r_k : D.r_v;
+  pp.n_stages = ptc::stages_for(pp.r_max);
   const int groups = 2 * D.Hkv;
   const int n_units = D.B * pp.tiles_per_b;
   int per_group = kNumSMs / groups;
   if (per_group < 1) per_group = 1;
   if (per_group > n_units) per_group = n_units;
-  const size_t smem = ptc::smem_bytes(pp.r_max);
+  const size_t smem = ptc::Layout(pp.r_max, pp.n_stages).bytes;
   if (!set_smem(ptc::project_tc_kernel, smem) || !set_smem(ptc::route_count_kernel, 0) ||
       !set_smem(ptc::route_scatter_kernel, 0))
     return LRKV_ERR_CUDA;
