@@ -537,40 +537,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     }
   }
   __syncthreads();
-  // lift on the tensor cores: A = merged acc_c split into hi (rows 0..3) / lo
-  // (rows 4..7) parts over k = r_v; B = U_v rows (n = output column); warp w
-  // owns the 8-column blocks w and w + 8
-  {
-    const int hh = g & 3;
-    const bool lo_row = g >= 4;
-#pragma unroll
-    for (int nbk = 0; nbk < 2; ++nbk) {
-      const int n0 = 8 * (warp + kWarps * nbk);
-      float l0[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ks = 0; ks < RV / 16; ++ks) {
-        uint32_t a0 = 0u, a2 = 0u;
-        if (hh < G) {
-          const float* row = merged + S::M_CC + hh * RV + ks * 16 + 2 * t;
-          a0 = pack_bf16(bf16_part(row[0], lo_row), bf16_part(row[1], lo_row));
-          a2 = pack_bf16(bf16_part(row[8], lo_row), bf16_part(row[9], lo_row));
-        }
-        uint32_t b0, b1, b2, b3;   // (cols n0.., k lo), (cols n0.., k hi), repeated
-        ldsm_x4(b0, b1, b2, b3, uv + (n0 + lr) * S::VS + (ks * 16 + (lm & 1) * 8) * 2);
-        mma_16816(l0, a0, 0u, a2, 0u, b0, b1);
-      }
-#pragma unroll
-      for (int x = 0; x < 2; ++x) l0[x] += __shfl_xor_sync(kFull, l0[x], 16);
-      if (g < G) {
-        const float L = merged[S::M_L + g];
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        const int i0 = n0 + 2 * t;
-        const float* cf = merged + S::M_CF + g * kD;
-        float* o = p.out + ((size_t)b * D.Hq + (size_t)h * G + g) * kD;
-        o[i0] = (l0[0] + cf[i0]) * inv;
-        o[i0 + 1] = (l0[1] + cf[i0 + 1]) * inv;
-      }
+  // lift on the CUDA cores (G x d outputs of r_v terms each, fp32 against the
+  // bf16 basis rows): o = (U_v acc_c + acc_f) / l
+#pragma unroll 1
+  for (int o = tid; o < G * kD; o += kThreads) {
+    const int gi = o / kD, i = o - gi * kD;
+    const uint32_t* urow = reinterpret_cast<const uint32_t*>(uv + i * S::VS);
+    const float2* cc = reinterpret_cast<const float2*>(merged + S::M_CC + gi * RV);
+    float x0 = 0.f, x1 = 0.f;
+#pragma unroll 8
+    for (int j2 = 0; j2 < RV / 2; ++j2) {
+      const uint32_t u = urow[j2];
+      const float2 c2 = cc[j2];
+      x0 = fmaf(bf_lo(u), c2.x, x0);
+      x1 = fmaf(bf_hi(u), c2.y, x1);
     }
+    const float L = merged[S::M_L + gi];
+    p.out[((size_t)b * D.Hq + (size_t)h * G + gi) * kD + i] =
+        L > 0.f ? (x0 + x1 + merged[S::M_CF + gi * kD + i]) / L : 0.f;
   }
   if (tid == 0) p.tickets[bh] = 0;
 }
