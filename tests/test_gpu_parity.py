@@ -227,3 +227,19 @@ def test_prefill_in_two_parts_unaligned_start():
     assert list(gc.seq_len) == [3000, 2500]
     out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
     assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
+
+
+@pytest.mark.parametrize("Hq,Hkv,r_k,r_v", [(16, 8, 48, 80), (4, 2, 64, 64), (6, 2, 48, 64),
+                                            (16, 2, 32, 32), (8, 8, 32, 48)],
+                         ids=["g2_48_80", "g2_64_64", "g3_simple", "g8_simple", "g1_rank_pair_simple"])
+def test_group_sizes_and_rank_pairs(Hq, Hkv, r_k, r_v):
+    """GQA groups of 1, 2, 3 and 8 query heads and a rank pair outside the
+    streaming kernel's instantiations (served by the CUDA-core kernel)."""
+    w = synth.workload(1, Hq=Hq, Hkv=Hkv, r_k=r_k, r_v=r_v, T=900, layers=1)
+    layer, D, cache, oc, ws = _setup(w, seed=13)
+    gc, band = _compress_both(D, cache, oc, layer["K"], layer["V"], w.tau, ws)
+    extra = synth.decode_tokens(w, layer["Qk"], layer["Qv"], 2, 13, 0, DEV)
+    gc, band = _compress_both(D, cache, oc, extra[0][:, :1].contiguous(), extra[1][:, :1].contiguous(),
+                              w.tau, ws, band=band)
+    out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
+    assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
