@@ -243,3 +243,31 @@ def test_group_sizes_and_rank_pairs(Hq, Hkv, r_k, r_v):
                               w.tau, ws, band=band)
     out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
     assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
+
+
+def test_degenerate_zero_rows_no_list_exact_fill():
+    """All-zero key/value rows (e := 0, never routed), a key-only zero row, a
+    cache with no full-rank list (F_cap = 0: every routed token overflows and
+    stays compressed), and a prefill that fills T_cap exactly."""
+    w = synth.workload(0, T=512)
+    layer, D, cache, oc, ws = _setup(w, seed=17, T_cap=512, F_cap=0)
+    K, V = layer["K"].clone(), layer["V"].clone()
+    K[:, 100:140] = 0
+    V[:, 100:140] = 0
+    K[:, 300] = 0
+    for f in ("full_idx", "full_k", "full_v"):
+        getattr(cache, f).fill_(0x3C3C)
+    gc, _ = _compress_both(D, cache, oc, K, V, w.tau, ws)
+    assert list(gc.seq_len) == [512]
+    assert gc.status == L.DEV_FULL_OVERFLOW and int(gc.full_cnt.sum()) == 0
+    assert not gc.route_mask.any()
+    for f in ("full_idx", "full_k", "full_v"):
+        assert (getattr(cache, f) == 0x3C3C).all(), f
+    assert not gc.coef_k[0, 0, 100:140].any() and not gc.coef_v[0, 0, 100:140].any()
+    out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
+    assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
+    # one more token: the sequence is full, the token is dropped
+    cache.dev_status.zero_()
+    oc.status = 0
+    gc, _ = _compress_both(D, cache, oc, K[:, :1].contiguous(), V[:, :1].contiguous(), w.tau, ws)
+    assert gc.status == L.DEV_SEQ_OVERFLOW and list(gc.seq_len) == [512]
