@@ -207,14 +207,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   const lrkv_bf16* fv = p.C.full_v + (bh * D.F_cap + f0) * kD;
   __syncthreads();   // mask words in; every warp is done with U_k (the last stage is free)
 
-  // this warp's tiles: full-rank ones first (they need only q), then compressed ones
+  // this warp's tiles: every kWarps-th compressed tile and every kWarps-th full-rank tile
   const int n_ct = (n_pos + kTileC - 1) / kTileC;
   const int n_ft = (n_full + kTileF - 1) / kTileF;
   const int nct_w = n_ct > warp ? (n_ct - warp + kWarps - 1) / kWarps : 0;
   const int nft_w = n_ft > warp ? (n_ft - warp + kWarps - 1) / kWarps : 0;
   const int n_tiles = nct_w + nft_w;
-  // tile i of this warp: i < nft_w -> full-rank tile warp + kWarps*i, else
-  // compressed tile warp + kWarps*(i - nft_w)
+  // The warp's sequence interleaves its compressed and full-rank tiles evenly
+  // (a Bresenham walk: step i is compressed when floor((i+1) nct_w / n_tiles)
+  // grows), so the bytes in flight stay near their mean even when a high routed
+  // fraction leaves compressed tiles nearly empty.  `Walk` yields, step by
+  // step, whether the tile is compressed and its index among the warp's tiles
+  // of that kind; the copy side and the compute side each keep one.
+  struct Walk {
+    int err, ic, jf;
+    __device__ __forceinline__ bool next(int nc, int n, int& k) {
+      err += nc;
+      if (err >= n) {
+        err -= n;
+        k = ic++;
+        return true;
+      }
+      k = jf++;
+      return false;
+    }
+  };
+  Walk wi_copy{0, 0, 0}, wi_comp{0, 0, 0};
 
   // positions of compressed tile k that are read: unmasked and before the end
   auto tile_bits = [&](int k) -> uint32_t {
@@ -224,8 +242,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   };
   auto issue = [&](int i) {
     unsigned char* slot = slot_of(i % NST, warp);
-    if (i >= nft_w) {
-      const int k = warp + kWarps * (i - nft_w);
+    int kw;
+    if (wi_copy.next(nct_w, n_tiles, kw)) {
+      const int k = warp + kWarps * kw;
       const uint32_t bits = tile_bits(k);
       const unsigned char* src_k = reinterpret_cast<const unsigned char*>(ck + (size_t)k * kTileC * RK);
       const unsigned char* src_v = reinterpret_cast<const unsigned char*>(cv + (size_t)k * kTileC * RV);
@@ -243,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
         cp_async16_zfill(vslot + r * S::VS + sg * 16, on ? src_v + q * 16 : src_v, on ? 16u : 0u);
       }
     } else {
-      const int k = warp + kWarps * i;
+      const int k = warp + kWarps * kw;
       const int r0 = k * kTileF;
       const int n = min(kTileF, n_full - r0);
       const unsigned char* src_k = reinterpret_cast<const unsigned char*>(fk + (size_t)r0 * kD);
@@ -321,9 +340,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     cp_async_wait<NST - 1>();
     __syncwarp();
     const unsigned char* slot = slot_of(i % NST, warp);
-    if (i >= nft_w) {
+    int kw;
+    if (wi_comp.next(nct_w, n_tiles, kw)) {
       // compressed tile: S^T[token][head part] = C_k q~^T, then O^T += C_v^T P^T
-      const uint32_t bits = tile_bits(warp + kWarps * (i - nft_w));
+      const uint32_t bits = tile_bits(warp + kWarps * kw);
       float st[2][4];
 #pragma unroll
       for (int nb = 0; nb < 2; ++nb) {
@@ -358,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
         }
     } else {
       // full-rank tile: 16 list rows
-      const int k = warp + kWarps * i;
+      const int k = warp + kWarps * kw;
       const int nrows = min(kTileF, n_full - k * kTileF);
       float st[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
