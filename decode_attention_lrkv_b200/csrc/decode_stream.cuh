@@ -31,9 +31,10 @@
 // Rows land in padded shared-memory rows (stride 2r+16 bytes) so ldmatrix is
 // conflict-free.  Three ring stages where shared memory allows, else two.
 // At the end each warp leaves its partial softmax state in its own slot, the
-// CTA merges its warps and writes one record (m, l, acc_c[r_v], acc_f[d]) per
-// query head, and the last CTA of the (batch row, kv head) merges all records
-// (atomic ticket, no waiting) and lifts once: o = (U_v acc_c + acc_f) / l.
+// CTA merges its warps, lifts its value sum on the tensor cores
+// (U_v acc_c + acc_f) and writes one record (m, l, o[d]) per query head; the
+// last CTA of the (batch row, kv head) (atomic ticket, no waiting) merges the
+// records in registers, straight from L2: o = sum_c w_c o_c / sum_c w_c l_c.
 //
 // Programmatic dependent launch: U_k and q are loaded and q~ is formed before
 // waiting on the preceding kernel of the stream (an append to the same
@@ -71,12 +72,19 @@ struct Shape {
   static constexpr int SLOT_C = kTileC * (KS + VS);
   static constexpr int SLOT_F = kTileF * 2 * FS;
   static constexpr int SLOT = al128(imax(SLOT_C, SLOT_F));
-  static constexpr int FIXED = (kMaxChunk / 32) * 4;               // mask words
-  static constexpr int STAGES = kWarps * 3 * SLOT + FIXED <= 227 * 1024 ? 3 : 2;
+  static constexpr int MASK_BYTES = (kMaxChunk / 32) * 4;          // mask words
+  static constexpr int SMEM_MAX = 227 * 1024 - 1024;               // static shared memory aside
+  static constexpr int STAGES = kWarps * 3 * SLOT + MASK_BYTES <= SMEM_MAX ? 3 : 2;
   static constexpr int RING = kWarps * STAGES * SLOT;             // [stage][warp][SLOT]
   static constexpr int OFF_MASK = RING;
-  static constexpr int SMEM = OFF_MASK + (kMaxChunk / 32) * 4;
-  static_assert(SMEM <= 227 * 1024, "shared memory of one CTA");
+  // U_v rows [d][VS] for the per-split lift: resident beside the ring (loaded
+  // in the prologue) where it fits, else loaded into the tail of the ring once
+  // the stream is done
+  static constexpr int UVB = kD * VS;
+  static constexpr bool UV_RES = RING + MASK_BYTES + UVB <= SMEM_MAX;
+  static constexpr int OFF_UV = UV_RES ? RING + MASK_BYTES : ((RING - UVB) & ~127);
+  static constexpr int SMEM = UV_RES ? OFF_UV + UVB : RING + MASK_BYTES;
+  static_assert(SMEM <= SMEM_MAX, "shared memory of one CTA");
   // U_k rows [d][KS] live in the last stage until every warp has its q~
   static constexpr int OFF_UK = (STAGES - 1) * kWarps * SLOT;
   static_assert(kD * KS <= kWarps * SLOT, "U_k fits in one stage");
@@ -86,15 +94,16 @@ struct Shape {
   static constexpr int W_M = W_PF + G * kD;         // [G]
   static constexpr int W_L = W_M + G;               // [G]
   static_assert((W_L + G) * 4 <= SLOT, "partials fit in a slot");
-  static constexpr int REC = 4 + RV + kD;           // record floats per query head
-  // final merge: U_v rows [d][VS] at the end of the ring, records staged before it
-  static constexpr int OFF_UV = (RING - kD * VS) & ~127;
-  static constexpr int STAGE_BYTES = OFF_UV;
-  // merged sums of the final merge, after the staged records' batch area (floats)
+  // the CTA's merged sums, in the first slot of stage 1 (floats)
+  static constexpr int OFF_MRG = kWarps * SLOT;
   static constexpr int M_CC = 0;                    // [G][RV]
   static constexpr int M_CF = M_CC + G * RV;        // [G][d]
-  static constexpr int M_L = M_CF + G * kD;         // [G]
-  static constexpr int MERGE_FLOATS = M_L + G;
+  static constexpr int MERGE_FLOATS = M_CF + G * kD;
+  static_assert(STAGES >= 2, "stage 1 holds the merged sums");
+  static_assert(OFF_MRG + MERGE_FLOATS * 4 <= (UV_RES ? RING : OFF_UV), "merged sums beside U_v");
+  static_assert(kD == 16 * kWarps, "one 16-row block of the lift per warp");
+  // record of one split per query head: m, l, two pad floats, o[d] = U_v acc_c + acc_f
+  static constexpr int REC = 4 + kD;
 };
 
 template <int G, int RK, int RV>
@@ -130,6 +139,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     }
     cp_async_commit();
   }
+  auto load_uv = [&]() {   // U_v into padded rows, 16-byte pieces over every thread
+    const unsigned char* Uv = reinterpret_cast<const unsigned char*>(p.C.U_v + (size_t)h * kD * RV);
+    for (int q = tid; q < kD * VP; q += kThreads) {
+      const int r = q / VP, sg = q - r * VP;
+      cp_async16(sm + S::OFF_UV + r * S::VS + sg * 16, Uv + q * 16);
+    }
+    cp_async_commit();
+  };
+  if constexpr (S::UV_RES) load_uv();
   // q as fragments over k = d: the B operand of the full-rank logits (column
   // n = 2h holds head h; q is bf16, hence exact, so the low-part columns are 0)
   // and the A operand (rows = heads) of q~ = U_k^T q
@@ -148,7 +166,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   // q~ = U_k^T q as this warp's B fragments over k = r_k (column n < 4 = bf16
   // high part of head n, n >= 4 = low part of head n - 4), on the tensor cores
   uint32_t qb0[KST], qb1[KST];
-  cp_async_wait<0>();
+  if constexpr (S::UV_RES) cp_async_wait<1>();   // U_k in (U_v may still be in flight)
+  else cp_async_wait<0>();
   __syncthreads();
   uint32_t qa0[8], qa1[8];   // q as the A operand: row m = head m < G
   {
@@ -182,16 +201,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
 
   // ---- cache state: after the preceding kernel (an append) has completed ------------
   griddep_wait();
-  // the split's mask words (at most one per thread; words past the sequence end
-  // are never used), the sequence length and the list length, all loaded at once
-  static_assert(kMaxChunk / 32 <= kThreads, "one mask word per thread");
+  // the split's mask words (words past the sequence end are never used), the
+  // sequence length and the list length, all loaded at once
+  constexpr int kMW = (kMaxChunk / 32 + kThreads - 1) / kThreads;   // mask words per thread
   const int c0 = c * p.chunk;
-  const int wi = c0 / 32 + tid;
-  const bool has_w = tid < p.chunk / 32 && wi < D.T_cap / 32;
-  const uint32_t mw = has_w ? p.C.route_mask[bh * (D.T_cap / 32) + wi] : 0u;
+  uint32_t mw[kMW];
+#pragma unroll
+  for (int u = 0; u < kMW; ++u) {
+    const int wl = tid + u * kThreads, wi = c0 / 32 + wl;
+    mw[u] = wl < p.chunk / 32 && wi < D.T_cap / 32 ? p.C.route_mask[bh * (D.T_cap / 32) + wi] : 0u;
+  }
   int T = p.C.seq_len[b];
   const int F_raw = p.C.full_cnt[bh];
-  if (has_w) maskw[tid] = mw;
+#pragma unroll
+  for (int u = 0; u < kMW; ++u)
+    if (tid + u * kThreads < kMaxChunk / 32) maskw[tid + u * kThreads] = mw[u];
   T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
   const int n_chunks = T > 0 ? (T + p.chunk - 1) / p.chunk : 1;
   if (c >= n_chunks) return;
@@ -436,10 +460,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   }
   __syncthreads();
 
-  // ---- merge the warps into this split's record --------------------------------------
+  // ---- merge the warps into this split's record, lift, write it -------------------
+  if constexpr (!S::UV_RES) load_uv();           // into the tail of the ring, behind stage 0
   auto wpart = [&](int w) { return reinterpret_cast<const float*>(slot_of(0, w)); };
   __shared__ float s_we[kWarps][G];
   float* rec0 = p.partials + (bh * p.n_chunk_max + c) * G * (size_t)S::REC;
+  float* mrg = reinterpret_cast<float*>(sm + S::OFF_MRG);
   if (tid < G) {
     float M = -INFINITY;
     for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wpart(w)[S::W_M + tid]);
@@ -460,7 +486,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     float x = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[src], s_we[w][gi], x);
-    rec0[gi * S::REC + 4 + j] = x;
+    mrg[src] = x;   // same [G][RV], [G][d] layout as a warp's partials
+  }
+  cp_async_wait<0>();   // U_v
+  __syncthreads();
+  // Lift on the tensor cores: O[d][head part] = U_v [d x r_v] * acc_c^T, warp w
+  // taking rows [16w, 16w + 16).  B column n = 2h + part holds the bf16 high
+  // or low part of head h's acc_c, so a lane's accumulator fragment (columns
+  // 2t, 2t + 1) is head t again: o = high + low + acc_f.
+  {
+    const unsigned char* uv = sm + S::OFF_UV;
+    const int hb = g >> 1;                       // B column g: head g / 2
+    const bool lo_n = g & 1;
+    const float* cc = mrg + S::M_CC + (hb < G ? hb : 0) * RV;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < RV / 16; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(a0, a1, a2, a3, uv + (16 * warp + (lm & 1) * 8 + lr) * S::VS + (ks * 16 + (lm >> 1) * 8) * 2);
+      const float2 x = *reinterpret_cast<const float2*>(cc + ks * 16 + 2 * t);
+      const float2 y = *reinterpret_cast<const float2*>(cc + ks * 16 + 8 + 2 * t);
+      const uint32_t b0 = hb < G ? pack_bf16(bf16_part(x.x, lo_n), bf16_part(x.y, lo_n)) : 0u;
+      const uint32_t b1 = hb < G ? pack_bf16(bf16_part(y.x, lo_n), bf16_part(y.y, lo_n)) : 0u;
+      mma_16816(acc, a0, a1, a2, a3, b0, b1);
+    }
+    if (live_t) {
+      const int i0 = 16 * warp + g;
+      const float* cf = mrg + S::M_CF + t * kD;
+      rec0[t * S::REC + 4 + i0] = acc[0] + acc[1] + cf[i0];
+      rec0[t * S::REC + 4 + i0 + 8] = acc[2] + acc[3] + cf[i0 + 8];
+    }
   }
 
   // ---- the last split of this (batch row, kv head) merges every record ------------
@@ -468,113 +523,65 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   if (tid == 0) s_last = atom_add_acq_rel_gpu(p.tickets + bh, 1) == n_chunks - 1;
   __syncthreads();
   if (!s_last) return;
-  // U_v for the lift, then the records in batches through the ring, merged
-  // with a running max per (head, element); all loads are 16-byte cp.async
-  // pieces over every thread
-  unsigned char* uv = sm + S::OFF_UV;
+  // Warp w serves query head w / (kWarps / G) and a block of its columns; each
+  // lane finds the head's global max and sum itself (lanes over records), then
+  // accumulates its columns over the records with the weights passed by
+  // shuffle.  Records come from L2 (ld.global.cg): other CTAs wrote them.
   {
-    const unsigned char* Uv = reinterpret_cast<const unsigned char*>(p.C.U_v + (size_t)h * kD * RV);
-    for (int q = tid; q < kD * VP; q += kThreads) {
-      const int r = q / VP, sg = q - r * VP;
-      cp_async16(uv + r * S::VS + sg * 16, Uv + q * 16);
-    }
-    cp_async_commit();
-  }
-  const float* recs = p.partials + bh * p.n_chunk_max * G * (size_t)S::REC;
-  constexpr int kRecBytes = G * S::REC * 4;
-  constexpr int per_batch = (S::STAGE_BYTES - S::MERGE_FLOATS * 4) / kRecBytes;
-  static_assert(per_batch >= 1, "one record batch fits");
-  float* stage = reinterpret_cast<float*>(sm);
-  float* merged = stage + per_batch * G * S::REC;   // [G][RV], [G][d], [G]
-  __shared__ float s_w[per_batch < 64 ? per_batch : 64][G];   // weights of one batch
-  __shared__ float s_run[2][G];                               // [1]: old-sum scale of a batch
-  constexpr int kWB = per_batch < 64 ? per_batch : 64;        // records per batch
-  constexpr int NE = G * (RV + kD);
-  constexpr int NO = (NE + kThreads - 1) / kThreads;
-  float acc_o[NO];
+    constexpr int WPH = kWarps / G;              // warps per head
+    constexpr int CPW = kD / WPH;                // columns per warp: 16, 32, 64
+    constexpr int CPL = CPW >= 32 ? CPW / 32 : 1;
+    const int gi = warp / WPH;
+    const int col = (warp - gi * WPH) * CPW + lane * CPL;
+    const bool on = lane * CPL < CPW;
+    const float* recs = p.partials + bh * p.n_chunk_max * G * (size_t)S::REC + gi * S::REC;
+    constexpr size_t kStride = (size_t)G * S::REC;   // floats between two records of a head
+    float acc[CPL];
 #pragma unroll
-  for (int u = 0; u < NO; ++u) acc_o[u] = 0.f;
-  float run_m = -INFINITY, run_l = 0.f;           // warps < G: head = warp
-  for (int cb = 0; cb < n_chunks; cb += kWB) {
-    const int nb = min(kWB, n_chunks - cb);
-    {
-      const unsigned char* src = reinterpret_cast<const unsigned char*>(recs + (size_t)cb * G * S::REC);
-      unsigned char* dst = reinterpret_cast<unsigned char*>(stage);
-      for (int q = tid; q < nb * kRecBytes / 16; q += kThreads) cp_async16(dst + q * 16, src + q * 16);
-      cp_async_commit();
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    // per (record, head) weights against the new running max: warp gi < G, lanes over records
-    if (warp < G) {
-      const int gi = warp;
-      float mx = run_m;
-      for (int k = lane; k < nb; k += 32) mx = fmaxf(mx, stage[(k * G + gi) * S::REC]);
+    for (int u = 0; u < CPL; ++u) acc[u] = 0.f;
+    float Lsum = 0.f;
+    // one batch of up to 32 records: every load is issued before the first use
+    auto batch = [&](int k0, float M) {
+      const int k = k0 + lane;
+      const int nk = min(32, n_chunks - k0);
+      float vals[32][CPL];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-      float l = 0.f;
-      for (int k = lane; k < nb; k += 32) {
-        const float* rc = stage + (k * G + gi) * S::REC;
-        const float w = rc[0] == -INFINITY ? 0.f : exp2f(rc[0] - mx);
-        s_w[k][gi] = w;
-        l = fmaf(w, rc[1], l);
-      }
-      l = warp_sum(l);
-      const float sc = run_m == -INFINITY ? 0.f : exp2f(run_m - mx);
-      if (lane == 0) s_run[1][gi] = sc;
-      run_l = fmaf(run_l, sc, l);
-      run_m = mx;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int u = 0; u < NO; ++u) {
-      const int o = tid + u * kThreads;
-      if (o < NE) {
-        const int gi = o / (RV + kD), j = o - gi * (RV + kD);
-        const float* col = stage + gi * S::REC + 4 + j;
-        constexpr int kStride = G * S::REC;
-        float x0 = acc_o[u] * s_run[1][gi], x1 = 0.f, x2 = 0.f, x3 = 0.f;
-        int k = 0;
-        for (; k + 4 <= nb; k += 4) {
-          x0 = fmaf(s_w[k][gi], col[k * kStride], x0);
-          x1 = fmaf(s_w[k + 1][gi], col[(k + 1) * kStride], x1);
-          x2 = fmaf(s_w[k + 2][gi], col[(k + 2) * kStride], x2);
-          x3 = fmaf(s_w[k + 3][gi], col[(k + 3) * kStride], x3);
+      for (int j = 0; j < 32; ++j) {
+        const float* v = recs + (size_t)(k0 + j) * kStride + 4 + col;
+        if constexpr (CPL == 2) {
+          const float2 x = j < nk && on ? __ldcg(reinterpret_cast<const float2*>(v)) : make_float2(0.f, 0.f);
+          vals[j][0] = x.x;
+          vals[j][CPL - 1] = x.y;
+        } else {
+          vals[j][0] = j < nk && on ? __ldcg(v) : 0.f;
         }
-        for (; k < nb; ++k) x0 = fmaf(s_w[k][gi], col[k * kStride], x0);
-        acc_o[u] = (x0 + x1) + (x2 + x3);
       }
-    }
-    __syncthreads();
-  }
-  if (warp < G && lane == 0) merged[S::M_L + warp] = run_l;
+      const float m = k < n_chunks ? __ldcg(recs + (size_t)k * kStride) : -INFINITY;
+      const float l = k < n_chunks ? __ldcg(recs + (size_t)k * kStride + 1) : 0.f;
+      if (M == -INFINITY) M = warp_max(m);      // a single batch: its own max is the max
+      const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+      Lsum = fmaf(w, l, Lsum);
 #pragma unroll
-  for (int u = 0; u < NO; ++u) {
-    const int o = tid + u * kThreads;
-    if (o < NE) {
-      const int gi = o / (RV + kD), j = o - gi * (RV + kD);
-      merged[j < RV ? S::M_CC + gi * RV + j : S::M_CF + gi * kD + (j - RV)] = acc_o[u];
+      for (int j = 0; j < 32; ++j) {
+        const float wj = __shfl_sync(kFull, w, j);
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) acc[u] = fmaf(wj, vals[j][u], acc[u]);
+      }
+    };
+    if (n_chunks <= 32) {
+      batch(0, -INFINITY);
+    } else {
+      float M = -INFINITY;
+      for (int k = lane; k < n_chunks; k += 32) M = fmaxf(M, __ldcg(recs + (size_t)k * kStride));
+      M = warp_max(M);
+      for (int k0 = 0; k0 < n_chunks; k0 += 32) batch(k0, M);
     }
-  }
-  __syncthreads();
-  // lift on the CUDA cores (G x d outputs of r_v terms each, fp32 against the
-  // bf16 basis rows): o = (U_v acc_c + acc_f) / l
-#pragma unroll 1
-  for (int o = tid; o < G * kD; o += kThreads) {
-    const int gi = o / kD, i = o - gi * kD;
-    const uint32_t* urow = reinterpret_cast<const uint32_t*>(uv + i * S::VS);
-    const float2* cc = reinterpret_cast<const float2*>(merged + S::M_CC + gi * RV);
-    float x0 = 0.f, x1 = 0.f;
-#pragma unroll 8
-    for (int j2 = 0; j2 < RV / 2; ++j2) {
-      const uint32_t u = urow[j2];
-      const float2 c2 = cc[j2];
-      x0 = fmaf(bf_lo(u), c2.x, x0);
-      x1 = fmaf(bf_hi(u), c2.y, x1);
+    Lsum = warp_sum(Lsum);
+    if (on) {
+      float* out = p.out + ((size_t)b * D.Hq + (size_t)h * G + gi) * kD + col;
+#pragma unroll
+      for (int u = 0; u < CPL; ++u) out[u] = Lsum > 0.f ? acc[u] / Lsum : 0.f;
     }
-    const float L = merged[S::M_L + gi];
-    p.out[((size_t)b * D.Hq + (size_t)h * G + gi) * kD + i] =
-        L > 0.f ? (x0 + x1 + merged[S::M_CF + gi * kD + i]) / L : 0.f;
   }
   if (tid == 0) p.tickets[bh] = 0;
 }

@@ -29,6 +29,12 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
 // Number of new tokens sequence b contributes, and the status bits it raises.
 __device__ __forceinline__ int new_tokens(const int32_t* t_new_b, int b, int t_new,
                                           uint32_t* flags) {
