@@ -108,7 +108,6 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
   __shared__ int s_cnt;
   __shared__ bool s_last;
   __shared__ float s_err[2];
-  __shared__ uint32_t s_mask[2];    // the (at most two) mask words the new positions touch
 
   // bases first: they do not depend on the preceding kernel of the stream
   if (tid == 0) {
@@ -124,25 +123,40 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
 
   uint32_t st = 0;
   const int n = new_tokens(p.t_new_b, b, p.t_new, &st);
-  const int start = min(max(p.C.seq_len[b], 0), D.T_cap);
-  int n_eff = D.T_cap - start;
-  if (n_eff > n) n_eff = n;
-  if (n_eff < 0) n_eff = 0;
   const size_t bh = (size_t)b * D.Hkv + h;
-  uint32_t* mask_row = p.C.route_mask + bh * (D.T_cap / 32);
-
+  // the new rows do not depend on the cache state: their copies go out first
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar, n_eff * 4u * kD);   // the arrival that closes the phase
-    for (int t = 0; t < n_eff; ++t) {
+    mbar_arrive_expect_tx(bar, n * 4u * kD);   // the arrival that closes the phase
+    for (int t = 0; t < n; ++t) {
       const size_t x = (((size_t)b * p.t_new + t) * D.Hkv + h) * kD;
       bulk_g2s(Xks + t * kD, p.k_new + x, 2u * kD, bar);
       bulk_g2s(Xvs + t * kD, p.v_new + x, 2u * kD, bar);
     }
-    if (n_eff > 0) {
-      s_cnt = min(max(p.C.full_cnt[bh], 0), D.F_cap);
-      s_mask[0] = mask_row[start >> 5];
-      s_mask[1] = ((start + n_eff - 1) >> 5) != (start >> 5) ? mask_row[(start >> 5) + 1] : 0u;
+  }
+  const int start = min(max(p.C.seq_len[b], 0), D.T_cap);
+  const int cnt0 = tid == 0 ? p.C.full_cnt[bh] : 0;
+  int n_eff = D.T_cap - start;
+  if (n_eff > n) n_eff = n;
+  if (n_eff < 0) n_eff = 0;
+  uint32_t* mask_row = p.C.route_mask + bh * (D.T_cap / 32);
+  if (tid == 0) s_cnt = min(max(cnt0, 0), D.F_cap);
+  // Every thread of this CTA holds its sequence's start: take the ticket now.
+  // The CTA that takes the last one advances every sequence's length; the
+  // other CTAs have all read theirs by then (acquire/release on the ticket).
+  __syncthreads();
+  if (tid == 0) s_last = atom_add_acq_rel_gpu(p.ticket, 1) == (int)(gridDim.x * gridDim.y) - 1;
+  __syncthreads();
+  if (s_last) {
+    for (int bb = tid; bb < D.B; bb += kAppendThreads) {
+      uint32_t dummy = 0;
+      const int nb = new_tokens(p.t_new_b, bb, p.t_new, &dummy);
+      const int sb = min(max(p.C.seq_len[bb], 0), D.T_cap);
+      int ne = D.T_cap - sb;
+      if (ne > nb) ne = nb;
+      if (ne < 0) ne = 0;
+      p.C.seq_len[bb] = sb + ne;
     }
+    if (tid == 0) *p.ticket = 0;
   }
   __syncthreads();
   // every copy (bases included) lands before anything else, also when there is no token
@@ -155,6 +169,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
   }
   if (n_eff > 0) {
     bool overflow = false;
+    uint32_t m_or[2] = {0u, 0u}, m_and[2] = {~0u, ~0u};   // edits of the (at most two) mask words
     for (int t = 0; t < n_eff; ++t) {
       const int pos = start + t;
       const size_t row = bh * D.T_cap + pos;
@@ -177,8 +192,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
       }
       if (tid == 0) {
         const uint32_t bit = 1u << (pos & 31);
-        uint32_t& mw = s_mask[(pos >> 5) - (start >> 5)];
-        mw = keep ? (mw | bit) : (mw & ~bit);
+        const int wsel = (pos >> 5) - (start >> 5);
+        if (keep) m_or[wsel] |= bit;
+        else m_and[wsel] &= ~bit;
         if (keep) {
           p.C.full_idx[bh * D.F_cap + slot] = pos;
           s_cnt = slot + 1;
@@ -189,34 +205,18 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
     }
     if (tid == 0) {
       p.C.full_cnt[bh] = s_cnt;
-      mask_row[start >> 5] = s_mask[0];
-      if (((start + n_eff - 1) >> 5) != (start >> 5)) mask_row[(start >> 5) + 1] = s_mask[1];
+      // bits of earlier positions in the same words stay as they are
+      const int nw = ((start + n_eff - 1) >> 5) - (start >> 5) + 1;
+      for (int u = 0; u < nw; ++u) {
+        if (m_or[u]) atomicOr(mask_row + (start >> 5) + u, m_or[u]);
+        if (m_and[u] != ~0u) atomicAnd(mask_row + (start >> 5) + u, m_and[u]);
+      }
       if (overflow) st |= LRKV_DEV_FULL_OVERFLOW;
     }
   }
   if (n_eff < n && !(st & LRKV_DEV_WAIT_TIMEOUT)) st |= LRKV_DEV_SEQ_OVERFLOW;
   if (h != 0) st &= LRKV_DEV_FULL_OVERFLOW;     // per-sequence conditions: reported once
   if (tid == 0 && st) atomicOr(p.C.dev_status, st);
-  // the last CTA advances every sequence's length (all CTAs have read them)
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    s_last = atomicAdd(p.ticket, 1) == (int)(gridDim.x * gridDim.y) - 1;
-  }
-  __syncthreads();
-  if (s_last) {
-    __threadfence();
-    for (int bb = tid; bb < D.B; bb += kAppendThreads) {
-      uint32_t dummy = 0;
-      const int nb = new_tokens(p.t_new_b, bb, p.t_new, &dummy);
-      const int sb = min(max(p.C.seq_len[bb], 0), D.T_cap);
-      int ne = D.T_cap - sb;
-      if (ne > nb) ne = nb;
-      if (ne < 0) ne = 0;
-      p.C.seq_len[bb] = sb + ne;
-    }
-    if (tid == 0) *p.ticket = 0;
-  }
 }
 
 }  // namespace lrkv
