@@ -9,12 +9,12 @@
 
 namespace lrkv {
 
-template <int G, int RK, int RV>
+template <int G, int RK, int RV, int W, int NS>
 inline lrkv_status launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t s) {
-  using S = ds::Shape<G, RK, RV>;
-  auto kern = ds::decode_stream_kernel<G, RK, RV>;
+  using S = ds::Shape<G, RK, RV, W, NS>;
+  auto kern = ds::decode_stream_kernel<G, RK, RV, W, NS>;
   if (!set_smem(kern, S::SMEM)) return LRKV_ERR_CUDA;
-  return launch_pdl(kern, grid, dim3(ds::kThreads), S::SMEM, s, p);
+  return launch_pdl(kern, grid, dim3(S::kThreads), S::SMEM, s, p);
 }
 
 template <int G>
@@ -29,11 +29,13 @@ template <int G>
 inline lrkv_status launch_stream_g(const DecodeParams& p, dim3 grid, cudaStream_t s, bool* done) {
   *done = true;
   const int rk = p.D.r_k, rv = p.D.r_v;
-  if (rk == 32 && rv == 32) return launch_stream<G, 32, 32>(p, grid, s);
-  if (rk == 48 && rv == 64) return launch_stream<G, 48, 64>(p, grid, s);
-  if (rk == 48 && rv == 80) return launch_stream<G, 48, 80>(p, grid, s);
-  if (rk == 64 && rv == 64) return launch_stream<G, 64, 64>(p, grid, s);
-  if (rk == 64 && rv == 96) return launch_stream<G, 64, 96>(p, grid, s);
+  // (warps per CTA, ring stages per warp) per shape: what shared memory holds
+  // beside the mask words and the resident U_v
+  if (rk == 32 && rv == 32) return launch_stream<G, 32, 32, 8, 3>(p, grid, s);
+  if (rk == 48 && rv == 64) return launch_stream<G, 48, 64, 8, 3>(p, grid, s);
+  if (rk == 48 && rv == 80) return launch_stream<G, 48, 80, 8, 2>(p, grid, s);
+  if (rk == 64 && rv == 64) return launch_stream<G, 64, 64, 8, 2>(p, grid, s);
+  if (rk == 64 && rv == 96) return launch_stream<G, 64, 96, 8, 2>(p, grid, s);
   *done = false;
   return LRKV_OK;
 }

@@ -50,8 +50,6 @@
 namespace lrkv {
 namespace ds {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
 constexpr int kTileC = 32;                       // positions per compressed tile (one mask word)
 constexpr int kTileF = 16;                       // rows per full-rank tile
 constexpr int kMaxChunk = kMaxDecodeChunk;       // positions per split (mask words in smem)
@@ -61,10 +59,15 @@ constexpr int al16(int x) { return (x + 15) & ~15; }
 constexpr int al128(int x) { return (x + 127) & ~127; }
 constexpr int imax(int a, int b) { return a > b ? a : b; }
 
-template <int G, int RK, int RV>
+// W warps per CTA and NS ring stages per warp: per shape, as many warps as
+// shared memory allows with U_v resident beside the ring.
+template <int G, int RK, int RV, int W, int NS>
 struct Shape {
   static_assert(G == 1 || G == 2 || G == 4, "1, 2 or 4 query heads per kv head");
   static_assert(RK % 16 == 0 && RV % 16 == 0 && RK <= kD && RV <= kD, "ranks");
+  static_assert(W >= 8 && NS >= 2, "at least 8 warps and 2 ring stages");
+  static constexpr int kWarps = W;
+  static constexpr int kThreads = W * 32;
   static constexpr int KP = RK / 8, VP = RV / 8;   // 16-byte pieces per row
   static constexpr int KS = 2 * RK + 16;           // padded row strides (bytes): odd multiples of 16
   static constexpr int VS = 2 * RV + 16;
@@ -74,41 +77,30 @@ struct Shape {
   static constexpr int SLOT = al128(imax(SLOT_C, SLOT_F));
   static constexpr int MASK_BYTES = (kMaxChunk / 32) * 4;          // mask words
   static constexpr int SMEM_MAX = 227 * 1024 - 1024;               // static shared memory aside
-  static constexpr int STAGES = kWarps * 3 * SLOT + MASK_BYTES <= SMEM_MAX ? 3 : 2;
-  static constexpr int RING = kWarps * STAGES * SLOT;             // [stage][warp][SLOT]
+  static constexpr int STAGES = NS;
+  static constexpr int RING = W * NS * SLOT;                      // [stage][warp][SLOT]
   static constexpr int OFF_MASK = RING;
-  // U_v rows [d][VS] for the per-split lift: resident beside the ring (loaded
-  // in the prologue) where it fits, else loaded into the tail of the ring once
-  // the stream is done
-  static constexpr int UVB = kD * VS;
-  static constexpr bool UV_RES = RING + MASK_BYTES + UVB <= SMEM_MAX;
-  static constexpr int OFF_UV = UV_RES ? RING + MASK_BYTES : ((RING - UVB) & ~127);
-  static constexpr int SMEM = UV_RES ? OFF_UV + UVB : RING + MASK_BYTES;
+  // U_v rows [d][VS], resident beside the ring (loaded in the prologue) for
+  // the per-warp lift
+  static constexpr int OFF_UV = RING + MASK_BYTES;
+  static constexpr int SMEM = OFF_UV + kD * VS;
   static_assert(SMEM <= SMEM_MAX, "shared memory of one CTA");
   // U_k rows [d][KS] live in the last stage until every warp has its q~
-  static constexpr int OFF_UK = (STAGES - 1) * kWarps * SLOT;
-  static_assert(kD * KS <= kWarps * SLOT, "U_k fits in one stage");
+  static constexpr int OFF_UK = (NS - 1) * W * SLOT;
+  static_assert(kD * KS <= W * SLOT, "U_k fits in one stage");
   // per-warp partial state in the warp's stage-0 slot (floats)
-  static constexpr int W_PC = 0;                    // [G][RV]
-  static constexpr int W_PF = W_PC + G * RV;        // [G][d]
+  static constexpr int W_PF = 0;                    // [G][d]
   static constexpr int W_M = W_PF + G * kD;         // [G]
   static constexpr int W_L = W_M + G;               // [G]
   static_assert((W_L + G) * 4 <= SLOT, "partials fit in a slot");
-  // the CTA's merged sums, in the first slot of stage 1 (floats)
-  static constexpr int OFF_MRG = kWarps * SLOT;
-  static constexpr int M_CC = 0;                    // [G][RV]
-  static constexpr int M_CF = M_CC + G * RV;        // [G][d]
-  static constexpr int MERGE_FLOATS = M_CF + G * kD;
-  static_assert(STAGES >= 2, "stage 1 holds the merged sums");
-  static_assert(OFF_MRG + MERGE_FLOATS * 4 <= (UV_RES ? RING : OFF_UV), "merged sums beside U_v");
-  static_assert(kD == 16 * kWarps, "one 16-row block of the lift per warp");
   // record of one split per query head: m, l, two pad floats, o[d] = U_v acc_c + acc_f
   static constexpr int REC = 4 + kD;
 };
 
-template <int G, int RK, int RV>
-__global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams p) {
-  using S = Shape<G, RK, RV>;
+template <int G, int RK, int RV, int W, int NS>
+__global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p) {
+  using S = Shape<G, RK, RV, W, NS>;
+  constexpr int kWarps = S::kWarps, kThreads = S::kThreads;
   constexpr int KST = RK / 16;                   // k-steps of the compressed logits
   constexpr int MVT = RV / 16;                   // m-tiles of the compressed value sum
   constexpr int KP = S::KP, VP = S::VP;
@@ -147,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     }
     cp_async_commit();
   };
-  if constexpr (S::UV_RES) load_uv();
+  load_uv();
   // q as fragments over k = d: the B operand of the full-rank logits (column
   // n = 2h holds head h; q is bf16, hence exact, so the low-part columns are 0)
   // and the A operand (rows = heads) of q~ = U_k^T q
@@ -166,8 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   // q~ = U_k^T q as this warp's B fragments over k = r_k (column n < 4 = bf16
   // high part of head n, n >= 4 = low part of head n - 4), on the tensor cores
   uint32_t qb0[KST], qb1[KST];
-  if constexpr (S::UV_RES) cp_async_wait<1>();   // U_k in (U_v may still be in flight)
-  else cp_async_wait<0>();
+  cp_async_wait<1>();   // U_k in (U_v may still be in flight)
   __syncthreads();
   uint32_t qa0[8], qa1[8];   // q as the A operand: row m = head m < G
   {
@@ -229,7 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   const lrkv_bf16* cv = p.C.coef_v + bh * D.T_cap * RV + (size_t)c0 * RV;
   const lrkv_bf16* fk = p.C.full_k + (bh * D.F_cap + f0) * kD;
   const lrkv_bf16* fv = p.C.full_v + (bh * D.F_cap + f0) * kD;
-  __syncthreads();   // mask words in; every warp is done with U_k (the last stage is free)
+  cp_async_wait<0>();   // U_v (in flight since the prologue)
+  __syncthreads();   // mask words and U_v in; every warp is done with U_k (the last stage is free)
 
   // this warp's tiles: every kWarps-th compressed tile and every kWarps-th full-rank tile
   const int n_ct = (n_pos + kTileC - 1) / kTileC;
@@ -433,39 +425,58 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   __syncwarp();
   griddep_launch_dependents();
 
+  // ---- lift: of += U_v acc_c^T on the tensor cores --------------------------------
+  // acc_c^T (rows = r_v, columns = head parts) becomes the B operand: lane
+  // (g, t) holds acc_c[head t][16 mt + g (+8)] (high + low part columns), packs
+  // it as bf16 high and low parts (columns 2t, 2t + 1 of an 8x8 tile) and one
+  // transpose gives the fragment (k = 2t, 2t + 1; n = g).  The product lands in
+  // the full-rank accumulators, whose layout is the same: o = both parts summed.
+  {
+    const unsigned char* uv = sm + S::OFF_UV;
+    uint32_t lb0[MVT], lb1[MVT];
+#pragma unroll
+    for (int mt = 0; mt < MVT; ++mt) {
+      const float x0 = oc[mt][0] + oc[mt][1], x1 = oc[mt][2] + oc[mt][3];
+      const float h0 = __uint_as_float(cvt_bf16x2(x0, x0) << 16);
+      const float h1 = __uint_as_float(cvt_bf16x2(x1, x1) << 16);
+      lb0[mt] = movmatrix_t(cvt_bf16x2(x0, x0 - h0));
+      lb1[mt] = movmatrix_t(cvt_bf16x2(x1, x1 - h1));
+    }
+#pragma unroll
+    for (int mi = 0; mi < 8; ++mi)
+#pragma unroll
+      for (int mt = 0; mt < MVT; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(a0, a1, a2, a3, uv + (16 * mi + (lm & 1) * 8 + lr) * S::VS + (mt * 16 + (lm >> 1) * 8) * 2);
+        mma_16816(of[mi], a0, a1, a2, a3, lb0[mt], lb1[mt]);
+      }
+  }
+
   // ---- this warp's partial state into its stage-0 slot -------------------------------
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) l_run += __shfl_xor_sync(kFull, l_run, o);
   {
-    float* W = reinterpret_cast<float*>(slot_of(0, warp));
+    float* Wp = reinterpret_cast<float*>(slot_of(0, warp));
     if (live_t) {
-      // lane (g, t): head t, value columns mt*16 + g and mt*16 + g + 8, high + low part
-      float* pc = W + S::W_PC + t * RV;
-      float* pf = W + S::W_PF + t * kD;
+      // lane (g, t): head t, output rows mi*16 + g and mi*16 + g + 8, high + low part
+      float* pf = Wp + S::W_PF + t * kD;
 #pragma unroll
-      for (int mt = 0; mt < MVT; ++mt) {
-        pc[mt * 16 + g] = oc[mt][0] + oc[mt][1];
-        pc[mt * 16 + g + 8] = oc[mt][2] + oc[mt][3];
-      }
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        pf[mt * 16 + g] = of[mt][0] + of[mt][1];
-        pf[mt * 16 + g + 8] = of[mt][2] + of[mt][3];
+      for (int mi = 0; mi < 8; ++mi) {
+        pf[mi * 16 + g] = of[mi][0] + of[mi][1];
+        pf[mi * 16 + g + 8] = of[mi][2] + of[mi][3];
       }
       if (g == 0) {
-        W[S::W_M + t] = m_run;
-        W[S::W_L + t] = l_run;
+        Wp[S::W_M + t] = m_run;
+        Wp[S::W_L + t] = l_run;
       }
     }
   }
   __syncthreads();
 
-  // ---- merge the warps into this split's record, lift, write it -------------------
-  if constexpr (!S::UV_RES) load_uv();           // into the tail of the ring, behind stage 0
+  // ---- merge the warps into this split's record ---------------------------------
   auto wpart = [&](int w) { return reinterpret_cast<const float*>(slot_of(0, w)); };
   __shared__ float s_we[kWarps][G];
   float* rec0 = p.partials + (bh * p.n_chunk_max + c) * G * (size_t)S::REC;
-  float* mrg = reinterpret_cast<float*>(sm + S::OFF_MRG);
   if (tid < G) {
     float M = -INFINITY;
     for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wpart(w)[S::W_M + tid]);
@@ -480,42 +491,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
     rec0[tid * S::REC + 1] = Ls;
   }
   __syncthreads();
-  for (int o = tid; o < G * (RV + kD); o += kThreads) {
-    const int gi = o / (RV + kD), j = o - gi * (RV + kD);
-    const int src = j < RV ? S::W_PC + gi * RV + j : S::W_PF + gi * kD + (j - RV);
+  for (int o = tid; o < G * kD; o += kThreads) {
+    const int gi = o / kD, i = o - gi * kD;
     float x = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[src], s_we[w][gi], x);
-    mrg[src] = x;   // same [G][RV], [G][d] layout as a warp's partials
-  }
-  cp_async_wait<0>();   // U_v
-  __syncthreads();
-  // Lift on the tensor cores: O[d][head part] = U_v [d x r_v] * acc_c^T, warp w
-  // taking rows [16w, 16w + 16).  B column n = 2h + part holds the bf16 high
-  // or low part of head h's acc_c, so a lane's accumulator fragment (columns
-  // 2t, 2t + 1) is head t again: o = high + low + acc_f.
-  {
-    const unsigned char* uv = sm + S::OFF_UV;
-    const int hb = g >> 1;                       // B column g: head g / 2
-    const bool lo_n = g & 1;
-    const float* cc = mrg + S::M_CC + (hb < G ? hb : 0) * RV;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < RV / 16; ++ks) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(a0, a1, a2, a3, uv + (16 * warp + (lm & 1) * 8 + lr) * S::VS + (ks * 16 + (lm >> 1) * 8) * 2);
-      const float2 x = *reinterpret_cast<const float2*>(cc + ks * 16 + 2 * t);
-      const float2 y = *reinterpret_cast<const float2*>(cc + ks * 16 + 8 + 2 * t);
-      const uint32_t b0 = hb < G ? pack_bf16(bf16_part(x.x, lo_n), bf16_part(x.y, lo_n)) : 0u;
-      const uint32_t b1 = hb < G ? pack_bf16(bf16_part(y.x, lo_n), bf16_part(y.y, lo_n)) : 0u;
-      mma_16816(acc, a0, a1, a2, a3, b0, b1);
-    }
-    if (live_t) {
-      const int i0 = 16 * warp + g;
-      const float* cf = mrg + S::M_CF + t * kD;
-      rec0[t * S::REC + 4 + i0] = acc[0] + acc[1] + cf[i0];
-      rec0[t * S::REC + 4 + i0 + 8] = acc[2] + acc[3] + cf[i0 + 8];
-    }
+    for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[S::W_PF + o], s_we[w][gi], x);
+    rec0[gi * S::REC + 4 + i] = x;
   }
 
   // ---- the last split of this (batch row, kv head) merges every record ------------
@@ -523,12 +504,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_stream_kernel(DecodeParams
   if (tid == 0) s_last = atom_add_acq_rel_gpu(p.tickets + bh, 1) == n_chunks - 1;
   __syncthreads();
   if (!s_last) return;
-  // Warp w serves query head w / (kWarps / G) and a block of its columns; each
+  // Warp w < 8 serves query head w / (8 / G) and a block of its columns; each
   // lane finds the head's global max and sum itself (lanes over records), then
   // accumulates its columns over the records with the weights passed by
   // shuffle.  Records come from L2 (ld.global.cg): other CTAs wrote them.
-  {
-    constexpr int WPH = kWarps / G;              // warps per head
+  if (warp < 8) {
+    constexpr int WPH = 8 / G;                   // warps per head (the first 8 warps)
     constexpr int CPW = kD / WPH;                // columns per warp: 16, 32, 64
     constexpr int CPL = CPW >= 32 ? CPW / 32 : 1;
     const int gi = warp / WPH;
