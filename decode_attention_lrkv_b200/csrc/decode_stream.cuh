@@ -36,9 +36,10 @@
 // last CTA of the (batch row, kv head) (atomic ticket, no waiting) merges the
 // records in registers, straight from L2: o = sum_c w_c o_c / sum_c w_c l_c.
 //
-// Programmatic dependent launch: U_k and q are loaded and q~ is formed before
-// waiting on the preceding kernel of the stream (an append to the same
-// cache); every read of cache state comes after the wait.
+// Programmatic dependent launch: the bases U_k and U_v are loaded before
+// waiting on the preceding kernel of the stream (they are not written by the
+// kernels around a decode); the query, produced upstream, and every piece of
+// cache state (an append to the same cache may precede) are read after it.
 #pragma once
 
 #include <type_traits>
@@ -76,7 +77,7 @@ struct Shape {
   static constexpr int SLOT_F = kTileF * 2 * FS;
   static constexpr int SLOT = al128(imax(SLOT_C, SLOT_F));
   static constexpr int MASK_BYTES = (kMaxChunk / 32) * 4;          // mask words
-  static constexpr int SMEM_MAX = 227 * 1024 - 1024;               // static shared memory aside
+  static constexpr int SMEM_MAX = 227 * 1024 - 2048;               // static shared memory aside
   static constexpr int STAGES = NS;
   static constexpr int RING = W * NS * SLOT;                      // [stage][warp][SLOT]
   static constexpr int OFF_MASK = RING;
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   auto slot_of = [&](int stage, int w) { return sm + (size_t)(stage * kWarps + w) * S::SLOT; };
   __shared__ int s_last;
 
-  // ---- prologue, independent of the preceding kernel: U_k, q and q~ ----------------
+  // ---- prologue, independent of the preceding kernel: the bases ------------------
   {  // U_k into padded rows, 16-byte pieces over every thread
     const unsigned char* Uk = reinterpret_cast<const unsigned char*>(p.C.U_k + (size_t)h * kD * RK);
     for (int q = tid; q < kD * KP; q += kThreads) {
@@ -140,6 +141,10 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     cp_async_commit();
   };
   load_uv();
+
+  // ---- after the preceding kernel of the stream: the query (produced upstream)
+  // and the cache state (an append may precede), all loaded in one batch ----------
+  griddep_wait();
   // q as fragments over k = d: the B operand of the full-rank logits (column
   // n = 2h holds head h; q is bf16, hence exact, so the low-part columns are 0)
   // and the A operand (rows = heads) of q~ = U_k^T q
@@ -154,12 +159,6 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       qf1[ks] = on ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
     }
   }
-  const float scale = kLog2e * rsqrtf((float)kD);
-  // q~ = U_k^T q as this warp's B fragments over k = r_k (column n < 4 = bf16
-  // high part of head n, n >= 4 = low part of head n - 4), on the tensor cores
-  uint32_t qb0[KST], qb1[KST];
-  cp_async_wait<1>();   // U_k in (U_v may still be in flight)
-  __syncthreads();
   uint32_t qa0[8], qa1[8];   // q as the A operand: row m = head m < G
   {
     const lrkv_bf16* qrow = p.q + ((size_t)b * D.Hq + (size_t)h * G + (g < G ? g : 0)) * kD;
@@ -169,8 +168,32 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       qa1[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
     }
   }
+  // the split's mask words (words past the sequence end are never used), the
+  // sequence length and the list length
+  constexpr int kMW = (kMaxChunk / 32 + kThreads - 1) / kThreads;   // mask words per thread
+  const int c0 = c * p.chunk;
+  uint32_t mw[kMW];
 #pragma unroll
-  for (int ks2 = 0; ks2 < KST; ++ks2) {        // columns [16 ks2, 16 ks2 + 16) of q~
+  for (int u = 0; u < kMW; ++u) {
+    const int wl = tid + u * kThreads, wi = c0 / 32 + wl;
+    mw[u] = wl < p.chunk / 32 && wi < D.T_cap / 32 ? p.C.route_mask[bh * (D.T_cap / 32) + wi] : 0u;
+  }
+  int T = p.C.seq_len[b];
+  const int F_raw = p.C.full_cnt[bh];
+#pragma unroll
+  for (int u = 0; u < kMW; ++u)
+    if (tid + u * kThreads < kMaxChunk / 32) maskw[tid + u * kThreads] = mw[u];
+
+  const float scale = kLog2e * rsqrtf((float)kD);
+  // q~ = U_k^T q as B fragments over k = r_k (column n = 2h + part: the bf16
+  // high or low part of head h), on the tensor cores: warp w < r_k / 16 forms
+  // columns [16w, 16w + 16) and leaves its fragments in shared memory for all
+  static_assert(KST <= kWarps, "one block of q~ columns per warp");
+  __shared__ uint32_t s_qb[KST][2][32];
+  cp_async_wait<1>();   // U_k in (U_v may still be in flight)
+  __syncthreads();
+  if (warp < KST) {
+    const int ks2 = warp;                      // columns [16 ks2, 16 ks2 + 16) of q~
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -186,29 +209,12 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     const float y0 = __shfl_sync(kFull, a1[0], src), y1 = __shfl_sync(kFull, a1[1], src);
     const bool lo_n = g & 1;
     const bool live = (g >> 1) < G;
-    qb0[ks2] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
-    qb1[ks2] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
+    s_qb[ks2][0][lane] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
+    s_qb[ks2][1][lane] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
   }
-
-  // ---- cache state: after the preceding kernel (an append) has completed ------------
-  griddep_wait();
-  // the split's mask words (words past the sequence end are never used), the
-  // sequence length and the list length, all loaded at once
-  constexpr int kMW = (kMaxChunk / 32 + kThreads - 1) / kThreads;   // mask words per thread
-  const int c0 = c * p.chunk;
-  uint32_t mw[kMW];
-#pragma unroll
-  for (int u = 0; u < kMW; ++u) {
-    const int wl = tid + u * kThreads, wi = c0 / 32 + wl;
-    mw[u] = wl < p.chunk / 32 && wi < D.T_cap / 32 ? p.C.route_mask[bh * (D.T_cap / 32) + wi] : 0u;
-  }
-  int T = p.C.seq_len[b];
-  const int F_raw = p.C.full_cnt[bh];
-#pragma unroll
-  for (int u = 0; u < kMW; ++u)
-    if (tid + u * kThreads < kMaxChunk / 32) maskw[tid + u * kThreads] = mw[u];
   T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
   const int n_chunks = T > 0 ? (T + p.chunk - 1) / p.chunk : 1;
+  cp_async_wait<0>();   // U_v (in flight since the prologue): none left behind on exit
   if (c >= n_chunks) return;
   const int c1 = min(T, c0 + p.chunk);
   const int n_pos = c1 > c0 ? c1 - c0 : 0;
@@ -220,8 +226,10 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   const lrkv_bf16* cv = p.C.coef_v + bh * D.T_cap * RV + (size_t)c0 * RV;
   const lrkv_bf16* fk = p.C.full_k + (bh * D.F_cap + f0) * kD;
   const lrkv_bf16* fv = p.C.full_v + (bh * D.F_cap + f0) * kD;
-  cp_async_wait<0>();   // U_v (in flight since the prologue)
-  __syncthreads();   // mask words and U_v in; every warp is done with U_k (the last stage is free)
+  __syncthreads();   // mask words, U_v and q~ in; every warp is done with U_k (the last stage is free)
+  uint32_t qb0[KST], qb1[KST];
+#pragma unroll
+  for (int ks2 = 0; ks2 < KST; ++ks2) qb0[ks2] = s_qb[ks2][0][lane], qb1[ks2] = s_qb[ks2][1][lane];
 
   // this warp's tiles: every kWarps-th compressed tile and every kWarps-th full-rank tile
   const int n_ct = (n_pos + kTileC - 1) / kTileC;

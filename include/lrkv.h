@@ -108,6 +108,13 @@ typedef struct {
    mask bit, coefficient row and list entry it covers, so stale contents past
    seq_len / full_cnt are harmless. */
 
+/* Stream ordering.  lrkv_compress's decode-time append and lrkv_decode_attn
+   launch with programmatic dependent launch: their kernels may begin on the
+   GPU while the preceding kernel of the stream is finishing.  Before waiting
+   for it they read only the bases U_k and U_v, so the kernel issued just
+   before a call must not write the bases.  Every other input (q, k_new,
+   v_new and all cache state) is read after the preceding kernel completed. */
+
 /* Bytes of device workspace that lrkv_compress and lrkv_decode_attn need for
    these sizes (0 for invalid sizes).  The workspace must be zero-filled once
    after allocation; the kernels leave it zeroed where it needs to be, so it
