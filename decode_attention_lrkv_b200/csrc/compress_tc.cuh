@@ -111,6 +111,20 @@ __device__ __forceinline__ int eff_tokens(const Params& p, int b, int* start) {
   return ne;
 }
 
+// eff_tokens of the last row asked for: a CTA's units are a contiguous range
+// of (row, tile), so the row changes rarely and its length is loaded once.
+struct RowLen {
+  int b = -1, ne = 0, start = 0;
+  __device__ __forceinline__ int get(const Params& p, int bb, int* st) {
+    if (bb != b) {
+      b = bb;
+      ne = eff_tokens(p, bb, &start);
+    }
+    *st = start;
+    return ne;
+  }
+};
+
 // Bounded wait that also gives up once another role has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag) {
@@ -244,10 +258,11 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
     // TMA producer
     if (lane == 0) {
       int i = 0;
+      RowLen rl;
       for (int u = u_begin; u < u_end && !*abort_flag; ++u) {
         const int b = u / p.tiles_per_b, t0 = (u - b * p.tiles_per_b) * kTile;
         int start;
-        if (t0 >= eff_tokens(p, b, &start)) continue;
+        if (t0 >= rl.get(p, b, &start)) continue;
         const int s = i % NS;
         if (i >= NS && !wait_or_abort(&empty[s], ((i / NS) - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
@@ -271,10 +286,11 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
       const uint32_t phb = smem_u32(sm + Lo.phi);
       const uint32_t plb = smem_u32(sm + Lo.plo);
       int i = 0;
+      RowLen rl;
       for (int u = u_begin; u < u_end && !*abort_flag; ++u) {
         const int b = u / p.tiles_per_b, t0 = (u - b * p.tiles_per_b) * kTile;
         int start;
-        if (t0 >= eff_tokens(p, b, &start)) continue;
+        if (t0 >= rl.get(p, b, &start)) continue;
         const int s = i % NS, buf = i & 1;
         if (!wait_or_abort(&full[s], (i / NS) & 1, abort_flag)) break;
         if (i >= 2 && !wait_or_abort(&tfree[buf], ((i >> 1) - 1) & 1, abort_flag)) break;
@@ -314,10 +330,11 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     float2* part = reinterpret_cast<float2*>(sm + Lo.part);   // [2][128]
     int i = 0;
+    RowLen rl;
     for (int u = u_begin; u < u_end; ++u) {
       const int b = u / p.tiles_per_b, t0 = (u - b * p.tiles_per_b) * kTile;
       int start;
-      const int ne = eff_tokens(p, b, &start);
+      const int ne = rl.get(p, b, &start);
       if (t0 >= ne) continue;
       const int s = i % NS, buf = i & 1;
       // every epilogue thread stops together, so the named barriers below
