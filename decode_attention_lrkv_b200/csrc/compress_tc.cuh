@@ -44,7 +44,7 @@ namespace lrkv {
 namespace ptc {
 
 constexpr int kTile = 128;                 // tokens per tile (MMA M)
-constexpr int kMaxStages = 3;              // input stages (2 when shared memory is short)
+constexpr int kMaxStages = 4;              // input stages (fewer when shared memory is short)
 constexpr int kThreads = 320;              // warps 0-7 epilogue, 8 TMA, 9 MMA + TMEM
 constexpr int kEpi = 256;                  // epilogue threads: two per token row
 constexpr int kTmaWarp = 8, kMmaWarp = 9;
@@ -76,7 +76,9 @@ struct Layout {
 };
 static_assert(kD * 128 * 2 <= kStageBytes, "U fits in one input stage");
 inline int stages_for(int rm) {
-  return Layout(rm, kMaxStages).bytes <= kSmemLimit ? kMaxStages : kMaxStages - 1;
+  int ns = kMaxStages;
+  while (ns > 2 && Layout(rm, ns).bytes > kSmemLimit) --ns;
+  return ns;
 }
 
 struct Params {
