@@ -11,6 +11,7 @@ Entry points (same names as the C ABI):
     lrkv_compress(dims, cache, k_new, v_new, tau, t_new_b=None, err_out=None, ws=...)
     lrkv_decode_attn(dims, cache, q, out, ws=...)
     lrkv_decode_attn_noalloc(dims, cache, q, out)   (scratch held by the library)
+    lrkv_append_decode_attn(dims, cache, k_new, v_new, tau, q, out, t_new_b=None, err_out=None, ws=...)
     lrkv_status_str(code) -> str
 plus ``LayerCache`` (allocates one layer's buffers with torch) and
 ``make_workspace``.
@@ -73,6 +74,9 @@ def load_library(path=None):
     lib.lrkv_decode_attn.restype = ctypes.c_int
     lib.lrkv_decode_attn_noalloc.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Cache), P, P, P]
     lib.lrkv_decode_attn_noalloc.restype = ctypes.c_int
+    lib.lrkv_append_decode_attn.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Cache), P, P, P,
+                                            ctypes.c_float, P, P, P, P, ctypes.c_size_t, P]
+    lib.lrkv_append_decode_attn.restype = ctypes.c_int
     lib.lrkv_status_str.argtypes = [ctypes.c_int]
     lib.lrkv_status_str.restype = ctypes.c_char_p
     if path is None:
@@ -190,4 +194,18 @@ def lrkv_decode_attn_noalloc(dims, cache, q, out, stream=None, check=True):
                                         _ptr(out), _stream_ptr(stream))
     if check and code != LRKV_OK:
         raise LrkvError(code, "lrkv_decode_attn_noalloc")
+    return code
+
+
+def lrkv_append_decode_attn(dims, cache, k_new, v_new, tau, q, out, t_new_b=None, err_out=None,
+                            ws=None, stream=None, check=True):
+    """Append one token per row (k_new/v_new [B,1,Hkv,d] bf16) and attend with q, in one launch."""
+    lib = load_library()
+    assert int(k_new.shape[1]) == 1, "one new token per row"
+    code = lib.lrkv_append_decode_attn(ctypes.byref(dims.c()), ctypes.byref(cache.c()), _ptr(k_new),
+                                       _ptr(v_new), _ptr(t_new_b), float(tau), _ptr(err_out),
+                                       _ptr(q), _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
+                                       _stream_ptr(stream))
+    if check and code != LRKV_OK:
+        raise LrkvError(code, "lrkv_append_decode_attn")
     return code

@@ -12,7 +12,8 @@ namespace lrkv {
 template <int G, int RK, int RV, int W, int NS>
 inline lrkv_status launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t s) {
   using S = ds::Shape<G, RK, RV, W, NS>;
-  auto kern = ds::decode_stream_kernel<G, RK, RV, W, NS>;
+  auto kern = p.k_new ? ds::decode_stream_kernel<G, RK, RV, W, NS, true>
+                      : ds::decode_stream_kernel<G, RK, RV, W, NS, false>;
   if (!set_smem(kern, S::SMEM)) return LRKV_ERR_CUDA;
   return launch_pdl(kern, grid, dim3(S::kThreads), S::SMEM, s, p);
 }
@@ -50,6 +51,8 @@ inline bool stream_decode_supported(const lrkv_dims& D, int chunk) {
          (rk == 64 && rv == 64) || (rk == 64 && rv == 96);
 }
 
+// p.k_new set: the fused append + decode, which only the streaming kernel has
+// (the caller checks stream_decode_supported first).
 inline lrkv_status launch_decode(const DecodeParams& p, cudaStream_t s) {
   const dim3 grid(p.n_chunk_max, p.D.Hkv, p.D.B);
   const int g = p.D.Hq / p.D.Hkv;
@@ -61,6 +64,7 @@ inline lrkv_status launch_decode(const DecodeParams& p, cudaStream_t s) {
     else st = launch_stream_g<4>(p, grid, s, &done);
     if (done) return st;
   }
+  if (p.k_new) return LRKV_ERR_UNSUPPORTED;
   switch (g) {
     case 1: return launch_simple<1>(p, grid, s);
     case 2: return launch_simple<2>(p, grid, s);

@@ -22,6 +22,13 @@ struct DecodeParams {
   float* partials;    // [B][Hkv][n_chunk_max][g][2 + r_v + d]
   int chunk;          // positions per split
   int n_chunk_max;
+  // fused decode-time append (lrkv_append_decode_attn); k_new null: plain decode
+  const lrkv_bf16* k_new;   // [B][1][Hkv][d]
+  const lrkv_bf16* v_new;   // [B][1][Hkv][d]
+  const int32_t* t_new_b;   // [B] tokens of row b (0 or 1), nullable: 1 for every row
+  float tau;
+  float* err_out;           // [B][Hkv][1], nullable
+  int32_t* seq_tickets;     // [B], zero between calls
 };
 
 constexpr int kDecThreads = 256;

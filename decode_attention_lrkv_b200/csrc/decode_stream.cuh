@@ -94,13 +94,120 @@ struct Shape {
   static constexpr int W_M = W_PF + G * kD;         // [G]
   static constexpr int W_L = W_M + G;               // [G]
   static_assert((W_L + G) * 4 <= SLOT, "partials fit in a slot");
-  // record of one split per query head: m, l, two pad floats, o[d] = U_v acc_c + acc_f
+  // record of one split per query head: m, l, flag, pad, o[d] = U_v acc_c + acc_f
+  // (flag, head 0 only: the split appended a full-rank row, fused append)
   static constexpr int REC = 4 + kD;
+  // fused append scratch in stage 0 (free until the stream starts), floats:
+  // c_k [RK], c_v [RV], q~ (scaled) [G][RK], x [2][d] (key, value), sums [16]
+  static constexpr int A_CK = 0, A_CV = RK, A_QT = RK + RV, A_X = A_QT + G * RK,
+                       A_RED = A_X + 2 * kD, A_FLOATS = A_RED + 16;
+  static_assert(A_FLOATS * 4 <= SLOT, "append scratch fits in a slot");
 };
 
-template <int G, int RK, int RV, int W, int NS>
+// The owner CTA's share of a fused decode-time append: one new token of row b,
+// kv head h, at position pos, with every thread of the CTA (the StaticPCA
+// write path and the OjaKV hybrid policy, as in the append kernel):
+//   c_k = U_k^T k is already in app[A_CK] (row 8 of the q~ product); c_v =
+//   U_v^T v on the tensor cores the same way; e = max(||k - U_k c_k|| / ||k||,
+//   ||v - U_v c_v|| / ||v||) by direct reconstruction from the unrounded c;
+//   routed iff e > tau: the rows go to list slot F when there is room (the
+//   mask bit set), else the token stays compressed (FULL_OVERFLOW).  bf16(c)
+//   is stored at pos either way.  Then the token's base-2 logit per head and
+//   its value row (v, or bf16(c_v)) for the fold after the stream.
+template <typename S, int G, int RK, int RV>
+__device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
+                                             const unsigned char* uk, const unsigned char* uv,
+                                             int b, int h, size_t bh, int pos, int F, float scale,
+                                             uint16_t xe, float* s_new, float* s_vals, int* s_keep) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3, lm = lane >> 3, lr = lane & 7;
+  const lrkv_dims& D = p.D;
+  constexpr int MVT = RV / 16;
+  app[S::A_X + tid] = bf2f(xe);   // key (threads < d), value (threads >= d)
+  __syncthreads();                // x, c_k, q~ and U_v in
+  if (warp < MVT) {               // c_v columns [16w, 16w + 16): v as row 8 of A
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* xv = app + S::A_X + kD;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t x0 = g == 0 ? pack_bf16(xv[ks * 16 + 2 * t], xv[ks * 16 + 2 * t + 1]) : 0u;
+      const uint32_t x1 = g == 0 ? pack_bf16(xv[ks * 16 + 8 + 2 * t], xv[ks * 16 + 9 + 2 * t]) : 0u;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(b0, b1, b2, b3, uv + (ks * 16 + (lm & 1) * 8 + lr) * S::VS + (16 * warp + (lm >> 1) * 8) * 2);
+      mma_16816(a0, 0u, x0, 0u, x1, b0, b1);
+      mma_16816(a1, 0u, x0, 0u, x1, b2, b3);
+    }
+    if (g == 0) {
+      app[S::A_CV + 16 * warp + 2 * t] = a0[2];
+      app[S::A_CV + 16 * warp + 2 * t + 1] = a0[3];
+      app[S::A_CV + 16 * warp + 8 + 2 * t] = a1[2];
+      app[S::A_CV + 16 * warp + 8 + 2 * t + 1] = a1[3];
+    }
+  }
+  __syncthreads();
+  {  // direct reconstruction: x_hat_i = sum_j U[i][j] c_j, residual and norm sums
+    const bool val = tid >= kD;
+    const int i = tid & (kD - 1);
+    const uint32_t* urow = reinterpret_cast<const uint32_t*>(val ? uv + i * S::VS : uk + i * S::KS);
+    const float* cc = app + (val ? S::A_CV : S::A_CK);
+    const int npair = (val ? RV : RK) / 2;
+    float h0 = 0.f, h1 = 0.f;
+    for (int j2 = 0; j2 < npair; ++j2) {
+      const uint32_t u = urow[j2];
+      h0 = fmaf(bf_lo(u), cc[2 * j2], h0);
+      h1 = fmaf(bf_hi(u), cc[2 * j2 + 1], h1);
+    }
+    const float x = app[S::A_X + tid];
+    const float dlt = x - (h0 + h1);
+    const float rs = warp_sum(dlt * dlt), ns = warp_sum(x * x);
+    if (lane == 0) app[S::A_RED + 2 * warp] = rs, app[S::A_RED + 2 * warp + 1] = ns;
+  }
+  __syncthreads();
+  const float* red = app + S::A_RED;
+  const float rk = (red[0] + red[2]) + (red[4] + red[6]), nk = (red[1] + red[3]) + (red[5] + red[7]);
+  const float rv = (red[8] + red[10]) + (red[12] + red[14]), nv = (red[9] + red[11]) + (red[13] + red[15]);
+  const float e = fmaxf(nk > 0.f ? sqrtf(rk / nk) : 0.f, nv > 0.f ? sqrtf(rv / nv) : 0.f);
+  const bool routed = e > p.tau;
+  const bool keep = routed && F < D.F_cap;
+  if (tid < RK) p.C.coef_k[(bh * D.T_cap + pos) * RK + tid] = f2bf(app[S::A_CK + tid]);
+  if (tid >= kD && tid - kD < RV)
+    p.C.coef_v[(bh * D.T_cap + pos) * RV + (tid - kD)] = f2bf(app[S::A_CV + tid - kD]);
+  if (keep) {
+    if (tid < kD) reinterpret_cast<uint16_t*>(p.C.full_k)[(bh * D.F_cap + F) * kD + tid] = xe;
+    else reinterpret_cast<uint16_t*>(p.C.full_v)[(bh * D.F_cap + F) * kD + tid - kD] = xe;
+  }
+  if (tid == 0) {
+    uint32_t* mword = p.C.route_mask + bh * (D.T_cap / 32) + (pos >> 5);
+    const uint32_t bit = 1u << (pos & 31);
+    if (keep) {
+      atomicOr(mword, bit);
+      p.C.full_idx[bh * D.F_cap + F] = pos;
+    } else {
+      atomicAnd(mword, ~bit);
+    }
+    if (routed && !keep) atomicOr(p.C.dev_status, LRKV_DEV_FULL_OVERFLOW);
+    if (p.err_out) p.err_out[bh] = e;
+    *s_keep = keep;
+  }
+  if (warp < G) {   // the token's logit for query head `warp`, base 2
+    float sd = 0.f;
+    if (keep) {     // full rank: q . k / sqrt(d)
+      const uint16_t* qrow = reinterpret_cast<const uint16_t*>(p.q) + ((size_t)b * D.Hq + (size_t)h * G + warp) * kD;
+      for (int i = lane; i < kD; i += 32) sd = fmaf(bf2f(qrow[i]), app[S::A_X + i], sd);
+      sd = warp_sum(sd) * scale;
+    } else {        // compressed: q~ . bf16(c_k), q~ already scaled
+      for (int j = lane; j < RK; j += 32) sd = fmaf(app[S::A_QT + warp * RK + j], bf2f(f2bf(app[S::A_CK + j])), sd);
+      sd = warp_sum(sd);
+    }
+    if (lane == 0) s_new[warp] = sd;
+  }
+  if (tid < kD) s_vals[tid] = keep ? app[S::A_X + kD + tid] : (tid < RV ? bf2f(f2bf(app[S::A_CV + tid])) : 0.f);
+}
+
+template <int G, int RK, int RV, int W, int NS, bool APP>
 __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p) {
   using S = Shape<G, RK, RV, W, NS>;
+  static_assert(!APP || W * 32 == 2 * kD, "the fused append maps one row element to a thread");
   constexpr int kWarps = S::kWarps, kThreads = S::kThreads;
   constexpr int KST = RK / 16;                   // k-steps of the compressed logits
   constexpr int MVT = RV / 16;                   // m-tiles of the compressed value sum
@@ -168,6 +275,27 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       qa1[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
     }
   }
+  // fused append: this (b, h)'s new key row as row 8 of the q~ product's A
+  // operand (lanes of fragment row 0), and one element of the new key or
+  // value row per thread
+  uint32_t xa0[8], xa1[8];
+  int n_b = 0;
+  uint32_t st_new = 0;
+  uint16_t xe = 0;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) xa0[ks] = xa1[ks] = 0u;
+  if constexpr (APP) {
+    n_b = new_tokens(p.t_new_b, b, 1, &st_new);
+    const lrkv_bf16* krow = p.k_new + bh * kD;   // [B][1][Hkv][d]: row (b, h)
+    if (g == 0) {
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        xa0[ks] = *reinterpret_cast<const uint32_t*>(krow + ks * 16 + 2 * t);
+        xa1[ks] = *reinterpret_cast<const uint32_t*>(krow + ks * 16 + 8 + 2 * t);
+      }
+    }
+    xe = reinterpret_cast<const uint16_t*>(tid < kD ? p.k_new : p.v_new)[bh * kD + (tid & (kD - 1))];
+  }
   // the split's mask words (words past the sequence end are never used), the
   // sequence length and the list length
   constexpr int kMW = (kMaxChunk / 32 + kThreads - 1) / kThreads;   // mask words per thread
@@ -190,6 +318,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   // columns [16w, 16w + 16) and leaves its fragments in shared memory for all
   static_assert(KST <= kWarps, "one block of q~ columns per warp");
   __shared__ uint32_t s_qb[KST][2][32];
+  float* app = reinterpret_cast<float*>(slot_of(0, 0));   // fused append scratch (stage 0)
   cp_async_wait<1>();   // U_k in (U_v may still be in flight)
   __syncthreads();
   if (warp < KST) {
@@ -199,8 +328,23 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     for (int ks = 0; ks < 8; ++ks) {
       uint32_t b0, b1, b2, b3;
       ldsm_x4_t(b0, b1, b2, b3, uk + (ks * 16 + (lm & 1) * 8 + lr) * S::KS + (16 * ks2 + (lm >> 1) * 8) * 2);
-      mma_16816(a0, qa0[ks], 0u, qa1[ks], 0u, b0, b1);
-      mma_16816(a1, qa0[ks], 0u, qa1[ks], 0u, b2, b3);
+      mma_16816(a0, qa0[ks], xa0[ks], qa1[ks], xa1[ks], b0, b1);
+      mma_16816(a1, qa0[ks], xa0[ks], qa1[ks], xa1[ks], b2, b3);
+    }
+    if constexpr (APP) {
+      if (g == 0) {   // row 8: the new key's coefficients c_k = U_k^T k (fp32, unrounded)
+        app[S::A_CK + 16 * ks2 + 2 * t] = a0[2];
+        app[S::A_CK + 16 * ks2 + 2 * t + 1] = a0[3];
+        app[S::A_CK + 16 * ks2 + 8 + 2 * t] = a1[2];
+        app[S::A_CK + 16 * ks2 + 8 + 2 * t + 1] = a1[3];
+      }
+      if (g < G) {    // q~ rows (scaled), for the new token's logit if it stays compressed
+        float* qt = app + S::A_QT + g * RK + 16 * ks2;
+        qt[2 * t] = a0[0] * scale;
+        qt[2 * t + 1] = a0[1] * scale;
+        qt[8 + 2 * t] = a1[0] * scale;
+        qt[8 + 2 * t + 1] = a1[1] * scale;
+      }
     }
     // lane (m, t) holds q~[head m][16 ks2 + 2t (+1)] in a0 and [+8] in a1 (rows m < 4).
     // B column g = 2h + part takes head h from lane 4h + t.
@@ -213,10 +357,31 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     s_qb[ks2][1][lane] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
   }
   T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
+  // fused append: the new token (if the row has one and there is room) takes
+  // position T_old; the split holding it (the last one) is its owner
+  int n_eff = 0;
+  if constexpr (APP) {
+    n_eff = n_b > 0 && T < D.T_cap ? 1 : 0;
+    if (n_b > 0 && T >= D.T_cap) st_new |= LRKV_DEV_SEQ_OVERFLOW;
+  }
+  const int T_old = T;
+  T += n_eff;
   const int n_chunks = T > 0 ? (T + p.chunk - 1) / p.chunk : 1;
+  const bool owner = APP && n_eff > 0 && c == n_chunks - 1;
+  if constexpr (APP) {
+    // every thread of this CTA has read seq_len[b] (the barrier above); the
+    // last CTA of the grid to get here advances every row's length
+    if (tid == 0) {
+      if (atom_add_acq_rel_gpu(p.seq_tickets + b, 1) == D.Hkv * (int)gridDim.x - 1) {
+        p.C.seq_len[b] = T;
+        p.seq_tickets[b] = 0;
+      }
+      if (h == 0 && c == 0 && st_new) atomicOr(p.C.dev_status, st_new);
+    }
+  }
   cp_async_wait<0>();   // U_v (in flight since the prologue): none left behind on exit
   if (c >= n_chunks) return;
-  const int c1 = min(T, c0 + p.chunk);
+  const int c1 = min(T_old, c0 + p.chunk);   // the new position is not read from the cache
   const int n_pos = c1 > c0 ? c1 - c0 : 0;
   const int F = min(max(F_raw, 0), D.F_cap);
   const int share = (F + n_chunks - 1) / n_chunks;
@@ -226,6 +391,14 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   const lrkv_bf16* cv = p.C.coef_v + bh * D.T_cap * RV + (size_t)c0 * RV;
   const lrkv_bf16* fk = p.C.full_k + (bh * D.F_cap + f0) * kD;
   const lrkv_bf16* fv = p.C.full_v + (bh * D.F_cap + f0) * kD;
+  // the new token for the fold after the stream: its logit per head, whether
+  // it went to the full-rank list, and its value row (v, or c_v as stored)
+  __shared__ float s_new[G];
+  __shared__ float s_vals[kD];
+  __shared__ int s_keep;
+  if constexpr (APP) {
+    if (owner) append_token<S, G, RK, RV>(p, app, uk, sm + S::OFF_UV, b, h, bh, T_old, F, scale, xe, s_new, s_vals, &s_keep);
+  }
   __syncthreads();   // mask words, U_v and q~ in; every warp is done with U_k (the last stage is free)
   uint32_t qb0[KST], qb1[KST];
 #pragma unroll
@@ -433,6 +606,35 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   __syncwarp();
   griddep_launch_dependents();
 
+  // ---- fused append: fold the new token into warp 0's state ---------------------
+  if (owner && warp == 0 && live_t) {
+    const float sv = s_new[t];
+    if (sv > m_run) {
+      const float sc = m_run == -INFINITY ? 0.f : exp2f(m_run - sv);
+      l_run *= sc;
+#pragma unroll
+      for (int mt = 0; mt < MVT; ++mt) oc[mt][0] *= sc, oc[mt][1] *= sc, oc[mt][2] *= sc, oc[mt][3] *= sc;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) of[mt][0] *= sc, of[mt][1] *= sc, of[mt][2] *= sc, of[mt][3] *= sc;
+      m_run = sv;
+    }
+    const float pn = exp2f(sv - m_run);
+    if (g == 0) l_run += pn;
+    if (s_keep) {
+#pragma unroll
+      for (int mi = 0; mi < 8; ++mi) {
+        of[mi][0] = fmaf(pn, s_vals[16 * mi + g], of[mi][0]);
+        of[mi][2] = fmaf(pn, s_vals[16 * mi + g + 8], of[mi][2]);
+      }
+    } else {
+#pragma unroll
+      for (int mt = 0; mt < MVT; ++mt) {
+        oc[mt][0] = fmaf(pn, s_vals[16 * mt + g], oc[mt][0]);
+        oc[mt][2] = fmaf(pn, s_vals[16 * mt + g + 8], oc[mt][2]);
+      }
+    }
+  }
+
   // ---- lift: of += U_v acc_c^T on the tensor cores --------------------------------
   // acc_c^T (rows = r_v, columns = head parts) becomes the B operand: lane
   // (g, t) holds acc_c[head t][16 mt + g (+8)] (high + low part columns), packs
@@ -497,6 +699,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     }
     rec0[tid * S::REC] = M;
     rec0[tid * S::REC + 1] = Ls;
+    if (APP && tid == 0) rec0[2] = owner && s_keep ? 1.f : 0.f;
   }
   __syncthreads();
   for (int o = tid; o < G * kD; o += kThreads) {
@@ -572,7 +775,13 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       for (int u = 0; u < CPL; ++u) out[u] = Lsum > 0.f ? acc[u] / Lsum : 0.f;
     }
   }
-  if (tid == 0) p.tickets[bh] = 0;
+  if (tid == 0) {
+    p.tickets[bh] = 0;
+    // fused append: every CTA of this (b, kv head) has read the list length;
+    // the new full-rank row (if the owner appended one) now counts
+    if (APP && __ldcg(p.partials + (bh * p.n_chunk_max + n_chunks - 1) * G * (size_t)S::REC + 2) != 0.f)
+      p.C.full_cnt[bh] = F + 1;
+  }
 }
 
 }  // namespace ds

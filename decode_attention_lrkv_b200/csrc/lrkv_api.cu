@@ -98,7 +98,7 @@ bool rows_map(CUtensorMap* map, const lrkv_bf16* base, const lrkv_dims& D, int t
 lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16* k_new,
                         const lrkv_bf16* v_new, int t_new, const int32_t* t_new_b, float tau,
                         float* err_out, char* w, const WsLayout& L, cudaStream_t s) {
-  ptc::Params pp;
+  ptc::Params pp = {};
   if (!rows_map(&pp.map_k, k_new, D, t_new) || !rows_map(&pp.map_v, v_new, D, t_new))
     return LRKV_ERR_CUDA;
   const int tmax = t_new < D.T_cap ? t_new : D.T_cap;
@@ -122,7 +122,7 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
   ptc::project_tc_kernel<<<dim3(per_group, groups), ptc::kThreads, smem, s>>>(pp);
   lrkv_status st = launched();
   if (st != LRKV_OK) return st;
-  ptc::RouteParams rp;
+  ptc::RouteParams rp = {};
   rp.D = D;
   rp.C = C;
   rp.k_new = k_new;
@@ -168,7 +168,7 @@ lrkv_status lrkv_compress(const lrkv_dims* dims, const lrkv_cache* cache,
   if (t_new == 0) return LRKV_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
-  CompressParams p;
+  CompressParams p = {};
   p.D = *dims;
   p.C = *cache;
   p.k_new = k_new;
@@ -197,7 +197,7 @@ lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache, con
   if ((st = check_ws(dims, ws, ws_bytes, &L)) != LRKV_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* w = static_cast<char*>(ws);
-  DecodeParams p;
+  DecodeParams p = {};
   p.D = *dims;
   p.C = *cache;
   p.q = q;
@@ -206,6 +206,45 @@ lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache, con
   p.partials = reinterpret_cast<float*>(w + L.partials);
   p.chunk = L.chunk;
   p.n_chunk_max = L.n_chunk_max;
+  return launch_decode(p, s);
+}
+
+lrkv_status lrkv_append_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache,
+                                    const lrkv_bf16* k_new, const lrkv_bf16* v_new,
+                                    const int32_t* t_new_b, float tau, float* err_out,
+                                    const lrkv_bf16* q, float* out, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  lrkv_status st = check_dims(dims);
+  if (st != LRKV_OK) return st;
+  if ((st = check_cache(dims, cache)) != LRKV_OK) return st;
+  if (!k_new || !v_new || !q || !out) return LRKV_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(t_new_b) || !aligned16(err_out) ||
+      !aligned16(q) || !aligned16(out))
+    return LRKV_ERR_ALIGNMENT;
+  WsLayout L;
+  if ((st = check_ws(dims, ws, ws_bytes, &L)) != LRKV_OK) return st;
+  if (!stream_decode_supported(*dims, L.chunk)) {   // the two launches it fuses
+    st = lrkv_compress(dims, cache, k_new, v_new, 1, t_new_b, tau, err_out, ws, ws_bytes, stream);
+    if (st != LRKV_OK) return st;
+    return lrkv_decode_attn(dims, cache, q, out, ws, ws_bytes, stream);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  DecodeParams p = {};
+  p.D = *dims;
+  p.C = *cache;
+  p.q = q;
+  p.out = out;
+  p.tickets = reinterpret_cast<int32_t*>(w + L.decode_tickets);
+  p.partials = reinterpret_cast<float*>(w + L.partials);
+  p.chunk = L.chunk;
+  p.n_chunk_max = L.n_chunk_max;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.t_new_b = t_new_b;
+  p.tau = tau;
+  p.err_out = err_out;
+  p.seq_tickets = reinterpret_cast<int32_t*>(w + L.seq_tickets);
   return launch_decode(p, s);
 }
 

@@ -53,6 +53,7 @@ __device__ __forceinline__ int new_tokens(const int32_t* t_new_b, int b, int t_n
 struct WsLayout {
   size_t decode_tickets;   // int32 [B][Hkv], zero between calls
   size_t compress_ticket;  // int32 [1], zero between calls
+  size_t seq_tickets;      // int32 [B], zero between calls (fused append + decode)
   size_t errs;             // float [2][B][Hkv][T_cap] e_k, e_v of a prefill compress call
   size_t tile_cnt;         // int32 [B][Hkv][n_tiles] routed tokens per 128-token tile
   size_t tile_bits;        // uint32 [B][Hkv][n_tiles][4] routed bits per tile
@@ -96,6 +97,8 @@ inline WsLayout ws_layout(const lrkv_dims& D) {
   off = align_up(off + sizeof(int32_t) * (size_t)D.B * D.Hkv, 256);
   L.compress_ticket = off;
   off = align_up(off + sizeof(int32_t), 256);
+  L.seq_tickets = off;
+  off = align_up(off + sizeof(int32_t) * (size_t)D.B, 256);
   L.n_tiles = (D.T_cap + 127) / 128;
   L.errs = off;
   off = align_up(off + sizeof(float) * 2 * (size_t)D.B * D.Hkv * D.T_cap, 256);

@@ -97,7 +97,7 @@ extern "C" LRKV_API lrkv_status lrkv_decode_attn_noalloc(const lrkv_dims* dims,
     cudaGetLastError();
     return LRKV_ERR_CUDA;
   }
-  DecodeParams p;
+  DecodeParams p = {};
   p.D = *dims;
   p.C = *cache;
   p.q = q;

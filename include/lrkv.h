@@ -154,6 +154,24 @@ LRKV_API lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* c
                                       const lrkv_bf16* q, float* out, void* ws,
                                       size_t ws_bytes, void* stream);
 
+/* One decode step with its append, in one launch: the same result as
+ *   lrkv_compress(dims, cache, k_new, v_new, 1, t_new_b, tau, err_out, ...)
+ *   lrkv_decode_attn(dims, cache, q, out, ...)
+ * issued back to back on `stream` (append-then-attend: the new token is
+ * attended).  k_new, v_new: [B][1][Hkv][d] bf16; t_new_b: nullable device [B]
+ * int32, each 0 or 1 (a row with 0 only attends); err_out: nullable device
+ * [B][Hkv][1] fp32.  The append is done inside the decode kernel by the CTA
+ * that holds the new position; the list length and seq_len are advanced on
+ * the device once every CTA has read them.  Shapes the streaming decode kernel
+ * does not cover run the two calls above instead (two launches).
+ * Arguments, layouts and errors otherwise as lrkv_compress / lrkv_decode_attn.
+ */
+LRKV_API lrkv_status lrkv_append_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache,
+                                             const lrkv_bf16* k_new, const lrkv_bf16* v_new,
+                                             const int32_t* t_new_b, float tau, float* err_out,
+                                             const lrkv_bf16* q, float* out, void* ws,
+                                             size_t ws_bytes, void* stream);
+
 /* Device scratch built into the library for lrkv_decode_attn_noalloc, bytes. */
 #define LRKV_NOALLOC_SCRATCH_BYTES (4u << 20)
 
