@@ -97,11 +97,13 @@ struct Shape {
   // record of one split per query head: m, l, flag, pad, o[d] = U_v acc_c + acc_f
   // (flag, head 0 only: the split appended a full-rank row, fused append)
   static constexpr int REC = 4 + kD;
-  // fused append scratch in stage 0 (free until the stream starts), floats:
-  // c_k [RK], c_v [RV], q~ (scaled) [G][RK], x [2][d] (key, value), sums [16]
+  // fused append scratch behind U_k in the last stage (untouched until the
+  // stream's first refill), floats: c_k [RK], c_v [RV], q~ (scaled) [G][RK],
+  // x [2][d] (key, value), sums [16]
+  static constexpr int OFF_APP = OFF_UK + al16(kD * KS);
   static constexpr int A_CK = 0, A_CV = RK, A_QT = RK + RV, A_X = A_QT + G * RK,
                        A_RED = A_X + 2 * kD, A_FLOATS = A_RED + 16;
-  static_assert(A_FLOATS * 4 <= SLOT, "append scratch fits in a slot");
+  static_assert(al16(kD * KS) + A_FLOATS * 4 <= W * SLOT, "U_k and the append scratch fit in a stage");
 };
 
 // The owner CTA's share of a fused decode-time append: one new token of row b,
@@ -318,7 +320,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   // columns [16w, 16w + 16) and leaves its fragments in shared memory for all
   static_assert(KST <= kWarps, "one block of q~ columns per warp");
   __shared__ uint32_t s_qb[KST][2][32];
-  float* app = reinterpret_cast<float*>(slot_of(0, 0));   // fused append scratch (stage 0)
+  float* app = reinterpret_cast<float*>(sm + S::OFF_APP);   // fused append scratch
   cp_async_wait<1>();   // U_k in (U_v may still be in flight)
   __syncthreads();
   if (warp < KST) {
@@ -396,9 +398,6 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   __shared__ float s_new[G];
   __shared__ float s_vals[kD];
   __shared__ int s_keep;
-  if constexpr (APP) {
-    if (owner) append_token<S, G, RK, RV>(p, app, uk, sm + S::OFF_UV, b, h, bh, T_old, F, scale, xe, s_new, s_vals, &s_keep);
-  }
   __syncthreads();   // mask words, U_v and q~ in; every warp is done with U_k (the last stage is free)
   uint32_t qb0[KST], qb1[KST];
 #pragma unroll
@@ -480,6 +479,16 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   for (int s = 0; s < NST - 1; ++s) {
     if (s < n_tiles) issue(s);
     cp_async_commit();
+  }
+  // the owner of a fused append does it while its first tiles are in flight
+  // (U_k and the scratch sit in the last stage, which the stream refills only
+  // from its first step on)
+  if constexpr (APP) {
+    if (owner) {
+      append_token<S, G, RK, RV>(p, app, uk, sm + S::OFF_UV, b, h, bh, T_old, F, scale, xe, s_new,
+                                 s_vals, &s_keep);
+      __syncthreads();   // the token's logits and value row in for warp 0
+    }
   }
 
   // ---- stream the tiles ------------------------------------------------------------
