@@ -370,19 +370,28 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   T += n_eff;
   const int n_chunks = T > 0 ? (T + p.chunk - 1) / p.chunk : 1;
   const bool owner = APP && n_eff > 0 && c == n_chunks - 1;
+  // Every thread of this CTA has read seq_len[b] (the barrier above): take the
+  // row's ticket now (release only, so nothing waits for it here) and look at
+  // it at the end; the last CTA of the grid for row b advances its length.
+  int seq_ticket = 0;
+  auto advance_len = [&]() {
+    if (seq_ticket == D.Hkv * (int)gridDim.x - 1) {
+      fence_acq_rel_gpu();
+      p.C.seq_len[b] = T;
+      p.seq_tickets[b] = 0;
+    }
+  };
   if constexpr (APP) {
-    // every thread of this CTA has read seq_len[b] (the barrier above); the
-    // last CTA of the grid to get here advances every row's length
     if (tid == 0) {
-      if (atom_add_acq_rel_gpu(p.seq_tickets + b, 1) == D.Hkv * (int)gridDim.x - 1) {
-        p.C.seq_len[b] = T;
-        p.seq_tickets[b] = 0;
-      }
+      seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
       if (h == 0 && c == 0 && st_new) atomicOr(p.C.dev_status, st_new);
     }
   }
   cp_async_wait<0>();   // U_v (in flight since the prologue): none left behind on exit
-  if (c >= n_chunks) return;
+  if (c >= n_chunks) {
+    if (APP && tid == 0) advance_len();
+    return;
+  }
   const int c1 = min(T_old, c0 + p.chunk);   // the new position is not read from the cache
   const int n_pos = c1 > c0 ? c1 - c0 : 0;
   const int F = min(max(F_raw, 0), D.F_cap);
@@ -612,6 +621,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     __syncwarp();
   }
   cp_async_wait<0>();
+  if (APP && tid == 0) advance_len();
   __syncwarp();
   griddep_launch_dependents();
 

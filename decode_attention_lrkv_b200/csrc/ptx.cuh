@@ -157,6 +157,17 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* addr, int v) {
   return old;
 }
 
+// Release-only add: later operations of the thread need not wait for it; a
+// thread that acts on the returned count issues fence_acq_rel_gpu() first.
+__device__ __forceinline__ int atom_add_release_gpu(int* addr, int v) {
+  int old;
+  asm volatile("atom.add.release.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 // Two floats -> bf16x2 (round to nearest even), the first in the low half.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
