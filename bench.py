@@ -4,19 +4,21 @@
                     [--workload 1] [--no-cpu-baseline]
 
 A step is one decode step of the whole model: for each of the workload's
-layers, append the step's new token through lrkv_compress (projection,
-error, routing) and then run lrkv_decode_attn over the layer's compressed
-cache (append-then-attend).  Caches are built first by a prefill
-lrkv_compress per layer, which is timed on its own (compress tokens/s).
+layers, append the step's new token (projection, error, routing) and attend
+over the layer's compressed cache with it included (append-then-attend), in
+one lrkv_append_decode_attn call.  The same step as two calls
+(lrkv_compress, then lrkv_decode_attn) is timed too and reported beside it.
+Caches are built first by a prefill lrkv_compress per layer, which is timed
+on its own (compress tokens/s).
 
 Printed JSON line (rank 0):
   value   = decode-step algorithmic HBM bytes (all ranks) / max-over-ranks time, GB/s
   e2e     = the same through host buffers: pinned-host -> device copy of
             the step's inputs and device -> host copy of its outputs inside
             the timed region
-  roofline: the decode kernel, algorithmic bytes per launch / its mean
-            duration from CUDA events around each launch, vs the measured
-            copy bandwidth
+  roofline: the decode kernel (with the fused append), algorithmic bytes per
+            launch / its mean duration from CUDA events around each launch,
+            vs the measured copy bandwidth
   cpu_baseline: the fp64 CPU oracle on a bounded sample of the same work.
 
 Multi-GPU (torchrun): every rank runs its own independent sequences (weak
@@ -44,8 +46,7 @@ from decode_attention_lrkv_b200 import accounting as A  # noqa: E402
 
 HBM_SPEC_GBS = 8000.0
 FALLBACK_PEAK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-COMPRESS_LAUNCHES = 1     # kernels one decode-time (one-token) lrkv_compress call launches
-DECODE_LAUNCHES = 1       # kernels one lrkv_decode_attn call launches
+FUSED_LAUNCHES = 1        # kernels one lrkv_append_decode_attn call launches
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -253,11 +254,12 @@ def build_layers(L, w, seed, steps_total, dev):
     return dims, ws, layers, comp_ms, lengths
 
 
-def capture_step_graph(L, dims, ws, layers, w, s, out, dec_events, host=None):
+def capture_step_graph(L, dims, ws, layers, w, s, out, dec_events, host=None, fused=True):
     """One CUDA graph: every layer's append + decode for step s.
 
-    host: optional (pinned inputs, pinned outputs, device staging) for the
-    end-to-end variant with copies in the graph.
+    fused: one lrkv_append_decode_attn call per layer, else lrkv_compress then
+    lrkv_decode_attn.  host: optional (pinned inputs, pinned outputs, device
+    staging) for the end-to-end variant with copies in the graph.
     """
     g = torch.cuda.CUDAGraph()
     stream = torch.cuda.Stream()
@@ -275,10 +277,15 @@ def capture_step_graph(L, dims, ws, layers, w, s, out, dec_events, host=None):
                     k = lay["K_app"][:, s:s + 1]
                     v = lay["V_app"][:, s:s + 1]
                     q = lay["q_app"][s]
-                L.lrkv_compress(dims, lay["cache"], k, v, w.tau, ws=ws, stream=stream)
+                if not fused:
+                    L.lrkv_compress(dims, lay["cache"], k, v, w.tau, ws=ws, stream=stream)
                 if dec_events is not None:
                     dec_events[li][0].record(stream)
-                L.lrkv_decode_attn(dims, lay["cache"], q, out[li], ws=ws, stream=stream)
+                if fused:
+                    L.lrkv_append_decode_attn(dims, lay["cache"], k, v, w.tau, q, out[li], ws=ws,
+                                              stream=stream)
+                else:
+                    L.lrkv_decode_attn(dims, lay["cache"], q, out[li], ws=ws, stream=stream)
                 if dec_events is not None:
                     dec_events[li][1].record(stream)
             if host is not None:   # the step's result for every layer: one copy back
@@ -294,7 +301,7 @@ def run_ours(args, rank, world, dev):
     K, W = args.steps, args.warmup
     steps_total = W + K
     seed = rank_seed(args.seed, rank)
-    dims, ws, layers, comp_ms, lengths = build_layers(L, w, seed, 3 * steps_total, dev)
+    dims, ws, layers, comp_ms, lengths = build_layers(L, w, seed, 4 * steps_total, dev)
     out = torch.empty(w.layers, w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
 
     # --- device-resident timed region: the step graphs carry no events (an event
@@ -348,6 +355,24 @@ def run_ours(args, rank, world, dev):
         g.reset()
     del graphs
 
+    # --- the same step as two calls per layer (lrkv_compress, lrkv_decode_attn) ---------
+    graphs = [capture_step_graph(L, dims, ws, layers, w, s, out, None, fused=False)
+              for s in range(steps_total)]
+    torch.cuda.synchronize()
+    for s in range(W):
+        graphs[s].replay()
+    torch.cuda.synchronize()
+    u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    u0.record()
+    for s in range(W, steps_total):
+        graphs[s].replay()
+    u1.record()
+    torch.cuda.synchronize()
+    unfused_ms = max_over_ranks(u0.elapsed_time(u1), dev, world) / K
+    for g in graphs:
+        g.reset()
+    del graphs
+
     # --- the decode kernel back to back: one graph of every layer's decode, K times
     # (no appends: the caches stay as they are), so consecutive decodes overlap as
     # they do behind an append -------------------------------------------------------
@@ -388,7 +413,7 @@ def run_ours(args, rank, world, dev):
     dec_launch_ms = float(np.mean(dec_ms))
     T_mid_k = [int(x) + (K + 1) / 2.0 for x in seq_k]
     dec_bytes_launch = float(np.mean([A.decode_bytes(w.B, w.Hq, w.Hkv, w.d, w.r_k, w.r_v, T_mid_k, fc)
-                                      for fc in full_cnt_k]))
+                                      for fc in full_cnt_k])) + app_bytes   # the fused append's too
     pk, pk_kind = peaks()
     achieved = dec_bytes_launch / (dec_launch_ms * 1e-3) / 1e9
     dec_bytes_chain = float(np.mean([A.decode_bytes(w.B, w.Hq, w.Hkv, w.d, w.r_k, w.r_v,
@@ -413,7 +438,7 @@ def run_ours(args, rank, world, dev):
                    "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d, "r_k": w.r_k, "r_v": w.r_v,
                    "tau": w.tau, "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB touched per step vs 126 MB L2",
-                   "graph": "one CUDA graph per step (all layers: append + decode)"},
+                   "graph": "one CUDA graph per step (all layers: fused append + decode)"},
         "us_per_step": round(ms_step * 1e3, 2),
         "frac_of_8TBs": round(value / world / HBM_SPEC_GBS, 4),
         "routed_fraction": round(routed_frac, 4),
@@ -426,13 +451,16 @@ def run_ours(args, rank, world, dev):
                      "tensor_frac_of_measured_bf16": round(comp_tflops / pk.get("bf16_tflops",
                                                                                 FALLBACK_PEAK["bf16_tflops"]), 4),
                      "tokens_per_layer": n_tok},
-        "roofline": {"kernel": "decode_attn", "bound": "hbm", "achieved": round(achieved, 2),
+        "unfused_step": {"us_per_step": round(unfused_ms * 1e3, 2),
+                         "value": round(sum_over_ranks(step_bytes, dev, world) / (unfused_ms * 1e-3) / 1e9, 2),
+                         "calls": "lrkv_compress then lrkv_decode_attn per layer (two launches)"},
+        "roofline": {"kernel": "decode_attn (fused append)", "bound": "hbm", "achieved": round(achieved, 2),
                      "peak": pk.get("hbm_gbs", FALLBACK_PEAK["hbm_gbs"]),
                      "peak_kind": pk_kind + " copy bandwidth", "unit": "GB/s",
                      "frac": round(achieved / pk.get("hbm_gbs", FALLBACK_PEAK["hbm_gbs"]), 4),
                      "traffic": stored_traffic("decode_attn", w.name),
                      "algorithmic_bytes_per_launch": round(dec_bytes_launch),
-                     "launch_timing": "CUDA events on the launching stream around every decode, "
+                     "launch_timing": "CUDA events on the launching stream around every fused call, "
                                       "in a second pass of the same steps (events are kept out of "
                                       "the timed step graphs)",
                      "mean_launch_us": round(dec_launch_ms * 1e3, 3),
@@ -442,7 +470,7 @@ def run_ours(args, rank, world, dev):
                                  "timing": "one CUDA graph of every layer's decode, K times back "
                                            "to back (no appends), CUDA events around the replay"}},
         "e2e": e2e,
-        "gpu_launches": K * w.layers * (COMPRESS_LAUNCHES + DECODE_LAUNCHES),
+        "gpu_launches": K * w.layers * FUSED_LAUNCHES,
         "clocks": clk,
     }
     return result, w, layers, dims

@@ -102,15 +102,15 @@ struct Shape {
   // x [2][d] (key, value), sums [16]
   static constexpr int OFF_APP = OFF_UK + al16(kD * KS);
   static constexpr int A_CK = 0, A_CV = RK, A_QT = RK + RV, A_X = A_QT + G * RK,
-                       A_RED = A_X + 2 * kD, A_FLOATS = A_RED + 16;
+                       A_RED = A_X + 2 * kD, A_FLOATS = A_RED + 24;
   static_assert(al16(kD * KS) + A_FLOATS * 4 <= W * SLOT, "U_k and the append scratch fit in a stage");
 };
 
 // The owner CTA's share of a fused decode-time append: one new token of row b,
 // kv head h, at position pos, with every thread of the CTA (the StaticPCA
 // write path and the OjaKV hybrid policy, as in the append kernel):
-//   c_k = U_k^T k is already in app[A_CK] (row 8 of the q~ product); c_v =
-//   U_v^T v on the tensor cores the same way; e = max(||k - U_k c_k|| / ||k||,
+//   c_k = U_k^T k and c_v = U_v^T v on the tensor cores (x as an A row,
+//   exact in bf16, fp32 accumulation); e = max(||k - U_k c_k|| / ||k||,
 //   ||v - U_v c_v|| / ||v||) by direct reconstruction from the unrounded c;
 //   routed iff e > tau: the rows go to list slot F when there is room (the
 //   mask bit set), else the token stays compressed (FULL_OVERFLOW).  bf16(c)
@@ -124,50 +124,73 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3, lm = lane >> 3, lr = lane & 7;
   const lrkv_dims& D = p.D;
-  constexpr int MVT = RV / 16;
-  app[S::A_X + tid] = bf2f(xe);   // key (threads < d), value (threads >= d)
-  __syncthreads();                // x, c_k, q~ and U_v in
-  if (warp < MVT) {               // c_v columns [16w, 16w + 16): v as row 8 of A
+  constexpr int KST = RK / 16, MVT = RV / 16;
+  app[S::A_X + tid] = bf2f(xe);   // new key (threads < d) and value (threads >= d) rows
+  __syncthreads();                // x and q~ in; U_k and U_v in since the prologue
+  // c = U^T x on the tensor cores, x as row 8 of the A operand: warp w forms
+  // columns [16w, 16w + 16) of c_k (w < r_k / 16) and of c_v (w < r_v / 16)
+  auto coef_block = [&](const unsigned char* U, int stride, const float* x, float* cdst) {
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-    const float* xv = app + S::A_X + kD;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t x0 = g == 0 ? pack_bf16(xv[ks * 16 + 2 * t], xv[ks * 16 + 2 * t + 1]) : 0u;
-      const uint32_t x1 = g == 0 ? pack_bf16(xv[ks * 16 + 8 + 2 * t], xv[ks * 16 + 9 + 2 * t]) : 0u;
+      const uint32_t x0 = g == 0 ? pack_bf16(x[ks * 16 + 2 * t], x[ks * 16 + 2 * t + 1]) : 0u;
+      const uint32_t x1 = g == 0 ? pack_bf16(x[ks * 16 + 8 + 2 * t], x[ks * 16 + 9 + 2 * t]) : 0u;
       uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(b0, b1, b2, b3, uv + (ks * 16 + (lm & 1) * 8 + lr) * S::VS + (16 * warp + (lm >> 1) * 8) * 2);
+      ldsm_x4_t(b0, b1, b2, b3, U + (ks * 16 + (lm & 1) * 8 + lr) * stride + (16 * warp + (lm >> 1) * 8) * 2);
       mma_16816(a0, 0u, x0, 0u, x1, b0, b1);
       mma_16816(a1, 0u, x0, 0u, x1, b2, b3);
     }
     if (g == 0) {
-      app[S::A_CV + 16 * warp + 2 * t] = a0[2];
-      app[S::A_CV + 16 * warp + 2 * t + 1] = a0[3];
-      app[S::A_CV + 16 * warp + 8 + 2 * t] = a1[2];
-      app[S::A_CV + 16 * warp + 8 + 2 * t + 1] = a1[3];
+      cdst[16 * warp + 2 * t] = a0[2];
+      cdst[16 * warp + 2 * t + 1] = a0[3];
+      cdst[16 * warp + 8 + 2 * t] = a1[2];
+      cdst[16 * warp + 8 + 2 * t + 1] = a1[3];
     }
-  }
+  };
+  if (warp < KST) coef_block(uk, S::KS, app + S::A_X, app + S::A_CK);
+  if (warp < MVT) coef_block(uv, S::VS, app + S::A_X + kD, app + S::A_CV);
   __syncthreads();
-  {  // direct reconstruction: x_hat_i = sum_j U[i][j] c_j, residual and norm sums
-    const bool val = tid >= kD;
-    const int i = tid & (kD - 1);
-    const uint32_t* urow = reinterpret_cast<const uint32_t*>(val ? uv + i * S::VS : uk + i * S::KS);
-    const float* cc = app + (val ? S::A_CV : S::A_CK);
-    const int npair = (val ? RV : RK) / 2;
-    float h0 = 0.f, h1 = 0.f;
-    for (int j2 = 0; j2 < npair; ++j2) {
-      const uint32_t u = urow[j2];
-      h0 = fmaf(bf_lo(u), cc[2 * j2], h0);
-      h1 = fmaf(bf_hi(u), cc[2 * j2 + 1], h1);
+  // direct reconstruction x_hat = U c on the tensor cores: A = U's rows
+  // [16w, 16w + 16) (warp w, keys then values), B = c split into bf16 high
+  // (column 0) and low (column 1) parts; lane (g, t = 0) gets x_hat of rows
+  // 16w + g and 16w + g + 8 as the sum of its two columns
+  auto recon_sq = [&](const unsigned char* U, int stride, int r, const float* cc, const float* x) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int ks = 0; ks < r / 16; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(a0, a1, a2, a3, U + (16 * warp + (lm & 1) * 8 + lr) * stride + (ks * 16 + (lm >> 1) * 8) * 2);
+      const bool lo = g & 1;
+      const float* c2 = cc + ks * 16 + 2 * t;
+      const uint32_t b0 = g < 2 ? pack_bf16(bf16_part(c2[0], lo), bf16_part(c2[1], lo)) : 0u;
+      const uint32_t b1 = g < 2 ? pack_bf16(bf16_part(c2[8], lo), bf16_part(c2[9], lo)) : 0u;
+      mma_16816(acc, a0, a1, a2, a3, b0, b1);
     }
+    float rr = 0.f;
+    if (t == 0) {
+      const float d0 = x[16 * warp + g] - (acc[0] + acc[1]);
+      const float d1 = x[16 * warp + g + 8] - (acc[2] + acc[3]);
+      rr = d0 * d0 + d1 * d1;
+    }
+    return warp_sum(rr);
+  };
+  {
+    const float rk = recon_sq(uk, S::KS, RK, app + S::A_CK, app + S::A_X);
+    const float rv = recon_sq(uv, S::VS, RV, app + S::A_CV, app + S::A_X + kD);
     const float x = app[S::A_X + tid];
-    const float dlt = x - (h0 + h1);
-    const float rs = warp_sum(dlt * dlt), ns = warp_sum(x * x);
-    if (lane == 0) app[S::A_RED + 2 * warp] = rs, app[S::A_RED + 2 * warp + 1] = ns;
+    const float ns = warp_sum(x * x);   // warps < 4: the key's squares, else the value's
+    if (lane == 0) {
+      app[S::A_RED + warp] = rk;
+      app[S::A_RED + 8 + warp] = rv;
+      app[S::A_RED + 16 + warp] = ns;
+    }
   }
   __syncthreads();
-  const float* red = app + S::A_RED;
-  const float rk = (red[0] + red[2]) + (red[4] + red[6]), nk = (red[1] + red[3]) + (red[5] + red[7]);
-  const float rv = (red[8] + red[10]) + (red[12] + red[14]), nv = (red[9] + red[11]) + (red[13] + red[15]);
+  const float* red = app + S::A_RED;   // [3][8]: key residual, value residual, squares per warp
+  float rk = 0.f, rv = 0.f, nk = 0.f, nv = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) rk += red[w], rv += red[8 + w];
+#pragma unroll
+  for (int w = 0; w < 4; ++w) nk += red[16 + w], nv += red[20 + w];
   const float e = fmaxf(nk > 0.f ? sqrtf(rk / nk) : 0.f, nv > 0.f ? sqrtf(rv / nv) : 0.f);
   const bool routed = e > p.tau;
   const bool keep = routed && F < D.F_cap;
@@ -277,26 +300,14 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       qa1[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
     }
   }
-  // fused append: this (b, h)'s new key row as row 8 of the q~ product's A
-  // operand (lanes of fragment row 0), and one element of the new key or
-  // value row per thread
-  uint32_t xa0[8], xa1[8];
+  // fused append: does row b have a new token; one element of its new key
+  // (threads < d) or value (threads >= d) row per thread, for the owner
   int n_b = 0;
   uint32_t st_new = 0;
   uint16_t xe = 0;
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) xa0[ks] = xa1[ks] = 0u;
   if constexpr (APP) {
     n_b = new_tokens(p.t_new_b, b, 1, &st_new);
-    const lrkv_bf16* krow = p.k_new + bh * kD;   // [B][1][Hkv][d]: row (b, h)
-    if (g == 0) {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        xa0[ks] = *reinterpret_cast<const uint32_t*>(krow + ks * 16 + 2 * t);
-        xa1[ks] = *reinterpret_cast<const uint32_t*>(krow + ks * 16 + 8 + 2 * t);
-      }
-    }
-    xe = reinterpret_cast<const uint16_t*>(tid < kD ? p.k_new : p.v_new)[bh * kD + (tid & (kD - 1))];
+    xe = (tid < kD ? p.k_new : p.v_new)[bh * kD + (tid & (kD - 1))];   // [B][1][Hkv][d]
   }
   // the split's mask words (words past the sequence end are never used), the
   // sequence length and the list length
@@ -330,16 +341,10 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     for (int ks = 0; ks < 8; ++ks) {
       uint32_t b0, b1, b2, b3;
       ldsm_x4_t(b0, b1, b2, b3, uk + (ks * 16 + (lm & 1) * 8 + lr) * S::KS + (16 * ks2 + (lm >> 1) * 8) * 2);
-      mma_16816(a0, qa0[ks], xa0[ks], qa1[ks], xa1[ks], b0, b1);
-      mma_16816(a1, qa0[ks], xa0[ks], qa1[ks], xa1[ks], b2, b3);
+      mma_16816(a0, qa0[ks], 0u, qa1[ks], 0u, b0, b1);
+      mma_16816(a1, qa0[ks], 0u, qa1[ks], 0u, b2, b3);
     }
     if constexpr (APP) {
-      if (g == 0) {   // row 8: the new key's coefficients c_k = U_k^T k (fp32, unrounded)
-        app[S::A_CK + 16 * ks2 + 2 * t] = a0[2];
-        app[S::A_CK + 16 * ks2 + 2 * t + 1] = a0[3];
-        app[S::A_CK + 16 * ks2 + 8 + 2 * t] = a1[2];
-        app[S::A_CK + 16 * ks2 + 8 + 2 * t + 1] = a1[3];
-      }
       if (g < G) {    // q~ rows (scaled), for the new token's logit if it stays compressed
         float* qt = app + S::A_QT + g * RK + 16 * ks2;
         qt[2 * t] = a0[0] * scale;
@@ -381,15 +386,16 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       p.seq_tickets[b] = 0;
     }
   };
+  const int tk = kThreads - 32;   // the thread that takes it: lane 0 of the last warp
   if constexpr (APP) {
-    if (tid == 0) {
-      seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
-      if (h == 0 && c == 0 && st_new) atomicOr(p.C.dev_status, st_new);
-    }
+    if (tid == 0 && h == 0 && c == 0 && st_new) atomicOr(p.C.dev_status, st_new);
   }
   cp_async_wait<0>();   // U_v (in flight since the prologue): none left behind on exit
   if (c >= n_chunks) {
-    if (APP && tid == 0) advance_len();
+    if (APP && tid == tk) {
+      seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
+      advance_len();
+    }
     return;
   }
   const int c1 = min(T_old, c0 + p.chunk);   // the new position is not read from the cache
@@ -493,9 +499,10 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   // (U_k and the scratch sit in the last stage, which the stream refills only
   // from its first step on)
   if constexpr (APP) {
+    if (tid == tk) seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
     if (owner) {
-      append_token<S, G, RK, RV>(p, app, uk, sm + S::OFF_UV, b, h, bh, T_old, F, scale, xe, s_new,
-                                 s_vals, &s_keep);
+      append_token<S, G, RK, RV>(p, app, uk, sm + S::OFF_UV, b, h, bh, T_old, F, scale, xe,
+                                 s_new, s_vals, &s_keep);
       __syncthreads();   // the token's logits and value row in for warp 0
     }
   }
@@ -621,7 +628,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     __syncwarp();
   }
   cp_async_wait<0>();
-  if (APP && tid == 0) advance_len();
+  if (APP && tid == tk) advance_len();
   __syncwarp();
   griddep_launch_dependents();
 
