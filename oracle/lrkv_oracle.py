@@ -149,6 +149,38 @@ def rel_error(U, X, C=None):
     return np.where(den > 0, num / np.where(den > 0, den, 1.0), 0.0)
 
 
+# ---------------------------------------------------------------------------
+# the offline basis (OjaKV README, Method Summary > StaticPCA; KV-CoRE page,
+# abstract: the Frobenius-optimal low-rank approximation)
+# ---------------------------------------------------------------------------
+
+def fit_basis(X, r):
+    """StaticPCA's offline basis of one kv head: the top-r eigenvectors of the
+    (uncentred, reading R1) scatter matrix G = X^T X of the calibration rows.
+
+    OjaKV README, "Method Summary > StaticPCA": an offline low-rank basis
+    computed from a calibration corpus.  KV-CoRE page, abstract: the optimal
+    low-rank approximation under the Frobenius norm; by Eckart-Young that is
+    the span of G's leading eigenvectors, and the residual sum of squares is
+    the discarded eigenvalue mass.
+
+    X: [N, d] rows (bfloat16 values as float64).  Returns (U [d, r], lam [d])
+    with lam descending and U's columns the matching unit eigenvectors.  Sign
+    (reading R18): each column's entry of largest magnitude is positive (the
+    lowest index on a tie).
+    """
+    X = np.asarray(X, np.float64)
+    G = X.T @ X
+    lam, V = np.linalg.eigh(G)               # ascending
+    order = np.argsort(-lam, kind="stable")
+    lam, V = lam[order], V[:, order]
+    for j in range(V.shape[1]):
+        i = int(np.argmax(np.abs(V[:, j])))  # first index of the largest magnitude
+        if V[i, j] < 0:
+            V[:, j] = -V[:, j]
+    return V[:, :r], lam
+
+
 def route(e_k, e_v, tau):
     """Full-rank decision per token: max(e_k, e_v) > tau (readings R2, R3)."""
     return np.maximum(e_k, e_v) > tau

@@ -323,3 +323,57 @@ def test_coefficient_space_equals_reconstruct_then_attend():
     a = O.decode_attn(cache, q)
     b = O.decode_attn_coef(cache, q)
     assert np.abs(a - b).max() <= 1e-12 * np.abs(a).max()
+
+
+# ---- the offline basis (StaticPCA; Frobenius-optimal subspace) --------------------------
+
+def _calib_rows(seed, N=600, d=32, rank_sig=12, noise=0.05):
+    rng = np.random.default_rng(seed)
+    Q, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    Z = rng.standard_normal((N, rank_sig)) * (np.arange(1, rank_sig + 1) ** -0.5)
+    return Z @ Q[:, :rank_sig].T + noise * rng.standard_normal((N, d))
+
+
+def test_fit_basis_matches_svd_and_eckart_young():
+    """Against numpy's SVD of X (another library routine): singular values squared are
+    the eigenvalues, the right singular vectors span the same subspace; the residual
+    sum of squares equals the discarded eigenvalue mass."""
+    X = _calib_rows(1)
+    r = 8
+    U, lam = O.fit_basis(X, r)
+    _, sv, Vt = np.linalg.svd(X, full_matrices=False)
+    assert np.allclose(lam[:len(sv)], sv ** 2, rtol=1e-10, atol=1e-9)
+    P, Ps = U @ U.T, Vt[:r].T @ Vt[:r]
+    assert np.abs(P - Ps).max() < 1e-10
+    resid = ((X - X @ U @ U.T) ** 2).sum()
+    assert abs(resid - lam[r:].sum()) <= 1e-10 * lam.sum()
+    assert np.allclose(U.T @ U, np.eye(r), atol=1e-12)
+    G = X.T @ X
+    assert np.allclose(G @ U, U * lam[:r], atol=1e-9 * lam[0])
+
+
+def test_fit_basis_beats_every_other_basis_and_sign_convention():
+    """No other r-dim orthonormal basis has a smaller residual (random trials), and
+    each column's largest-magnitude entry is positive."""
+    X = _calib_rows(2)
+    r = 6
+    U, lam = O.fit_basis(X, r)
+    best = ((X - X @ U @ U.T) ** 2).sum()
+    rng = np.random.default_rng(3)
+    for _ in range(50):
+        Q, _ = np.linalg.qr(rng.standard_normal((X.shape[1], r)))
+        assert ((X - X @ Q @ Q.T) ** 2).sum() >= best - 1e-9
+    for j in range(r):
+        i = int(np.argmax(np.abs(U[:, j])))
+        assert U[i, j] > 0
+
+
+def test_fit_basis_exact_low_rank_data():
+    """Rows exactly in a rank-r span: the basis spans it and the rest of the spectrum is 0."""
+    rng = np.random.default_rng(4)
+    d, r = 16, 5
+    Q, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    X = rng.standard_normal((200, r)) @ Q[:, :r].T
+    U, lam = O.fit_basis(X, r)
+    assert np.abs(U @ U.T - Q[:, :r] @ Q[:, :r].T).max() < 1e-10
+    assert np.abs(lam[r:]).max() < 1e-9 * lam[0]
