@@ -12,6 +12,8 @@ Entry points (same names as the C ABI):
     lrkv_decode_attn(dims, cache, q, out, ws=...)
     lrkv_decode_attn_noalloc(dims, cache, q, out)   (scratch held by the library)
     lrkv_append_decode_attn(dims, cache, k_new, v_new, tau, q, out, t_new_b=None, err_out=None, ws=...)
+    lrkv_fit_workspace_size(dims, n_rows) -> int
+    lrkv_fit_basis(dims, X, r, ...) -> (U [Hkv,d,r] bf16, eigenvalues [Hkv,d] fp32)
     lrkv_status_str(code) -> str
 plus ``LayerCache`` (allocates one layer's buffers with torch) and
 ``make_workspace``.
@@ -77,6 +79,11 @@ def load_library(path=None):
     lib.lrkv_append_decode_attn.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Cache), P, P, P,
                                             ctypes.c_float, P, P, P, P, ctypes.c_size_t, P]
     lib.lrkv_append_decode_attn.restype = ctypes.c_int
+    lib.lrkv_fit_workspace_size.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int32]
+    lib.lrkv_fit_workspace_size.restype = ctypes.c_size_t
+    lib.lrkv_fit_basis.argtypes = [ctypes.POINTER(_Dims), P, ctypes.c_int32, ctypes.c_int32, P, P, P,
+                                   ctypes.c_size_t, P]
+    lib.lrkv_fit_basis.restype = ctypes.c_int
     lib.lrkv_status_str.argtypes = [ctypes.c_int]
     lib.lrkv_status_str.restype = ctypes.c_char_p
     if path is None:
@@ -209,3 +216,27 @@ def lrkv_append_decode_attn(dims, cache, k_new, v_new, tau, q, out, t_new_b=None
     if check and code != LRKV_OK:
         raise LrkvError(code, "lrkv_append_decode_attn")
     return code
+
+
+def lrkv_fit_workspace_size(dims, n_rows):
+    return int(load_library().lrkv_fit_workspace_size(ctypes.byref(dims.c()), int(n_rows)))
+
+
+def lrkv_fit_basis(dims, X, r, U_out=None, eigvals_out=None, ws=None, stream=None, check=True):
+    """StaticPCA basis of every kv head from calibration rows X [..., Hkv, d] (bf16, device).
+
+    Returns (U [Hkv, d, r] bf16, eigenvalues [Hkv, d] fp32 descending); see include/lrkv.h."""
+    lib = load_library()
+    n_rows = X.numel() // (dims.Hkv * dims.d)
+    dev = X.device
+    if U_out is None:
+        U_out = torch.empty(dims.Hkv, dims.d, r, dtype=torch.bfloat16, device=dev)
+    if eigvals_out is None:
+        eigvals_out = torch.empty(dims.Hkv, dims.d, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.empty(max(lrkv_fit_workspace_size(dims, n_rows), 16), dtype=torch.uint8, device=dev)
+    code = lib.lrkv_fit_basis(ctypes.byref(dims.c()), _ptr(X), int(n_rows), int(r), _ptr(U_out),
+                              _ptr(eigvals_out), _ptr(ws), ws.numel(), _stream_ptr(stream))
+    if check and code != LRKV_OK:
+        raise LrkvError(code, "lrkv_fit_basis")
+    return U_out, eigvals_out

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 
+#include "basis_fit.cuh"
 #include "compress_append.cuh"
 #include "compress_params.cuh"
 #include "compress_tc.cuh"
@@ -144,6 +145,18 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
   return launched();
 }
 
+// Row splits of the Gram pass: about one wave of CTAs over the kv heads, each
+// split a multiple of the ring's 64-row tile.
+inline void fit_splits(int Hkv, int n_rows, int* splits, int* rows_per_split) {
+  const int tiles = (n_rows + fit::kTileRows - 1) / fit::kTileRows;
+  int sp = kNumSMs / (Hkv > 0 ? Hkv : 1);
+  if (sp < 1) sp = 1;
+  if (sp > tiles) sp = tiles;
+  const int tiles_per = (tiles + sp - 1) / sp;
+  *rows_per_split = tiles_per * fit::kTileRows;
+  *splits = (tiles + tiles_per - 1) / tiles_per;
+}
+
 }  // namespace
 
 extern "C" {
@@ -246,6 +259,49 @@ lrkv_status lrkv_append_decode_attn(const lrkv_dims* dims, const lrkv_cache* cac
   p.err_out = err_out;
   p.seq_tickets = reinterpret_cast<int32_t*>(w + L.seq_tickets);
   return launch_decode(p, s);
+}
+
+size_t lrkv_fit_workspace_size(const lrkv_dims* dims, int32_t n_rows) {
+  if (!dims || dims->Hkv < 1 || dims->Hkv > 65535 || dims->d != kD || n_rows < 1) return 0;
+  int splits, rps;
+  fit_splits(dims->Hkv, n_rows, &splits, &rps);
+  return sizeof(float) * (size_t)dims->Hkv * splits * kD * kD;
+}
+
+lrkv_status lrkv_fit_basis(const lrkv_dims* dims, const lrkv_bf16* X, int32_t n_rows, int32_t r,
+                           lrkv_bf16* U_out, float* eigvals_out, void* ws, size_t ws_bytes,
+                           void* stream) {
+  if (!dims || !X || !U_out || n_rows < 1) return LRKV_ERR_INVALID_ARG;
+  if (dims->Hkv < 1 || dims->Hkv > 65535) return LRKV_ERR_INVALID_ARG;
+  if (dims->d != kD) return LRKV_ERR_UNSUPPORTED;
+  if (r < 1 || r > kD) return LRKV_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(U_out) || !aligned16(eigvals_out) || !aligned16(ws))
+    return LRKV_ERR_ALIGNMENT;
+  const size_t need = lrkv_fit_workspace_size(dims, n_rows);
+  if (!ws || ws_bytes < need) return LRKV_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  fit::GramParams gp;
+  gp.X = X;
+  gp.n_rows = n_rows;
+  gp.Hkv = dims->Hkv;
+  gp.partials = static_cast<float*>(ws);
+  int splits;
+  fit_splits(dims->Hkv, n_rows, &splits, &gp.rows_per_split);
+  const size_t gsmem = 2 * fit::kStageBytes;
+  if (!set_smem(fit::gram_kernel, gsmem)) return LRKV_ERR_CUDA;
+  fit::gram_kernel<<<dim3(splits, dims->Hkv), fit::kThreads, gsmem, s>>>(gp);
+  lrkv_status st = launched();
+  if (st != LRKV_OK) return st;
+  fit::EigParams ep;
+  ep.partials = gp.partials;
+  ep.splits = splits;
+  ep.r = r;
+  ep.U = U_out;
+  ep.eigvals = eigvals_out;
+  const size_t esmem = fit::eig_smem_bytes();
+  if (!set_smem(fit::eig_kernel, esmem)) return LRKV_ERR_CUDA;
+  fit::eig_kernel<<<dims->Hkv, fit::kEigThreads, esmem, s>>>(ep);
+  return launched();
 }
 
 const char* lrkv_status_str(lrkv_status status) {

@@ -172,6 +172,31 @@ LRKV_API lrkv_status lrkv_append_decode_attn(const lrkv_dims* dims, const lrkv_c
                                              const lrkv_bf16* q, float* out, void* ws,
                                              size_t ws_bytes, void* stream);
 
+/* StaticPCA's offline basis (OjaKV repository README, "Method Summary >
+ * StaticPCA": a fixed basis computed offline from calibration rows; KV-CoRE
+ * page, abstract: the Frobenius-optimal low-rank approximation).  For every
+ * kv head h, the top-r eigenvectors of the uncentred scatter matrix
+ * G_h = sum over rows n of x_{n,h} x_{n,h}^T, computed on the GPU: G in fp32 on
+ * the tensor cores (exact bf16 products), summed in fp64, cyclic Jacobi in
+ * fp64 (eigenvectors in fp32).
+ *
+ * X:        [n_rows][Hkv][d] bf16 calibration rows (keys or values; the layout
+ *           of lrkv_compress's k_new with B * t_new rows).  Only dims->Hkv and
+ *           dims->d (128) are used.
+ * r:        1..d columns to keep.
+ * U_out:    [Hkv][d][r] bf16, unit eigenvectors by decreasing eigenvalue, each
+ *           signed so that its largest-magnitude entry is positive (the lowest
+ *           index on a tie), rounded to nearest even: a basis for lrkv_cache.
+ * eigvals_out: nullable [Hkv][d] fp32, every eigenvalue of G_h, descending (the
+ *           discarded mass of a rank-r basis is the sum past index r).
+ * ws:       lrkv_fit_workspace_size(dims, n_rows) bytes (any contents).
+ * Returns LRKV_OK when the work was enqueued (two kernels on `stream`).
+ */
+LRKV_API size_t lrkv_fit_workspace_size(const lrkv_dims* dims, int32_t n_rows);
+LRKV_API lrkv_status lrkv_fit_basis(const lrkv_dims* dims, const lrkv_bf16* X, int32_t n_rows,
+                                    int32_t r, lrkv_bf16* U_out, float* eigvals_out, void* ws,
+                                    size_t ws_bytes, void* stream);
+
 /* Device scratch built into the library for lrkv_decode_attn_noalloc, bytes. */
 #define LRKV_NOALLOC_SCRATCH_BYTES (4u << 20)
 

@@ -30,7 +30,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["lrkv_workspace_size", "lrkv_compress", "lrkv_decode_attn", "lrkv_decode_attn_noalloc",
-         "lrkv_append_decode_attn", "lrkv_status_str"])
+         "lrkv_append_decode_attn", "lrkv_fit_workspace_size", "lrkv_fit_basis",
+         "lrkv_status_str"])
 
 
 def test_every_declared_symbol_is_exported(lib):
