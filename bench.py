@@ -84,11 +84,16 @@ def peaks():
     return FALLBACK_PEAK, "fallback"
 
 
+# the decode kernel's sources: the stored ncu traffic is of the kernel built from these
+DECODE_SOURCES = ("decode_stream.cuh", "decode_launch.cuh", "decode_simple.cuh", "lrkv_common.cuh",
+                  "ptx.cuh", "launch_util.cuh")
+
+
 def source_hash():
-    """Hash of the library sources: ties stored ncu traffic to the kernel it was taken on."""
+    """Hash of the decode kernel's sources: ties stored ncu traffic to the kernel it was taken on."""
     h = hashlib.sha256()
     cs = os.path.join(ROOT, "decode_attention_lrkv_b200", "csrc")
-    for f in sorted(os.listdir(cs)):
+    for f in DECODE_SOURCES:
         with open(os.path.join(cs, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
