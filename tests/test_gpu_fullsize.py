@@ -6,7 +6,8 @@ case at 131072), with the cache capacity bench.py uses, so the kernels run in
 the launch configuration bench.py times: a prefill through lrkv_compress,
 three one-token appends, then one decode.  The oracle cannot redo whole
 layers in seconds, so sampled (batch row, kv head) pairs are recomputed one
-by one and compared element by element:
+by one and compared element by element (then two more steps through the fused
+append + decode call, the launch bench.py times, are checked the same way):
   - every coefficient of the head: 1 bf16 ulp + the fp32 accumulation bound;
   - the routed set: identical except tokens within 1e-4 of tau;
   - the full-rank list: ascending positions, rows bit-exact, length;
@@ -25,9 +26,9 @@ from tests import lrkv_testutil as U
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
-# bench.py's cache capacity: the context plus three passes of its default
+# bench.py's cache capacity: the context plus four passes of its default
 # 100 timed + 5 warm-up decode steps, plus one
-BENCH_EXTRA = 3 * (100 + 5) + 1
+BENCH_EXTRA = 4 * (100 + 5) + 1
 N_APPEND = 3
 
 
@@ -94,6 +95,7 @@ def test_full_size_sampled_heads(wi, w):
     U_k, U_v = U.f64(layer["U_k"]), U.f64(layer["U_v"])
     g = w.Hq // w.Hkv
     q = U.f64(layer["q"])
+    heads = {}
     for b, h in sorted(picks):
         Kh = U.f64(layer["K"][b:b + 1, :, h:h + 1])
         Vh = U.f64(layer["V"][b:b + 1, :, h:h + 1])
@@ -127,3 +129,32 @@ def test_full_size_sampled_heads(wi, w):
         # decode over the GPU-written cache
         ref = O.decode_attn(gc, q[b:b + 1, h * g:(h + 1) * g])
         assert U.out_rel_err(out[b, h * g:(h + 1) * g], ref[0]) <= U.OUT_RTOL, (b, h)
+        heads[(b, h)] = (oc, band)
+
+    # two fused steps (lrkv_append_decode_attn): the same checks on the sampled heads
+    Kf, Vf = synth.decode_tokens(w, layer["Qk"], layer["Qv"], N_APPEND + 2, seed, 0, DEV)
+    qf = synth.decode_queries(w, 2, seed + 1, 0, DEV)
+    for s in range(2):
+        k = Kf[:, N_APPEND + s:N_APPEND + s + 1].contiguous()
+        v = Vf[:, N_APPEND + s:N_APPEND + s + 1].contiguous()
+        out = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=DEV)
+        L.lrkv_append_decode_attn(D, cache, k, v, w.tau, qf[s], out, ws=ws)
+        torch.cuda.synchronize()
+        assert int(cache.dev_status[0]) == 0
+        assert cache.seq_len.tolist() == [n + N_APPEND + s + 1 for n in lengths]
+        out = U.f64(out)
+        kq, vq, qq = U.f64(k), U.f64(v), U.f64(qf[s])
+        for (b, h), (oc, band) in heads.items():
+            e1, _, _ = O.compress(oc, kq[b:b + 1, :, h:h + 1], vq[b:b + 1, :, h:h + 1], w.tau)
+            gc = _gpu_head(D, cache, b, h)
+            T = int(oc.seq_len[0])
+            assert int(gc.seq_len[0]) == T
+            for got, want, x, Ub in ((gc.coef_k[0, 0, T - 1], oc.coef_k[0, 0, T - 1], kq[b, 0, h], U_k[h]),
+                                     (gc.coef_v[0, 0, T - 1], oc.coef_v[0, 0, T - 1], vq[b, 0, h], U_v[h])):
+                tol = O.bf16_ulp(np.maximum(np.abs(got), np.abs(want)))
+                tol = tol + U.COEF_ABS_SAFETY * U.GAMMA_128 * (np.abs(x) @ np.abs(Ub))
+                assert (np.abs(got - want) <= tol).all(), (b, h, s)
+            rg, ro = set(U.routed_positions(gc, 0, 0)), set(U.routed_positions(oc, 0, 0))
+            assert (rg ^ ro) <= band | ({T - 1} if abs(float(e1.ravel()[0]) - w.tau) < U.BAND else set())
+            ref = O.decode_attn(gc, qq[b:b + 1, h * g:(h + 1) * g])
+            assert U.out_rel_err(out[b, h * g:(h + 1) * g], ref[0]) <= U.OUT_RTOL, (b, h, s)
