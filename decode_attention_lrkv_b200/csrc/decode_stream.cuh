@@ -205,10 +205,10 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
     uint32_t* mword = p.C.route_mask + bh * (D.T_cap / 32) + (pos >> 5);
     const uint32_t bit = 1u << (pos & 31);
     if (keep) {
-      atomicOr(mword, bit);
+      red_or_u32(mword, bit);
       p.C.full_idx[bh * D.F_cap + F] = pos;
     } else {
-      atomicAnd(mword, ~bit);
+      red_and_u32(mword, ~bit);
     }
     if (routed && !keep) atomicOr(p.C.dev_status, LRKV_DEV_FULL_OVERFLOW);
     if (p.err_out) p.err_out[bh] = e;
@@ -375,9 +375,9 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   T += n_eff;
   const int n_chunks = T > 0 ? (T + p.chunk - 1) / p.chunk : 1;
   const bool owner = APP && n_eff > 0 && c == n_chunks - 1;
-  // Every thread of this CTA has read seq_len[b] (the barrier above): take the
-  // row's ticket now (release only, so nothing waits for it here) and look at
-  // it at the end; the last CTA of the grid for row b advances its length.
+  // Every thread of this CTA has read seq_len[b] (the barrier above): each CTA
+  // takes the row's ticket once (release only) and looks at it later; the last
+  // CTA of the grid for row b advances its length.
   int seq_ticket = 0;
   auto advance_len = [&]() {
     if (seq_ticket == D.Hkv * (int)gridDim.x - 1) {
@@ -499,7 +499,6 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   // (U_k and the scratch sit in the last stage, which the stream refills only
   // from its first step on)
   if constexpr (APP) {
-    if (tid == tk) seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
     if (owner) {
       append_token<S, G, RK, RV>(p, app, uk, sm + S::OFF_UV, b, h, bh, T_old, F, scale, xe,
                                  s_new, s_vals, &s_keep);
@@ -628,7 +627,9 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     __syncwarp();
   }
   cp_async_wait<0>();
-  if (APP && tid == tk) advance_len();
+  // the row's length ticket: release-only, taken now that this thread has no
+  // copy in flight (a release waits for them); looked at after the record
+  if (APP && tid == tk) seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
   __syncwarp();
   griddep_launch_dependents();
 
@@ -735,6 +736,8 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[S::W_PF + o], s_we[w][gi], x);
     rec0[gi * S::REC + 4 + i] = x;
   }
+
+  if (APP && tid == tk) advance_len();
 
   // ---- the last split of this (batch row, kv head) merges every record ------------
   __syncthreads();

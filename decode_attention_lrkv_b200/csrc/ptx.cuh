@@ -157,6 +157,15 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* addr, int v) {
   return old;
 }
 
+// Fire-and-forget bitwise OR / AND on a global word (no value returned, so the
+// thread never waits for it).
+__device__ __forceinline__ void red_or_u32(uint32_t* addr, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.or.b32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_and_u32(uint32_t* addr, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.and.b32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+
 // Release-only add: later operations of the thread need not wait for it; a
 // thread that acts on the returned count issues fence_acq_rel_gpu() first.
 __device__ __forceinline__ int atom_add_release_gpu(int* addr, int v) {
