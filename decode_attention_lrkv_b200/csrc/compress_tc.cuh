@@ -15,12 +15,17 @@
 // (U U^T) and split into bf16 high and low parts (P = P_hi + P_lo to 2^-17).
 // Per tile, TMA brings the 128 x 128 input rows (128-byte swizzle); one
 // thread issues
-//     D1 = X U        (M 128, N r, K 128)      -> coefficients
-//     D2 = X P_hi^T + X P_lo^T  (M 128, N 128) -> residual vectors
-// into tensor memory (double-buffered), and four epilogue warps (one token
-// row per thread) store bf16(c), sum the squared residual and the squared
-// input, and write e.  Three input stages and two accumulator buffers let
-// the loads, the MMAs and the epilogue of consecutive tiles overlap.
+//     [D2 | D1] = X [P_hi | U]   (M 128, N 128 + r, K 128)
+//     D2       += X P_lo^T       (M 128, N 128)
+// into tensor memory (double-buffered): D1 = X U holds the coefficients and
+// D2 = X P^T the residual vectors.  P_hi and U^T sit back to back in shared
+// memory as one B operand, so each K slice of X is read twice per tile, not
+// three times: the MMAs read their operands from shared memory at close to
+// its bandwidth, and every byte saved there also speeds up the loads and the
+// epilogue, which share it.  Eight epilogue warps (two per token row) store
+// bf16(c), sum the squared residual and the squared input, and write e.  Up
+// to four input stages and two accumulator buffers let the loads, the MMAs
+// and the epilogue of consecutive tiles overlap.
 //
 // Kernel 2, route_count_kernel: e_t = max(e_k, e_v); routed iff e_t > tau.
 // Per 128-token tile: err_out, the routed bits (warp ballots) and their count.
@@ -56,8 +61,9 @@ constexpr size_t kSmemLimit = 227 * 1024;
 
 // Shared memory (bytes) for rank rm (the larger rank of the launch: both
 // tensors share one layout) and ns input stages; operand regions 1024-aligned.
-//   X stages [ns][128][128] (128-byte swizzle), P_hi, P_lo [128][128],
-//   U^T [rm][128], mbarriers, group B's per-row sums [2][128].
+//   X stages [ns][128][128] (128-byte swizzle), P_hi [128][128] directly
+//   followed by U^T [rm][128] (rows 128.. of the merged B operand),
+//   P_lo [128][128], mbarriers, group B's per-row sums [2][128].
 // U [128][rm] for U U^T is needed only before the first tile: it borrows the
 // last input stage.
 struct Layout {
@@ -66,10 +72,10 @@ struct Layout {
   __host__ __device__ Layout(int rm, int ns) {
     x = 0;
     phi = ns * kStageBytes;
-    plo = phi + kD * kD * 2;
-    ut = plo + kD * kD * 2;
+    ut = phi + kD * kD * 2;
+    plo = ut + rm * kD * 2;
     u = (ns - 1) * kStageBytes;
-    bar = ut + rm * kD * 2;
+    bar = plo + kD * kD * 2;
     part = bar + 128;
     bytes = (size_t)part + 2 * kTile * 8 + 1024;   // + slack to align the base to 1024
   }
@@ -281,11 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   } else if (warp == kMmaWarp) {
     // MMA issuer
     if (lane == 0) {
-      const uint32_t idesc1 = tc5::idesc_bf16_f32(128, R);
+      const uint32_t idesc1 = tc5::idesc_bf16_f32(128, 128 + R);
       const uint32_t idesc2 = tc5::idesc_bf16_f32(128, 128);
       const uint32_t xbase = smem_u32(sm + Lo.x);
-      const uint32_t utb = smem_u32(sm + Lo.ut);
-      const uint32_t phb = smem_u32(sm + Lo.phi);
+      const uint32_t phb = smem_u32(sm + Lo.phi);   // P_hi rows, then U^T rows
       const uint32_t plb = smem_u32(sm + Lo.plo);
       int i = 0;
       RowLen rl;
@@ -297,20 +302,13 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
         if (!wait_or_abort(&full[s], (i / NS) & 1, abort_flag)) break;
         if (i >= 2 && !wait_or_abort(&tfree[buf], ((i >> 1) - 1) & 1, abort_flag)) break;
         tc5::fence_after_sync();
-        const uint32_t d1 = tmem + buf * 256, d2 = d1 + 128;
+        const uint32_t d2 = tmem + buf * 256;   // D2 columns [0, 128), D1 [128, 128 + R)
         const uint32_t xs = xbase + s * kStageBytes;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint64_t a = tc5::smem_desc(xs + (j >> 2) * kBoxBytes + (j & 3) * 32, 16, 1024,
                                             tc5::kSwizzle128B);
-          tc5::mma_bf16(d1, a, tc5::smem_desc(utb + j * 256, 128, 2048, tc5::kSwizzleNone), idesc1,
-                        j > 0);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint64_t a = tc5::smem_desc(xs + (j >> 2) * kBoxBytes + (j & 3) * 32, 16, 1024,
-                                            tc5::kSwizzle128B);
-          tc5::mma_bf16(d2, a, tc5::smem_desc(phb + j * 256, 128, 2048, tc5::kSwizzleNone), idesc2,
+          tc5::mma_bf16(d2, a, tc5::smem_desc(phb + j * 256, 128, 2048, tc5::kSwizzleNone), idesc1,
                         j > 0);
           tc5::mma_bf16(d2, a, tc5::smem_desc(plb + j * 256, 128, 2048, tc5::kSwizzleNone), idesc2,
                         1);
@@ -347,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
       const int t = t0 + m;
       const bool valid = t < ne;
       const size_t bh = (size_t)b * D.Hkv + h;
-      const uint32_t d1 = lane_base + buf * 256, d2 = d1 + 128;
+      const uint32_t d2 = lane_base + buf * 256, d1 = d2 + 128;
       float rs = 0.f, xs = 0.f;
       if (grp_a) {
         // coefficients, 64 columns per batch of loads
