@@ -14,6 +14,7 @@ Entry points (same names as the C ABI):
     lrkv_append_decode_attn(dims, cache, k_new, v_new, tau, q, out, t_new_b=None, err_out=None, ws=...)
     lrkv_fit_workspace_size(dims, n_rows) -> int
     lrkv_fit_basis(dims, X, r, ...) -> (U [Hkv,d,r] bf16, eigenvalues [Hkv,d] fp32)
+    lrkv_rank_for_budget(eigvals, budget) -> int32 ranks   (host call)
     lrkv_status_str(code) -> str
 plus ``LayerCache`` (allocates one layer's buffers with torch) and
 ``make_workspace``.
@@ -30,6 +31,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "liblrkv.so")
 
 LRKV_OK = 0
+LRKV_ERR_INVALID_ARG = 1
 STATUS_NAMES = {0: "LRKV_OK", 1: "LRKV_ERR_INVALID_ARG", 2: "LRKV_ERR_UNSUPPORTED",
                 3: "LRKV_ERR_ALIGNMENT", 4: "LRKV_ERR_CUDA"}
 DEV_FULL_OVERFLOW = 0x1
@@ -84,6 +86,8 @@ def load_library(path=None):
     lib.lrkv_fit_basis.argtypes = [ctypes.POINTER(_Dims), P, ctypes.c_int32, ctypes.c_int32, P, P, P,
                                    ctypes.c_size_t, P]
     lib.lrkv_fit_basis.restype = ctypes.c_int
+    lib.lrkv_rank_for_budget.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_double, P]
+    lib.lrkv_rank_for_budget.restype = ctypes.c_int
     lib.lrkv_status_str.argtypes = [ctypes.c_int]
     lib.lrkv_status_str.restype = ctypes.c_char_p
     if path is None:
@@ -143,6 +147,23 @@ class LayerCache:
 
     def nbytes(self):
         return sum(getattr(self, f).numel() * getattr(self, f).element_size() for f in self.FIELDS)
+
+
+def lrkv_rank_for_budget(eigvals, budget, check=True):
+    """Smallest rank per head whose discarded eigenvalue mass is within `budget`
+    of the total (host call; see include/lrkv.h).
+
+    eigvals: [n_heads, d] fp32 on the host or the device (copied to the host),
+    as returned by lrkv_fit_basis.  Returns an int32 tensor [n_heads] (CPU)."""
+    lam = eigvals.detach().to("cpu", torch.float32).contiguous()
+    if lam.dim() == 1:
+        lam = lam.unsqueeze(0)
+    r = torch.zeros(lam.shape[0], dtype=torch.int32)
+    code = load_library().lrkv_rank_for_budget(lam.data_ptr(), int(lam.shape[0]), int(lam.shape[1]),
+                                               float(budget), r.data_ptr())
+    if check and code != LRKV_OK:
+        raise LrkvError(code, "lrkv_rank_for_budget")
+    return r
 
 
 def lrkv_status_str(code):

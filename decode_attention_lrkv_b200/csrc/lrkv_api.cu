@@ -304,6 +304,24 @@ lrkv_status lrkv_fit_basis(const lrkv_dims* dims, const lrkv_bf16* X, int32_t n_
   return launched();
 }
 
+lrkv_status lrkv_rank_for_budget(const float* eigvals, int32_t n_heads, int32_t d, double budget,
+                                 int32_t* r_out) {
+  if (!eigvals || !r_out || n_heads < 1 || d < 1 || d > 4096) return LRKV_ERR_INVALID_ARG;
+  if (!(budget >= 0.0 && budget <= 1.0)) return LRKV_ERR_INVALID_ARG;   // NaN fails too
+  double tail[4097];
+  for (int32_t h = 0; h < n_heads; ++h) {
+    const float* lam = eigvals + (size_t)h * d;
+    // tail[j] = mass of eigenvalues j..d-1, summed from the smallest up
+    tail[d] = 0.0;
+    for (int32_t j = d - 1; j >= 0; --j) tail[j] = tail[j + 1] + (lam[j] > 0.f ? (double)lam[j] : 0.0);
+    const double limit = budget * tail[0];
+    int32_t r = 1;
+    while (r < d && tail[r] > limit) ++r;
+    r_out[h] = r;
+  }
+  return LRKV_OK;
+}
+
 const char* lrkv_status_str(lrkv_status status) {
   switch (status) {
     case LRKV_OK: return "ok";

@@ -197,6 +197,29 @@ LRKV_API lrkv_status lrkv_fit_basis(const lrkv_dims* dims, const lrkv_bf16* X, i
                                     int32_t r, lrkv_bf16* U_out, float* eigvals_out, void* ws,
                                     size_t ws_bytes, void* stream);
 
+/* Rank by error budget for a StaticPCA basis (OjaKV repository README, the
+ * calibration command's `--error_budget`; KV-CoRE page, abstract: the
+ * Frobenius-optimal rank-r approximation).  By Eckart-Young the relative
+ * squared Frobenius error of the best rank-r approximation of the calibration
+ * rows is the discarded eigenvalue mass over the total; for each head the
+ * call returns the smallest r in 1..d with
+ *     sum_{j >= r} max(lambda_j, 0) <= budget * sum_j max(lambda_j, 0),
+ * sums in fp64 taken from the smallest eigenvalue up (j = d-1 first).
+ * Negative eigenvalues (rounding of a positive semi-definite matrix) count as
+ * zero; a head whose eigenvalues are all zero gets r = 1.
+ *
+ * Host call: no GPU work, nothing is enqueued.
+ * eigvals: HOST [n_heads][d] fp32, each row descending (lrkv_fit_basis's
+ *          eigvals_out, copied to the host).
+ * d:       eigenvalues per head, 1..4096.
+ * budget:  0 <= budget <= 1 (not NaN); 0 keeps every direction with mass.
+ * r_out:   HOST [n_heads] int32.
+ * Returns LRKV_ERR_INVALID_ARG for null pointers, n_heads < 1, d out of range
+ * or a budget outside [0, 1]; r_out is then untouched.
+ */
+LRKV_API lrkv_status lrkv_rank_for_budget(const float* eigvals, int32_t n_heads, int32_t d,
+                                          double budget, int32_t* r_out);
+
 /* Device scratch built into the library for lrkv_decode_attn_noalloc, bytes. */
 #define LRKV_NOALLOC_SCRATCH_BYTES (4u << 20)
 

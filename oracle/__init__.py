@@ -5,6 +5,6 @@ Test infrastructure only: ``tests/``, ``__graft_entry__.smoke()`` and
 and its Python binding never do.
 """
 from .bf16 import bf16_round, bf16_bits, bf16_from_bits, bf16_ulp
-from .lrkv_oracle import (Dims, Cache, project, reconstruct, rel_error, route, fit_basis,
+from .lrkv_oracle import (Dims, Cache, project, reconstruct, rel_error, route, fit_basis, rank_for_budget,
                           compress, effective_kv, softmax, decode_attn,
                           decode_attn_coef, FULL_OVERFLOW, SEQ_OVERFLOW)

@@ -181,6 +181,33 @@ def fit_basis(X, r):
     return V[:, :r], lam
 
 
+def rank_for_budget(lam, budget):
+    """Smallest rank whose discarded eigenvalue mass is within the error budget.
+
+    OjaKV README (calibration command, `--error_budget`) and KV-CoRE page,
+    abstract (Frobenius-optimal low-rank approximation).  Reading R20: the
+    budget bounds the relative squared Frobenius error of the rank-r
+    approximation of the calibration rows, which by Eckart-Young is the mass
+    of the discarded eigenvalues over the total:
+        r = min { r in 1..d : sum_{j >= r} lam_j <= budget * sum_j lam_j }
+    with negative eigenvalues (rounding of a positive semi-definite matrix)
+    counted as zero; the sums run from the smallest eigenvalue up, in fp64.
+
+    lam: [d] eigenvalues, descending.  Returns an int.
+    """
+    lam = np.asarray(lam, np.float64)
+    lam = np.where(lam > 0.0, lam, 0.0)
+    d = lam.shape[0]
+    tail = [0.0] * (d + 1)
+    for j in range(d - 1, -1, -1):
+        tail[j] = tail[j + 1] + float(lam[j])
+    limit = float(budget) * tail[0]
+    for r in range(1, d + 1):
+        if tail[r] <= limit:
+            return r
+    return d
+
+
 def route(e_k, e_v, tau):
     """Full-rank decision per token: max(e_k, e_v) > tau (readings R2, R3)."""
     return np.maximum(e_k, e_v) > tau

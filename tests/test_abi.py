@@ -31,7 +31,7 @@ def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["lrkv_workspace_size", "lrkv_compress", "lrkv_decode_attn", "lrkv_decode_attn_noalloc",
          "lrkv_append_decode_attn", "lrkv_fit_workspace_size", "lrkv_fit_basis",
-         "lrkv_status_str"])
+         "lrkv_rank_for_budget", "lrkv_status_str"])
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -122,3 +122,43 @@ def test_host_validation_rejects_before_launch(lib):
     assert _call_compress(lib, _dims(F_cap=0), _FakeCache(full_k=None, full_v=None, full_idx=None),
                           t_new=0) == 0
     assert _call_compress(lib, D, _FakeCache(full_v=None)) == INVALID
+
+
+def test_rank_for_budget_matches_the_oracle(lib):
+    """Host call: the same rank as the oracle on fp32 spectra, bit for bit, including
+    budgets that land exactly on a discarded-mass boundary."""
+    import numpy as np
+    import torch
+    import oracle as O
+    rng = np.random.default_rng(11)
+    spectra = [np.sort(rng.gamma(a, 1.0, 128).astype(np.float32))[::-1] for a in (0.3, 1.0, 3.0)]
+    spectra.append(np.array([2.0 ** -j for j in range(128)], np.float32))   # exact binary fractions
+    z = np.zeros(128, np.float32)
+    z[:3] = [5.0, 2.0, 1.0]
+    z[-1] = -1e-6                                                             # rounding below zero
+    spectra.append(z)
+    spectra.append(np.zeros(128, np.float32))
+    lam = np.stack(spectra)
+    for budget in (0.0, 1e-6, 0.01, 0.075, 0.125, 0.25, 0.5, 1.0, 0.5 ** 10):
+        got = L.lrkv_rank_for_budget(torch.from_numpy(lam.copy()), budget)
+        want = [O.rank_for_budget(row, budget) for row in lam]
+        assert got.tolist() == want, budget
+
+
+def test_rank_for_budget_rejects_bad_arguments(lib):
+    import ctypes
+    import numpy as np
+    lam = np.ones((2, 8), np.float32)
+    r = np.full(2, -7, np.int32)
+    P = lambda a: a.ctypes.data
+    bad = L.LRKV_ERR_INVALID_ARG
+    assert lib.lrkv_rank_for_budget(None, 2, 8, 0.1, P(r)) == bad
+    assert lib.lrkv_rank_for_budget(P(lam), 2, 8, 0.1, None) == bad
+    assert lib.lrkv_rank_for_budget(P(lam), 0, 8, 0.1, P(r)) == bad
+    assert lib.lrkv_rank_for_budget(P(lam), 2, 0, 0.1, P(r)) == bad
+    assert lib.lrkv_rank_for_budget(P(lam), 2, 4097, 0.1, P(r)) == bad
+    for b in (-0.01, 1.01, float("nan")):
+        assert lib.lrkv_rank_for_budget(P(lam), 2, 8, b, P(r)) == bad
+    assert (r == -7).all()
+    assert lib.lrkv_rank_for_budget(P(lam), 2, 8, 0.5, P(r)) == L.LRKV_OK
+    assert r.tolist() == [4, 4]

@@ -113,3 +113,30 @@ def test_fitted_basis_feeds_compress_and_decode():
                             abs_v=U.coef_abs_bound(oc.U_v, U.f64(layer["V"])))
     out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
     assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
+
+
+@pytest.mark.parametrize("budget", [0.3, 0.1, 0.03])
+def test_rank_for_budget_on_fitted_spectra(budget):
+    """Rank by error budget from the GPU's eigenvalues: the oracle's rank on its own fp64
+    spectrum (or a neighbour, only where the discarded mass is within the eigenvalue
+    tolerance of the limit), and the chosen columns' residual within the budget."""
+    w = synth.workload(1, T=2048, layers=1)
+    layer = synth.make_layer(w, 0, 61, device=DEV)
+    D = U.dims_of(w, synth.pad_to(2048, 32))
+    Ug, lam_g = L.lrkv_fit_basis(D, layer["K"], 128)
+    torch.cuda.synchronize()
+    r_g = L.lrkv_rank_for_budget(lam_g, budget).tolist()
+    Xf = U.f64(layer["K"])
+    for h in range(min(w.Hkv, 4)):
+        Xh = Xf[:, :, h].reshape(-1, w.d)
+        _, lam = O.fit_basis(Xh, 1)
+        lp = np.where(lam > 0, lam, 0.0)
+        tot = lp.sum()
+        r_o = O.rank_for_budget(lam, budget)
+        if r_g[h] != r_o:
+            r = min(r_g[h], r_o)
+            assert abs(max(r_g[h], r_o) - r) == 1
+            assert abs(lp[r:].sum() - budget * tot) <= 2e-3 * lam[0], (h, r_g[h], r_o)
+        Q, _ = np.linalg.qr(U.f64(Ug[h])[:, :r_g[h]])
+        resid = ((Xh - Xh @ Q @ Q.T) ** 2).sum()
+        assert resid <= budget * tot + 2e-3 * lam[0], (h, resid / tot)

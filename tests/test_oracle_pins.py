@@ -377,3 +377,46 @@ def test_fit_basis_exact_low_rank_data():
     U, lam = O.fit_basis(X, r)
     assert np.abs(U @ U.T - Q[:, :r] @ Q[:, :r].T).max() < 1e-10
     assert np.abs(lam[r:]).max() < 1e-9 * lam[0]
+
+
+def test_rank_for_budget_worked_by_hand():
+    """Spectrum 8, 4, 2, 1, 1 (total 16): discarded mass after r = 1..5 is 8, 4, 2, 1, 0."""
+    lam = [8.0, 4.0, 2.0, 1.0, 1.0]
+    assert O.rank_for_budget(lam, 0.5) == 1        # 8 <= 8
+    assert O.rank_for_budget(lam, 0.49) == 2       # 4 <= 7.84
+    assert O.rank_for_budget(lam, 0.125) == 3      # 2 <= 2, boundary inclusive
+    assert O.rank_for_budget(lam, 0.1) == 4        # 2 > 1.6, 1 <= 1.6
+    assert O.rank_for_budget(lam, 0.0) == 5
+    assert O.rank_for_budget(lam, 1.0) == 1
+    assert O.rank_for_budget([0.0, 0.0, 0.0], 0.0) == 1
+    # a negative eigenvalue from rounding counts as zero
+    assert O.rank_for_budget([3.0, 1.0, -1e-12], 0.0) == 2
+
+
+def test_rank_for_budget_is_the_eckart_young_rank():
+    """The chosen rank's projection residual, computed directly from the rows, is
+    within the budget and one rank less is not (Eckart-Young: the discarded mass
+    is the best rank-r residual)."""
+    X = _calib_rows(5)
+    total = (X ** 2).sum()
+    for budget in (0.3, 0.1, 0.05, 0.02, 0.01, 0.004):
+        U, lam = O.fit_basis(X, X.shape[1])
+        r = O.rank_for_budget(lam, budget)
+        res = lambda k: ((X - X @ U[:, :k] @ U[:, :k].T) ** 2).sum() / total
+        assert res(r) <= budget + 1e-12
+        if r > 1:
+            assert res(r - 1) > budget - 1e-12
+
+
+def test_rank_for_budget_monotone_and_exact_rank():
+    rng = np.random.default_rng(6)
+    lam = np.sort(rng.gamma(0.5, 1.0, 64))[::-1]
+    ranks = [O.rank_for_budget(lam, b) for b in np.linspace(0.0, 1.0, 101)]
+    assert all(a >= b for a, b in zip(ranks, ranks[1:]))
+    assert ranks[0] == 64 and ranks[-1] == 1
+    # rows exactly in a rank-5 span: any small budget gives 5
+    d, k = 16, 5
+    Q, _ = np.linalg.qr(rng.standard_normal((d, d)))
+    X = rng.standard_normal((200, k)) @ Q[:, :k].T
+    _, lam = O.fit_basis(X, d)
+    assert O.rank_for_budget(lam, 1e-9) == k
