@@ -199,14 +199,33 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   // U into two K-major no-swizzle operand layouts:
   //   U   as [m = i][k = j]   (A and B of U U^T), 8-row groups 16 r bytes apart
   //   U^T as [n = j][k = i]   (B of X U),         8-row groups 2048 bytes apart
+  // Every 16-byte piece of U (8 columns of one row, r a multiple of 16) is
+  // loaded before the first store, so the loads share one memory latency.
   {
     unsigned char* su = sm + Lo.u;
     unsigned char* sut = sm + Lo.ut;
-    for (int idx = tid; idx < kD * R; idx += kThreads) {
-      const int i = idx / R, j = idx - (idx / R) * R;
-      const uint16_t u = Ug[idx];
-      *reinterpret_cast<uint16_t*>(su + core_off(i, j, 16 * R)) = u;
-      *reinterpret_cast<uint16_t*>(sut + core_off(j, i, 2048)) = u;
+    constexpr int kMaxPieces = (kD * kD / 8 + kThreads - 1) / kThreads;
+    const int n_pieces = kD * R / 8;
+    const uint4* ug = reinterpret_cast<const uint4*>(Ug);
+    uint4 piece[kMaxPieces];
+#pragma unroll
+    for (int k = 0; k < kMaxPieces; ++k) {
+      const int c = tid + k * kThreads;
+      if (c < n_pieces) piece[k] = ug[c];
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxPieces; ++k) {
+      const int c = tid + k * kThreads;
+      if (c < n_pieces) {
+        const int i = (c * 8) / R, j0 = c * 8 - i * R;
+        *reinterpret_cast<uint4*>(su + core_off(i, j0, 16 * R)) = piece[k];
+        const uint32_t w[4] = {piece[k].x, piece[k].y, piece[k].z, piece[k].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          *reinterpret_cast<uint16_t*>(sut + core_off(j0 + 2 * q, i, 2048)) = (uint16_t)(w[q] & 0xffffu);
+          *reinterpret_cast<uint16_t*>(sut + core_off(j0 + 2 * q + 1, i, 2048)) = (uint16_t)(w[q] >> 16);
+        }
+      }
     }
   }
   fence_proxy_async_smem();
