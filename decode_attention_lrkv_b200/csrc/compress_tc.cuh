@@ -561,19 +561,34 @@ __global__ void __launch_bounds__(128) route_scatter_kernel(RouteParams p) {
         }
       }
     }
-    // copy the kept rows, one row per warp pass (32 lanes x 8 bytes)
+    // copy the kept rows (32 lanes x 8 bytes per row), up to kBatch rows per
+    // pass with every load of the pass issued before its first store
+    constexpr int kBatch = 8;
     uint32_t todo = keep_b;
     const int wslot0 = base + wbefore;
     while (todo) {
-      const int src = __ffs(todo) - 1;
-      todo &= todo - 1;
-      const int ts = t0 + warp * 32 + src;
-      const int sl = wslot0 + __popc(wbits & ((1u << src) - 1u));
-      const size_t x = (((size_t)b * p.t_new + ts) * D.Hkv + h) * kD;
-      const uint2* ks = reinterpret_cast<const uint2*>(p.k_new + x);
-      const uint2* vs = reinterpret_cast<const uint2*>(p.v_new + x);
-      reinterpret_cast<uint2*>(p.C.full_k + (bh * D.F_cap + sl) * kD)[lane] = ks[lane];
-      reinterpret_cast<uint2*>(p.C.full_v + (bh * D.F_cap + sl) * kD)[lane] = vs[lane];
+      uint2 kr[kBatch], vr[kBatch];
+      int sl[kBatch];
+#pragma unroll
+      for (int q = 0; q < kBatch; ++q) {
+        sl[q] = -1;
+        if (todo) {
+          const int src = __ffs(todo) - 1;
+          todo &= todo - 1;
+          const int ts = t0 + warp * 32 + src;
+          sl[q] = wslot0 + __popc(wbits & ((1u << src) - 1u));
+          const size_t x = (((size_t)b * p.t_new + ts) * D.Hkv + h) * kD;
+          kr[q] = reinterpret_cast<const uint2*>(p.k_new + x)[lane];
+          vr[q] = reinterpret_cast<const uint2*>(p.v_new + x)[lane];
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < kBatch; ++q) {
+        if (sl[q] >= 0) {
+          reinterpret_cast<uint2*>(p.C.full_k + (bh * D.F_cap + sl[q]) * kD)[lane] = kr[q];
+          reinterpret_cast<uint2*>(p.C.full_v + (bh * D.F_cap + sl[q]) * kD)[lane] = vr[q];
+        }
+      }
     }
   }
   if (__syncthreads_or(overflow)) st |= LRKV_DEV_FULL_OVERFLOW;
