@@ -11,3 +11,4 @@ from .lrkv_oracle import (Dims, Cache, project, reconstruct, rel_error, route, f
 from .coef_quant import (QMAX, quantize_coef, dequantize_coef, pack_int4, unpack_int4,
                          quantize_cache, dequantized_cache, decode_attn_quant,
                          decode_attn_quant_coef, quant_bytes_per_token)
+from .attn_aware import KeyTransform, key_transform, weighted_key_error
