@@ -12,3 +12,4 @@ from .coef_quant import (QMAX, quantize_coef, dequantize_coef, pack_int4, unpack
                          quantize_cache, dequantized_cache, decode_attn_quant,
                          decode_attn_quant_coef, quant_bytes_per_token)
 from .attn_aware import KeyTransform, key_transform, weighted_key_error
+from .oja import oja_direction, oja_step, oja_stream
