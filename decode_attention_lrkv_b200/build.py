@@ -1,10 +1,12 @@
 """Builds liblrkv.so in-tree with nvcc for sm_100a.
 
-    python -m decode_attention_lrkv_b200.build [--force]
+    python -m decode_attention_lrkv_b200.build [--force] [--ptxas-v]
 
-The library is compiled from csrc/*.cu against include/lrkv.h and linked
-with the static CUDA runtime, so it carries no run-time path dependencies.
+Every csrc/*.cu is compiled to an object on its own (in parallel, into
+_build/) against include/lrkv.h, then the objects are linked with the static
+CUDA runtime, so the library carries no run-time path dependencies.
 """
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -15,11 +17,12 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
+OBJ = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "liblrkv.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
-         "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden", "-shared"]
+         "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden"]
 
 
 def nvcc():
@@ -33,9 +36,13 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _inputs():
-    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + \
+def _headers():
+    return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))) + \
         [os.path.join(INCLUDE, "lrkv.h"), os.path.abspath(__file__)]
+
+
+def _inputs():
+    return sources() + _headers()
 
 
 def up_to_date():
@@ -45,19 +52,35 @@ def up_to_date():
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
+def _compile(src, extra):
+    obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, *extra, "-c", src, "-o", obj]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    return obj, cmd, r
+
+
 def build(force=False, verbose=False, extra=()):
     """Compile liblrkv.so unless it is newer than every source; returns its path."""
     if not force and up_to_date():
         return LIB
+    os.makedirs(OBJ, exist_ok=True)
+    srcs = sources()
+    workers = max(1, min(len(srcs), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(workers) as ex:
+        results = list(ex.map(lambda s: _compile(s, list(extra)), srcs))
+    for obj, cmd, r in results:
+        if verbose:
+            print(" ".join(cmd))
+            if r.stdout or r.stderr:
+                print(r.stdout + r.stderr)
+        if r.returncode != 0:
+            raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + r.stdout + r.stderr)
     tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, *extra, *sources(), "-o", tmp]
-    if verbose:
-        print(" ".join(cmd))
+    cmd = [nvcc(), *ARCH, "-shared", "-Xcompiler", "-fvisibility=hidden",
+           *[o for o, _, _ in results], "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
-    if verbose and (r.stdout or r.stderr):
-        print(r.stdout + r.stderr)
+        raise RuntimeError("nvcc link failed:\n" + r.stdout + r.stderr)
     os.replace(tmp, LIB)
     return LIB
 

@@ -9,27 +9,11 @@
 // accumulated in r_v-space and lifted by U_v once at the end.
 #pragma once
 
+#include "decode_params.cuh"
 #include "lrkv_common.cuh"
 
 namespace lrkv {
 
-struct DecodeParams {
-  lrkv_dims D;
-  lrkv_cache C;
-  const lrkv_bf16* q;
-  float* out;
-  int32_t* tickets;   // [B][Hkv]
-  float* partials;    // [B][Hkv][n_chunk_max][g][2 + r_v + d]
-  int chunk;          // positions per split
-  int n_chunk_max;
-  // fused decode-time append (lrkv_append_decode_attn); k_new null: plain decode
-  const lrkv_bf16* k_new;   // [B][1][Hkv][d]
-  const lrkv_bf16* v_new;   // [B][1][Hkv][d]
-  const int32_t* t_new_b;   // [B] tokens of row b (0 or 1), nullable: 1 for every row
-  float tau;
-  float* err_out;           // [B][Hkv][1], nullable
-  int32_t* seq_tickets;     // [B], zero between calls
-};
 
 constexpr int kDecThreads = 256;
 constexpr int kDecWarps = kDecThreads / 32;
@@ -58,7 +42,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(DecodeParams
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int T = p.C.seq_len[b];
   T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
-  const int n_chunks = T > 0 ? (T + p.chunk - 1) / p.chunk : 1;
+  int chunk;   // positions per split, from the live length
+  const int n_chunks = decode_split(T, p.n_chunk_max, (long long)D.B * D.Hkv, p.num_sms, &chunk);
   if (c >= n_chunks) return;
   const int r_k = D.r_k, r_v = D.r_v;
   const size_t bh = (size_t)b * D.Hkv + h;
@@ -93,8 +78,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(DecodeParams
   }
 
   // compressed tokens of this split
-  const int c0 = c * p.chunk;
-  const int c1 = min(T, c0 + p.chunk);
+  const int c0 = c * chunk;
+  const int c1 = min(T, c0 + chunk);
   const uint32_t* mask = p.C.route_mask + bh * (D.T_cap / 32);
   const lrkv_bf16* ck = p.C.coef_k + bh * D.T_cap * r_k;
   const lrkv_bf16* cv = p.C.coef_v + bh * D.T_cap * r_v;

@@ -309,21 +309,34 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     n_b = new_tokens(p.t_new_b, b, 1, &st_new);
     xe = (tid < kD ? p.k_new : p.v_new)[bh * kD + (tid & (kD - 1))];   // [B][1][Hkv][d]
   }
-  // the split's mask words (words past the sequence end are never used), the
-  // sequence length and the list length
+  // the sequence length and the list length; the split's mask words follow
+  // once the live length has fixed the split
+  int T = p.C.seq_len[b];
+  const int F_raw = p.C.full_cnt[bh];
+  T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
+  // fused append: the new token (if the row has one and there is room) takes
+  // position T_old; the split holding it (the last one) is its owner
+  int n_eff = 0;
+  if constexpr (APP) {
+    n_eff = n_b > 0 && T < D.T_cap ? 1 : 0;
+    if (n_b > 0 && T >= D.T_cap) st_new |= LRKV_DEV_SEQ_OVERFLOW;
+  }
+  const int T_old = T;
+  T += n_eff;
+  // splits from the live length (every CTA of the (b, kv head) finds the same)
+  int chunk;
+  const int n_chunks = decode_split(T, p.n_chunk_max, (long long)D.B * D.Hkv, p.num_sms, &chunk);
+  const bool active = c < n_chunks;
+  const int c0 = c * chunk;
+  // this split's mask words (words past the sequence end are never used): the
+  // loads go out now and land while q~ is formed
   constexpr int kMW = (kMaxChunk / 32 + kThreads - 1) / kThreads;   // mask words per thread
-  const int c0 = c * p.chunk;
   uint32_t mw[kMW];
 #pragma unroll
   for (int u = 0; u < kMW; ++u) {
     const int wl = tid + u * kThreads, wi = c0 / 32 + wl;
-    mw[u] = wl < p.chunk / 32 && wi < D.T_cap / 32 ? p.C.route_mask[bh * (D.T_cap / 32) + wi] : 0u;
+    mw[u] = active && wl < chunk / 32 && wi < D.T_cap / 32 ? p.C.route_mask[bh * (D.T_cap / 32) + wi] : 0u;
   }
-  int T = p.C.seq_len[b];
-  const int F_raw = p.C.full_cnt[bh];
-#pragma unroll
-  for (int u = 0; u < kMW; ++u)
-    if (tid + u * kThreads < kMaxChunk / 32) maskw[tid + u * kThreads] = mw[u];
 
   const float scale = kLog2e * rsqrtf((float)kD);
   // q~ = U_k^T q as B fragments over k = r_k (column n = 2h + part: the bf16
@@ -334,7 +347,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   float* app = reinterpret_cast<float*>(sm + S::OFF_APP);   // fused append scratch
   cp_async_wait<1>();   // U_k in (U_v may still be in flight)
   __syncthreads();
-  if (warp < KST) {
+  if (active && warp < KST) {
     const int ks2 = warp;                      // columns [16 ks2, 16 ks2 + 16) of q~
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -363,17 +376,6 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     s_qb[ks2][0][lane] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
     s_qb[ks2][1][lane] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
   }
-  T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
-  // fused append: the new token (if the row has one and there is room) takes
-  // position T_old; the split holding it (the last one) is its owner
-  int n_eff = 0;
-  if constexpr (APP) {
-    n_eff = n_b > 0 && T < D.T_cap ? 1 : 0;
-    if (n_b > 0 && T >= D.T_cap) st_new |= LRKV_DEV_SEQ_OVERFLOW;
-  }
-  const int T_old = T;
-  T += n_eff;
-  const int n_chunks = T > 0 ? (T + p.chunk - 1) / p.chunk : 1;
   const bool owner = APP && n_eff > 0 && c == n_chunks - 1;
   // Every thread of this CTA has read seq_len[b] (the barrier above): each CTA
   // takes the row's ticket once (release only) and looks at it later; the last
@@ -391,14 +393,17 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     if (tid == 0 && h == 0 && c == 0 && st_new) atomicOr(p.C.dev_status, st_new);
   }
   cp_async_wait<0>();   // U_v (in flight since the prologue): none left behind on exit
-  if (c >= n_chunks) {
+  if (!active) {
     if (APP && tid == tk) {
       seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
       advance_len();
     }
     return;
   }
-  const int c1 = min(T_old, c0 + p.chunk);   // the new position is not read from the cache
+#pragma unroll
+  for (int u = 0; u < kMW; ++u)
+    if (tid + u * kThreads < kMaxChunk / 32) maskw[tid + u * kThreads] = mw[u];
+  const int c1 = min(T_old, c0 + chunk);   // the new position is not read from the cache
   const int n_pos = c1 > c0 ? c1 - c0 : 0;
   const int F = min(max(F_raw, 0), D.F_cap);
   const int share = (F + n_chunks - 1) / n_chunks;

@@ -9,48 +9,15 @@
 #include "compress_append.cuh"
 #include "compress_params.cuh"
 #include "compress_tc.cuh"
-#include "decode_launch.cuh"
+#include "decode_dispatch.h"
 #include "launch_util.cuh"
 #include "lrkv.h"
 #include "lrkv_common.cuh"
+#include "lrkv_host.cuh"
 
 namespace {
 
 using namespace lrkv;
-
-constexpr int kMaxG = 8;
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-lrkv_status check_dims(const lrkv_dims* D) {
-  if (!D) return LRKV_ERR_INVALID_ARG;
-  if (D->B < 1 || D->Hq < 1 || D->Hkv < 1 || D->T_cap < 32 || D->F_cap < 0)
-    return LRKV_ERR_INVALID_ARG;
-  if (D->B > 65535 || D->Hkv > 65535) return LRKV_ERR_UNSUPPORTED;
-  if (D->Hq % D->Hkv != 0) return LRKV_ERR_INVALID_ARG;
-  if (D->T_cap % 32 != 0) return LRKV_ERR_INVALID_ARG;
-  if (D->d != kD) return LRKV_ERR_UNSUPPORTED;
-  if (D->r_k < 16 || D->r_k > D->d || D->r_k % 16 || D->r_v < 16 || D->r_v > D->d || D->r_v % 16)
-    return LRKV_ERR_INVALID_ARG;
-  if (D->Hq / D->Hkv > kMaxG) return LRKV_ERR_UNSUPPORTED;
-  return LRKV_OK;
-}
-
-lrkv_status check_cache(const lrkv_dims* D, const lrkv_cache* C) {
-  if (!C) return LRKV_ERR_INVALID_ARG;
-  const void* need[] = {C->U_k, C->U_v, C->coef_k, C->coef_v, C->route_mask,
-                        C->full_cnt, C->seq_len, C->dev_status};
-  for (const void* p : need)
-    if (!p) return LRKV_ERR_INVALID_ARG;
-  const void* full[] = {C->full_idx, C->full_k, C->full_v};
-  for (const void* p : full)
-    if (!p && D->F_cap > 0) return LRKV_ERR_INVALID_ARG;
-  for (const void* p : need)
-    if (!aligned16(p)) return LRKV_ERR_ALIGNMENT;
-  for (const void* p : full)
-    if (!aligned16(p)) return LRKV_ERR_ALIGNMENT;
-  return LRKV_OK;
-}
 
 lrkv_status check_ws(const lrkv_dims* D, void* ws, size_t ws_bytes, WsLayout* L) {
   *L = ws_layout(*D);
@@ -113,7 +80,7 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
   pp.n_stages = ptc::stages_for(pp.r_max);
   const int groups = 2 * D.Hkv;
   const int n_units = D.B * pp.tiles_per_b;
-  int per_group = kNumSMs / groups;
+  int per_group = num_sms() / groups;
   if (per_group < 1) per_group = 1;
   if (per_group > n_units) per_group = n_units;
   const size_t smem = ptc::Layout(pp.r_max, pp.n_stages).bytes;
@@ -149,7 +116,7 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
 // split a multiple of the ring's 64-row tile.
 inline void fit_splits(int Hkv, int n_rows, int* splits, int* rows_per_split) {
   const int tiles = (n_rows + fit::kTileRows - 1) / fit::kTileRows;
-  int sp = kNumSMs / (Hkv > 0 ? Hkv : 1);
+  int sp = num_sms() / (Hkv > 0 ? Hkv : 1);
   if (sp < 1) sp = 1;
   if (sp > tiles) sp = tiles;
   const int tiles_per = (tiles + sp - 1) / sp;
@@ -204,8 +171,7 @@ lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache, con
   lrkv_status st = check_dims(dims);
   if (st != LRKV_OK) return st;
   if ((st = check_cache(dims, cache)) != LRKV_OK) return st;
-  if (!q || !out) return LRKV_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(out)) return LRKV_ERR_ALIGNMENT;
+  if ((st = check_q_out(q, out)) != LRKV_OK) return st;
   WsLayout L;
   if ((st = check_ws(dims, ws, ws_bytes, &L)) != LRKV_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -217,8 +183,8 @@ lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache, con
   p.out = out;
   p.tickets = reinterpret_cast<int32_t*>(w + L.decode_tickets);
   p.partials = reinterpret_cast<float*>(w + L.partials);
-  p.chunk = L.chunk;
   p.n_chunk_max = L.n_chunk_max;
+  p.num_sms = num_sms();
   return launch_decode(p, s);
 }
 
@@ -236,7 +202,7 @@ lrkv_status lrkv_append_decode_attn(const lrkv_dims* dims, const lrkv_cache* cac
     return LRKV_ERR_ALIGNMENT;
   WsLayout L;
   if ((st = check_ws(dims, ws, ws_bytes, &L)) != LRKV_OK) return st;
-  if (!stream_decode_supported(*dims, L.chunk)) {   // the two launches it fuses
+  if (!stream_decode_supported(*dims)) {   // the two launches it fuses
     st = lrkv_compress(dims, cache, k_new, v_new, 1, t_new_b, tau, err_out, ws, ws_bytes, stream);
     if (st != LRKV_OK) return st;
     return lrkv_decode_attn(dims, cache, q, out, ws, ws_bytes, stream);
@@ -250,8 +216,8 @@ lrkv_status lrkv_append_decode_attn(const lrkv_dims* dims, const lrkv_cache* cac
   p.out = out;
   p.tickets = reinterpret_cast<int32_t*>(w + L.decode_tickets);
   p.partials = reinterpret_cast<float*>(w + L.partials);
-  p.chunk = L.chunk;
   p.n_chunk_max = L.n_chunk_max;
+  p.num_sms = num_sms();
   p.k_new = k_new;
   p.v_new = v_new;
   p.t_new_b = t_new_b;

@@ -5,13 +5,17 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "lrkv.h"
 
 namespace lrkv {
 
 constexpr int kD = 128;            // head dimension handled by this build
-constexpr int kNumSMs = 148;       // B200; only used to size work splits
+constexpr int kDefaultSMs = 148;   // B200: used only when no device can be queried
 constexpr int kMaxDecodeChunk = 8192;   // positions per decode split, at most
+constexpr int kMinDecodeChunk = 128;    // positions per decode split, at least (when T allows)
+constexpr int kDecodeOverhead = 1024;   // a decode CTA's fixed cost, in streamed positions
 constexpr float kLog2e = 1.4426950408889634f;
 
 // bf16 <-> fp32.  A bf16 value is the top half of the fp32 with the same
@@ -60,34 +64,66 @@ struct WsLayout {
   int n_tiles;             // ceil(T_cap / 128)
   size_t partials;         // float [B][Hkv][n_chunk_max][g][4 + r_v + d]
   size_t total;
-  int chunk;               // decode: positions per split
-  int n_chunk_max;         // decode: splits per (b, kv head)
+  int chunk;               // decode: positions per split of a full cache
+  int n_chunk_max;         // decode: splits per (b, kv head) in the grid
   int partial_floats;      // floats per (split, q head)
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Positions per decode split: at least 128, a multiple of 32 (one mask word),
-// at most kMaxDecodeChunk.  The split count n minimises the modelled makespan
-//   ceil(B*Hkv*n / SMs) * (chunk + overhead)
-// with one CTA per SM resident at a time; `overhead` is a CTA's fixed cost
-// (bases, q~, merge) expressed in streamed positions.
-inline int decode_chunk(const lrkv_dims& D) {
-  const long long bh = (long long)D.B * D.Hkv;
-  const long long overhead = 1024;
-  long long best_cost = -1, best = kMaxDecodeChunk;
-  const long long n_max = (D.T_cap + 127) / 128;
-  for (long long n = 1; n <= n_max && n <= 1024; ++n) {
-    long long ch = (D.T_cap + n - 1) / n;
-    ch = (ch + 31) / 32 * 32;
-    if (ch < 128) ch = 128;
-    if (ch > kMaxDecodeChunk) continue;
-    const long long splits = (D.T_cap + ch - 1) / ch;
-    const long long waves = (bh * splits + kNumSMs - 1) / kNumSMs;
-    const long long cost = waves * (ch + overhead);
-    if (best_cost < 0 || cost < best_cost) best_cost = cost, best = ch;
+// Streaming multiprocessors of the current device, queried once per device.
+// kDefaultSMs when no device is visible (a host-only size query).
+inline int num_sms() {
+  static std::atomic<int> cached[64];   // 0 until queried
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return kDefaultSMs;
   }
-  return (int)best;
+  if (dev >= 0 && dev < 64) {
+    const int v = cached[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return kDefaultSMs;
+  }
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// How one (batch row, kv head) with T positions is split for decode: n splits
+// of `chunk` positions (a multiple of 32, one mask word; at most
+// kMaxDecodeChunk), n in [n_min, n_max] minimising the modelled makespan
+//   ceil(BH * n / sms) * (chunk + kDecodeOverhead)
+// with BH (batch row, kv head) pairs and one CTA per SM resident at a time.
+// The cost only drops where n fills a wave, so the candidates are the largest
+// n of the first four wave counts that n_min allows, and n_max.  Returns the
+// splits that hold positions (ceil(T / chunk) <= n).
+__host__ __device__ inline int decode_split(long long T, int n_max_grid, long long BH, int sms,
+                                            int* chunk_out) {
+  if (T <= 0) {
+    *chunk_out = kMinDecodeChunk;
+    return 1;
+  }
+  const long long n_min = (T + kMaxDecodeChunk - 1) / kMaxDecodeChunk;
+  long long n_max = (T + kMinDecodeChunk - 1) / kMinDecodeChunk;
+  if (n_max > n_max_grid) n_max = n_max_grid;
+  if (n_max < n_min) n_max = n_min;
+  const long long w0 = (BH * n_min + sms - 1) / sms;   // waves at n_min
+  long long best_cost = -1, best_chunk = kMaxDecodeChunk;
+  for (int k = 0; k <= 4; ++k) {
+    long long n = k < 4 ? (w0 + k) * sms / BH : n_max;
+    if (n < n_min) n = n_min;
+    if (n > n_max) n = n_max;
+    const long long ch = ((T + n - 1) / n + 31) / 32 * 32;
+    const long long waves = (BH * ((T + ch - 1) / ch) + sms - 1) / sms;
+    const long long cost = waves * (ch + kDecodeOverhead);
+    if (best_cost < 0 || cost < best_cost) best_cost = cost, best_chunk = ch;
+  }
+  *chunk_out = (int)best_chunk;
+  return (int)((T + best_chunk - 1) / best_chunk);
 }
 
 inline WsLayout ws_layout(const lrkv_dims& D) {
@@ -106,8 +142,9 @@ inline WsLayout ws_layout(const lrkv_dims& D) {
   off = align_up(off + sizeof(int32_t) * (size_t)D.B * D.Hkv * L.n_tiles, 256);
   L.tile_bits = off;
   off = align_up(off + sizeof(uint32_t) * 4 * (size_t)D.B * D.Hkv * L.n_tiles, 256);
-  L.chunk = decode_chunk(D);
-  L.n_chunk_max = (D.T_cap + L.chunk - 1) / L.chunk;
+  // decode: the grid has the splits of a full cache; each CTA re-splits the
+  // live length (decode_split) within them
+  L.n_chunk_max = decode_split(D.T_cap, 1024, (long long)D.B * D.Hkv, num_sms(), &L.chunk);
   L.partial_floats = 4 + D.r_v + D.d;   // m, l, pad, pad, acc_c[r_v], acc_f[d]
   L.partials = off;
   int g = D.Hkv > 0 ? D.Hq / D.Hkv : 0;

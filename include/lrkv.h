@@ -116,10 +116,13 @@ typedef struct {
    v_new and all cache state) is read after the preceding kernel completed. */
 
 /* Bytes of device workspace that lrkv_compress and lrkv_decode_attn need for
-   these sizes (0 for invalid sizes).  The workspace must be zero-filled once
-   after allocation; the kernels leave it zeroed where it needs to be, so it
-   can be reused by any later call with the same dims.  One workspace serves
-   one stream of calls: concurrent calls need their own. */
+   these sizes (0 for invalid sizes).  The decode part depends on the current
+   device's number of SMs (the split-K grid is sized for it; 148 is assumed
+   when no device is visible): query it with the device current on which the
+   calls will run.  The workspace must be zero-filled once after allocation;
+   the kernels leave it zeroed where it needs to be, so it can be reused by any
+   later call with the same dims.  One workspace serves one stream of calls:
+   concurrent calls need their own. */
 LRKV_API size_t lrkv_workspace_size(const lrkv_dims* dims);
 
 /* Append new tokens to every sequence of the cache (prefill or a decode step).
@@ -147,7 +150,10 @@ LRKV_API lrkv_status lrkv_compress(const lrkv_dims* dims, const lrkv_cache* cach
  * out: [B][Hq][d] fp32, the attention output (0 for an empty sequence).
  * Attends to positions 0..seq_len[b]-1 as the cache holds them on the
  * device when the kernel runs (so an append issued earlier on the same
- * stream is included).
+ * stream is included).  The split-K grid is sized for a full cache (T_cap
+ * positions); each sequence's splits are cut from its live length on the
+ * device, so a cache allocated far larger than it holds costs no more than a
+ * snug one.
  * ws: workspace of at least lrkv_workspace_size(dims) bytes (ws_bytes).
  */
 LRKV_API lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache,
@@ -243,12 +249,17 @@ LRKV_API lrkv_status lrkv_rank_for_budget(const float* eigvals, int32_t n_heads,
  * launches the decode kernel there.
  *
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress), once per device, with that device current: make
- * that first call before any stream capture starts.
+ * (cudaGetSymbolAddress), with that device current: make that first call
+ * before any stream capture starts.  The address is kept once the lookup has
+ * succeeded; a failed lookup returns LRKV_ERR_CUDA and is tried again by the
+ * next call.
  * All calls on one device share the array.  Calls whose executions overlap on
  * the GPU (different streams, or host threads without ordering) race on it
  * and give wrong results: order them, e.g. issue them on one stream.
- * Arguments, layouts and synchronous errors are those of lrkv_decode_attn.
+ * Arguments and layouts are those of lrkv_decode_attn.  Checks, in order: the
+ * sizes (as lrkv_decode_attn checks them), then the scratch limit
+ * (LRKV_ERR_UNSUPPORTED, nothing else looked at), then the cache, q and out
+ * pointers (as lrkv_decode_attn checks them).
  */
 LRKV_API lrkv_status lrkv_decode_attn_noalloc(const lrkv_dims* dims, const lrkv_cache* cache,
                                               const lrkv_bf16* q, float* out, void* stream);

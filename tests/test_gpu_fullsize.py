@@ -67,12 +67,18 @@ def _gpu_head(D, cache, b, h):
 WORKLOADS = [(i, synth.workload(i, layers=1)) for i in (1, 2, 3, 4)]
 
 
+def bench_f_cap(wi, T_cap):
+    """bench.py's full-rank list capacity: all positions on the 32K workload (81%
+    routed), a quarter of them elsewhere (7-11% routed)."""
+    return T_cap if wi == 2 else synth.pad_to(T_cap // 4, 32)
+
+
 @pytest.mark.parametrize("wi,w", WORKLOADS, ids=[w.name for _, w in WORKLOADS])
 def test_full_size_sampled_heads(wi, w):
     seed = 31 + wi
     layer = synth.make_layer(w, 0, seed, device=DEV)
     T_cap = synth.pad_to(w.T + BENCH_EXTRA, 32)
-    D = U.dims_of(w, T_cap)
+    D = U.dims_of(w, T_cap, bench_f_cap(wi, T_cap))
     cache = L.LayerCache(D, layer["U_k"], layer["U_v"], device=DEV)
     ws = L.make_workspace(D, DEV)
     lengths = layer["lengths"].tolist()
@@ -158,3 +164,36 @@ def test_full_size_sampled_heads(wi, w):
             assert (rg ^ ro) <= band | ({T - 1} if abs(float(e1.ravel()[0]) - w.tau) < U.BAND else set())
             ref = O.decode_attn(gc, qq[b:b + 1, h * g:(h + 1) * g])
             assert U.out_rel_err(out[b, h * g:(h + 1) * g], ref[0]) <= U.OUT_RTOL, (b, h, s)
+
+
+def test_long_capacity_holding_8k():
+    """A cache allocated for 131072 positions that holds the 8K workload's
+    context (the serving case: capacity for the longest request): the decode
+    splits follow the live length.  Sampled heads against the oracle, then one
+    fused append + decode step."""
+    wi, w = 1, synth.workload(1, layers=1)
+    seed = 41
+    layer = synth.make_layer(w, 0, seed, device=DEV)
+    D = U.dims_of(w, 131072, 32768)
+    cache = L.LayerCache(D, layer["U_k"], layer["U_v"], device=DEV)
+    ws = L.make_workspace(D, DEV)
+    L.lrkv_compress(D, cache, layer["K"], layer["V"], w.tau, ws=ws)
+    out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
+    Kf, Vf = synth.decode_tokens(w, layer["Qk"], layer["Qv"], 1, seed, 0, DEV)
+    o2 = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=DEV)
+    # the decode above read the prefilled cache; gather those heads before the fused step
+    g = w.Hq // w.Hkv
+    q = U.f64(layer["q"])
+    torch.cuda.synchronize()
+    for h in (0, 5):
+        gc = _gpu_head(D, cache, 0, h)
+        ref = O.decode_attn(gc, q[0:1, h * g:(h + 1) * g])
+        assert U.out_rel_err(out[0, h * g:(h + 1) * g], ref[0]) <= U.OUT_RTOL, h
+    L.lrkv_append_decode_attn(D, cache, Kf.contiguous(), Vf.contiguous(), w.tau, layer["q"], o2, ws=ws)
+    torch.cuda.synchronize()
+    assert int(cache.dev_status[0]) == 0 and int(cache.seq_len[0]) == w.T + 1
+    o2 = U.f64(o2)
+    for h in (0, 3, 7):
+        gc = _gpu_head(D, cache, 0, h)
+        ref = O.decode_attn(gc, q[0:1, h * g:(h + 1) * g])
+        assert U.out_rel_err(o2[0, h * g:(h + 1) * g], ref[0]) <= U.OUT_RTOL, h

@@ -245,6 +245,27 @@ def test_group_sizes_and_rank_pairs(Hq, Hkv, r_k, r_v):
     assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
 
 
+@pytest.mark.parametrize("Hq,Hkv,r_k,r_v", [(32, 8, 64, 96), (24, 8, 64, 96), (4, 4, 48, 64)])
+def test_capacity_far_above_the_live_length(Hq, Hkv, r_k, r_v):
+    """A cache allocated for 16384 positions that holds 600: the decode splits
+    follow the live length (the grid is sized for the capacity), with the
+    streaming kernel (GQA 4, MHA) and the CUDA-core kernel (GQA 3); then a
+    fused append + decode step on the same cache."""
+    w = synth.workload(1, Hq=Hq, Hkv=Hkv, r_k=r_k, r_v=r_v, T=600, layers=1)
+    layer, D, cache, oc, ws = _setup(w, seed=19, T_cap=16384, F_cap=4096)
+    gc, band = _compress_both(D, cache, oc, layer["K"], layer["V"], w.tau, ws)
+    out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
+    assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
+    Ka, Va = synth.decode_tokens(w, layer["Qk"], layer["Qv"], 1, 19, 0, DEV)
+    o2 = torch.empty(D.B, D.Hq, D.d, dtype=torch.float32, device=DEV)
+    L.lrkv_append_decode_attn(D, cache, Ka.contiguous(), Va.contiguous(), w.tau, layer["q"], o2, ws=ws)
+    O.compress(oc, U.f64(Ka), U.f64(Va), w.tau)
+    torch.cuda.synchronize()
+    gc = U.gpu_to_oracle(D, cache)
+    assert list(gc.seq_len) == [601] and gc.status == 0
+    assert U.out_rel_err(U.f64(o2), O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
+
+
 def test_degenerate_zero_rows_no_list_exact_fill():
     """All-zero key/value rows (e := 0, never routed), a key-only zero row, a
     cache with no full-rank list (F_cap = 0: every routed token overflows and

@@ -211,6 +211,40 @@ def test_span_inputs_are_exact():
     np.testing.assert_allclose(O.decode_attn(cache, q), ref, rtol=1e-12, atol=1e-13)
 
 
+def test_mixed_cache_equals_dense_attention():
+    """Both token sets at once, against a library routine: tokens whose K and V lie
+    in span(U) (U a signed column subset of I, so c and the reconstruction are exact
+    in bf16) stay compressed; the other tokens are off the span (error well above
+    tau) and go to the full-rank list.  The oracle's decode over that mixed cache
+    must be dense attention over the raw K, V -- a wrong joint softmax, a lost
+    full-rank row or a misplaced one would break it."""
+    rng = np.random.default_rng(18)
+    B, T, Hkv, Hq, d, r = 2, 77, 2, 8, 128, 32
+    cols = [rng.choice(d, r, replace=False) for _ in range(Hkv)]
+    U = np.zeros((Hkv, d, r))
+    for h in range(Hkv):
+        U[h, cols[h], np.arange(r)] = rng.choice([-1.0, 1.0], r)
+    K = O.bf16_round(rng.standard_normal((B, T, Hkv, d)))
+    V = O.bf16_round(rng.standard_normal((B, T, Hkv, d)))
+    in_span = rng.random((B, T, Hkv)) < 0.6
+    for b in range(B):
+        for h in range(Hkv):
+            off = np.setdiff1d(np.arange(d), cols[h])
+            for t in np.flatnonzero(in_span[b, :, h]):
+                K[b, t, h, off] = 0.0
+                V[b, t, h, off] = 0.0
+    q = O.bf16_round(rng.standard_normal((B, Hq, d)))
+    cache = _cache_from(K, V, U, U, tau=0.5, Hq=Hq)
+    for b in range(B):
+        for h in range(Hkv):
+            routed = cache.routed(b, h, np.arange(T))
+            assert np.array_equal(routed, ~in_span[b, :, h])
+            assert 0 < routed.sum() < T
+    ref = _sdpa(q, K.transpose(0, 2, 1, 3), V.transpose(0, 2, 1, 3), Hq // Hkv)
+    np.testing.assert_allclose(O.decode_attn(cache, q), ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(O.decode_attn_coef(cache, q), ref, rtol=1e-12, atol=1e-13)
+
+
 def test_negative_tau_routes_everything_and_attends_raw_rows():
     rng = np.random.default_rng(9)
     B, T, Hkv, Hq, d = 1, 50, 1, 4, 128
