@@ -52,7 +52,7 @@ class _Dims(ctypes.Structure):
 class _Cache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "U_k", "U_v", "coef_k", "coef_v", "route_mask", "full_idx", "full_k", "full_v",
-        "full_cnt", "seq_len", "dev_status")]
+        "full_cnt", "seq_len", "dev_status", "U_kq", "mu_k")]
 
 
 _lib = None
@@ -123,15 +123,20 @@ class LayerCache:
     full_cnt [B,Hkv], seq_len [B]; dev_status int32 [4] (word 0 used).
     """
     FIELDS = ("U_k", "U_v", "coef_k", "coef_v", "route_mask", "full_idx", "full_k", "full_v",
-              "full_cnt", "seq_len", "dev_status")
+              "full_cnt", "seq_len", "dev_status", "U_kq", "mu_k")
 
-    def __init__(self, dims, U_k, U_v, device="cuda"):
+    def __init__(self, dims, U_k, U_v, device="cuda", U_kq=None, mu_k=None):
         D = dims
         self.dims = D
         z = lambda *s, dt=torch.bfloat16: torch.zeros(*s, dtype=dt, device=device)
         self.U_k = U_k.to(device=device, dtype=torch.bfloat16).contiguous()
         self.U_v = U_v.to(device=device, dtype=torch.bfloat16).contiguous()
         assert tuple(self.U_k.shape) == (D.Hkv, D.d, D.r_k) and tuple(self.U_v.shape) == (D.Hkv, D.d, D.r_v)
+        # attention-aware key basis (optional): query-side basis and key mean
+        self.U_kq = None if U_kq is None else U_kq.to(device=device, dtype=torch.bfloat16).contiguous()
+        self.mu_k = None if mu_k is None else mu_k.to(device=device, dtype=torch.float32).contiguous()
+        assert self.U_kq is None or tuple(self.U_kq.shape) == (D.Hkv, D.d, D.r_k)
+        assert self.mu_k is None or tuple(self.mu_k.shape) == (D.Hkv, D.d)
         self.coef_k = z(D.B, D.Hkv, D.T_cap, D.r_k)
         self.coef_v = z(D.B, D.Hkv, D.T_cap, D.r_v)
         self.route_mask = z(D.B, D.Hkv, D.T_cap // 32, dt=torch.int32)
@@ -143,10 +148,12 @@ class LayerCache:
         self.dev_status = z(4, dt=torch.int32)
 
     def c(self):
-        return _Cache(*[getattr(self, f).data_ptr() for f in self.FIELDS])
+        return _Cache(*[None if getattr(self, f) is None else getattr(self, f).data_ptr()
+                        for f in self.FIELDS])
 
     def nbytes(self):
-        return sum(getattr(self, f).numel() * getattr(self, f).element_size() for f in self.FIELDS)
+        return sum(getattr(self, f).numel() * getattr(self, f).element_size() for f in self.FIELDS
+                   if getattr(self, f) is not None)
 
 
 def lrkv_rank_for_budget(eigvals, budget, check=True):

@@ -22,19 +22,23 @@ constexpr int kAppendThreads = 256;    // two halves of 128: keys and values sid
 constexpr int kAppendMaxTokens = 16;   // larger appends take the tiled path
 constexpr uint32_t kAppendWaitIters = 1u << 24;
 
-// Shared memory: U_k, U_v as stored (bf16 [d][r]) and the new tokens' key and
-// value rows (bf16 [kAppendMaxTokens][d] each), all filled by bulk copies; then
-// per half: x [d], partial c [4][d], c [d], reduction scratch; one mbarrier.
-inline size_t append_smem_bytes(int r_k, int r_v) {
-  return sizeof(uint16_t) * (size_t)kD * (r_k + r_v + 2 * kAppendMaxTokens) +
+// Shared memory: U_k, U_v as stored (bf16 [d][r]), the new tokens' key and
+// value rows (bf16 [kAppendMaxTokens][d] each) and, with an attention-aware key
+// basis, U_kq (bf16 [d][r_k]), all filled by bulk copies; then per half: x [d],
+// partial c [4][d], c [d], reduction scratch; one mbarrier.
+inline size_t append_smem_bytes(int r_k, int r_v, bool aware) {
+  return sizeof(uint16_t) * (size_t)kD * (r_k + r_v + 2 * kAppendMaxTokens + (aware ? r_k : 0)) +
          sizeof(float) * 2 * (6 * kD + 8) + 16;
 }
 
 // One tensor (the key for half 0, the value for half 1) of one token: x (bf16
-// [d] in shared memory) -> coefficients (bf16, global); returns the relative error
-// to every thread of the half.  All 256 threads call it together.
+// [d] in shared memory) -> coefficients c = Us^T (x - mu) (bf16, global);
+// returns the relative error ||x - mu - Urec c|| / ||x|| to every thread of the
+// half (Urec = Us and mu = null except for an attention-aware key basis).  All
+// 256 threads call it together.
 __device__ __forceinline__ float append_project(const uint16_t* __restrict__ x_s,
-                                                const uint16_t* Us, int r,
+                                                const uint16_t* Us, const uint16_t* Urec,
+                                                const float* mu, int r,
                                                 lrkv_bf16* __restrict__ coef_g, float* ws) {
   const int tid = threadIdx.x & 127;
   const int warp = tid >> 5, lane = tid & 31;
@@ -42,7 +46,8 @@ __device__ __forceinline__ float append_project(const uint16_t* __restrict__ x_s
   float* part = xs + kD;          // [4][d]
   float* cs = part + 4 * kD;      // [d]
   float* red = cs + kD;           // [8]
-  const float x = bf2f(x_s[tid]);
+  const float xraw = bf2f(x_s[tid]);
+  const float x = mu ? xraw - mu[tid] : xraw;
   xs[tid] = x;
   __syncthreads();
   // c_j = sum_i U[i][j] x_i: warp w sums rows 32w..32w+31, lane owns columns lane + 32k
@@ -70,7 +75,7 @@ __device__ __forceinline__ float append_project(const uint16_t* __restrict__ x_s
   // x_hat_i = sum_j U[i][j] c_j: thread i walks row i two columns at a time,
   // starting at column pair (i mod r/2), so a warp's 32 rows hit 32 banks.
   const int npair = r >> 1;
-  const uint32_t* row = reinterpret_cast<const uint32_t*>(Us) + tid * npair;
+  const uint32_t* row = reinterpret_cast<const uint32_t*>(Urec) + tid * npair;
   const float2* c2 = reinterpret_cast<const float2*>(cs);
   float h0 = 0.f, h1 = 0.f;
   int w = tid % npair;
@@ -83,7 +88,7 @@ __device__ __forceinline__ float append_project(const uint16_t* __restrict__ x_s
     w = (w + 1 == npair) ? 0 : w + 1;
   }
   const float dlt = x - (h0 + h1);
-  const float rs = warp_sum(dlt * dlt), ns = warp_sum(x * x);
+  const float rs = warp_sum(dlt * dlt), ns = warp_sum(xraw * xraw);
   if (lane == 0) red[warp] = rs, red[4 + warp] = ns;
   __syncthreads();
   const float rsum = (red[0] + red[1]) + (red[2] + red[3]);
@@ -101,7 +106,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
   uint16_t* Uvs = Uks + kD * r_k;
   uint16_t* Xks = Uvs + kD * r_v;                          // new key rows
   uint16_t* Xvs = Xks + kD * kAppendMaxTokens;             // new value rows
-  float* ws0 = reinterpret_cast<float*>(Xvs + kD * kAppendMaxTokens);   // per-half scratch
+  const bool aware = p.C.U_kq != nullptr;
+  uint16_t* Ukqs = Xvs + kD * kAppendMaxTokens;            // query-side key basis (aware only)
+  float* ws0 = reinterpret_cast<float*>(Ukqs + (aware ? kD * r_k : 0));   // per-half scratch
   const int half = tid >> 7;
   float* ws = ws0 + half * (6 * kD + 8);
   uint64_t* bar = reinterpret_cast<uint64_t*>(ws0 + 2 * (6 * kD + 8));
@@ -114,9 +121,10 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
     mbar_init(bar, 1);
     fence_mbar_init();
     const uint32_t bk = kD * r_k * 2, bv = kD * r_v * 2;
-    mbar_expect_tx(bar, bk + bv);
+    mbar_expect_tx(bar, bk + bv + (aware ? bk : 0));
     bulk_g2s(Uks, p.C.U_k + (size_t)h * kD * r_k, bk, bar);
     bulk_g2s(Uvs, p.C.U_v + (size_t)h * kD * r_v, bv, bar);
+    if (aware) bulk_g2s(Ukqs, p.C.U_kq + (size_t)h * kD * r_k, bk, bar);
   }
   griddep_launch_dependents();
   griddep_wait();   // the new rows and the cache state come from earlier kernels
@@ -175,7 +183,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
       const size_t row = bh * D.T_cap + pos;
       // one call site for both halves: every __syncthreads inside is reached by all threads
       const float eh = append_project(half == 0 ? Xks + t * kD : Xvs + t * kD,
-                                      half == 0 ? Uks : Uvs, half == 0 ? r_k : r_v,
+                                      half == 0 ? Uks : Uvs, half == 0 ? (aware ? Ukqs : Uks) : Uvs,
+                                      half == 0 && p.C.mu_k ? p.C.mu_k + (size_t)h * kD : nullptr,
+                                      half == 0 ? r_k : r_v,
                                       half == 0 ? p.C.coef_k + row * r_k : p.C.coef_v + row * r_v,
                                       ws);
       if ((tid & 127) == 0) s_err[half] = eh;

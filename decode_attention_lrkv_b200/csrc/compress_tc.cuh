@@ -63,11 +63,13 @@ constexpr size_t kSmemLimit = 227 * 1024;
 // tensors share one layout) and ns input stages; operand regions 1024-aligned.
 //   X stages [ns][128][128] (128-byte swizzle), P_hi [128][128] directly
 //   followed by U^T [rm][128] (rows 128.. of the merged B operand),
-//   P_lo [128][128], mbarriers, group B's per-row sums [2][128].
+//   P_lo [128][128], mbarriers, group B's per-row sums [2][128], the key
+//   mean's constants [2][128] (U^T mu and P mu, attention-aware keys only).
 // U [128][rm] for U U^T is needed only before the first tile: it borrows the
-// last input stage.
+// last input stage; the query-side key basis U_q of an attention-aware key
+// basis (P = I - U_q U^T) borrows the one before.
 struct Layout {
-  int x, phi, plo, ut, u, bar, part;
+  int x, phi, plo, ut, u, uq, bar, part, mu;
   size_t bytes;
   __host__ __device__ Layout(int rm, int ns) {
     x = 0;
@@ -75,9 +77,11 @@ struct Layout {
     ut = phi + kD * kD * 2;
     plo = ut + rm * kD * 2;
     u = (ns - 1) * kStageBytes;
+    uq = (ns - 2) * kStageBytes;
     bar = plo + kD * kD * 2;
     part = bar + 128;
-    bytes = (size_t)part + 2 * kTile * 8 + 1024;   // + slack to align the base to 1024
+    mu = part + 2 * kTile * 8;
+    bytes = (size_t)mu + 2 * kD * 4 + 1024;   // + slack to align the base to 1024
   }
 };
 static_assert(kD * 128 * 2 <= kStageBytes, "U fits in one input stage");
@@ -159,6 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   const int NS = p.n_stages;
   const Layout Lo(p.r_max, NS);
   const lrkv_bf16* Ug = (tensor == 0 ? p.C.U_k : p.C.U_v) + (size_t)h * kD * R;
+  // attention-aware keys: the query-side basis reconstructs, the mean is subtracted
+  const lrkv_bf16* Uqg = tensor == 0 && p.C.U_kq ? p.C.U_kq + (size_t)h * kD * R : nullptr;
+  const float* mug = tensor == 0 && p.C.mu_k ? p.C.mu_k + (size_t)h * kD : nullptr;
   lrkv_bf16* coef = tensor == 0 ? p.C.coef_k : p.C.coef_v;
   float* errs = p.errs + (size_t)tensor * D.B * D.Hkv * D.T_cap;
 
@@ -227,6 +234,22 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
         }
       }
     }
+    if (Uqg) {   // the query-side key basis, in U's layout (the A operand of U_q U^T)
+      const uint4* uq = reinterpret_cast<const uint4*>(Uqg);
+#pragma unroll
+      for (int k = 0; k < kMaxPieces; ++k) {
+        const int c = tid + k * kThreads;
+        if (c < n_pieces) piece[k] = uq[c];
+      }
+#pragma unroll
+      for (int k = 0; k < kMaxPieces; ++k) {
+        const int c = tid + k * kThreads;
+        if (c < n_pieces) {
+          const int i = (c * 8) / R, j0 = c * 8 - i * R;
+          *reinterpret_cast<uint4*>(sm + Lo.uq + core_off(i, j0, 16 * R)) = piece[k];
+        }
+      }
+    }
   }
   fence_proxy_async_smem();
   tc5::fence_before_sync();
@@ -234,14 +257,35 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   tc5::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  // ---- P = I - U U^T, split into bf16 high and low parts ----------------------------
+  // ---- P = I - U_q U^T (U_q = U unless an attention-aware key basis is given),
+  // split into bf16 high and low parts -----------------------------------------------
   if (warp == kMmaWarp && lane == 0) {
     const uint32_t ub = smem_u32(sm + Lo.u);
+    const uint32_t uqb = smem_u32(sm + (Uqg ? Lo.uq : Lo.u));
     for (int j = 0; j < R / 16; ++j) {
-      const uint64_t d = tc5::smem_desc(ub + j * 256, 128, 16 * R, tc5::kSwizzleNone);
-      tc5::mma_bf16(tmem + 128, d, d, tc5::idesc_bf16_f32(128, 128), j > 0);
+      const uint64_t db = tc5::smem_desc(ub + j * 256, 128, 16 * R, tc5::kSwizzleNone);
+      const uint64_t da = tc5::smem_desc(uqb + j * 256, 128, 16 * R, tc5::kSwizzleNone);
+      tc5::mma_bf16(tmem + 128, da, db, tc5::idesc_bf16_f32(128, 128), j > 0);
     }
     tc5::mma_commit(pready);
+  }
+  // attention-aware keys with a mean: the per-column constants U^T mu (from the
+  // coefficients) and P mu = mu - U_q U^T mu (from the residual vectors)
+  float* cmu = reinterpret_cast<float*>(sm + Lo.mu);   // [128]: U^T mu, columns < R
+  float* rmu = cmu + kD;                               // [128]: P mu
+  if (mug && warp < 8) {
+    if (tid < R) {
+      float a = 0.f;
+      for (int i = 0; i < kD; ++i) a = fmaf(bf2f(Ug[i * R + tid]), mug[i], a);
+      cmu[tid] = a;
+    }
+    tc5::named_bar_sync(1, kEpi);
+    if (tid < kD) {
+      const lrkv_bf16* uq = Uqg ? Uqg : Ug;
+      float a = 0.f;
+      for (int j = 0; j < R; ++j) a = fmaf(bf2f(uq[tid * R + j]), cmu[j], a);
+      rmu[tid] = mug[tid] - a;
+    }
   }
   if (warp < 8) {
     // row m of U U^T = TMEM lane m; warps w and w + 4 share the rows, columns split
@@ -376,6 +420,12 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
           for (int q = 0; q < 4; ++q)
             if (c0 + 16 * q < R) tc5::tmem_ld16(d1 + c0 + 16 * q, v[q]);
           tc5::tmem_wait_ld();
+          if (mug) {   // c = U^T x - U^T mu
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+              for (int k = 0; k < 16; ++k) v[q][k] -= cmu[(c0 + 16 * q + k) & (kD - 1)];
+          }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             if (valid && c0 + 16 * q < R) {
@@ -395,6 +445,12 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
 #pragma unroll
         for (int q = 0; q < 4; ++q) tc5::tmem_ld16(d2 + (grp_a ? 0 : 64) + 16 * q, v[q]);
         tc5::tmem_wait_ld();
+        if (mug) {   // residual P (x - mu) = P x - P mu
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[q][k] -= rmu[(grp_a ? 0 : 64) + 16 * q + k];
+        }
         float r0 = 0.f, r1 = 0.f;
 #pragma unroll
         for (int q = 0; q < 4; ++q)

@@ -49,9 +49,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(DecodeParams
   const size_t bh = (size_t)b * D.Hkv + h;
 
   float* qs = sm;                  // [G][d]  q * log2(e)/sqrt(d)
-  float* qt = qs + G * kD;         // [G][d]  U_k^T q * log2(e)/sqrt(d)  (r_k used)
+  float* qt = qs + G * kD;         // [G][d]  U_kq^T q * log2(e)/sqrt(d)  (r_k used)
   float* ws = qt + G * kD;         // per-warp state
   float* wts = ws + kDecWarps * G * (2 + 2 * kD);
+  __shared__ float s_bias[G];      // q . mu_k * log2(e)/sqrt(d): added to compressed logits
   const float scale = kLog2e * rsqrtf((float)kD);
 
   for (int o = tid; o < G * kD; o += kDecThreads) {
@@ -59,12 +60,20 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(DecodeParams
     qs[o] = bf2f(p.q[((size_t)b * D.Hq + h * G + gi) * kD + i]) * scale;
   }
   __syncthreads();
-  const lrkv_bf16* Uk = p.C.U_k + (size_t)h * kD * r_k;
+  // q~ in the query-side key basis (U_k unless an attention-aware U_kq is given)
+  const lrkv_bf16* Uk = (p.C.U_kq ? p.C.U_kq : p.C.U_k) + (size_t)h * kD * r_k;
   for (int o = tid; o < G * r_k; o += kDecThreads) {
     const int gi = o / r_k, j = o % r_k;
     float acc = 0.f;
     for (int i = 0; i < kD; ++i) acc = fmaf(bf2f(Uk[i * r_k + j]), qs[gi * kD + i], acc);
     qt[gi * kD + j] = acc;
+  }
+  if (warp < G) {
+    float s = 0.f;
+    if (p.C.mu_k)
+      for (int i = lane; i < kD; i += 32) s = fmaf(qs[warp * kD + i], p.C.mu_k[(size_t)h * kD + i], s);
+    s = warp_sum(s);
+    if (lane == 0) s_bias[warp] = s;
   }
   __syncthreads();
 
@@ -100,7 +109,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(DecodeParams
         const int j = lane + 32 * k;
         if (j < r_k) s = fmaf(qt[gi * kD + j], kv[k], s);
       }
-      s = warp_sum(s);
+      s = warp_sum(s) + s_bias[gi];
       const float mn = fmaxf(m[gi], s);
       const float sc = exp2f(m[gi] - mn);
       const float pr = exp2f(s - mn);

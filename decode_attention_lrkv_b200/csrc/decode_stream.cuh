@@ -86,8 +86,11 @@ struct Shape {
   static constexpr int OFF_UV = RING + MASK_BYTES;
   static constexpr int SMEM = OFF_UV + kD * VS;
   static_assert(SMEM <= SMEM_MAX, "shared memory of one CTA");
-  // U_k rows [d][KS] live in the last stage until every warp has its q~
+  // U_k rows [d][KS] (the query-side basis U_kq when the cache has one) live in
+  // the last stage until every warp has its q~; with an attention-aware key
+  // basis the fused append also needs the key-side U_k: second copy behind it
   static constexpr int OFF_UK = (NS - 1) * W * SLOT;
+  static constexpr int OFF_UK2 = OFF_UK + al16(kD * KS);
   static_assert(kD * KS <= W * SLOT, "U_k fits in one stage");
   // per-warp partial state in the warp's stage-0 slot (floats)
   static constexpr int W_PF = 0;                    // [G][d]
@@ -97,13 +100,14 @@ struct Shape {
   // record of one split per query head: m, l, flag, pad, o[d] = U_v acc_c + acc_f
   // (flag, head 0 only: the split appended a full-rank row, fused append)
   static constexpr int REC = 4 + kD;
-  // fused append scratch behind U_k in the last stage (untouched until the
-  // stream's first refill), floats: c_k [RK], c_v [RV], q~ (scaled) [G][RK],
-  // x [2][d] (key, value), sums [16]
-  static constexpr int OFF_APP = OFF_UK + al16(kD * KS);
+  // fused append scratch behind the two key bases in the last stage (untouched
+  // until the stream's first refill), floats: c_k [RK], c_v [RV], q~ (scaled)
+  // [G][RK], x [2][d] (key, value), the key minus its mean [d], sums [24]
+  static constexpr int OFF_APP = OFF_UK2 + al16(kD * KS);
   static constexpr int A_CK = 0, A_CV = RK, A_QT = RK + RV, A_X = A_QT + G * RK,
-                       A_RED = A_X + 2 * kD, A_FLOATS = A_RED + 24;
-  static_assert(al16(kD * KS) + A_FLOATS * 4 <= W * SLOT, "U_k and the append scratch fit in a stage");
+                       A_XC = A_X + 2 * kD, A_RED = A_XC + kD, A_FLOATS = A_RED + 24;
+  static_assert(2 * al16(kD * KS) + A_FLOATS * 4 <= W * SLOT,
+                "both key bases and the append scratch fit in a stage");
 };
 
 // The owner CTA's share of a fused decode-time append: one new token of row b,
@@ -118,7 +122,8 @@ struct Shape {
 //   its value row (v, or bf16(c_v)) for the fold after the stream.
 template <typename S, int G, int RK, int RV>
 __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
-                                             const unsigned char* uk, const unsigned char* uv,
+                                             const unsigned char* uk, const unsigned char* ukq,
+                                             const unsigned char* uv, const float* s_bias,
                                              int b, int h, size_t bh, int pos, int F, float scale,
                                              uint16_t xe, float* s_new, float* s_vals, int* s_keep) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -126,29 +131,50 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
   const lrkv_dims& D = p.D;
   constexpr int KST = RK / 16, MVT = RV / 16;
   app[S::A_X + tid] = bf2f(xe);   // new key (threads < d) and value (threads >= d) rows
-  __syncthreads();                // x and q~ in; U_k and U_v in since the prologue
-  // c = U^T x on the tensor cores, x as row 8 of the A operand: warp w forms
-  // columns [16w, 16w + 16) of c_k (w < r_k / 16) and of c_v (w < r_v / 16)
-  auto coef_block = [&](const unsigned char* U, int stride, const float* x, float* cdst) {
+  // the key as projected: minus the key mean of an attention-aware basis
+  if (tid < kD) app[S::A_XC + tid] = bf2f(xe) - (p.C.mu_k ? p.C.mu_k[(size_t)h * kD + tid] : 0.f);
+  __syncthreads();                // x and q~ in; the bases in since the prologue
+  // c = U^T (x - mu) on the tensor cores: x (bf16, exact) is row 8 of the A
+  // operand; a key mean (fp32) enters as its bf16 high and low parts in rows 9
+  // and 10, so U^T mu is fp32-accurate and c = row 8 - (row 9 + row 10).  Warp
+  // w forms columns [16w, 16w + 16) of c_k (w < r_k / 16) and of c_v (w < r_v / 16).
+  auto coef_block = [&](const unsigned char* U, int stride, const float* x, const float* mu,
+                        float* cdst) {
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t x0 = g == 0 ? pack_bf16(x[ks * 16 + 2 * t], x[ks * 16 + 2 * t + 1]) : 0u;
-      const uint32_t x1 = g == 0 ? pack_bf16(x[ks * 16 + 8 + 2 * t], x[ks * 16 + 9 + 2 * t]) : 0u;
+      const int i0 = ks * 16 + 2 * t, i1 = i0 + 8;
+      uint32_t x0 = 0u, x1 = 0u;
+      if (g == 0) {
+        x0 = pack_bf16(x[i0], x[i0 + 1]);
+        x1 = pack_bf16(x[i1], x[i1 + 1]);
+      } else if (mu && g <= 2) {
+        const bool lo = g == 2;
+        x0 = pack_bf16(bf16_part(mu[i0], lo), bf16_part(mu[i0 + 1], lo));
+        x1 = pack_bf16(bf16_part(mu[i1], lo), bf16_part(mu[i1 + 1], lo));
+      }
       uint32_t b0, b1, b2, b3;
       ldsm_x4_t(b0, b1, b2, b3, U + (ks * 16 + (lm & 1) * 8 + lr) * stride + (16 * warp + (lm >> 1) * 8) * 2);
       mma_16816(a0, 0u, x0, 0u, x1, b0, b1);
       mma_16816(a1, 0u, x0, 0u, x1, b2, b3);
     }
+    float m[4] = {0.f, 0.f, 0.f, 0.f};   // U^T mu: rows 9 and 10, from lanes 4 + t and 8 + t
+    if (mu) {
+      const float v[4] = {a0[2], a0[3], a1[2], a1[3]};
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        m[e] = __shfl_sync(kFull, v[e], (lane + 4) & 31) + __shfl_sync(kFull, v[e], (lane + 8) & 31);
+    }
     if (g == 0) {
-      cdst[16 * warp + 2 * t] = a0[2];
-      cdst[16 * warp + 2 * t + 1] = a0[3];
-      cdst[16 * warp + 8 + 2 * t] = a1[2];
-      cdst[16 * warp + 8 + 2 * t + 1] = a1[3];
+      cdst[16 * warp + 2 * t] = a0[2] - m[0];
+      cdst[16 * warp + 2 * t + 1] = a0[3] - m[1];
+      cdst[16 * warp + 8 + 2 * t] = a1[2] - m[2];
+      cdst[16 * warp + 8 + 2 * t + 1] = a1[3] - m[3];
     }
   };
-  if (warp < KST) coef_block(uk, S::KS, app + S::A_X, app + S::A_CK);
-  if (warp < MVT) coef_block(uv, S::VS, app + S::A_X + kD, app + S::A_CV);
+  const float* mu_h = p.C.mu_k ? p.C.mu_k + (size_t)h * kD : nullptr;
+  if (warp < KST) coef_block(uk, S::KS, app + S::A_X, mu_h, app + S::A_CK);
+  if (warp < MVT) coef_block(uv, S::VS, app + S::A_X + kD, nullptr, app + S::A_CV);
   __syncthreads();
   // direct reconstruction x_hat = U c on the tensor cores: A = U's rows
   // [16w, 16w + 16) (warp w, keys then values), B = c split into bf16 high
@@ -174,7 +200,7 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
     return warp_sum(rr);
   };
   {
-    const float rk = recon_sq(uk, S::KS, RK, app + S::A_CK, app + S::A_X);
+    const float rk = recon_sq(ukq, S::KS, RK, app + S::A_CK, app + S::A_XC);
     const float rv = recon_sq(uv, S::VS, RV, app + S::A_CV, app + S::A_X + kD);
     const float x = app[S::A_X + tid];
     const float ns = warp_sum(x * x);   // warps < 4: the key's squares, else the value's
@@ -220,9 +246,9 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
       const uint16_t* qrow = reinterpret_cast<const uint16_t*>(p.q) + ((size_t)b * D.Hq + (size_t)h * G + warp) * kD;
       for (int i = lane; i < kD; i += 32) sd = fmaf(bf2f(qrow[i]), app[S::A_X + i], sd);
       sd = warp_sum(sd) * scale;
-    } else {        // compressed: q~ . bf16(c_k), q~ already scaled
+    } else {        // compressed: q . mu_k + q~ . bf16(c_k), both already scaled
       for (int j = lane; j < RK; j += 32) sd = fmaf(app[S::A_QT + warp * RK + j], bf2f(f2bf(app[S::A_CK + j])), sd);
-      sd = warp_sum(sd);
+      sd = warp_sum(sd) + s_bias[warp];
     }
     if (lane == 0) s_new[warp] = sd;
   }
@@ -256,12 +282,18 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   __shared__ int s_last;
 
   // ---- prologue, independent of the preceding kernel: the bases ------------------
-  {  // U_k into padded rows, 16-byte pieces over every thread
-    const unsigned char* Uk = reinterpret_cast<const unsigned char*>(p.C.U_k + (size_t)h * kD * RK);
-    for (int q = tid; q < kD * KP; q += kThreads) {
-      const int r = q / KP, sg = q - r * KP;
-      cp_async16(uk + r * S::KS + sg * 16, Uk + q * 16);
-    }
+  {  // U_k into padded rows, 16-byte pieces over every thread: the query-side
+     // basis for q~ (U_kq when given), and the key-side basis for the fused
+     // append when it differs
+    auto load_uk = [&](const lrkv_bf16* src, unsigned char* dst) {
+      const unsigned char* Uk = reinterpret_cast<const unsigned char*>(src + (size_t)h * kD * RK);
+      for (int q = tid; q < kD * KP; q += kThreads) {
+        const int r = q / KP, sg = q - r * KP;
+        cp_async16(dst + r * S::KS + sg * 16, Uk + q * 16);
+      }
+    };
+    load_uk(p.C.U_kq ? p.C.U_kq : p.C.U_k, uk);
+    if (APP && p.C.U_kq) load_uk(p.C.U_k, sm + S::OFF_UK2);
     cp_async_commit();
   }
   auto load_uv = [&]() {   // U_v into padded rows, 16-byte pieces over every thread
@@ -338,73 +370,11 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     mw[u] = active && wl < chunk / 32 && wi < D.T_cap / 32 ? p.C.route_mask[bh * (D.T_cap / 32) + wi] : 0u;
   }
 
-  const float scale = kLog2e * rsqrtf((float)kD);
-  // q~ = U_k^T q as B fragments over k = r_k (column n = 2h + part: the bf16
-  // high or low part of head h), on the tensor cores: warp w < r_k / 16 forms
-  // columns [16w, 16w + 16) and leaves its fragments in shared memory for all
-  static_assert(KST <= kWarps, "one block of q~ columns per warp");
-  __shared__ uint32_t s_qb[KST][2][32];
-  float* app = reinterpret_cast<float*>(sm + S::OFF_APP);   // fused append scratch
-  cp_async_wait<1>();   // U_k in (U_v may still be in flight)
-  __syncthreads();
-  if (active && warp < KST) {
-    const int ks2 = warp;                      // columns [16 ks2, 16 ks2 + 16) of q~
-    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(b0, b1, b2, b3, uk + (ks * 16 + (lm & 1) * 8 + lr) * S::KS + (16 * ks2 + (lm >> 1) * 8) * 2);
-      mma_16816(a0, qa0[ks], 0u, qa1[ks], 0u, b0, b1);
-      mma_16816(a1, qa0[ks], 0u, qa1[ks], 0u, b2, b3);
-    }
-    if constexpr (APP) {
-      if (g < G) {    // q~ rows (scaled), for the new token's logit if it stays compressed
-        float* qt = app + S::A_QT + g * RK + 16 * ks2;
-        qt[2 * t] = a0[0] * scale;
-        qt[2 * t + 1] = a0[1] * scale;
-        qt[8 + 2 * t] = a1[0] * scale;
-        qt[8 + 2 * t + 1] = a1[1] * scale;
-      }
-    }
-    // lane (m, t) holds q~[head m][16 ks2 + 2t (+1)] in a0 and [+8] in a1 (rows m < 4).
-    // B column g = 2h + part takes head h from lane 4h + t.
-    const int src = ((g >> 1) << 2) | t;
-    const float x0 = __shfl_sync(kFull, a0[0], src), x1 = __shfl_sync(kFull, a0[1], src);
-    const float y0 = __shfl_sync(kFull, a1[0], src), y1 = __shfl_sync(kFull, a1[1], src);
-    const bool lo_n = g & 1;
-    const bool live = (g >> 1) < G;
-    s_qb[ks2][0][lane] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
-    s_qb[ks2][1][lane] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
-  }
-  const bool owner = APP && n_eff > 0 && c == n_chunks - 1;
-  // Every thread of this CTA has read seq_len[b] (the barrier above): each CTA
-  // takes the row's ticket once (release only) and looks at it later; the last
-  // CTA of the grid for row b advances its length.
-  int seq_ticket = 0;
-  auto advance_len = [&]() {
-    if (seq_ticket == D.Hkv * (int)gridDim.x - 1) {
-      fence_acq_rel_gpu();
-      p.C.seq_len[b] = T;
-      p.seq_tickets[b] = 0;
-    }
-  };
-  const int tk = kThreads - 32;   // the thread that takes it: lane 0 of the last warp
-  if constexpr (APP) {
-    if (tid == 0 && h == 0 && c == 0 && st_new) atomicOr(p.C.dev_status, st_new);
-  }
-  cp_async_wait<0>();   // U_v (in flight since the prologue): none left behind on exit
-  if (!active) {
-    if (APP && tid == tk) {
-      seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
-      advance_len();
-    }
-    return;
-  }
-#pragma unroll
-  for (int u = 0; u < kMW; ++u)
-    if (tid + u * kThreads < kMaxChunk / 32) maskw[tid + u * kThreads] = mw[u];
+  // ---- this warp's tiles; the first ones are issued before the mask words and
+  // the query projection, so their copies overlap both ------------------------------
   const int c1 = min(T_old, c0 + chunk);   // the new position is not read from the cache
-  const int n_pos = c1 > c0 ? c1 - c0 : 0;
+  const int n_pos = active && c1 > c0 ? c1 - c0 : 0;
+  // this split's share of the full-rank list
   const int F = min(max(F_raw, 0), D.F_cap);
   const int share = (F + n_chunks - 1) / n_chunks;
   const int f0 = min(F, c * share), f1 = min(F, f0 + share);
@@ -413,15 +383,6 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   const lrkv_bf16* cv = p.C.coef_v + bh * D.T_cap * RV + (size_t)c0 * RV;
   const lrkv_bf16* fk = p.C.full_k + (bh * D.F_cap + f0) * kD;
   const lrkv_bf16* fv = p.C.full_v + (bh * D.F_cap + f0) * kD;
-  // the new token for the fold after the stream: its logit per head, whether
-  // it went to the full-rank list, and its value row (v, or c_v as stored)
-  __shared__ float s_new[G];
-  __shared__ float s_vals[kD];
-  __shared__ int s_keep;
-  __syncthreads();   // mask words, U_v and q~ in; every warp is done with U_k (the last stage is free)
-  uint32_t qb0[KST], qb1[KST];
-#pragma unroll
-  for (int ks2 = 0; ks2 < KST; ++ks2) qb0[ks2] = s_qb[ks2][0][lane], qb1[ks2] = s_qb[ks2][1][lane];
 
   // this warp's tiles: every kWarps-th compressed tile and every kWarps-th full-rank tile
   const int n_ct = (n_pos + kTileC - 1) / kTileC;
@@ -450,18 +411,22 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   };
   Walk wi_copy{0, 0, 0}, wi_comp{0, 0, 0};
 
-  // positions of compressed tile k that are read: unmasked and before the end
-  auto tile_bits = [&](int k) -> uint32_t {
+  // positions of compressed tile k before the end, and those of them that are
+  // read: unmasked (compressed) too
+  auto valid_bits = [&](int k) -> uint32_t {
     const int nv = n_pos - k * kTileC;
-    const uint32_t valid = nv >= 32 ? kFull : ((1u << nv) - 1u);
-    return ~maskw[k] & valid;
+    return nv >= 32 ? kFull : ((1u << nv) - 1u);
   };
-  auto issue = [&](int i) {
+  auto tile_bits = [&](int k) -> uint32_t { return ~maskw[k] & valid_bits(k); };
+  // masked: skip routed positions (zero-filled, not read).  The prologue's tiles
+  // go out before the mask words have arrived and copy every valid row: the
+  // routed ones hold finite coefficients too and their logits are -inf.
+  auto issue = [&](int i, bool masked) {
     unsigned char* slot = slot_of(i % NST, warp);
     int kw;
     if (wi_copy.next(nct_w, n_tiles, kw)) {
       const int k = warp + kWarps * kw;
-      const uint32_t bits = tile_bits(k);
+      const uint32_t bits = masked ? tile_bits(k) : valid_bits(k);
       const unsigned char* src_k = reinterpret_cast<const unsigned char*>(ck + (size_t)k * kTileC * RK);
       const unsigned char* src_v = reinterpret_cast<const unsigned char*>(cv + (size_t)k * kTileC * RV);
 #pragma unroll
@@ -497,16 +462,106 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   };
 #pragma unroll
   for (int s = 0; s < NST - 1; ++s) {
-    if (s < n_tiles) issue(s);
+    if (active && s < n_tiles) issue(s, false);
     cp_async_commit();
   }
+
+  const float scale = kLog2e * rsqrtf((float)kD);
+  // q~ = U_k^T q as B fragments over k = r_k (column n = 2h + part: the bf16
+  // high or low part of head h), on the tensor cores: warp w < r_k / 16 forms
+  // columns [16w, 16w + 16) and leaves its fragments in shared memory for all
+  static_assert(KST <= kWarps, "one block of q~ columns per warp");
+  __shared__ uint32_t s_qb[KST][2][32];
+  float* app = reinterpret_cast<float*>(sm + S::OFF_APP);   // fused append scratch
+  cp_async_wait<NST>();   // U_k in (U_v and the prologue's tiles may still be in flight)
+  __syncthreads();
+  if (active && warp < KST) {
+    const int ks2 = warp;                      // columns [16 ks2, 16 ks2 + 16) of q~
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(b0, b1, b2, b3, uk + (ks * 16 + (lm & 1) * 8 + lr) * S::KS + (16 * ks2 + (lm >> 1) * 8) * 2);
+      mma_16816(a0, qa0[ks], 0u, qa1[ks], 0u, b0, b1);
+      mma_16816(a1, qa0[ks], 0u, qa1[ks], 0u, b2, b3);
+    }
+    if constexpr (APP) {
+      if (g < G) {    // q~ rows (scaled), for the new token's logit if it stays compressed
+        float* qt = app + S::A_QT + g * RK + 16 * ks2;
+        qt[2 * t] = a0[0] * scale;
+        qt[2 * t + 1] = a0[1] * scale;
+        qt[8 + 2 * t] = a1[0] * scale;
+        qt[8 + 2 * t + 1] = a1[1] * scale;
+      }
+    }
+    // lane (m, t) holds q~[head m][16 ks2 + 2t (+1)] in a0 and [+8] in a1 (rows m < 4).
+    // B column g = 2h + part takes head h from lane 4h + t.
+    const int src = ((g >> 1) << 2) | t;
+    const float x0 = __shfl_sync(kFull, a0[0], src), x1 = __shfl_sync(kFull, a0[1], src);
+    const float y0 = __shfl_sync(kFull, a1[0], src), y1 = __shfl_sync(kFull, a1[1], src);
+    const bool lo_n = g & 1;
+    const bool live = (g >> 1) < G;
+    s_qb[ks2][0][lane] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
+    s_qb[ks2][1][lane] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
+  }
+  // q . mu_k per query head (scaled), added to every compressed logit: 0 unless
+  // the cache has an attention-aware key basis with a mean
+  __shared__ float s_bias[G];
+  if (warp >= kWarps - G) {
+    const int gi = warp - (kWarps - G);
+    float sb = 0.f;
+    if (p.C.mu_k) {
+      const lrkv_bf16* qrow = p.q + ((size_t)b * D.Hq + (size_t)h * G + gi) * kD;
+      for (int i = lane; i < kD; i += 32) sb = fmaf(bf2f(qrow[i]), p.C.mu_k[(size_t)h * kD + i], sb);
+    }
+    sb = warp_sum(sb);
+    if (lane == 0) s_bias[gi] = sb * scale;
+  }
+  const bool owner = APP && n_eff > 0 && c == n_chunks - 1;
+  // Every thread of this CTA has read seq_len[b] (the barrier above): each CTA
+  // takes the row's ticket once (release only) and looks at it later; the last
+  // CTA of the grid for row b advances its length.
+  int seq_ticket = 0;
+  auto advance_len = [&]() {
+    if (seq_ticket == D.Hkv * (int)gridDim.x - 1) {
+      fence_acq_rel_gpu();
+      p.C.seq_len[b] = T;
+      p.seq_tickets[b] = 0;
+    }
+  };
+  const int tk = kThreads - 32;   // the thread that takes it: lane 0 of the last warp
+  if constexpr (APP) {
+    if (tid == 0 && h == 0 && c == 0 && st_new) atomicOr(p.C.dev_status, st_new);
+  }
+  if (!active) {
+    cp_async_wait<0>();   // U_v (in flight since the prologue): none left behind on exit
+    if (APP && tid == tk) {
+      seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
+      advance_len();
+    }
+    return;
+  }
+#pragma unroll
+  for (int u = 0; u < kMW; ++u)
+    if (tid + u * kThreads < kMaxChunk / 32) maskw[tid + u * kThreads] = mw[u];
+  cp_async_wait<NST - 1>();   // U_v in (only the prologue's tiles may be in flight)
+  // the new token for the fold after the stream: its logit per head, whether
+  // it went to the full-rank list, and its value row (v, or c_v as stored)
+  __shared__ float s_new[G];
+  __shared__ float s_vals[kD];
+  __shared__ int s_keep;
+  __syncthreads();   // mask words, U_v and q~ in; every warp is done with U_k (the last stage is free)
+  uint32_t qb0[KST], qb1[KST];
+#pragma unroll
+  for (int ks2 = 0; ks2 < KST; ++ks2) qb0[ks2] = s_qb[ks2][0][lane], qb1[ks2] = s_qb[ks2][1][lane];
+  const float bias = live_t ? s_bias[t] : 0.f;   // this lane's head
   // the owner of a fused append does it while its first tiles are in flight
   // (U_k and the scratch sit in the last stage, which the stream refills only
   // from its first step on)
   if constexpr (APP) {
     if (owner) {
-      append_token<S, G, RK, RV>(p, app, uk, sm + S::OFF_UV, b, h, bh, T_old, F, scale, xe,
-                                 s_new, s_vals, &s_keep);
+      append_token<S, G, RK, RV>(p, app, p.C.U_kq ? sm + S::OFF_UK2 : uk, uk, sm + S::OFF_UV, s_bias,
+                                 b, h, bh, T_old, F, scale, xe, s_new, s_vals, &s_keep);
       __syncthreads();   // the token's logits and value row in for warp 0
     }
   }
@@ -561,7 +616,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   };
 
   for (int i = 0; i < n_tiles; ++i) {
-    if (i + NST - 1 < n_tiles) issue(i + NST - 1);
+    if (i + NST - 1 < n_tiles) issue(i + NST - 1, true);
     cp_async_commit();
     cp_async_wait<NST - 1>();
     __syncwarp();
@@ -587,7 +642,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
         for (int x = 0; x < 2; ++x) {   // rows g, g + 8: high + low part of head t
-          const float v = st[nb][2 * x] + st[nb][2 * x + 1];
+          const float v = st[nb][2 * x] + st[nb][2 * x + 1] + bias;
           s[nb][x] = live_t && ((bits >> (16 * nb + g + x * 8)) & 1u) ? v : -INFINITY;
         }
       uint32_t pb0[2], pb1[2];

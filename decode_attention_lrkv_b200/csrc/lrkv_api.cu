@@ -159,7 +159,7 @@ lrkv_status lrkv_compress(const lrkv_dims* dims, const lrkv_cache* cache,
   p.err_out = err_out;
   p.ticket = reinterpret_cast<int32_t*>(w + L.compress_ticket);
   if (t_new <= kAppendMaxTokens) {  // decode-time appends: one fused launch
-    const size_t smem = append_smem_bytes(dims->r_k, dims->r_v);
+    const size_t smem = append_smem_bytes(dims->r_k, dims->r_v, cache->U_kq != nullptr);
     if (!set_smem(append_kernel, smem)) return LRKV_ERR_CUDA;
     return launch_pdl(append_kernel, dim3(dims->Hkv, dims->B), dim3(kAppendThreads), smem, s, p);
   }

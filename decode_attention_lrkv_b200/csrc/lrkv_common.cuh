@@ -99,31 +99,37 @@ inline int num_sms() {
 //   ceil(BH * n / sms) * (chunk + kDecodeOverhead)
 // with BH (batch row, kv head) pairs and one CTA per SM resident at a time.
 // The cost only drops where n fills a wave, so the candidates are the largest
-// n of the first four wave counts that n_min allows, and n_max.  Returns the
-// splits that hold positions (ceil(T / chunk) <= n).
-__host__ __device__ inline int decode_split(long long T, int n_max_grid, long long BH, int sms,
+// n of the first four wave counts that n_min allows, and n_max.  Every CTA
+// evaluates this for its own sequence, so the model is evaluated in fp32 (the
+// choice only has to be good) and the chosen split in exact 32-bit integers.
+// Returns the splits that hold positions (ceil(T / chunk) <= n).
+__host__ __device__ inline int decode_split(int T, int n_max_grid, long long BH, int sms,
                                             int* chunk_out) {
   if (T <= 0) {
     *chunk_out = kMinDecodeChunk;
     return 1;
   }
-  const long long n_min = (T + kMaxDecodeChunk - 1) / kMaxDecodeChunk;
-  long long n_max = (T + kMinDecodeChunk - 1) / kMinDecodeChunk;
+  const unsigned uT = (unsigned)T;
+  const int n_min = (int)((uT + kMaxDecodeChunk - 1) / kMaxDecodeChunk);
+  int n_max = (int)((uT + kMinDecodeChunk - 1) / kMinDecodeChunk);
   if (n_max > n_max_grid) n_max = n_max_grid;
   if (n_max < n_min) n_max = n_min;
-  const long long w0 = (BH * n_min + sms - 1) / sms;   // waves at n_min
-  long long best_cost = -1, best_chunk = kMaxDecodeChunk;
+  const float fbh = (float)BH, fsm = (float)sms, ft = (float)T;
+  const float w0 = ceilf(fbh * (float)n_min / fsm);   // waves at n_min
+  float best_cost = -1.f;
+  int best_n = n_min;
   for (int k = 0; k <= 4; ++k) {
-    long long n = k < 4 ? (w0 + k) * sms / BH : n_max;
-    if (n < n_min) n = n_min;
-    if (n > n_max) n = n_max;
-    const long long ch = ((T + n - 1) / n + 31) / 32 * 32;
-    const long long waves = (BH * ((T + ch - 1) / ch) + sms - 1) / sms;
-    const long long cost = waves * (ch + kDecodeOverhead);
-    if (best_cost < 0 || cost < best_cost) best_cost = cost, best_chunk = ch;
+    float nf = k < 4 ? floorf((w0 + (float)k) * fsm / fbh) : (float)n_max;
+    nf = fminf(fmaxf(nf, (float)n_min), (float)n_max);
+    const float ch = ceilf(ft / (32.f * nf)) * 32.f;
+    const float waves = ceilf(fbh * ceilf(ft / ch) / fsm);
+    const float cost = waves * (ch + (float)kDecodeOverhead);
+    if (best_cost < 0.f || cost < best_cost) best_cost = cost, best_n = (int)nf;
   }
-  *chunk_out = (int)best_chunk;
-  return (int)((T + best_chunk - 1) / best_chunk);
+  const unsigned n = (unsigned)best_n;
+  const unsigned ch = ((uT + n - 1) / n + 31) / 32 * 32;
+  *chunk_out = (int)ch;
+  return (int)((uT + ch - 1) / ch);
 }
 
 inline WsLayout ws_layout(const lrkv_dims& D) {

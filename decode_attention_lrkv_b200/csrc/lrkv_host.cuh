@@ -44,6 +44,7 @@ inline lrkv_status check_cache(const lrkv_dims* D, const lrkv_cache* C) {
     if (!aligned16(p)) return LRKV_ERR_ALIGNMENT;
   for (const void* p : full)
     if (!aligned16(p)) return LRKV_ERR_ALIGNMENT;
+  if (!aligned16(C->U_kq) || !aligned16(C->mu_k)) return LRKV_ERR_ALIGNMENT;   // optional
   return LRKV_OK;
 }
 

@@ -103,6 +103,18 @@ typedef struct {
   int32_t* full_cnt;    /* [B][Hkv] rows in use in the full-rank list */
   int32_t* seq_len;     /* [B] tokens already in the cache (positions 0..seq_len-1) */
   uint32_t* dev_status; /* 1 word, LRKV_DEV_* bits */
+  /* Attention-aware key basis (NOVA-KV summary, "Methodology > Key Transform
+     Derivation", Theorem 1: the optimal rank-p key transform R = M_q^{1/2} E_p,
+     non-orthogonal, with the query side projected by M_q^{-1/2} E_p).  Both
+     null: the plain StaticPCA cache described above.  When given:
+       c_k   = U_k^T (k - mu_k)                 U_k: the key-side basis R
+       k_hat = mu_k + U_kq c_k                  U_kq: the query-side basis
+       e_k   = ||k - k_hat|| / ||k||
+       q~    = U_kq^T q,  compressed logit (q . mu_k + q~ . c_k) / sqrt(d).
+     Either may be null on its own (U_kq = U_k, or mu_k = 0).  Values are not
+     transformed.  A cache must keep the same choice for all its calls. */
+  const lrkv_bf16* U_kq; /* nullable [Hkv][d][r_k] query-side / key reconstruction basis */
+  const float* mu_k;     /* nullable [Hkv][d] fp32 key mean */
 } lrkv_cache;
 /* A new cache is all zeros (seq_len = full_cnt = 0).  The library writes every
    mask bit, coefficient row and list entry it covers, so stale contents past
@@ -111,8 +123,8 @@ typedef struct {
 /* Stream ordering.  lrkv_compress's decode-time append and lrkv_decode_attn
    launch with programmatic dependent launch: their kernels may begin on the
    GPU while the preceding kernel of the stream is finishing.  Before waiting
-   for it they read only the bases U_k and U_v, so the kernel issued just
-   before a call must not write the bases.  Every other input (q, k_new,
+   for it they read only the bases (U_k, U_v, U_kq) and mu_k, so the kernel
+   issued just before a call must not write them.  Every other input (q, k_new,
    v_new and all cache state) is read after the preceding kernel completed. */
 
 /* Bytes of device workspace that lrkv_compress and lrkv_decode_attn need for

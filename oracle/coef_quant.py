@@ -90,7 +90,7 @@ def quantize_cache(cache, bits):
 
 def dequantized_cache(cache, codes):
     """A copy of ``cache`` whose coefficient rows are the dequantised codes."""
-    return Cache(dims=cache.dims, U_k=cache.U_k, U_v=cache.U_v,
+    return Cache(dims=cache.dims, U_k=cache.U_k, U_v=cache.U_v, U_kq=cache.U_kq, mu_k=cache.mu_k,
                  coef_k=dequantize_coef(codes["qk"], codes["sk"]),
                  coef_v=dequantize_coef(codes["qv"], codes["sv"]),
                  route_mask=cache.route_mask, full_idx=cache.full_idx, full_k=cache.full_k,
@@ -129,8 +129,9 @@ def decode_attn_quant_coef(cache, codes, q):
             Qv = codes["qv"][b, kvh, :T][comp].astype(np.float64)
             Sv = codes["sv"][b, kvh, :T][comp].astype(np.float64)
             for h in range(kvh * D.g, (kvh + 1) * D.g):
-                q_t = cache.U_k[kvh].T @ q[b, h]
-                s = np.concatenate([Sk * (Qk @ q_t), Fk @ q[b, h]]) / np.sqrt(D.d)
+                q_t = cache.key_rec_basis(kvh).T @ q[b, h]
+                bias = q[b, h] @ cache.key_mean(kvh)
+                s = np.concatenate([Sk * (Qk @ q_t) + bias, Fk @ q[b, h]]) / np.sqrt(D.d)
                 p = softmax(s)
                 pc, pf = p[:len(Sk)], p[len(Sk):]
                 out[b, h] = cache.U_v[kvh] @ ((pc * Sv) @ Qv) + pf @ Fv

@@ -33,6 +33,13 @@ reason in the design notes of the repository):
   R8  logits are scaled by 1/sqrt(d), d the head dimension.
   R10 a decode step appends first, then attends (the new token included).
   R12 every bfloat16 rounding is round-to-nearest-even.
+Attention-aware key basis (NOVA-KV summary, Theorem 1 and Proposition 1;
+reading R24 of how a cache uses it): a cache may carry a second key basis
+U_kq (the query-side / reconstruction basis) and a key mean mu_k.  Then
+c_k = U_k^T (k - mu_k), k_hat = mu_k + U_kq c_k, the key error is
+||k - k_hat|| / ||k||, and the decode reads q~ = U_kq^T q with compressed
+logits (q . mu_k + q~ . c_k) / sqrt(d).  Without them U_kq = U_k, mu_k = 0:
+the plain StaticPCA cache above.  Values are never transformed this way.
 Capacity: a sequence never grows past T_cap (the tokens that do not fit are
 dropped and SEQ_OVERFLOW is raised); routed tokens beyond F_cap are kept
 compressed instead (mask bit clear) and FULL_OVERFLOW is raised.  Routing is
@@ -93,21 +100,33 @@ class Cache:
     full_cnt: np.ndarray = field(default=None)
     seq_len: np.ndarray = field(default=None)
     status: int = 0
+    U_kq: np.ndarray = field(default=None)    # [Hkv,d,r_k] key reconstruction basis, None: U_k
+    mu_k: np.ndarray = field(default=None)    # [Hkv,d] key mean, None: 0
 
     @staticmethod
-    def empty(dims, U_k, U_v):
+    def empty(dims, U_k, U_v, U_kq=None, mu_k=None):
         D = dims
         if D.T_cap % 32:
             raise ValueError("T_cap must be a multiple of 32")
         z = np.zeros
         return Cache(
             dims=D,
+            U_kq=None if U_kq is None else np.asarray(U_kq, np.float64),
+            mu_k=None if mu_k is None else np.asarray(mu_k, np.float64),
             U_k=np.asarray(U_k, np.float64), U_v=np.asarray(U_v, np.float64),
             coef_k=z((D.B, D.Hkv, D.T_cap, D.r_k)), coef_v=z((D.B, D.Hkv, D.T_cap, D.r_v)),
             route_mask=z((D.B, D.Hkv, D.T_cap // 32), np.uint32),
             full_idx=z((D.B, D.Hkv, D.F_cap), np.int32),
             full_k=z((D.B, D.Hkv, D.F_cap, D.d)), full_v=z((D.B, D.Hkv, D.F_cap, D.d)),
             full_cnt=z((D.B, D.Hkv), np.int32), seq_len=z((D.B,), np.int32), status=0)
+
+    def key_rec_basis(self, h):
+        """The basis keys of kv head h are reconstructed with (and q~ taken in)."""
+        return self.U_k[h] if self.U_kq is None else self.U_kq[h]
+
+    def key_mean(self, h):
+        """The mean subtracted from keys of kv head h before projection."""
+        return np.zeros(self.dims.d) if self.mu_k is None else self.mu_k[h]
 
     def routed(self, b, h, pos):
         """True where the mask marks position(s) ``pos`` of (b, h) as full rank."""
@@ -120,31 +139,37 @@ class Cache:
 # write path: projection, error, routing (OjaKV README, Method Summary)
 # ---------------------------------------------------------------------------
 
-def project(U, X):
-    """Coefficients c = U^T x for every row x of X.  U [d,r], X [...,d] -> [...,r].
+def project(U, X, mu=None):
+    """Coefficients c = U^T (x - mu) for every row x of X.  U [d,r], X [...,d] -> [...,r].
 
     StaticPCA (OjaKV README, Method Summary): tokens are represented by their
-    coordinates in the fixed per-head basis.  Reading R1: no mean-centring.
+    coordinates in the fixed per-head basis.  Reading R1: no mean-centring
+    (mu = None); an attention-aware key basis (reading R24) subtracts its mean.
     """
-    return np.asarray(X, np.float64) @ np.asarray(U, np.float64)
+    X = np.asarray(X, np.float64)
+    if mu is not None:
+        X = X - np.asarray(mu, np.float64)
+    return X @ np.asarray(U, np.float64)
 
 
-def reconstruct(U, C):
-    """x_hat = U c for every row c of C (the on-the-fly reconstruction)."""
-    return np.asarray(C, np.float64) @ np.asarray(U, np.float64).T
+def reconstruct(U, C, mu=None):
+    """x_hat = mu + U c for every row c of C (the on-the-fly reconstruction)."""
+    Xh = np.asarray(C, np.float64) @ np.asarray(U, np.float64).T
+    return Xh if mu is None else Xh + np.asarray(mu, np.float64)
 
 
-def rel_error(U, X, C=None):
-    """Per-token relative reconstruction error ||x - U c|| / ||x|| (readings R4, R6).
+def rel_error(U, X, C=None, U_rec=None, mu=None):
+    """Per-token relative reconstruction error ||x - x_hat|| / ||x|| (readings R4, R6).
 
     OjaKV README, Method Summary > OjaKV: "reconstruction error" decides which
-    tokens stay in full rank.  Computed by direct reconstruction; ||x|| = 0
-    gives 0.
+    tokens stay in full rank.  Computed by direct reconstruction,
+    x_hat = mu + U_rec c with c = U^T (x - mu) (U_rec = U and mu = 0 unless an
+    attention-aware key basis is used, reading R24); ||x|| = 0 gives 0.
     """
     X = np.asarray(X, np.float64)
     if C is None:
-        C = project(U, X)
-    num = np.linalg.norm(X - reconstruct(U, C), axis=-1)
+        C = project(U, X, mu)
+    num = np.linalg.norm(X - reconstruct(U if U_rec is None else U_rec, C, mu), axis=-1)
     den = np.linalg.norm(X, axis=-1)
     return np.where(den > 0, num / np.where(den > 0, den, 1.0), 0.0)
 
@@ -244,9 +269,10 @@ def compress(cache, k_new, v_new, tau, t_new_b=None):
         for h in range(Hkv):
             K = k_new[b, :n_eff, h, :]
             V = v_new[b, :n_eff, h, :]
-            ck = project(cache.U_k[h], K)
+            mu = cache.key_mean(h)
+            ck = project(cache.U_k[h], K, mu)
             cv = project(cache.U_v[h], V)
-            ek = rel_error(cache.U_k[h], K, ck)
+            ek = rel_error(cache.U_k[h], K, ck, U_rec=cache.key_rec_basis(h), mu=mu)
             ev = rel_error(cache.U_v[h], V, cv)
             full = route(ek, ev, tau)
             pos = start + np.arange(n_eff)
@@ -289,7 +315,7 @@ def effective_kv(cache, b, h):
     """
     T = int(cache.seq_len[b])
     pos = np.arange(T)
-    K = reconstruct(cache.U_k[h], cache.coef_k[b, h, :T])
+    K = reconstruct(cache.key_rec_basis(h), cache.coef_k[b, h, :T], cache.key_mean(h))
     V = reconstruct(cache.U_v[h], cache.coef_v[b, h, :T])
     n_full = int(cache.full_cnt[b, h])
     idx = cache.full_idx[b, h, :n_full]
@@ -336,7 +362,8 @@ def decode_attn_coef(cache, q):
 
     q_tilde = U_k^T q;  s_t = q_tilde.c_k,t / sqrt(d) for compressed t,
     s_t = q.k_t / sqrt(d) for full-rank t; one softmax over both sets;
-    o = U_v (sum_C p_t c_v,t) + sum_F p_t v_t.
+    o = U_v (sum_C p_t c_v,t) + sum_F p_t v_t.  With an attention-aware key
+    basis (reading R24): q_tilde = U_kq^T q and s_t = (q.mu_k + q_tilde.c_k,t) / sqrt(d).
     """
     D = cache.dims
     q = np.asarray(q, np.float64)
@@ -355,8 +382,9 @@ def decode_attn_coef(cache, q):
             Ck = cache.coef_k[b, kvh, :T][comp]
             Cv = cache.coef_v[b, kvh, :T][comp]
             for h in range(kvh * D.g, (kvh + 1) * D.g):
-                q_t = cache.U_k[kvh].T @ q[b, h]
-                s = np.concatenate([Ck @ q_t, Fk @ q[b, h]]) / np.sqrt(D.d)
+                q_t = cache.key_rec_basis(kvh).T @ q[b, h]
+                bias = q[b, h] @ cache.key_mean(kvh)
+                s = np.concatenate([Ck @ q_t + bias, Fk @ q[b, h]]) / np.sqrt(D.d)
                 p = softmax(s)
                 pc, pf = p[:Ck.shape[0]], p[Ck.shape[0]:]
                 out[b, h] = cache.U_v[kvh] @ (pc @ Cv) + pf @ Fv

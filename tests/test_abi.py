@@ -122,6 +122,10 @@ def test_host_validation_rejects_before_launch(lib):
     assert _call_compress(lib, _dims(F_cap=0), _FakeCache(full_k=None, full_v=None, full_idx=None),
                           t_new=0) == 0
     assert _call_compress(lib, D, _FakeCache(full_v=None)) == INVALID
+    # the attention-aware key basis and mean are optional, aligned when given
+    assert _call_compress(lib, D, _FakeCache(U_kq=None, mu_k=None), t_new=0) == 0
+    assert _call_compress(lib, D, _FakeCache(mu_k=0x50000004)) == ALIGN
+    assert _call_decode(lib, D, _FakeCache(U_kq=0x50000002)) == ALIGN
 
 
 def test_rank_for_budget_matches_the_oracle(lib):
