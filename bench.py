@@ -68,6 +68,10 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (testing)")
     ap.add_argument("--context", type=int, default=0,
                     help="override the context length (small profiling cases)")
+    ap.add_argument("--quant", type=int, default=0, choices=[0, 8, 4],
+                    help="stored coefficients as 8- or 4-bit codes with per-row scales (0: bf16)")
+    ap.add_argument("--aware", action="store_true",
+                    help="attention-aware key basis (query-side basis and key mean) in every layer")
     ap.add_argument("--seed", type=int, default=1234)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -230,7 +234,26 @@ def sum_over_ranks(x, dev, world):
 # our arm
 # ---------------------------------------------------------------------------
 
-def build_layers(L, w, seed, steps_total, dev, workload_id, t_cap=0):
+def aware_key_basis(U_k, seed, layer):
+    """An attention-aware key basis of Theorem 1's form (NOVA-KV summary) for a
+    query covariance whose eigenvectors are U_k's columns: the key-side basis
+    W_k = U_k diag(s), the query-side basis W_q = U_k diag(1/s), s the square
+    roots of seeded query-covariance eigenvalues, and a seeded key mean inside
+    span(U_k).  Then W_q W_k^T = U_k U_k^T (up to bf16 rounding) and the mean
+    lies in the span, so the routed set is that of the plain basis and the step
+    moves the same bytes: what the timing shows is the cost of the query-side
+    basis and the mean in the kernels."""
+    g = torch.Generator(device=U_k.device).manual_seed(int(seed) * 7919 + int(layer))
+    Hkv, d, r = U_k.shape
+    s = torch.exp(0.5 * torch.randn(Hkv, 1, r, generator=g, device=U_k.device))
+    W_k = (U_k.float() * s).to(torch.bfloat16)
+    W_q = (U_k.float() / s).to(torch.bfloat16)
+    m = 0.05 * torch.randn(Hkv, r, 1, generator=g, device=U_k.device)
+    mu = torch.matmul(U_k.float(), m).squeeze(-1)
+    return W_k, W_q, mu
+
+
+def build_layers(L, w, seed, steps_total, dev, workload_id, t_cap=0, aware=False, quant=0):
     """Prefill every layer's cache through lrkv_compress; time each prefill.
 
     Each timed prefill starts with a cold L2 (a 256 MB buffer is written first)
@@ -239,7 +262,8 @@ def build_layers(L, w, seed, steps_total, dev, workload_id, t_cap=0):
     untimed prefill into a scratch cache first loads the kernels."""
     T_cap = synth.pad_to(max(w.T + steps_total + 1, t_cap), 32)
     F_cap = synth.pad_to(int(F_CAP_FRAC.get(workload_id, F_CAP_FRAC_DEFAULT) * T_cap), 32)
-    dims = L.Dims(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, r_k=w.r_k, r_v=w.r_v, T_cap=T_cap, F_cap=F_cap)
+    dims = L.Dims(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, r_k=w.r_k, r_v=w.r_v, T_cap=T_cap, F_cap=F_cap,
+                  coef_bits=quant)
     ws = L.make_workspace(dims, dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     layers = []
@@ -249,12 +273,17 @@ def build_layers(L, w, seed, steps_total, dev, workload_id, t_cap=0):
         lay = synth.make_layer(w, li, seed, device=dev)
         lengths = lay["lengths"]
         t_new_b = (lengths.to(torch.int32).to(dev) if w.ragged_min else None)
+        kb = {}
+        if aware:
+            W_k, W_q, mu = aware_key_basis(lay["U_k"], seed, li)
+            kb = dict(U_kq=W_q, mu_k=mu)
+            lay["U_k"] = W_k
         if li == 0:
-            scratch = L.LayerCache(dims, lay["U_k"], lay["U_v"], device=dev)
+            scratch = L.LayerCache(dims, lay["U_k"], lay["U_v"], device=dev, **kb)
             L.lrkv_compress(dims, scratch, lay["K"], lay["V"], w.tau, t_new_b=t_new_b, ws=ws)
             torch.cuda.synchronize()
             del scratch
-        cache = L.LayerCache(dims, lay["U_k"], lay["U_v"], device=dev)
+        cache = L.LayerCache(dims, lay["U_k"], lay["U_v"], device=dev, **kb)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         flush.zero_()
@@ -320,7 +349,7 @@ def run_ours(args, rank, world, dev):
     steps_total = W + K
     seed = rank_seed(args.seed, rank)
     dims, ws, layers, comp_ms, lengths = build_layers(L, w, seed, 4 * steps_total, dev, args.workload,
-                                                      args.t_cap)
+                                                      args.t_cap, aware=args.aware, quant=args.quant)
     out = torch.empty(w.layers, w.B, w.Hq, w.d, dtype=torch.float32, device=dev)
 
     # --- device-resident timed region: the step graphs carry no events (an event
@@ -423,15 +452,16 @@ def run_ours(args, rank, world, dev):
 
     # algorithmic bytes of the timed steps: step s attends over seq_len + 1 tokens
     T_mid = [int(x) + (K + 1) / 2.0 for x in seq_before]
-    dec_bytes = [A.decode_bytes(w.B, w.Hq, w.Hkv, w.d, w.r_k, w.r_v, T_mid, fc) for fc in full_cnt]
+    dec_bytes = [A.decode_bytes(w.B, w.Hq, w.Hkv, w.d, w.r_k, w.r_v, T_mid, fc, coef_bits=dims.bits) for fc in full_cnt]
     routed_frac = float(sum(fc.sum() for fc in full_cnt)) / (w.layers * w.Hkv * sum(T_mid))
-    app_bytes = A.compress_bytes(w.Hkv, w.d, w.r_k, w.r_v, w.B, w.B * w.Hkv * routed_frac)
+    app_bytes = A.compress_bytes(w.Hkv, w.d, w.r_k, w.r_v, w.B, w.B * w.Hkv * routed_frac,
+                                 coef_bits=dims.bits)
     step_bytes = sum(dec_bytes) + w.layers * app_bytes
     ms_step = ms / K
     value = sum_over_ranks(step_bytes, dev, world) / (ms_step * 1e-3) / 1e9
     dec_launch_ms = float(np.mean(dec_ms))
     T_mid_k = [int(x) + (K + 1) / 2.0 for x in seq_k]
-    dec_bytes_launch = float(np.mean([A.decode_bytes(w.B, w.Hq, w.Hkv, w.d, w.r_k, w.r_v, T_mid_k, fc)
+    dec_bytes_launch = float(np.mean([A.decode_bytes(w.B, w.Hq, w.Hkv, w.d, w.r_k, w.r_v, T_mid_k, fc, coef_bits=dims.bits)
                                       for fc in full_cnt_k])) + app_bytes   # the fused append's too
     pk, pk_kind = peaks()
     peak = pk.get("hbm_gbs", FALLBACK_PEAK["hbm_gbs"])
@@ -442,14 +472,15 @@ def run_ours(args, rank, world, dev):
     achieved = layer_bytes / (layer_ms * 1e-3) / 1e9
     isolated = dec_bytes_launch / (dec_launch_ms * 1e-3) / 1e9
     dec_bytes_chain = float(np.mean([A.decode_bytes(w.B, w.Hq, w.Hkv, w.d, w.r_k, w.r_v,
-                                                    [int(x) for x in seq_c], fc) for fc in full_cnt_c]))
+                                                    [int(x) for x in seq_c], fc, coef_bits=dims.bits) for fc in full_cnt_c]))
     chained = dec_bytes_chain / (chain_launch_ms * 1e-3) / 1e9
     status = max(int(lay["cache"].dev_status[0].item()) for lay in layers)
 
     # --- prefill compress rate ----------------------------------------------------------
     n_tok = float(sum(int(x) for x in lengths))
     comp_tok_s = n_tok / (float(np.mean(comp_ms)) * 1e-3)
-    comp_bytes = A.compress_bytes(w.Hkv, w.d, w.r_k, w.r_v, n_tok, n_tok * w.Hkv * routed_frac)
+    comp_bytes = A.compress_bytes(w.Hkv, w.d, w.r_k, w.r_v, n_tok, n_tok * w.Hkv * routed_frac,
+                                  coef_bits=dims.bits)
     comp_tflops = A.compress_tc_flops(w.Hkv, w.d, w.r_k, w.r_v, n_tok) / (float(np.mean(comp_ms)) * 1e-3) / 1e12
 
     # --- end-to-end through host buffers --------------------------------------------------
@@ -462,6 +493,11 @@ def run_ours(args, rank, world, dev):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "layers": w.layers, "batch": w.B, "context": w.T,
                    "T_cap": dims.T_cap, "F_cap": dims.F_cap,
+                   "key_basis": ("attention-aware (query-side basis + key mean)" if args.aware
+                                 else "orthonormal (StaticPCA)"),
+                   "coefficients": "bf16" if dims.bits == 16 else f"int{dims.bits} codes + fp32 row scales",
+                   "bytes_per_compressed_token_head": A.compressed_bytes_per_token_head(
+                       w.r_k, w.r_v, coef_bits=dims.bits),
                    "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d, "r_k": w.r_k, "r_v": w.r_v,
                    "tau": w.tau, "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": f"inputs larger than L2: {step_bytes / 1e9:.2f} GB touched per step vs 126 MB L2",
@@ -506,7 +542,8 @@ def run_ours(args, rank, world, dev):
                                  "timing": "one CUDA graph of every layer's decode, K times back "
                                            "to back (no appends), CUDA events around the replay"}},
         "e2e": e2e,
-        "gpu_launches": K * w.layers * FUSED_LAUNCHES,
+        "gpu_launches": K * w.layers * (FUSED_LAUNCHES if dims.bits != 4 and w.g in (1, 2, 4)
+                                        else 2),   # 4-bit codes or other groups: append + decode
         "clocks": clk,
     }
     return result, w, layers, dims
@@ -548,8 +585,8 @@ def run_e2e(L, args, w, dims, ws, layers, dev, world, steps_total):
     T_now = [int(x) for x in layers[0]["cache"].seq_len.cpu()]
     T_mid = [t - (K - 1) / 2.0 for t in T_now]
     full_cnt = [lay["cache"].full_cnt.cpu().numpy() for lay in layers]
-    step_bytes = sum(A.decode_bytes(w.B, w.Hq, w.Hkv, w.d, w.r_k, w.r_v, T_mid, fc) for fc in full_cnt)
-    step_bytes += w.layers * A.compress_bytes(w.Hkv, w.d, w.r_k, w.r_v, w.B, 0)
+    step_bytes = sum(A.decode_bytes(w.B, w.Hq, w.Hkv, w.d, w.r_k, w.r_v, T_mid, fc, coef_bits=dims.bits) for fc in full_cnt)
+    step_bytes += w.layers * A.compress_bytes(w.Hkv, w.d, w.r_k, w.r_v, w.B, 0, coef_bits=dims.bits)
     h2d = sum(t[0].numel() * t[0].element_size() for t in hin.values())
     d2h = hout[0].numel() * hout[0].element_size()
     job_bytes = sum_over_ranks(step_bytes, dev, world)

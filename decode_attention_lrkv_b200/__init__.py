@@ -46,13 +46,14 @@ class LrkvError(RuntimeError):
 
 
 class _Dims(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hq", "Hkv", "d", "r_k", "r_v", "T_cap", "F_cap")]
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hq", "Hkv", "d", "r_k", "r_v", "T_cap", "F_cap",
+                                               "coef_bits")]
 
 
 class _Cache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "U_k", "U_v", "coef_k", "coef_v", "route_mask", "full_idx", "full_k", "full_v",
-        "full_cnt", "seq_len", "dev_status", "U_kq", "mu_k")]
+        "full_cnt", "seq_len", "dev_status", "U_kq", "mu_k", "scale_k", "scale_v")]
 
 
 _lib = None
@@ -105,25 +106,32 @@ class Dims:
     r_v: int
     T_cap: int
     F_cap: int
+    coef_bits: int = 0     # stored coefficients: 0/16 bf16, 8 int8 codes, 4 int4 codes
 
     @property
     def g(self):
         return self.Hq // self.Hkv
 
+    @property
+    def bits(self):
+        return 16 if self.coef_bits == 0 else self.coef_bits
+
     def c(self):
-        return _Dims(self.B, self.Hq, self.Hkv, self.d, self.r_k, self.r_v, self.T_cap, self.F_cap)
+        return _Dims(self.B, self.Hq, self.Hkv, self.d, self.r_k, self.r_v, self.T_cap, self.F_cap,
+                     self.coef_bits)
 
 
 class LayerCache:
     """One layer of compressed cache as torch tensors, in the C ABI's layout.
 
     bf16 tensors: U_k [Hkv,d,r_k], U_v [Hkv,d,r_v], coef_k [B,Hkv,T_cap,r_k],
-    coef_v [B,Hkv,T_cap,r_v], full_k/full_v [B,Hkv,F_cap,d];
+    coef_v [B,Hkv,T_cap,r_v] (quantised caches: uint8 code bytes [B,Hkv,T_cap,r*bits/8]
+    with fp32 scale_k/scale_v [B,Hkv,T_cap]), full_k/full_v [B,Hkv,F_cap,d];
     int32: route_mask [B,Hkv,T_cap/32] (bit patterns), full_idx [B,Hkv,F_cap],
     full_cnt [B,Hkv], seq_len [B]; dev_status int32 [4] (word 0 used).
     """
     FIELDS = ("U_k", "U_v", "coef_k", "coef_v", "route_mask", "full_idx", "full_k", "full_v",
-              "full_cnt", "seq_len", "dev_status", "U_kq", "mu_k")
+              "full_cnt", "seq_len", "dev_status", "U_kq", "mu_k", "scale_k", "scale_v")
 
     def __init__(self, dims, U_k, U_v, device="cuda", U_kq=None, mu_k=None):
         D = dims
@@ -137,8 +145,15 @@ class LayerCache:
         self.mu_k = None if mu_k is None else mu_k.to(device=device, dtype=torch.float32).contiguous()
         assert self.U_kq is None or tuple(self.U_kq.shape) == (D.Hkv, D.d, D.r_k)
         assert self.mu_k is None or tuple(self.mu_k.shape) == (D.Hkv, D.d)
-        self.coef_k = z(D.B, D.Hkv, D.T_cap, D.r_k)
-        self.coef_v = z(D.B, D.Hkv, D.T_cap, D.r_v)
+        if D.bits == 16:
+            self.coef_k = z(D.B, D.Hkv, D.T_cap, D.r_k)
+            self.coef_v = z(D.B, D.Hkv, D.T_cap, D.r_v)
+            self.scale_k = self.scale_v = None
+        else:   # integer codes (bytes; 4-bit codes two per byte) and per-row scales
+            self.coef_k = z(D.B, D.Hkv, D.T_cap, D.r_k * D.bits // 8, dt=torch.uint8)
+            self.coef_v = z(D.B, D.Hkv, D.T_cap, D.r_v * D.bits // 8, dt=torch.uint8)
+            self.scale_k = z(D.B, D.Hkv, D.T_cap, dt=torch.float32)
+            self.scale_v = z(D.B, D.Hkv, D.T_cap, dt=torch.float32)
         self.route_mask = z(D.B, D.Hkv, D.T_cap // 32, dt=torch.int32)
         self.full_idx = z(D.B, D.Hkv, max(D.F_cap, 1), dt=torch.int32)
         self.full_k = z(D.B, D.Hkv, max(D.F_cap, 1), D.d)

@@ -18,9 +18,13 @@ def dense_kv_bytes_per_token(layers, kv_heads, d, elem_bytes=BF16):
     return layers * kv_heads * d * 2 * elem_bytes
 
 
-def compressed_bytes_per_token_head(r_k, r_v, elem_bytes=BF16):
-    """Coefficient bytes of one compressed token in one kv head: (r_k + r_v) values."""
-    return (r_k + r_v) * elem_bytes
+def compressed_bytes_per_token_head(r_k, r_v, elem_bytes=BF16, coef_bits=16):
+    """Coefficient bytes of one compressed token in one kv head: (r_k + r_v) values
+    (bf16), or their codes plus one fp32 scale for keys and one for values
+    (coef_bits 8 or 4)."""
+    if coef_bits in (0, 16):
+        return (r_k + r_v) * elem_bytes
+    return (r_k + r_v) * coef_bits // 8 + 2 * FP32
 
 
 def full_row_bytes(d, elem_bytes=BF16):
@@ -28,7 +32,7 @@ def full_row_bytes(d, elem_bytes=BF16):
     return 2 * d * elem_bytes + INT32
 
 
-def decode_bytes(B, Hq, Hkv, d, r_k, r_v, lengths, full_cnt):
+def decode_bytes(B, Hq, Hkv, d, r_k, r_v, lengths, full_cnt, coef_bits=16):
     """Algorithmic bytes of one decode-attention call over one layer.
 
     lengths: B sequence lengths; full_cnt: B x Hkv routed-token counts.
@@ -42,7 +46,7 @@ def decode_bytes(B, Hq, Hkv, d, r_k, r_v, lengths, full_cnt):
         T = int(lengths[b])
         for h in range(Hkv):
             F = int(full_cnt[b][h])
-            total += (T - F) * compressed_bytes_per_token_head(r_k, r_v)
+            total += (T - F) * compressed_bytes_per_token_head(r_k, r_v, coef_bits=coef_bits)
             total += F * 2 * d * BF16
             total += math.ceil(T / 32) * 4
     total += Hkv * d * (r_k + r_v) * BF16
@@ -50,14 +54,16 @@ def decode_bytes(B, Hq, Hkv, d, r_k, r_v, lengths, full_cnt):
     return total
 
 
-def compress_bytes(Hkv, d, r_k, r_v, n_tokens, n_routed):
+def compress_bytes(Hkv, d, r_k, r_v, n_tokens, n_routed, coef_bits=16):
     """Algorithmic bytes of compressing n_tokens positions (summed over batch rows).
 
     Each (token, kv head) reads its key and value rows and writes its
-    coefficients and its mask bit; each routed (token, kv head) also writes
-    its key and value rows and list index.  The basis is read once per kv head.
+    coefficients (or codes and scales) and its mask bit; each routed (token,
+    kv head) also writes its key and value rows and list index.  The basis is
+    read once per kv head.
     """
-    per_tok = Hkv * (2 * d * BF16 + (r_k + r_v) * BF16) + Hkv / 8.0
+    per_tok = Hkv * (2 * d * BF16 + compressed_bytes_per_token_head(r_k, r_v, coef_bits=coef_bits)) \
+        + Hkv / 8.0
     return int(n_tokens * per_tok + n_routed * full_row_bytes(d) + Hkv * d * (r_k + r_v) * BF16)
 
 

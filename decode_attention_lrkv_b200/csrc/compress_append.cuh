@@ -36,10 +36,13 @@ inline size_t append_smem_bytes(int r_k, int r_v, bool aware) {
 // returns the relative error ||x - mu - Urec c|| / ||x|| to every thread of the
 // half (Urec = Us and mu = null except for an attention-aware key basis).  All
 // 256 threads call it together.
+// bits 16: coef_g receives the row as bf16; bits 8 or 4: as codes, with the
+// row's scale in *scale_g (per-row quantisation of the stored row).
 __device__ __forceinline__ float append_project(const uint16_t* __restrict__ x_s,
                                                 const uint16_t* Us, const uint16_t* Urec,
-                                                const float* mu, int r,
-                                                lrkv_bf16* __restrict__ coef_g, float* ws) {
+                                                const float* mu, int r, int bits,
+                                                unsigned char* __restrict__ coef_g,
+                                                float* __restrict__ scale_g, float* ws) {
   const int tid = threadIdx.x & 127;
   const int warp = tid >> 5, lane = tid & 31;
   float* xs = ws;                 // [d]
@@ -66,10 +69,26 @@ __device__ __forceinline__ float append_project(const uint16_t* __restrict__ x_s
       if (lane + 32 * k < r) part[warp * kD + lane + 32 * k] = a[k];
   }
   __syncthreads();
+  float c = 0.f;
   if (tid < r) {
-    const float c = (part[tid] + part[kD + tid]) + (part[2 * kD + tid] + part[3 * kD + tid]);
+    c = (part[tid] + part[kD + tid]) + (part[2 * kD + tid] + part[3 * kD + tid]);
     cs[tid] = c;
-    coef_g[tid] = f2bf(c);
+  }
+  if (bits == 16) {
+    if (tid < r) reinterpret_cast<lrkv_bf16*>(coef_g)[tid] = f2bf(c);
+  } else {   // per-row codes: the row's amax over the half's warps, then one code per column
+    const float cb = tid < r ? bf16_round(c) : 0.f;
+    const float a = warp_max(fabsf(cb));
+    if (lane == 0) red[warp] = a;
+    __syncthreads();
+    const float s = quant_scale(fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])), bits);
+    const int qv = quant_code(cb, s, bits);
+    const int qn = __shfl_down_sync(0xffffffffu, qv, 1);   // the odd neighbour's code (4-bit pairs)
+    if (tid < r) {
+      if (bits == 8) coef_g[tid] = (unsigned char)(qv & 0xff);
+      else if ((tid & 1) == 0) coef_g[tid >> 1] = (unsigned char)((qv & 0xf) | ((qn & 0xf) << 4));
+    }
+    if (tid == 0) *scale_g = s;
   }
   __syncthreads();
   // x_hat_i = sum_j U[i][j] c_j: thread i walks row i two columns at a time,
@@ -102,6 +121,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
   const lrkv_dims& D = p.D;
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int r_k = D.r_k, r_v = D.r_v;
+  const int bits = coef_bits_of(D);   // stored coefficient format
   uint16_t* Uks = reinterpret_cast<uint16_t*>(sm_app);
   uint16_t* Uvs = Uks + kD * r_k;
   uint16_t* Xks = Uvs + kD * r_v;                          // new key rows
@@ -182,11 +202,14 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(CompressParams p
       const int pos = start + t;
       const size_t row = bh * D.T_cap + pos;
       // one call site for both halves: every __syncthreads inside is reached by all threads
+      const int r = half == 0 ? r_k : r_v;
       const float eh = append_project(half == 0 ? Xks + t * kD : Xvs + t * kD,
                                       half == 0 ? Uks : Uvs, half == 0 ? (aware ? Ukqs : Uks) : Uvs,
                                       half == 0 && p.C.mu_k ? p.C.mu_k + (size_t)h * kD : nullptr,
-                                      half == 0 ? r_k : r_v,
-                                      half == 0 ? p.C.coef_k + row * r_k : p.C.coef_v + row * r_v,
+                                      r, bits,
+                                      static_cast<unsigned char*>(half == 0 ? p.C.coef_k : p.C.coef_v) +
+                                          row * (size_t)(r * bits / 8),
+                                      bits < 16 ? (half == 0 ? p.C.scale_k : p.C.scale_v) + row : nullptr,
                                       ws);
       if ((tid & 127) == 0) s_err[half] = eh;
       __syncthreads();

@@ -149,7 +149,9 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
   return false;
 }
 
-// grid (CTAs per group, 2 * Hkv): group = 2 h + tensor (0 keys, 1 values)
+// grid (CTAs per group, 2 * Hkv): group = 2 h + tensor (0 keys, 1 values).
+// CB: stored coefficient format, 16 (bf16) or 8, 4 (codes with per-row scales).
+template <int CB>
 __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // the dynamic window is only guaranteed 16-byte aligned: round up to 1024
@@ -166,7 +168,9 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   // attention-aware keys: the query-side basis reconstructs, the mean is subtracted
   const lrkv_bf16* Uqg = tensor == 0 && p.C.U_kq ? p.C.U_kq + (size_t)h * kD * R : nullptr;
   const float* mug = tensor == 0 && p.C.mu_k ? p.C.mu_k + (size_t)h * kD : nullptr;
-  lrkv_bf16* coef = tensor == 0 ? p.C.coef_k : p.C.coef_v;
+  unsigned char* coef = static_cast<unsigned char*>(tensor == 0 ? p.C.coef_k : p.C.coef_v);
+  constexpr int bits = CB;                        // 16: bf16; 8, 4: codes + per-row scales
+  float* scales = tensor == 0 ? p.C.scale_k : p.C.scale_v;
   float* errs = p.errs + (size_t)tensor * D.B * D.Hkv * D.T_cap;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lo.bar);
@@ -411,31 +415,67 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
       const uint32_t d2 = lane_base + buf * 256, d1 = d2 + 128;
       float rs = 0.f, xs = 0.f;
       if (grp_a) {
-        // coefficients, 64 columns per batch of loads
-        lrkv_bf16* crow = coef + (bh * D.T_cap + start + t) * R;
-#pragma unroll 1
-        for (int c0 = 0; c0 < R; c0 += 64) {
-          float v[4][16];
+        // coefficients (c = U^T x - U^T mu with a key mean), in batches of NC
+        // columns (NC = 64 for bf16 rows; 32 for codes, whose rows take a first
+        // pass for the row's amax)
+        constexpr int NC = CB == 16 ? 64 : 32;
+        const size_t row = bh * D.T_cap + start + t;
+        auto load_c = [&](int c0, float (&v)[NC / 16][16]) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
+          for (int q = 0; q < NC / 16; ++q)
             if (c0 + 16 * q < R) tc5::tmem_ld16(d1 + c0 + 16 * q, v[q]);
           tc5::tmem_wait_ld();
-          if (mug) {   // c = U^T x - U^T mu
+          if (mug) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < NC / 16; ++q)
 #pragma unroll
               for (int k = 0; k < 16; ++k) v[q][k] -= cmu[(c0 + 16 * q + k) & (kD - 1)];
           }
+        };
+        float qs = 0.f;   // the row's scale (quantised rows)
+        if constexpr (CB < 16) {
+          float amax = 0.f;
+#pragma unroll 1
+          for (int c0 = 0; c0 < R; c0 += NC) {
+            float v[NC / 16][16];
+            load_c(c0, v);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            if (valid && c0 + 16 * q < R) {
-              const float* w = v[q];
+            for (int q = 0; q < NC / 16; ++q)
+              if (c0 + 16 * q < R)
+#pragma unroll
+                for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(bf16_round(v[q][k])));
+          }
+          qs = quant_scale(amax, CB);
+          if (valid) scales[row] = qs;
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < R; c0 += NC) {
+          float v[NC / 16][16];
+          load_c(c0, v);
+#pragma unroll
+          for (int q = 0; q < NC / 16; ++q) {
+            if (!valid || c0 + 16 * q >= R) continue;
+            const float* w = v[q];
+            if constexpr (CB == 16) {
+              lrkv_bf16* crow = reinterpret_cast<lrkv_bf16*>(coef) + row * R;
               *reinterpret_cast<uint4*>(crow + c0 + 16 * q) =
                   make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]),
                              pack_bf16(w[6], w[7]));
               *reinterpret_cast<uint4*>(crow + c0 + 16 * q + 8) =
                   make_uint4(pack_bf16(w[8], w[9]), pack_bf16(w[10], w[11]),
                              pack_bf16(w[12], w[13]), pack_bf16(w[14], w[15]));
+            } else {
+              uint32_t cw[4] = {0u, 0u, 0u, 0u};   // 16 codes: 16 bytes (8-bit) or 8 (4-bit)
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                const uint32_t cq = (uint32_t)quant_code(bf16_round(w[k]), qs, CB);
+                if (CB == 8) cw[k >> 2] |= (cq & 0xffu) << (8 * (k & 3));
+                else cw[k >> 3] |= (cq & 0xfu) << (4 * (k & 7));
+              }
+              if (CB == 8)
+                *reinterpret_cast<uint4*>(coef + row * R + c0 + 16 * q) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+              else
+                *reinterpret_cast<uint2*>(coef + row * (R / 2) + (c0 + 16 * q) / 2) = make_uint2(cw[0], cw[1]);
             }
           }
         }

@@ -8,13 +8,20 @@
 
 namespace lrkv {
 
-template <int G, int RK, int RV, int W, int NS>
-inline lrkv_status launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t s) {
-  using S = ds::Shape<G, RK, RV, W, NS>;
-  auto kern = p.k_new ? ds::decode_stream_kernel<G, RK, RV, W, NS, true>
-                      : ds::decode_stream_kernel<G, RK, RV, W, NS, false>;
+template <int G, int RK, int RV, int W, int NS, int CB>
+inline lrkv_status launch_stream_cb(const DecodeParams& p, dim3 grid, cudaStream_t s) {
+  using S = ds::Shape<G, RK, RV, W, NS, CB>;
+  auto kern = p.k_new ? ds::decode_stream_kernel<G, RK, RV, W, NS, true, CB>
+                      : ds::decode_stream_kernel<G, RK, RV, W, NS, false, CB>;
   if (!set_smem(kern, S::SMEM)) return LRKV_ERR_CUDA;
   return launch_pdl(kern, grid, dim3(S::kThreads), S::SMEM, s, p);
+}
+
+// bf16 coefficients or int8 codes (4-bit codes take the CUDA-core kernel)
+template <int G, int RK, int RV, int W, int NS>
+inline lrkv_status launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t s) {
+  if (coef_bits_of(p.D) == 8) return launch_stream_cb<G, RK, RV, W, NS, 8>(p, grid, s);
+  return launch_stream_cb<G, RK, RV, W, NS, 16>(p, grid, s);
 }
 
 template <int G>
@@ -29,6 +36,10 @@ template <int G>
 inline lrkv_status launch_stream_g(const DecodeParams& p, dim3 grid, cudaStream_t s, bool* done) {
   *done = true;
   const int rk = p.D.r_k, rv = p.D.r_v;
+  if (coef_bits_of(p.D) == 4) {   // 4-bit codes: the CUDA-core kernel
+    *done = false;
+    return LRKV_OK;
+  }
   // (warps per CTA, ring stages per warp) per shape: what shared memory holds
   // beside the mask words and the resident U_v
   if (rk == 32 && rv == 32) return launch_stream<G, 32, 32, 8, 3>(p, grid, s);

@@ -90,17 +90,28 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(DecodeParams
   const int c0 = c * chunk;
   const int c1 = min(T, c0 + chunk);
   const uint32_t* mask = p.C.route_mask + bh * (D.T_cap / 32);
-  const lrkv_bf16* ck = p.C.coef_k + bh * D.T_cap * r_k;
-  const lrkv_bf16* cv = p.C.coef_v + bh * D.T_cap * r_v;
+  // stored coefficients: bf16, or integer codes (8 or 4 bits) with per-row scales
+  const int bits = coef_bits_of(D);
+  const unsigned char* ck = static_cast<const unsigned char*>(p.C.coef_k) + bh * D.T_cap * (size_t)(r_k * bits / 8);
+  const unsigned char* cv = static_cast<const unsigned char*>(p.C.coef_v) + bh * D.T_cap * (size_t)(r_v * bits / 8);
+  auto coef_at = [&](const unsigned char* rows, int t, int j, int r) -> float {
+    if (bits == 16) return bf2f(reinterpret_cast<const uint16_t*>(rows)[(size_t)t * r + j]);
+    if (bits == 8) return (float)(int8_t)rows[(size_t)t * r + j];
+    const int byte = rows[(size_t)t * (r / 2) + (j >> 1)];
+    const int nib = (j & 1) ? (byte >> 4) : (byte & 0xf);
+    return (float)(nib >= 8 ? nib - 16 : nib);
+  };
   for (int t = c0 + warp; t < c1; t += kDecWarps) {
     if ((mask[t >> 5] >> (t & 31)) & 1u) continue;
     float kv[4], vv[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int j = lane + 32 * k;
-      kv[k] = j < r_k ? bf2f(ck[(size_t)t * r_k + j]) : 0.f;
-      vv[k] = j < r_v ? bf2f(cv[(size_t)t * r_v + j]) : 0.f;
+      kv[k] = j < r_k ? coef_at(ck, t, j, r_k) : 0.f;
+      vv[k] = j < r_v ? coef_at(cv, t, j, r_v) : 0.f;
     }
+    const float sk = bits < 16 ? p.C.scale_k[bh * D.T_cap + t] : 1.f;   // code scales
+    const float sv = bits < 16 ? p.C.scale_v[bh * D.T_cap + t] : 1.f;
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
       float s = 0.f;
@@ -109,14 +120,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(DecodeParams
         const int j = lane + 32 * k;
         if (j < r_k) s = fmaf(qt[gi * kD + j], kv[k], s);
       }
-      s = warp_sum(s) + s_bias[gi];
+      s = fmaf(warp_sum(s), sk, s_bias[gi]);
       const float mn = fmaxf(m[gi], s);
       const float sc = exp2f(m[gi] - mn);
       const float pr = exp2f(s - mn);
       l[gi] = l[gi] * sc + pr;
+      const float pv = pr * sv;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        accc[gi][k] = fmaf(pr, vv[k], accc[gi][k] * sc);
+        accc[gi][k] = fmaf(pv, vv[k], accc[gi][k] * sc);
         accf[gi][k] *= sc;
       }
       m[gi] = mn;

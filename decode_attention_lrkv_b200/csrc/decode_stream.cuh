@@ -62,18 +62,32 @@ constexpr int imax(int a, int b) { return a > b ? a : b; }
 
 // W warps per CTA and NS ring stages per warp: per shape, as many warps as
 // shared memory allows with U_v resident beside the ring.
-template <int G, int RK, int RV, int W, int NS>
+// x (a multiple of 16) raised to an odd multiple of 16: rows that far apart
+// put the 8 rows an ldmatrix reads in distinct shared-memory banks
+constexpr int odd16(int x) { return (x / 16) % 2 ? x : x + 16; }
+
+// CB: bits of a stored coefficient, 16 (bf16) or 8 (int8 codes with per-row
+// fp32 scales).
+template <int G, int RK, int RV, int W, int NS, int CB = 16>
 struct Shape {
   static_assert(G == 1 || G == 2 || G == 4, "1, 2 or 4 query heads per kv head");
   static_assert(RK % 16 == 0 && RV % 16 == 0 && RK <= kD && RV <= kD, "ranks");
   static_assert(W >= 8 && NS >= 2, "at least 8 warps and 2 ring stages");
+  static_assert(CB == 16 || CB == 8, "bf16 coefficients or int8 codes");
   static constexpr int kWarps = W;
   static constexpr int kThreads = W * 32;
-  static constexpr int KP = RK / 8, VP = RV / 8;   // 16-byte pieces per row
-  static constexpr int KS = 2 * RK + 16;           // padded row strides (bytes): odd multiples of 16
+  // the bases in shared memory: bf16 rows, padded
+  static constexpr int UKP = RK / 8, UVP = RV / 8;  // 16-byte pieces per basis row
+  static constexpr int KS = 2 * RK + 16;           // padded basis row strides (bytes)
   static constexpr int VS = 2 * RV + 16;
+  // a compressed tile: 32 stored rows of keys, then of values, then (codes
+  // only) their 32 + 32 fp32 scales
+  static constexpr int TKB = RK * CB / 8, TVB = RV * CB / 8;   // bytes per stored row
+  static constexpr int KP = TKB / 16, VP = TVB / 16;          // 16-byte pieces per stored row
+  static constexpr int TKS = odd16(TKB), TVS = odd16(TVB);    // padded tile row strides
+  static constexpr int T_SC = kTileC * (TKS + TVS);           // scales: [2][32] fp32
   static constexpr int FS = 2 * kD + 16;
-  static constexpr int SLOT_C = kTileC * (KS + VS);
+  static constexpr int SLOT_C = T_SC + (CB < 16 ? 2 * kTileC * 4 : 0);
   static constexpr int SLOT_F = kTileF * 2 * FS;
   static constexpr int SLOT = al128(imax(SLOT_C, SLOT_F));
   static constexpr int MASK_BYTES = (kMaxChunk / 32) * 4;          // mask words
@@ -105,7 +119,8 @@ struct Shape {
   // [G][RK], x [2][d] (key, value), the key minus its mean [d], sums [24]
   static constexpr int OFF_APP = OFF_UK2 + al16(kD * KS);
   static constexpr int A_CK = 0, A_CV = RK, A_QT = RK + RV, A_X = A_QT + G * RK,
-                       A_XC = A_X + 2 * kD, A_RED = A_XC + kD, A_FLOATS = A_RED + 24;
+                       A_XC = A_X + 2 * kD, A_RED = A_XC + kD, A_QR = A_RED + 24,
+                       A_FLOATS = A_QR + 8;
   static_assert(2 * al16(kD * KS) + A_FLOATS * 4 <= W * SLOT,
                 "both key bases and the append scratch fit in a stage");
 };
@@ -117,10 +132,11 @@ struct Shape {
 //   exact in bf16, fp32 accumulation); e = max(||k - U_k c_k|| / ||k||,
 //   ||v - U_v c_v|| / ||v||) by direct reconstruction from the unrounded c;
 //   routed iff e > tau: the rows go to list slot F when there is room (the
-//   mask bit set), else the token stays compressed (FULL_OVERFLOW).  bf16(c)
-//   is stored at pos either way.  Then the token's base-2 logit per head and
-//   its value row (v, or bf16(c_v)) for the fold after the stream.
-template <typename S, int G, int RK, int RV>
+//   mask bit set), else the token stays compressed (FULL_OVERFLOW).  bf16(c),
+//   or its per-row codes and scale (CB 8 or 4), is stored at pos either way.
+//   Then the token's base-2 logit per head and its value row (v, or c_v as
+//   stored) for the fold after the stream.
+template <typename S, int G, int RK, int RV, int CB>
 __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
                                              const unsigned char* uk, const unsigned char* ukq,
                                              const unsigned char* uv, const float* s_bias,
@@ -220,9 +236,34 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
   const float e = fmaxf(nk > 0.f ? sqrtf(rk / nk) : 0.f, nv > 0.f ? sqrtf(rv / nv) : 0.f);
   const bool routed = e > p.tau;
   const bool keep = routed && F < D.F_cap;
-  if (tid < RK) p.C.coef_k[(bh * D.T_cap + pos) * RK + tid] = f2bf(app[S::A_CK + tid]);
-  if (tid >= kD && tid - kD < RV)
-    p.C.coef_v[(bh * D.T_cap + pos) * RV + (tid - kD)] = f2bf(app[S::A_CV + tid - kD]);
+  {  // the stored rows: thread j of each half owns column j of its tensor's row
+    const bool kside = tid < kD;
+    const int j = tid & (kD - 1), r = kside ? RK : RV;
+    float* cval = app + (kside ? S::A_CK : S::A_CV) + j;
+    const size_t row = bh * D.T_cap + pos;
+    const float cb = j < r ? bf16_round(*cval) : 0.f;
+    if constexpr (CB == 16) {
+      if (j < r) reinterpret_cast<uint16_t*>(kside ? p.C.coef_k : p.C.coef_v)[row * r + j] = f2bf(cb);
+      if (j < r) *cval = cb;
+    } else {   // per-row codes: the row's amax over its half's warps, one code per column
+      const float wm = warp_max(fabsf(cb));
+      if (lane == 0) app[S::A_QR + warp] = wm;
+      __syncthreads();
+      const float* qr = app + S::A_QR + (kside ? 0 : 4);
+      const float s = quant_scale(fmaxf(fmaxf(qr[0], qr[1]), fmaxf(qr[2], qr[3])), CB);
+      const int qv = quant_code(cb, s, CB);
+      const int qn = __shfl_down_sync(kFull, qv, 1);   // the odd neighbour's code (4-bit pairs)
+      unsigned char* codes = static_cast<unsigned char*>(kside ? p.C.coef_k : p.C.coef_v) +
+                             row * (size_t)(r * CB / 8);
+      if (j < r) {
+        if (CB == 8) codes[j] = (unsigned char)(qv & 0xff);
+        else if ((j & 1) == 0) codes[j >> 1] = (unsigned char)((qv & 0xf) | ((qn & 0xf) << 4));
+        *cval = s * (float)qv;   // the coefficient as the decode reads it
+      }
+      if (j == 0) (kside ? p.C.scale_k : p.C.scale_v)[row] = s;
+    }
+  }
+  __syncthreads();   // every stored coefficient in, for the token's logit and value row
   if (keep) {
     if (tid < kD) reinterpret_cast<uint16_t*>(p.C.full_k)[(bh * D.F_cap + F) * kD + tid] = xe;
     else reinterpret_cast<uint16_t*>(p.C.full_v)[(bh * D.F_cap + F) * kD + tid - kD] = xe;
@@ -246,23 +287,24 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
       const uint16_t* qrow = reinterpret_cast<const uint16_t*>(p.q) + ((size_t)b * D.Hq + (size_t)h * G + warp) * kD;
       for (int i = lane; i < kD; i += 32) sd = fmaf(bf2f(qrow[i]), app[S::A_X + i], sd);
       sd = warp_sum(sd) * scale;
-    } else {        // compressed: q . mu_k + q~ . bf16(c_k), both already scaled
-      for (int j = lane; j < RK; j += 32) sd = fmaf(app[S::A_QT + warp * RK + j], bf2f(f2bf(app[S::A_CK + j])), sd);
+    } else {        // compressed: q . mu_k + q~ . c_k as stored, both already scaled
+      for (int j = lane; j < RK; j += 32) sd = fmaf(app[S::A_QT + warp * RK + j], app[S::A_CK + j], sd);
       sd = warp_sum(sd) + s_bias[warp];
     }
     if (lane == 0) s_new[warp] = sd;
   }
-  if (tid < kD) s_vals[tid] = keep ? app[S::A_X + kD + tid] : (tid < RV ? bf2f(f2bf(app[S::A_CV + tid])) : 0.f);
+  if (tid < kD) s_vals[tid] = keep ? app[S::A_X + kD + tid] : (tid < RV ? app[S::A_CV + tid] : 0.f);
 }
 
-template <int G, int RK, int RV, int W, int NS, bool APP>
+template <int G, int RK, int RV, int W, int NS, bool APP, int CB>
 __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p) {
-  using S = Shape<G, RK, RV, W, NS>;
+  using S = Shape<G, RK, RV, W, NS, CB>;
   static_assert(!APP || W * 32 == 2 * kD, "the fused append maps one row element to a thread");
   constexpr int kWarps = S::kWarps, kThreads = S::kThreads;
   constexpr int KST = RK / 16;                   // k-steps of the compressed logits
   constexpr int MVT = RV / 16;                   // m-tiles of the compressed value sum
-  constexpr int KP = S::KP, VP = S::VP;
+  constexpr int KP = S::KP, VP = S::VP;          // 16-byte pieces per stored row
+  constexpr int UKP = S::UKP, UVP = S::UVP;      // 16-byte pieces per basis row
   constexpr int NST = S::STAGES;
   extern __shared__ __align__(128) unsigned char sm[];
   const lrkv_dims& D = p.D;
@@ -287,8 +329,8 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
      // append when it differs
     auto load_uk = [&](const lrkv_bf16* src, unsigned char* dst) {
       const unsigned char* Uk = reinterpret_cast<const unsigned char*>(src + (size_t)h * kD * RK);
-      for (int q = tid; q < kD * KP; q += kThreads) {
-        const int r = q / KP, sg = q - r * KP;
+      for (int q = tid; q < kD * UKP; q += kThreads) {
+        const int r = q / UKP, sg = q - r * UKP;
         cp_async16(dst + r * S::KS + sg * 16, Uk + q * 16);
       }
     };
@@ -298,8 +340,8 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   }
   auto load_uv = [&]() {   // U_v into padded rows, 16-byte pieces over every thread
     const unsigned char* Uv = reinterpret_cast<const unsigned char*>(p.C.U_v + (size_t)h * kD * RV);
-    for (int q = tid; q < kD * VP; q += kThreads) {
-      const int r = q / VP, sg = q - r * VP;
+    for (int q = tid; q < kD * UVP; q += kThreads) {
+      const int r = q / UVP, sg = q - r * UVP;
       cp_async16(sm + S::OFF_UV + r * S::VS + sg * 16, Uv + q * 16);
     }
     cp_async_commit();
@@ -379,8 +421,10 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   const int share = (F + n_chunks - 1) / n_chunks;
   const int f0 = min(F, c * share), f1 = min(F, f0 + share);
   const int n_full = f1 - f0;
-  const lrkv_bf16* ck = p.C.coef_k + bh * D.T_cap * RK + (size_t)c0 * RK;
-  const lrkv_bf16* cv = p.C.coef_v + bh * D.T_cap * RV + (size_t)c0 * RV;
+  const unsigned char* ck = static_cast<const unsigned char*>(p.C.coef_k) + (bh * D.T_cap + c0) * S::TKB;
+  const unsigned char* cv = static_cast<const unsigned char*>(p.C.coef_v) + (bh * D.T_cap + c0) * S::TVB;
+  const float* sck = CB < 16 ? p.C.scale_k + bh * D.T_cap + c0 : nullptr;   // code scales
+  const float* scv = CB < 16 ? p.C.scale_v + bh * D.T_cap + c0 : nullptr;
   const lrkv_bf16* fk = p.C.full_k + (bh * D.F_cap + f0) * kD;
   const lrkv_bf16* fv = p.C.full_v + (bh * D.F_cap + f0) * kD;
 
@@ -427,20 +471,26 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     if (wi_copy.next(nct_w, n_tiles, kw)) {
       const int k = warp + kWarps * kw;
       const uint32_t bits = masked ? tile_bits(k) : valid_bits(k);
-      const unsigned char* src_k = reinterpret_cast<const unsigned char*>(ck + (size_t)k * kTileC * RK);
-      const unsigned char* src_v = reinterpret_cast<const unsigned char*>(cv + (size_t)k * kTileC * RV);
+      const unsigned char* src_k = ck + (size_t)k * kTileC * S::TKB;
+      const unsigned char* src_v = cv + (size_t)k * kTileC * S::TVB;
 #pragma unroll
       for (int j = 0; j < KP; ++j) {   // piece q = lane + 32 j of the tile's key rows
         const int q = lane + 32 * j, r = q / KP, sg = q - r * KP;
         const bool on = (bits >> r) & 1u;
-        cp_async16_zfill(slot + r * S::KS + sg * 16, on ? src_k + q * 16 : src_k, on ? 16u : 0u);
+        cp_async16_zfill(slot + r * S::TKS + sg * 16, on ? src_k + q * 16 : src_k, on ? 16u : 0u);
       }
-      unsigned char* vslot = slot + kTileC * S::KS;
+      unsigned char* vslot = slot + kTileC * S::TKS;
 #pragma unroll
       for (int j = 0; j < VP; ++j) {
         const int q = lane + 32 * j, r = q / VP, sg = q - r * VP;
         const bool on = (bits >> r) & 1u;
-        cp_async16_zfill(vslot + r * S::VS + sg * 16, on ? src_v + q * 16 : src_v, on ? 16u : 0u);
+        cp_async16_zfill(vslot + r * S::TVS + sg * 16, on ? src_v + q * 16 : src_v, on ? 16u : 0u);
+      }
+      if constexpr (CB < 16) {   // the tile's 32 key and 32 value scales: 16 pieces
+        if (lane < 16) {
+          const float* src = (lane < 8 ? sck : scv) + (size_t)k * kTileC + (lane & 7) * 4;
+          cp_async16(slot + S::T_SC + lane * 16, src);
+        }
       }
     } else {
       const int k = warp + kWarps * kw;
@@ -495,10 +545,26 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       }
     }
     // lane (m, t) holds q~[head m][16 ks2 + 2t (+1)] in a0 and [+8] in a1 (rows m < 4).
-    // B column g = 2h + part takes head h from lane 4h + t.
-    const int src = ((g >> 1) << 2) | t;
-    const float x0 = __shfl_sync(kFull, a0[0], src), x1 = __shfl_sync(kFull, a0[1], src);
-    const float y0 = __shfl_sync(kFull, a1[0], src), y1 = __shfl_sync(kFull, a1[1], src);
+    // B column g = 2h + part takes head h from lane 4h + t'.  The B fragment of
+    // k = 2t, 2t+1 (b0) and 2t+8, 2t+9 (b1) is the q~ columns of those k in the
+    // tiles' contraction order: the same columns for bf16 rows; for int8 codes a
+    // thread's four bytes 4t..4t+3 are k = 2t, 2t+1, 2t+8, 2t+9, so b0 holds
+    // columns 4t, 4t+1 and b1 columns 4t+2, 4t+3.
+    const int hq4 = (g >> 1) << 2;
+    const int sa = hq4 | (CB == 16 ? t : (t < 2 ? 2 * t : 2 * t - 4));
+    const int sb = hq4 | (CB == 16 ? t : (t < 2 ? 2 * t + 1 : 2 * t - 3));
+    const bool from_a1 = CB == 16 ? false : t >= 2;   // columns 8..15 of the block
+    const float pa0 = __shfl_sync(kFull, a0[0], sa), pa1 = __shfl_sync(kFull, a0[1], sa);
+    const float qa0_ = __shfl_sync(kFull, a1[0], sa), qa1_ = __shfl_sync(kFull, a1[1], sa);
+    const float pb0 = __shfl_sync(kFull, a0[0], sb), pb1 = __shfl_sync(kFull, a0[1], sb);
+    const float qb0_ = __shfl_sync(kFull, a1[0], sb), qb1_ = __shfl_sync(kFull, a1[1], sb);
+    float x0, x1, y0, y1;   // b0's and b1's two columns
+    if (CB == 16) {
+      x0 = pa0, x1 = pa1, y0 = qb0_, y1 = qb1_;
+    } else {
+      x0 = from_a1 ? qa0_ : pa0, x1 = from_a1 ? qa1_ : pa1;
+      y0 = from_a1 ? qb0_ : pb0, y1 = from_a1 ? qb1_ : pb1;
+    }
     const bool lo_n = g & 1;
     const bool live = (g >> 1) < G;
     s_qb[ks2][0][lane] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
@@ -560,7 +626,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   // from its first step on)
   if constexpr (APP) {
     if (owner) {
-      append_token<S, G, RK, RV>(p, app, p.C.U_kq ? sm + S::OFF_UK2 : uk, uk, sm + S::OFF_UV, s_bias,
+      append_token<S, G, RK, RV, CB>(p, app, p.C.U_kq ? sm + S::OFF_UK2 : uk, uk, sm + S::OFF_UV, s_bias,
                                  b, h, bh, T_old, F, scale, xe, s_new, s_vals, &s_keep);
       __syncthreads();   // the token's logits and value row in for warp 0
     }
@@ -580,8 +646,9 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   // Online softmax over NB 16-row blocks: s[nb] = {row g, row g + 8} of head t
   // (-inf = no token).  Rescales this lane's accumulators when the max grows,
   // and returns the probabilities packed as the P^T B fragments of each block
-  // (column 2t = bf16 high part, 2t + 1 = low part).
-  auto softmax_pack = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag) {
+  // (column 2t = bf16 high part, 2t + 1 = low part); with value weights wv
+  // (the rows' code scales) the packed entries are p * wv, the sum l takes p.
+  auto softmax_pack_w = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag, const float (*wv)[2]) {
     constexpr int NB = decltype(nb_tag)::value;
     float x = -INFINITY;
 #pragma unroll
@@ -604,15 +671,19 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     __syncwarp();
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
-      const float p0 = s[nb][0] == -INFINITY ? 0.f : exp2f(s[nb][0] - m_run);
-      const float p1 = s[nb][1] == -INFINITY ? 0.f : exp2f(s[nb][1] - m_run);
+      float p0 = s[nb][0] == -INFINITY ? 0.f : exp2f(s[nb][0] - m_run);
+      float p1 = s[nb][1] == -INFINITY ? 0.f : exp2f(s[nb][1] - m_run);
       l_run += p0 + p1;
+      if (wv) p0 *= wv[nb][0], p1 *= wv[nb][1];
       // (high part, low part) of p: bf16(p) and bf16(p - bf16(p))
       const float h0 = __uint_as_float(cvt_bf16x2(p0, p0) << 16);
       const float h1 = __uint_as_float(cvt_bf16x2(p1, p1) << 16);
       pb0[nb] = movmatrix_t(cvt_bf16x2(p0, p0 - h0));
       pb1[nb] = movmatrix_t(cvt_bf16x2(p1, p1 - h1));
     }
+  };
+  auto softmax_pack = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag) {
+    softmax_pack_w(s, pb0, pb1, nb_tag, static_cast<const float (*)[2]>(nullptr));
   };
 
   for (int i = 0; i < n_tiles; ++i) {
@@ -626,37 +697,92 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       // compressed tile: S^T[token][head part] = C_k q~^T, then O^T += C_v^T P^T
       const uint32_t bits = tile_bits(warp + kWarps * kw);
       float st[2][4];
-#pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-        st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < KST; ++ks) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(a0, a1, a2, a3,
-                  slot + (16 * nb + (lm & 1) * 8 + lr) * S::KS + (ks * 16 + (lm >> 1) * 8) * 2);
-          mma_16816(st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
-        }
-      }
-      float s[2][2];
-#pragma unroll
-      for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {   // rows g, g + 8: high + low part of head t
-          const float v = st[nb][2 * x] + st[nb][2 * x + 1] + bias;
-          s[nb][x] = live_t && ((bits >> (16 * nb + g + x * 8)) & 1u) ? v : -INFINITY;
-        }
-      uint32_t pb0[2], pb1[2];
-      softmax_pack(s, pb0, pb1, std::integral_constant<int, 2>{});
-      const unsigned char* vrows = slot + kTileC * S::KS;
-#pragma unroll
-      for (int mt = 0; mt < MVT; ++mt)
+      if constexpr (CB == 16) {
 #pragma unroll
         for (int nb = 0; nb < 2; ++nb) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(a0, a1, a2, a3,
-                    vrows + (16 * nb + (lm >> 1) * 8 + lr) * S::VS + (mt * 16 + (lm & 1) * 8) * 2);
-          mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
+          st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
+#pragma unroll
+          for (int ks = 0; ks < KST; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(a0, a1, a2, a3,
+                    slot + (16 * nb + (lm & 1) * 8 + lr) * S::TKS + (ks * 16 + (lm >> 1) * 8) * 2);
+            mma_16816(st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
+          }
         }
+        float s[2][2];
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {   // rows g, g + 8: high + low part of head t
+            const float v = st[nb][2 * x] + st[nb][2 * x + 1] + bias;
+            s[nb][x] = live_t && ((bits >> (16 * nb + g + x * 8)) & 1u) ? v : -INFINITY;
+          }
+        uint32_t pb0[2], pb1[2];
+        softmax_pack(s, pb0, pb1, std::integral_constant<int, 2>{});
+        const unsigned char* vrows = slot + kTileC * S::TKS;
+#pragma unroll
+        for (int mt = 0; mt < MVT; ++mt)
+#pragma unroll
+          for (int nb = 0; nb < 2; ++nb) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(a0, a1, a2, a3,
+                      vrows + (16 * nb + (lm >> 1) * 8 + lr) * S::TVS + (mt * 16 + (lm & 1) * 8) * 2);
+            mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
+          }
+      } else {
+        // int8 codes, converted to bf16 in registers (exact).  Logits: an
+        // ldmatrix of a k-step's 16 code bytes gives a thread bytes 4t..4t+3 of
+        // its row, k = 2t, 2t+1 (a0/a1) and 2t+8, 2t+9 (a2/a3) in the order q~'s
+        // B fragments were built in; the row's key scale multiplies the logit.
+        const float* scl = reinterpret_cast<const float*>(slot + S::T_SC);   // [2][32]
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+          st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
+          const unsigned char* rows = slot + (16 * nb + (lm & 1) * 8 + lr) * S::TKS;
+#pragma unroll
+          for (int kp = 0; kp < KST; kp += 2) {
+            uint32_t r0, r1, r2 = 0u, r3 = 0u, e0, e1, f0, f1;
+            if (kp + 1 < KST) ldsm_x4(r0, r1, r2, r3, rows + kp * 16 + (lm >> 1) * 16);
+            else ldsm_x2(r0, r1, rows + kp * 16);
+            s8x4_pairs(r0, e0, f0);
+            s8x4_pairs(r1, e1, f1);
+            mma_16816(st[nb], e0, e1, f0, f1, qb0[kp], qb1[kp]);
+            if (kp + 1 < KST) {
+              s8x4_pairs(r2, e0, f0);
+              s8x4_pairs(r3, e1, f1);
+              mma_16816(st[nb], e0, e1, f0, f1, qb0[kp + 1], qb1[kp + 1]);
+            }
+          }
+        }
+        float s[2][2], wv[2][2];
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {   // rows g, g + 8: high + low part of head t
+            const int row = 16 * nb + g + x * 8;
+            const bool on = live_t && ((bits >> row) & 1u);
+            const float v = st[nb][2 * x] + st[nb][2 * x + 1];
+            s[nb][x] = on ? fmaf(v, scl[row], bias) : -INFINITY;
+            wv[nb][x] = on ? scl[kTileC + row] : 0.f;   // scales of unread rows are never used
+          }
+        uint32_t pb0[2], pb1[2];
+        softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv);
+        // values: one transposing ldmatrix per 16 value columns covers the 32
+        // tokens; a thread's bytes are (token 2t | 2t+1) x (column 2g | 2g+1), so
+        // accumulator row g is column 2g of the block and row g + 8 column 2g + 1
+        const unsigned char* vrows = slot + kTileC * S::TKS;
+#pragma unroll
+        for (int mt = 0; mt < MVT; ++mt) {
+          uint32_t r0, r1, r2, r3, a0, a1, a2, a3;
+          ldsm_x4_t(r0, r1, r2, r3, vrows + (8 * lm + lr) * S::TVS + mt * 16);
+          s8x4_evenodd(r0, a0, a1);
+          s8x4_evenodd(r1, a2, a3);
+          mma_16816(oc[mt], a0, a1, a2, a3, pb0[0], pb1[0]);
+          s8x4_evenodd(r2, a0, a1);
+          s8x4_evenodd(r3, a2, a3);
+          mma_16816(oc[mt], a0, a1, a2, a3, pb0[1], pb1[1]);
+        }
+      }
     } else {
       // full-rank tile: 16 list rows
       const int k = warp + kWarps * kw;
@@ -713,11 +839,11 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
         of[mi][0] = fmaf(pn, s_vals[16 * mi + g], of[mi][0]);
         of[mi][2] = fmaf(pn, s_vals[16 * mi + g + 8], of[mi][2]);
       }
-    } else {
+    } else {   // accumulator rows g, g + 8 are value columns g, g + 8 (bf16) or 2g, 2g + 1 (codes)
 #pragma unroll
       for (int mt = 0; mt < MVT; ++mt) {
-        oc[mt][0] = fmaf(pn, s_vals[16 * mt + g], oc[mt][0]);
-        oc[mt][2] = fmaf(pn, s_vals[16 * mt + g + 8], oc[mt][2]);
+        oc[mt][0] = fmaf(pn, s_vals[16 * mt + (CB == 16 ? g : 2 * g)], oc[mt][0]);
+        oc[mt][2] = fmaf(pn, s_vals[16 * mt + (CB == 16 ? g + 8 : 2 * g + 1)], oc[mt][2]);
       }
     }
   }
@@ -744,7 +870,19 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
 #pragma unroll
       for (int mt = 0; mt < MVT; ++mt) {
         uint32_t a0, a1, a2, a3;
-        ldsm_x4(a0, a1, a2, a3, uv + (16 * mi + (lm & 1) * 8 + lr) * S::VS + (mt * 16 + (lm >> 1) * 8) * 2);
+        if constexpr (CB == 16) {
+          ldsm_x4(a0, a1, a2, a3, uv + (16 * mi + (lm & 1) * 8 + lr) * S::VS + (mt * 16 + (lm >> 1) * 8) * 2);
+        } else {
+          // accumulator row k of the block is value column 2k (k < 8) or
+          // 2(k - 8) + 1: A[i][k] = U_v[i][that column], so a thread's k = 2t,
+          // 2t+1 are columns 4t, 4t+2 and k = 2t+8, 2t+9 columns 4t+1, 4t+3
+          const uint2 w0 = *reinterpret_cast<const uint2*>(uv + (16 * mi + g) * S::VS + (mt * 16 + 4 * t) * 2);
+          const uint2 w1 = *reinterpret_cast<const uint2*>(uv + (16 * mi + g + 8) * S::VS + (mt * 16 + 4 * t) * 2);
+          a0 = __byte_perm(w0.x, w0.y, 0x5410);
+          a2 = __byte_perm(w0.x, w0.y, 0x7632);
+          a1 = __byte_perm(w1.x, w1.y, 0x5410);
+          a3 = __byte_perm(w1.x, w1.y, 0x7632);
+        }
         mma_16816(of[mi], a0, a1, a2, a3, lb0[mt], lb1[mt]);
       }
   }

@@ -26,6 +26,10 @@ __device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float(uint3
 __device__ __forceinline__ uint16_t f2bf(float x) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
+// x rounded to bf16 (nearest even), as fp32
+__device__ __forceinline__ float bf16_round(float x) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -37,6 +41,29 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
+}
+
+// Stored coefficient format: bits per coefficient (16 bf16, 8 or 4 integer codes).
+__host__ __device__ __forceinline__ int coef_bits_of(const lrkv_dims& D) {
+  return D.coef_bits == 0 ? 16 : D.coef_bits;
+}
+__host__ __device__ __forceinline__ bool coef_quantised(const lrkv_dims& D) {
+  return coef_bits_of(D) < 16;
+}
+
+// Per-row quantisation of a stored coefficient row (codes with per-vector
+// scales): Q = 127 for 8 bits, 7 for 4 bits; s = amax / Q with amax the largest
+// |bf16(c_j)|; q_j = round_half_even(bf16(c_j) / s) clamped to [-Q, Q]; s = 0
+// gives q = 0.  Every step is IEEE fp32 (correctly rounded division), so the
+// decisions are those of any implementation of the same steps.
+__device__ __forceinline__ float quant_scale(float amax, int bits) {
+  return __fdiv_rn(amax, bits == 8 ? 127.f : 7.f);
+}
+__device__ __forceinline__ int quant_code(float cb, float s, int bits) {
+  if (!(s > 0.f)) return 0;
+  const int Q = bits == 8 ? 127 : 7;
+  const int qv = __float2int_rn(__fdiv_rn(cb, s));
+  return qv > Q ? Q : (qv < -Q ? -Q : qv);
 }
 
 // Number of new tokens sequence b contributes, and the status bits it raises.

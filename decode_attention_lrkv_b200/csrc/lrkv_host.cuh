@@ -26,6 +26,8 @@ inline lrkv_status check_dims(const lrkv_dims* D) {
   if (D->r_k < 16 || D->r_k > D->d || D->r_k % 16 || D->r_v < 16 || D->r_v > D->d || D->r_v % 16)
     return LRKV_ERR_INVALID_ARG;
   if (D->Hq / D->Hkv > kMaxG) return LRKV_ERR_UNSUPPORTED;
+  if (D->coef_bits != 0 && D->coef_bits != 16 && D->coef_bits != 8 && D->coef_bits != 4)
+    return LRKV_ERR_INVALID_ARG;
   return LRKV_OK;
 }
 
@@ -45,6 +47,10 @@ inline lrkv_status check_cache(const lrkv_dims* D, const lrkv_cache* C) {
   for (const void* p : full)
     if (!aligned16(p)) return LRKV_ERR_ALIGNMENT;
   if (!aligned16(C->U_kq) || !aligned16(C->mu_k)) return LRKV_ERR_ALIGNMENT;   // optional
+  if (coef_quantised(*D)) {   // per-row scales of the codes
+    if (!C->scale_k || !C->scale_v) return LRKV_ERR_INVALID_ARG;
+    if (!aligned16(C->scale_k) || !aligned16(C->scale_v)) return LRKV_ERR_ALIGNMENT;
+  }
   return LRKV_OK;
 }
 

@@ -123,6 +123,11 @@ __device__ __forceinline__ void ldsm_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(smem_u32(row_addr)));
 }
+__device__ __forceinline__ void ldsm_x2(uint32_t& r0, uint32_t& r1, const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(smem_u32(row_addr)));
+}
 __device__ __forceinline__ void ldsm_x4_t(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
                                           const void* row_addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -212,6 +217,33 @@ __device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
   uint32_t d;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
   return d;
+}
+
+}  // namespace lrkv
+
+namespace lrkv {
+
+// int8 codes -> bf16, exactly.  A byte b read as unsigned after flipping its
+// sign bit is b + 128; placed in the low mantissa bits of 2^23 that fp32 is
+// 2^23 + b + 128, so subtracting 2^23 + 128 gives b as fp32.  An integer of
+// magnitude <= 128 has its bf16 value in the upper half of its fp32 bits.
+__device__ __forceinline__ float s8_byte_f32(uint32_t flipped, uint32_t sel) {
+  return __uint_as_float(__byte_perm(flipped, 0x4B000000u, sel)) - 8388736.f;
+}
+__device__ __forceinline__ uint32_t bf16x2_upper(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x7632);
+}
+// Four int8 codes in w: bf16x2 of bytes (0, 1) and of bytes (2, 3).
+__device__ __forceinline__ void s8x4_pairs(uint32_t w, uint32_t& b01, uint32_t& b23) {
+  const uint32_t u = w ^ 0x80808080u;
+  b01 = bf16x2_upper(s8_byte_f32(u, 0x7440), s8_byte_f32(u, 0x7441));
+  b23 = bf16x2_upper(s8_byte_f32(u, 0x7442), s8_byte_f32(u, 0x7443));
+}
+// Four int8 codes in w: bf16x2 of bytes (0, 2) and of bytes (1, 3).
+__device__ __forceinline__ void s8x4_evenodd(uint32_t w, uint32_t& b02, uint32_t& b13) {
+  const uint32_t u = w ^ 0x80808080u;
+  b02 = bf16x2_upper(s8_byte_f32(u, 0x7440), s8_byte_f32(u, 0x7442));
+  b13 = bf16x2_upper(s8_byte_f32(u, 0x7441), s8_byte_f32(u, 0x7443));
 }
 
 }  // namespace lrkv

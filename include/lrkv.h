@@ -88,14 +88,32 @@ typedef struct {
   int32_t r_v;   /* value rank, multiple of 16 in [16, d] */
   int32_t T_cap; /* positions per sequence the cache can hold, multiple of 32 */
   int32_t F_cap; /* full-rank rows per (sequence, kv head) the list can hold, >= 0 */
+  int32_t coef_bits; /* stored coefficient format: 0 or 16 = bf16; 8 = int8 codes;
+                        4 = int4 codes (see "Quantised coefficients" below) */
 } lrkv_dims;
+
+/* Quantised coefficients (coef_bits 8 or 4).  KVQuant record ("Quant method":
+ * sub-8-bit codes with a per-vector scale) and NOVA-KV summary (fixed-width
+ * codes read inside attention), applied to this cache's coefficient rows: each
+ * stored row (c_k or c_v of one token and kv head) is quantised on its own,
+ * symmetric and absmax-scaled, from its bf16 value c (round to nearest even):
+ *     Q = 127 (8 bits) or 7 (4 bits)
+ *     s = max_j |c_j| / Q                     (fp32 division, correctly rounded)
+ *     q_j = round_half_even(c_j / s)          (fp32 division), clamped to [-Q, Q]
+ *     s = 0 (an all-zero row) gives q = 0;    c_hat_j = s q_j
+ * with no flush of subnormals, so any implementation of these IEEE steps takes
+ * the same decisions.  Codes are two's complement; 4-bit codes are packed two
+ * per byte, element 2i in the low nibble.  The decode reads c_hat: compressed
+ * logits s_k,t (q~ . q_k,t) / sqrt(d), value weights p_t s_v,t.  The routing
+ * error is still that of the unrounded projection. */
 
 /* One layer of compressed cache.  Every pointer is a device pointer. */
 typedef struct {
   const lrkv_bf16* U_k; /* [Hkv][d][r_k] key basis (orthonormal columns, rounded to bf16) */
   const lrkv_bf16* U_v; /* [Hkv][d][r_v] value basis */
-  lrkv_bf16* coef_k;    /* [B][Hkv][T_cap][r_k] key coefficients, indexed by position */
-  lrkv_bf16* coef_v;    /* [B][Hkv][T_cap][r_v] value coefficients */
+  void* coef_k;         /* [B][Hkv][T_cap][r_k] key coefficients, indexed by position: bf16,
+                           or [B][Hkv][T_cap][r_k * coef_bits / 8] bytes of codes */
+  void* coef_v;         /* [B][Hkv][T_cap][r_v] value coefficients, likewise */
   uint32_t* route_mask; /* [B][Hkv][T_cap/32]; bit p%32 of word p/32 = position p is full rank */
   int32_t* full_idx;    /* [B][Hkv][F_cap] positions of the full-rank rows, ascending */
   lrkv_bf16* full_k;    /* [B][Hkv][F_cap][d] key rows of full-rank tokens */
@@ -115,6 +133,9 @@ typedef struct {
      transformed.  A cache must keep the same choice for all its calls. */
   const lrkv_bf16* U_kq; /* nullable [Hkv][d][r_k] query-side / key reconstruction basis */
   const float* mu_k;     /* nullable [Hkv][d] fp32 key mean */
+  float* scale_k;        /* [B][Hkv][T_cap] fp32 per-row scales of quantised key codes
+                            (coef_bits 8 or 4; unused, may be null, for bf16) */
+  float* scale_v;        /* [B][Hkv][T_cap] likewise for the value codes */
 } lrkv_cache;
 /* A new cache is all zeros (seq_len = full_cnt = 0).  The library writes every
    mask bit, coefficient row and list entry it covers, so stale contents past

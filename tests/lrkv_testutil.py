@@ -27,9 +27,9 @@ def f64(t):
     return t.detach().float().cpu().double().numpy()
 
 
-def dims_of(w, T_cap, F_cap=None, B=None):
+def dims_of(w, T_cap, F_cap=None, B=None, coef_bits=0):
     return L.Dims(B=B or w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, r_k=w.r_k, r_v=w.r_v, T_cap=T_cap,
-                  F_cap=T_cap if F_cap is None else F_cap)
+                  F_cap=T_cap if F_cap is None else F_cap, coef_bits=coef_bits)
 
 
 def oracle_dims(D):

@@ -62,8 +62,10 @@ def test_workspace_size(lib):
     n = L.lrkv_workspace_size(_dims())
     assert n > 0 and n % 256 == 0
     assert L.lrkv_workspace_size(_dims(T_cap=16384)) > n
+    assert L.lrkv_workspace_size(_dims(coef_bits=8)) == n       # the format needs no workspace
     for bad in (dict(d=64), dict(r_k=40), dict(r_v=0), dict(r_k=144), dict(Hq=30),
-                dict(T_cap=100), dict(T_cap=0), dict(F_cap=-1), dict(B=0), dict(Hq=72, Hkv=8)):
+                dict(T_cap=100), dict(T_cap=0), dict(F_cap=-1), dict(B=0), dict(Hq=72, Hkv=8),
+                dict(coef_bits=3), dict(coef_bits=32)):
         assert L.lrkv_workspace_size(_dims(**bad)) == 0, bad
     assert lib.lrkv_workspace_size(None) == 0
 
@@ -122,6 +124,11 @@ def test_host_validation_rejects_before_launch(lib):
     assert _call_compress(lib, _dims(F_cap=0), _FakeCache(full_k=None, full_v=None, full_idx=None),
                           t_new=0) == 0
     assert _call_compress(lib, D, _FakeCache(full_v=None)) == INVALID
+    # quantised coefficients need their per-row scales
+    Dq = _dims(coef_bits=8)
+    assert _call_compress(lib, Dq, _FakeCache(scale_v=None)) == INVALID
+    assert _call_decode(lib, Dq, _FakeCache(scale_k=0x50000008)) == ALIGN
+    assert _call_compress(lib, D, _FakeCache(scale_k=None, scale_v=None), t_new=0) == 0   # bf16: unused
     # the attention-aware key basis and mean are optional, aligned when given
     assert _call_compress(lib, D, _FakeCache(U_kq=None, mu_k=None), t_new=0) == 0
     assert _call_compress(lib, D, _FakeCache(mu_k=0x50000004)) == ALIGN
