@@ -485,6 +485,7 @@ def run_ours(args, rank, world, dev):
 
     # --- end-to-end through host buffers --------------------------------------------------
     e2e = run_e2e(L, args, w, dims, ws, layers, dev, world, steps_total)
+    side = side_measurements(L, w, dims, layers, dev, pk)
 
     result = {
         "metric": "compressed-KV decode attn µs/step & HBM GB/s vs 8 TB/s; compress tok/s",
@@ -542,11 +543,63 @@ def run_ours(args, rank, world, dev):
                                  "timing": "one CUDA graph of every layer's decode, K times back "
                                            "to back (no appends), CUDA events around the replay"}},
         "e2e": e2e,
+        "side": side,
         "gpu_launches": K * w.layers * (FUSED_LAUNCHES if dims.bits != 4 and w.g in (1, 2, 4)
                                         else 2),   # 4-bit codes or other groups: append + decode
         "clocks": clk,
     }
     return result, w, layers, dims
+
+
+def _event_time_ms(fn, reps, warm=3):
+    """Mean device time of fn() over reps calls, CUDA events around the batch."""
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def side_measurements(L, w, dims, layers, dev, pk):
+    """Timings of the calls the step does not use, on this workload's geometry:
+    the online basis update (one Oja batch step of every kv head's key basis
+    over 4096 rows) and the CUDA-core decode kernel, which serves query groups
+    the streaming kernel has no instantiation for (GQA 3 and 8 on layer 0's
+    cache; the cache does not depend on the query heads)."""
+    out = {}
+    g = torch.Generator(device=dev).manual_seed(99)
+    n_rows = 4096
+    X = torch.randn(n_rows, w.Hkv, w.d, generator=g, device=dev).to(torch.bfloat16)
+    U = torch.linalg.qr(torch.randn(w.Hkv, w.d, w.r_k, generator=g, device=dev, dtype=torch.float64))[0].float()
+    Ub = torch.empty(w.Hkv, w.d, w.r_k, dtype=torch.bfloat16, device=dev)
+    ows = torch.empty(L.lrkv_oja_workspace_size(dims, n_rows, w.r_k), dtype=torch.uint8, device=dev)
+    ms = _event_time_ms(lambda: L.lrkv_oja_update(dims, X, U, 1e-3, U_out=Ub, ws=ows), 10)
+    flops = 4.0 * n_rows * w.d * w.r_k * w.Hkv
+    out["oja_update"] = {"us_per_call": round(ms * 1e3, 2), "rows": n_rows, "kv_heads": w.Hkv,
+                         "rank": w.r_k, "tflops": round(flops / (ms * 1e-3) / 1e12, 3),
+                         "note": "one batch step (sums on CUDA cores in fp32, fp64 step + Gram-Schmidt)"}
+    lay = layers[0]
+    fb = {}
+    for gg in (3, 8):
+        Dg = L.Dims(B=dims.B, Hq=gg * dims.Hkv, Hkv=dims.Hkv, d=dims.d, r_k=dims.r_k, r_v=dims.r_v,
+                    T_cap=dims.T_cap, F_cap=dims.F_cap, coef_bits=dims.coef_bits)
+        wsg = L.make_workspace(Dg, dev)
+        q = torch.randn(dims.B, Dg.Hq, dims.d, generator=g, device=dev).to(torch.bfloat16)
+        o = torch.empty(dims.B, Dg.Hq, dims.d, dtype=torch.float32, device=dev)
+        ms = _event_time_ms(lambda: L.lrkv_decode_attn(Dg, lay["cache"], q, o, ws=wsg), 10)
+        fc = lay["cache"].full_cnt.cpu().numpy()
+        nb = A.decode_bytes(Dg.B, Dg.Hq, Dg.Hkv, Dg.d, Dg.r_k, Dg.r_v, lay["cache"].seq_len.cpu().tolist(), fc,
+                            coef_bits=dims.bits)
+        fb[f"gqa{gg}"] = {"us_per_launch": round(ms * 1e3, 2), "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+                          "frac_of_measured_hbm": round(nb / (ms * 1e-3) / 1e9 / pk.get("hbm_gbs", 6549.1), 4)}
+        del wsg
+    out["cuda_core_decode"] = fb
+    return out
 
 
 def run_e2e(L, args, w, dims, ws, layers, dev, world, steps_total):

@@ -15,6 +15,8 @@ Entry points (same names as the C ABI):
     lrkv_fit_workspace_size(dims, n_rows) -> int
     lrkv_fit_basis(dims, X, r, ...) -> (U [Hkv,d,r] bf16, eigenvalues [Hkv,d] fp32)
     lrkv_rank_for_budget(eigvals, budget) -> int32 ranks   (host call)
+    lrkv_oja_workspace_size(dims, n_rows, r) -> int
+    lrkv_oja_update(dims, X, U, eta, U_out=None)   (online basis update, U fp32 in place)
     lrkv_status_str(code) -> str
 plus ``LayerCache`` (allocates one layer's buffers with torch) and
 ``make_workspace``.
@@ -37,6 +39,7 @@ STATUS_NAMES = {0: "LRKV_OK", 1: "LRKV_ERR_INVALID_ARG", 2: "LRKV_ERR_UNSUPPORTE
 DEV_FULL_OVERFLOW = 0x1
 DEV_SEQ_OVERFLOW = 0x2
 DEV_BAD_COUNT = 0x4
+DEV_WAIT_TIMEOUT = 0x8
 
 
 class LrkvError(RuntimeError):
@@ -87,6 +90,11 @@ def load_library(path=None):
     lib.lrkv_fit_basis.argtypes = [ctypes.POINTER(_Dims), P, ctypes.c_int32, ctypes.c_int32, P, P, P,
                                    ctypes.c_size_t, P]
     lib.lrkv_fit_basis.restype = ctypes.c_int
+    lib.lrkv_oja_workspace_size.argtypes = [ctypes.POINTER(_Dims), ctypes.c_int32, ctypes.c_int32]
+    lib.lrkv_oja_workspace_size.restype = ctypes.c_size_t
+    lib.lrkv_oja_update.argtypes = [ctypes.POINTER(_Dims), P, ctypes.c_int32, ctypes.c_int32,
+                                    ctypes.c_float, P, P, P, ctypes.c_size_t, P]
+    lib.lrkv_oja_update.restype = ctypes.c_int
     lib.lrkv_rank_for_budget.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_double, P]
     lib.lrkv_rank_for_budget.restype = ctypes.c_int
     lib.lrkv_status_str.argtypes = [ctypes.c_int]
@@ -259,6 +267,27 @@ def lrkv_append_decode_attn(dims, cache, k_new, v_new, tau, q, out, t_new_b=None
     if check and code != LRKV_OK:
         raise LrkvError(code, "lrkv_append_decode_attn")
     return code
+
+
+def lrkv_oja_workspace_size(dims, n_rows, r):
+    return int(load_library().lrkv_oja_workspace_size(ctypes.byref(dims.c()), int(n_rows), int(r)))
+
+
+def lrkv_oja_update(dims, X, U, eta, U_out=None, ws=None, stream=None, check=True):
+    """One Oja step of every kv head's basis U [Hkv, d, r] (fp32, updated in place)
+    from rows X [..., Hkv, d] (bf16, device); U_out (optional bf16) receives the
+    rounded basis.  See include/lrkv.h."""
+    lib = load_library()
+    n_rows = X.numel() // (dims.Hkv * dims.d)
+    r = int(U.shape[-1])
+    if ws is None:
+        ws = torch.empty(max(lrkv_oja_workspace_size(dims, n_rows, r), 16), dtype=torch.uint8,
+                         device=X.device)
+    code = lib.lrkv_oja_update(ctypes.byref(dims.c()), _ptr(X), int(n_rows), r, float(eta), _ptr(U),
+                               _ptr(U_out), _ptr(ws), ws.numel(), _stream_ptr(stream))
+    if check and code != LRKV_OK:
+        raise LrkvError(code, "lrkv_oja_update")
+    return U_out
 
 
 def lrkv_fit_workspace_size(dims, n_rows):

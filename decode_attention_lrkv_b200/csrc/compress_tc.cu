@@ -2,6 +2,8 @@
 // passes, in their own translation unit (declared in compress_tc.h).
 #include <cuda.h>
 
+#include <cstdlib>
+
 #include "compress_tc.cuh"
 #include "compress_tc.h"
 #include "launch_util.cuh"
@@ -11,6 +13,21 @@ namespace {
 
 lrkv_status launched() {
   return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+}
+
+// Limit of the projection's main-loop wait for each input tile.  The
+// environment variable LRKV_MAIN_WAIT_ITERS (a positive integer) lowers it, so
+// a test can make that bounded wait run out and check that the call reports
+// LRKV_DEV_WAIT_TIMEOUT and leaves the GPU usable; the waits that drain copies
+// and MMAs in flight keep their own limit.
+uint32_t main_wait_iters() {
+  const char* e = std::getenv("LRKV_MAIN_WAIT_ITERS");
+  if (e && *e) {
+    char* end = nullptr;
+    const unsigned long v = std::strtoul(e, &end, 10);
+    if (end && *end == '\0' && v > 0 && v < ptc::kWaitIters) return (uint32_t)v;
+  }
+  return ptc::kWaitIters;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
@@ -63,6 +80,7 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
   pp.tiles_per_b = (tmax + ptc::kTile - 1) / ptc::kTile;
   pp.r_max = D.r_k > D.r_v ? D.r_k : D.r_v;
   pp.n_stages = ptc::stages_for(pp.r_max);
+  pp.wait_iters = main_wait_iters();
   const int groups = 2 * D.Hkv;
   const int n_units = D.B * pp.tiles_per_b;
   int per_group = num_sms() / groups;

@@ -102,6 +102,7 @@ struct Params {
   int tiles_per_b;       // ceil(min(t_new, T_cap) / 128)
   int r_max;             // max(r_k, r_v): the shared-memory layout
   int n_stages;          // input stages: stages_for(r_max)
+  uint32_t wait_iters;   // limit of the MMA issuer's wait for each input tile (kWaitIters)
 };
 
 // Byte offset of element (row n, column k) in a no-swizzle K-major operand:
@@ -139,8 +140,9 @@ struct RowLen {
 
 // Bounded wait that also gives up once another role has aborted.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
-                                              volatile int* abort_flag) {
-  for (uint32_t i = 0; i < kWaitIters; ++i) {
+                                              volatile int* abort_flag,
+                                              uint32_t max_iters = kWaitIters) {
+  for (uint32_t i = 0; i < max_iters; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63) == 63 && *abort_flag) return false;
     if (i > 64) __nanosleep(32);
@@ -366,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
         int start;
         if (t0 >= rl.get(p, b, &start)) continue;
         const int s = i % NS, buf = i & 1;
-        if (!wait_or_abort(&full[s], (i / NS) & 1, abort_flag)) break;
+        if (!wait_or_abort(&full[s], (i / NS) & 1, abort_flag, p.wait_iters)) break;
         if (i >= 2 && !wait_or_abort(&tfree[buf], ((i >> 1) - 1) & 1, abort_flag)) break;
         tc5::fence_after_sync();
         const uint32_t d2 = tmem + buf * 256;   // D2 columns [0, 128), D1 [128, 128 + R)
@@ -448,6 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
           qs = quant_scale(amax, CB);
           if (valid) scales[row] = qs;
         }
+        const float qinv = CB < 16 && qs > 0.f ? 1.f / qs : 0.f;
 #pragma unroll 1
         for (int c0 = 0; c0 < R; c0 += NC) {
           float v[NC / 16][16];
@@ -468,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
               uint32_t cw[4] = {0u, 0u, 0u, 0u};   // 16 codes: 16 bytes (8-bit) or 8 (4-bit)
 #pragma unroll
               for (int k = 0; k < 16; ++k) {
-                const uint32_t cq = (uint32_t)quant_code(bf16_round(w[k]), qs, CB);
+                const uint32_t cq = (uint32_t)quant_code_fast(bf16_round(w[k]), qs, qinv, CB);
                 if (CB == 8) cw[k >> 2] |= (cq & 0xffu) << (8 * (k & 3));
                 else cw[k >> 3] |= (cq & 0xfu) << (4 * (k & 7));
               }

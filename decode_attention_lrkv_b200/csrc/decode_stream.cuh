@@ -52,6 +52,7 @@ namespace lrkv {
 namespace ds {
 
 constexpr int kTileC = 32;                       // positions per compressed tile (one mask word)
+constexpr int kAppendTail = 256;                 // positions the fused append's split gives up
 constexpr int kTileF = 16;                       // rows per full-rank tile
 constexpr int kMaxChunk = kMaxDecodeChunk;       // positions per split (mask words in smem)
 constexpr unsigned kFull = 0xffffffffu;
@@ -397,9 +398,11 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   }
   const int T_old = T;
   T += n_eff;
-  // splits from the live length (every CTA of the (b, kv head) finds the same)
+  // splits from the live length (every CTA of the (b, kv head) finds the same);
+  // with a fused append the owner's split is kept shorter by the append's cost
   int chunk;
-  const int n_chunks = decode_split(T, p.n_chunk_max, (long long)D.B * D.Hkv, p.num_sms, &chunk);
+  const int n_chunks = decode_split(T, p.n_chunk_max, (long long)D.B * D.Hkv, p.num_sms, &chunk,
+                                    APP && n_eff > 0 ? kAppendTail : 0);
   const bool active = c < n_chunks;
   const int c0 = c * chunk;
   // this split's mask words (words past the sequence end are never used): the

@@ -65,6 +65,18 @@ __device__ __forceinline__ int quant_code(float cb, float s, int bits) {
   const int qv = __float2int_rn(__fdiv_rn(cb, s));
   return qv > Q ? Q : (qv < -Q ? -Q : qv);
 }
+// The same code from inv = 1/s (any rounding): t = cb * inv is within a few
+// ulps of the correctly rounded quotient, so the nearest integer is the same
+// unless t lies within 2^-15 of a half-integer (|t| <= Q + 1 < 128, where an
+// ulp is at most 2^-17); those cases take the correctly rounded division.
+__device__ __forceinline__ int quant_code_fast(float cb, float s, float inv, int bits) {
+  if (!(s > 0.f)) return 0;
+  const int Q = bits == 8 ? 127 : 7;
+  float t = cb * inv;
+  if (fabsf(fabsf(t - rintf(t)) - 0.5f) <= 3.0517578125e-05f || fabsf(t) > 128.f) t = __fdiv_rn(cb, s);
+  const int qv = __float2int_rn(t);
+  return qv > Q ? Q : (qv < -Q ? -Q : qv);
+}
 
 // Number of new tokens sequence b contributes, and the status bits it raises.
 __device__ __forceinline__ int new_tokens(const int32_t* t_new_b, int b, int t_new,
@@ -129,9 +141,12 @@ inline int num_sms() {
 // n of the first four wave counts that n_min allows, and n_max.  Every CTA
 // evaluates this for its own sequence, so the model is evaluated in fp32 (the
 // choice only has to be good) and the chosen split in exact 32-bit integers.
-// Returns the splits that hold positions (ceil(T / chunk) <= n).
+// Returns the splits that hold positions (ceil(T / chunk) <= n).  tail_short:
+// the chunk is sized for T + tail_short positions (still at most
+// kMaxDecodeChunk), which leaves the last split that many positions fewer on
+// average -- room for extra work its CTA does (the fused append).
 __host__ __device__ inline int decode_split(int T, int n_max_grid, long long BH, int sms,
-                                            int* chunk_out) {
+                                            int* chunk_out, int tail_short = 0) {
   if (T <= 0) {
     *chunk_out = kMinDecodeChunk;
     return 1;
@@ -154,7 +169,9 @@ __host__ __device__ inline int decode_split(int T, int n_max_grid, long long BH,
     if (best_cost < 0.f || cost < best_cost) best_cost = cost, best_n = (int)nf;
   }
   const unsigned n = (unsigned)best_n;
-  const unsigned ch = ((uT + n - 1) / n + 31) / 32 * 32;
+  unsigned ch = ((uT + (unsigned)tail_short + n - 1) / n + 31) / 32 * 32;
+  const unsigned ch_min = ((uT + n - 1) / n + 31) / 32 * 32;
+  if (ch > kMaxDecodeChunk) ch = ch_min > kMaxDecodeChunk ? ch_min : kMaxDecodeChunk;
   *chunk_out = (int)ch;
   return (int)((uT + ch - 1) / ch);
 }

@@ -76,7 +76,13 @@ typedef enum {
                                        T_cap were dropped */
 #define LRKV_DEV_BAD_COUNT 0x4u     /* a t_new_b entry outside [0, t_new]: clamped into it */
 #define LRKV_DEV_WAIT_TIMEOUT 0x8u  /* a kernel gave up waiting for its own copies (bounded
-                                       wait): its outputs for that call are not valid */
+                                       wait): its outputs for that call are not valid.
+                                       The environment variable LRKV_MAIN_WAIT_ITERS
+                                       (a positive integer, read by each prefill-sized
+                                       lrkv_compress) lowers the limit of the prefill
+                                       projection's wait for each input tile, so a test
+                                       can make it run out; the waits that drain copies
+                                       and MMAs in flight keep their full limit. */
 
 /* Problem sizes of one layer. */
 typedef struct {
@@ -258,6 +264,33 @@ LRKV_API lrkv_status lrkv_fit_basis(const lrkv_dims* dims, const lrkv_bf16* X, i
  */
 LRKV_API lrkv_status lrkv_rank_for_budget(const float* eigvals, int32_t n_heads, int32_t d,
                                           double budget, int32_t* r_out);
+
+/* Online basis update (OjaKV repository README, "Method Summary > OjaKV": the
+ * low-rank subspace is updated online with Oja's algorithm during prefill and
+ * decoding).  The page gives no rule, step size or normalisation; this is
+ * Oja's subspace rule for every kv head h, over a batch of N = n_rows rows x_n
+ * (a prefill chunk; N = 1 per decode step):
+ *     y_n = U^T x_n,   V = U + eta (1/N) sum_n (x_n - U y_n) y_n^T,
+ *     U <- Q of V = Q R with R's diagonal positive (columns kept orthonormal).
+ * The sums are taken in fp32, the step and the orthonormalisation (Gram-
+ * Schmidt with a second pass) in fp64.
+ *
+ * X:     [n_rows][Hkv][d] bf16 rows (keys or values: lrkv_compress's k_new
+ *        layout with B * t_new rows).  Only dims->Hkv and dims->d (128) are used.
+ * r:     columns of the basis, a multiple of 16 in [16, d].
+ * eta:   step size, >= 0 and finite.
+ * U:     [Hkv][d][r] fp32, the basis, updated in place.  Kept in fp32 so that
+ *        small steps accumulate (a bf16 basis would round most of them away).
+ * U_out: nullable [Hkv][d][r] bf16, the updated basis rounded to nearest even:
+ *        what lrkv_cache takes as U_k or U_v.
+ * ws:    lrkv_oja_workspace_size(dims, n_rows, r) bytes (any contents).
+ * A cache keeps one basis per kv head: after an update, compressed rows stored
+ * earlier are read with the new basis (the library does not rewrite them).
+ * Returns LRKV_OK when the work was enqueued (two kernels on `stream`). */
+LRKV_API size_t lrkv_oja_workspace_size(const lrkv_dims* dims, int32_t n_rows, int32_t r);
+LRKV_API lrkv_status lrkv_oja_update(const lrkv_dims* dims, const lrkv_bf16* X, int32_t n_rows,
+                                     int32_t r, float eta, float* U, lrkv_bf16* U_out, void* ws,
+                                     size_t ws_bytes, void* stream);
 
 /* Device scratch built into the library for lrkv_decode_attn_noalloc, bytes. */
 #define LRKV_NOALLOC_SCRATCH_BYTES (4u << 20)

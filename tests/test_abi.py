@@ -31,7 +31,7 @@ def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["lrkv_workspace_size", "lrkv_compress", "lrkv_decode_attn", "lrkv_decode_attn_noalloc",
          "lrkv_append_decode_attn", "lrkv_fit_workspace_size", "lrkv_fit_basis",
-         "lrkv_rank_for_budget", "lrkv_status_str"])
+         "lrkv_rank_for_budget", "lrkv_status_str", "lrkv_oja_workspace_size", "lrkv_oja_update"])
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -173,3 +173,19 @@ def test_rank_for_budget_rejects_bad_arguments(lib):
     assert (r == -7).all()
     assert lib.lrkv_rank_for_budget(P(lam), 2, 8, 0.5, P(r)) == L.LRKV_OK
     assert r.tolist() == [4, 4]
+
+
+def test_oja_update_rejects_bad_arguments(lib):
+    D = _dims()
+    INVALID, UNSUP, ALIGN = 1, 2, 3
+    n = L.lrkv_oja_workspace_size(D, 1000, 64)
+    assert n > 0 and L.lrkv_oja_workspace_size(D, 1000, 40) == 0 and L.lrkv_oja_workspace_size(D, 0, 64) == 0
+    call = lambda dims=D, X=0x20000000, n_rows=1000, r=64, eta=0.1, U=0x30000000, U_out=None, \
+        ws=0x40000000, ws_bytes=n: lib.lrkv_oja_update(ctypes.byref(dims.c()), X, n_rows, r, eta, U, U_out,
+                                                       ws, ws_bytes, None)
+    assert call(X=None) == INVALID and call(U=None) == INVALID and call(r=8) == INVALID
+    assert call(r=144) == INVALID and call(n_rows=0) == INVALID
+    assert call(eta=-0.5) == INVALID and call(eta=float("nan")) == INVALID and call(eta=float("inf")) == INVALID
+    assert call(dims=_dims(d=64)) == UNSUP
+    assert call(X=0x20000008) == ALIGN and call(U_out=0x50000004) == ALIGN
+    assert call(ws_bytes=n - 1) == INVALID and call(ws=None) == INVALID
