@@ -416,70 +416,89 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
       const size_t bh = (size_t)b * D.Hkv + h;
       const uint32_t d2 = lane_base + buf * 256, d1 = d2 + 128;
       float rs = 0.f, xs = 0.f;
-      if (grp_a) {
-        // coefficients (c = U^T x - U^T mu with a key mean), in batches of NC
-        // columns (NC = 64 for bf16 rows; 32 for codes, whose rows take a first
-        // pass for the row's amax)
-        constexpr int NC = CB == 16 ? 64 : 32;
+      if (CB < 16 && grp_a) {
+        // quantised rows: group A takes two TMEM passes over the coefficients
+        // (c = U^T x - U^T mu with a key mean), 32 columns per wait: the row's
+        // amax of bf16(c), then its codes and scale
         const size_t row = bh * D.T_cap + start + t;
-        auto load_c = [&](int c0, float (&v)[NC / 16][16]) {
+        float amax = 0.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < R; c0 += 32) {
+          float v[2][16];
 #pragma unroll
-          for (int q = 0; q < NC / 16; ++q)
+          for (int q = 0; q < 2; ++q)
+            if (c0 + 16 * q < R) tc5::tmem_ld16(d1 + c0 + 16 * q, v[q]);
+          tc5::tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+            if (c0 + 16 * q < R)
+#pragma unroll
+              for (int k = 0; k < 16; k += 2) {
+                const float m0 = mug ? cmu[(c0 + 16 * q + k) & (kD - 1)] : 0.f;
+                const float m1 = mug ? cmu[(c0 + 16 * q + k + 1) & (kD - 1)] : 0.f;
+                const uint32_t pr = cvt_bf16x2(v[q][k] - m0, v[q][k + 1] - m1);   // bf16 pair
+                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(pr << 16)),
+                                         fabsf(__uint_as_float(pr & 0xffff0000u))));
+              }
+        }
+        const float qs = quant_scale(amax, CB);
+        const float qinv = qs > 0.f ? 1.f / qs : 0.f;
+        if (valid) scales[row] = qs;
+#pragma unroll 1
+        for (int c0 = 0; c0 < R; c0 += 32) {
+          float v[2][16];
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+            if (c0 + 16 * q < R) tc5::tmem_ld16(d1 + c0 + 16 * q, v[q]);
+          tc5::tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            if (!valid || c0 + 16 * q >= R) continue;
+            uint32_t bw[8];
+#pragma unroll
+            for (int k = 0; k < 16; k += 2) {
+              const float m0 = mug ? cmu[(c0 + 16 * q + k) & (kD - 1)] : 0.f;
+              const float m1 = mug ? cmu[(c0 + 16 * q + k + 1) & (kD - 1)] : 0.f;
+              bw[k >> 1] = cvt_bf16x2(v[q][k] - m0, v[q][k + 1] - m1);
+            }
+            uint32_t cw[4];   // 16 codes: 16 bytes (8-bit) or 8 (4-bit)
+            quant_pack16_bf(bw, qs, qinv, CB, cw);
+            const int c = c0 + 16 * q;
+            if (CB == 8)
+              *reinterpret_cast<uint4*>(coef + row * R + c) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            else
+              *reinterpret_cast<uint2*>(coef + row * (R / 2) + c / 2) = make_uint2(cw[0], cw[1]);
+          }
+        }
+      }
+      if (CB == 16 && grp_a) {
+        // bf16 rows: group A stores the coefficients (c = U^T x - U^T mu with a
+        // key mean), 64 columns per batch of TMEM loads (one wait per batch)
+        const size_t row = bh * D.T_cap + start + t;
+#pragma unroll 1
+        for (int c0 = 0; c0 < R; c0 += 64) {
+          float v[4][16];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
             if (c0 + 16 * q < R) tc5::tmem_ld16(d1 + c0 + 16 * q, v[q]);
           tc5::tmem_wait_ld();
           if (mug) {
 #pragma unroll
-            for (int q = 0; q < NC / 16; ++q)
+            for (int q = 0; q < 4; ++q)
 #pragma unroll
               for (int k = 0; k < 16; ++k) v[q][k] -= cmu[(c0 + 16 * q + k) & (kD - 1)];
           }
-        };
-        float qs = 0.f;   // the row's scale (quantised rows)
-        if constexpr (CB < 16) {
-          float amax = 0.f;
-#pragma unroll 1
-          for (int c0 = 0; c0 < R; c0 += NC) {
-            float v[NC / 16][16];
-            load_c(c0, v);
 #pragma unroll
-            for (int q = 0; q < NC / 16; ++q)
-              if (c0 + 16 * q < R)
-#pragma unroll
-                for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(bf16_round(v[q][k])));
-          }
-          qs = quant_scale(amax, CB);
-          if (valid) scales[row] = qs;
-        }
-        const float qinv = CB < 16 && qs > 0.f ? 1.f / qs : 0.f;
-#pragma unroll 1
-        for (int c0 = 0; c0 < R; c0 += NC) {
-          float v[NC / 16][16];
-          load_c(c0, v);
-#pragma unroll
-          for (int q = 0; q < NC / 16; ++q) {
+          for (int q = 0; q < 4; ++q) {
             if (!valid || c0 + 16 * q >= R) continue;
             const float* w = v[q];
-            if constexpr (CB == 16) {
-              lrkv_bf16* crow = reinterpret_cast<lrkv_bf16*>(coef) + row * R;
-              *reinterpret_cast<uint4*>(crow + c0 + 16 * q) =
-                  make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]),
-                             pack_bf16(w[6], w[7]));
-              *reinterpret_cast<uint4*>(crow + c0 + 16 * q + 8) =
-                  make_uint4(pack_bf16(w[8], w[9]), pack_bf16(w[10], w[11]),
-                             pack_bf16(w[12], w[13]), pack_bf16(w[14], w[15]));
-            } else {
-              uint32_t cw[4] = {0u, 0u, 0u, 0u};   // 16 codes: 16 bytes (8-bit) or 8 (4-bit)
-#pragma unroll
-              for (int k = 0; k < 16; ++k) {
-                const uint32_t cq = (uint32_t)quant_code_fast(bf16_round(w[k]), qs, qinv, CB);
-                if (CB == 8) cw[k >> 2] |= (cq & 0xffu) << (8 * (k & 3));
-                else cw[k >> 3] |= (cq & 0xfu) << (4 * (k & 7));
-              }
-              if (CB == 8)
-                *reinterpret_cast<uint4*>(coef + row * R + c0 + 16 * q) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-              else
-                *reinterpret_cast<uint2*>(coef + row * (R / 2) + (c0 + 16 * q) / 2) = make_uint2(cw[0], cw[1]);
-            }
+            lrkv_bf16* crow = reinterpret_cast<lrkv_bf16*>(coef) + row * R;
+            *reinterpret_cast<uint4*>(crow + c0 + 16 * q) =
+                make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]),
+                           pack_bf16(w[6], w[7]));
+            *reinterpret_cast<uint4*>(crow + c0 + 16 * q + 8) =
+                make_uint4(pack_bf16(w[8], w[9]), pack_bf16(w[10], w[11]),
+                           pack_bf16(w[12], w[13]), pack_bf16(w[14], w[15]));
           }
         }
       }

@@ -73,9 +73,41 @@ __device__ __forceinline__ int quant_code_fast(float cb, float s, float inv, int
   if (!(s > 0.f)) return 0;
   const int Q = bits == 8 ? 127 : 7;
   float t = cb * inv;
-  if (fabsf(fabsf(t - rintf(t)) - 0.5f) <= 3.0517578125e-05f || fabsf(t) > 128.f) t = __fdiv_rn(cb, s);
+  if (fabsf(fabsf(t - rintf(t)) - 0.5f) <= 3.0517578125e-05f || fabsf(t) > 128.f)
+    t = __fdiv_rn(cb, s);   // rare
   const int qv = __float2int_rn(t);
   return qv > Q ? Q : (qv < -Q ? -Q : qv);
+}
+
+// The codes of 16 values w (fp32, rounded to bf16 here) of a row with scale s
+// and inv = 1/s (any rounding), packed: 8-bit codes into cw[0..3] (byte k),
+// 4-bit codes into cw[0..1] (nibble k).  The same decisions as quant_code,
+// with plain ALU/FMA steps: the nearest integer (half to even) of t = bf16(w) *
+// inv comes from adding 1.5 * 2^23 (|t| < 2^22), and t is within 2^-15 of the
+// correctly rounded quotient bf16(w) / s (|t| <= 128), so only a t that close
+// to a half-integer redoes the correctly rounded division.
+// bw: the 16 values already rounded, as bf16 pairs (element 2i in the low half of bw[i]).
+__device__ __forceinline__ void quant_pack16_bf(const uint32_t (&bw)[8], float s, float inv, int bits,
+                                                uint32_t (&cw)[4]) {
+  const int Q = bits == 8 ? 127 : 7;
+  cw[0] = cw[1] = cw[2] = cw[3] = 0u;
+#pragma unroll
+  for (int k = 0; k < 16; k += 2) {
+    const uint32_t pr = bw[k >> 1];
+    const float b[2] = {__uint_as_float(pr << 16), __uint_as_float(pr & 0xffff0000u)};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float t = b[e] * inv;
+      const float rr = t + 12582912.f;
+      int qi = __float_as_int(rr) - 0x4B400000;
+      if (fabsf(fabsf(t - (rr - 12582912.f)) - 0.5f) <= 3.0517578125e-05f || fabsf(t) > 128.f)
+        qi = s > 0.f ? __float2int_rn(__fdiv_rn(b[e], s)) : 0;   // rare
+      qi = qi > Q ? Q : (qi < -Q ? -Q : qi);
+      const int kk = k + e;
+      if (bits == 8) cw[kk >> 2] |= ((uint32_t)qi & 0xffu) << (8 * (kk & 3));
+      else cw[kk >> 3] |= ((uint32_t)qi & 0xfu) << (4 * (kk & 7));
+    }
+  }
 }
 
 // Number of new tokens sequence b contributes, and the status bits it raises.
