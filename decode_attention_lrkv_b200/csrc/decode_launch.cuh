@@ -17,10 +17,12 @@ inline lrkv_status launch_stream_cb(const DecodeParams& p, dim3 grid, cudaStream
   return launch_pdl(kern, grid, dim3(S::kThreads), S::SMEM, s, p);
 }
 
-// bf16 coefficients or int8 codes (4-bit codes take the CUDA-core kernel)
+// bf16 coefficients, int8 or int4 codes
 template <int G, int RK, int RV, int W, int NS>
 inline lrkv_status launch_stream(const DecodeParams& p, dim3 grid, cudaStream_t s) {
-  if (coef_bits_of(p.D) == 8) return launch_stream_cb<G, RK, RV, W, NS, 8>(p, grid, s);
+  const int bits = coef_bits_of(p.D);
+  if (bits == 8) return launch_stream_cb<G, RK, RV, W, NS, 8>(p, grid, s);
+  if (bits == 4) return launch_stream_cb<G, RK, RV, W, NS, 4>(p, grid, s);
   return launch_stream_cb<G, RK, RV, W, NS, 16>(p, grid, s);
 }
 
@@ -36,10 +38,6 @@ template <int G>
 inline lrkv_status launch_stream_g(const DecodeParams& p, dim3 grid, cudaStream_t s, bool* done) {
   *done = true;
   const int rk = p.D.r_k, rv = p.D.r_v;
-  if (coef_bits_of(p.D) == 4) {   // 4-bit codes: the CUDA-core kernel
-    *done = false;
-    return LRKV_OK;
-  }
   // (warps per CTA, ring stages per warp) per shape: what shared memory holds
   // beside the mask words and the resident U_v
   if (rk == 32 && rv == 32) return launch_stream<G, 32, 32, 8, 3>(p, grid, s);

@@ -22,7 +22,6 @@ lrkv_status launch_simple_any(const DecodeParams& p, dim3 grid, cudaStream_t s) 
 bool stream_decode_supported(const lrkv_dims& D) {
   const int g = D.Hq / D.Hkv;
   if (g != 1 && g != 2 && g != 4) return false;
-  if (coef_bits_of(D) == 4) return false;
   const int rk = D.r_k, rv = D.r_v;
   return (rk == 32 && rv == 32) || (rk == 48 && rv == 64) || (rk == 48 && rv == 80) ||
          (rk == 64 && rv == 64) || (rk == 64 && rv == 96);

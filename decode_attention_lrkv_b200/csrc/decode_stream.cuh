@@ -67,14 +67,14 @@ constexpr int imax(int a, int b) { return a > b ? a : b; }
 // put the 8 rows an ldmatrix reads in distinct shared-memory banks
 constexpr int odd16(int x) { return (x / 16) % 2 ? x : x + 16; }
 
-// CB: bits of a stored coefficient, 16 (bf16) or 8 (int8 codes with per-row
-// fp32 scales).
+// CB: bits of a stored coefficient, 16 (bf16), 8 or 4 (int8 / int4 codes
+// with per-row fp32 scales).
 template <int G, int RK, int RV, int W, int NS, int CB = 16>
 struct Shape {
   static_assert(G == 1 || G == 2 || G == 4, "1, 2 or 4 query heads per kv head");
   static_assert(RK % 16 == 0 && RV % 16 == 0 && RK <= kD && RV <= kD, "ranks");
   static_assert(W >= 8 && NS >= 2, "at least 8 warps and 2 ring stages");
-  static_assert(CB == 16 || CB == 8, "bf16 coefficients or int8 codes");
+  static_assert(CB == 16 || CB == 8 || CB == 4, "bf16 coefficients or int8 / int4 codes");
   static constexpr int kWarps = W;
   static constexpr int kThreads = W * 32;
   // the bases in shared memory: bf16 rows, padded
@@ -84,8 +84,14 @@ struct Shape {
   // a compressed tile: 32 stored rows of keys, then of values, then (codes
   // only) their 32 + 32 fp32 scales
   static constexpr int TKB = RK * CB / 8, TVB = RV * CB / 8;   // bytes per stored row
-  static constexpr int KP = TKB / 16, VP = TVB / 16;          // 16-byte pieces per stored row
-  static constexpr int TKS = odd16(TKB), TVS = odd16(TVB);    // padded tile row strides
+  // bf16 and int8 rows are copied piece by piece into padded rows (16-byte
+  // pieces per row; routed rows zero-filled); int4 rows (8 bytes per 16 codes)
+  // are copied as the tile's flat block (16-byte pieces per tile) and read
+  // with plain shared loads, rows TKB apart
+  static constexpr int KP = CB == 4 ? 2 * TKB : TKB / 16;     // pieces per row, or per tile / 16
+  static constexpr int VP = CB == 4 ? 2 * TVB : TVB / 16;
+  static constexpr int TKS = CB == 4 ? TKB : odd16(TKB);      // tile row strides
+  static constexpr int TVS = CB == 4 ? TVB : odd16(TVB);
   static constexpr int T_SC = kTileC * (TKS + TVS);           // scales: [2][32] fp32
   static constexpr int FS = 2 * kD + 16;
   static constexpr int SLOT_C = T_SC + (CB < 16 ? 2 * kTileC * 4 : 0);
@@ -476,18 +482,27 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       const uint32_t bits = masked ? tile_bits(k) : valid_bits(k);
       const unsigned char* src_k = ck + (size_t)k * kTileC * S::TKB;
       const unsigned char* src_v = cv + (size_t)k * kTileC * S::TVB;
-#pragma unroll
-      for (int j = 0; j < KP; ++j) {   // piece q = lane + 32 j of the tile's key rows
-        const int q = lane + 32 * j, r = q / KP, sg = q - r * KP;
-        const bool on = (bits >> r) & 1u;
-        cp_async16_zfill(slot + r * S::TKS + sg * 16, on ? src_k + q * 16 : src_k, on ? 16u : 0u);
-      }
       unsigned char* vslot = slot + kTileC * S::TKS;
+      if constexpr (CB == 4) {
+        // the tile's rows are one block of 32 * TKB (32 * TVB) bytes: 16-byte
+        // pieces, no per-row zero-fill (routed and past-the-end rows hold
+        // finite codes; their logits are -inf and their weights 0)
+        for (int q = lane; q < kTileC * S::TKB / 16; q += 32) cp_async16(slot + q * 16, src_k + q * 16);
+        for (int q = lane; q < kTileC * S::TVB / 16; q += 32) cp_async16(vslot + q * 16, src_v + q * 16);
+        (void)bits;
+      } else {
 #pragma unroll
-      for (int j = 0; j < VP; ++j) {
-        const int q = lane + 32 * j, r = q / VP, sg = q - r * VP;
-        const bool on = (bits >> r) & 1u;
-        cp_async16_zfill(vslot + r * S::TVS + sg * 16, on ? src_v + q * 16 : src_v, on ? 16u : 0u);
+        for (int j = 0; j < KP; ++j) {   // piece q = lane + 32 j of the tile's key rows
+          const int q = lane + 32 * j, r = q / KP, sg = q - r * KP;
+          const bool on = (bits >> r) & 1u;
+          cp_async16_zfill(slot + r * S::TKS + sg * 16, on ? src_k + q * 16 : src_k, on ? 16u : 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < VP; ++j) {
+          const int q = lane + 32 * j, r = q / VP, sg = q - r * VP;
+          const bool on = (bits >> r) & 1u;
+          cp_async16_zfill(vslot + r * S::TVS + sg * 16, on ? src_v + q * 16 : src_v, on ? 16u : 0u);
+        }
       }
       if constexpr (CB < 16) {   // the tile's 32 key and 32 value scales: 16 pieces
         if (lane < 16) {
@@ -730,6 +745,68 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
             uint32_t a0, a1, a2, a3;
             ldsm_x4_t(a0, a1, a2, a3,
                       vrows + (16 * nb + (lm >> 1) * 8 + lr) * S::TVS + (mt * 16 + (lm & 1) * 8) * 2);
+            mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
+          }
+      } else if constexpr (CB == 4) {
+        // int4 codes, converted to bf16 in registers (exact): a nibble n with
+        // its sign bit flipped is u = n + 8, the bf16 0x4300 | u is 128 + u, and
+        // subtracting 136 gives n.  Logits: a 16-bit load of a row gives a
+        // thread the k-step's codes 4t..4t+3 (k = 2t, 2t+1 | 2t+8, 2t+9, the
+        // order of q~'s B fragments, as for int8).  Values: a byte of a row holds
+        // columns 2g, 2g+1 of a 16-column block (accumulator rows g, g + 8).
+        const float* scl = reinterpret_cast<const float*>(slot + S::T_SC);   // [2][32]
+        const uint32_t k136 = 0xC308C308u, k1 = 0x3F803F80u;                 // bf16x2 (-136, -136), (1, 1)
+        auto nib_pairs = [&](uint32_t x16, uint32_t& lo01, uint32_t& lo23) {
+          // x16: four nibbles (codes c0..c3 from the low end) -> bf16x2 (c0, c1), (c2, c3)
+          const uint32_t u = x16 ^ 0x8888u;
+          lo01 = 0x43004300u | (u & 0xFu) | ((u & 0xF0u) << 12);
+          lo23 = 0x43004300u | ((u >> 8) & 0xFu) | ((u & 0xF000u) << 4);
+          asm("fma.rn.bf16x2 %0, %0, %1, %2;" : "+r"(lo01) : "r"(k1), "r"(k136));
+          asm("fma.rn.bf16x2 %0, %0, %1, %2;" : "+r"(lo23) : "r"(k1), "r"(k136));
+        };
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+          st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
+          const unsigned char* r_lo = slot + (16 * nb + g) * S::TKS + 2 * t;
+          const unsigned char* r_hi = r_lo + 8 * S::TKS;
+#pragma unroll
+          for (int ks = 0; ks < KST; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            nib_pairs(*reinterpret_cast<const uint16_t*>(r_lo + 8 * ks), a0, a2);
+            nib_pairs(*reinterpret_cast<const uint16_t*>(r_hi + 8 * ks), a1, a3);
+            mma_16816(st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
+          }
+        }
+        float s[2][2], wv[2][2];
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            const int row = 16 * nb + g + x * 8;
+            const bool on = live_t && ((bits >> row) & 1u);
+            const float v = st[nb][2 * x] + st[nb][2 * x + 1];
+            s[nb][x] = on ? fmaf(v, scl[row], bias) : -INFINITY;
+            wv[nb][x] = on ? scl[kTileC + row] : 0.f;
+          }
+        uint32_t pb0[2], pb1[2];
+        softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv);
+        const unsigned char* vrows = slot + kTileC * S::TKS;
+#pragma unroll
+        for (int mt = 0; mt < MVT; ++mt)
+#pragma unroll
+          for (int nb = 0; nb < 2; ++nb) {
+            // tokens 16 nb + 2t, 2t+1 (a0, a1) and 2t+8, 2t+9 (a2, a3), byte g of the block
+            const unsigned char* c0p = vrows + (16 * nb + 2 * t) * S::TVS + 8 * mt + g;
+            const uint32_t x01 = (uint32_t)c0p[0] | ((uint32_t)c0p[S::TVS] << 8);
+            const uint32_t x89 = (uint32_t)c0p[8 * S::TVS] | ((uint32_t)c0p[9 * S::TVS] << 8);
+            // nibbles of x01: (token 2t: col 2g, 2g+1), (token 2t+1: col 2g, 2g+1)
+            uint32_t a0, a1, a2, a3, e, o;
+            nib_pairs(x01, e, o);   // e = (2t:2g, 2t:2g+1), o = (2t+1:2g, 2t+1:2g+1)
+            a0 = __byte_perm(e, o, 0x5410);   // (2t:2g, 2t+1:2g)
+            a1 = __byte_perm(e, o, 0x7632);   // (2t:2g+1, 2t+1:2g+1)
+            nib_pairs(x89, e, o);
+            a2 = __byte_perm(e, o, 0x5410);
+            a3 = __byte_perm(e, o, 0x7632);
             mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
           }
       } else {
