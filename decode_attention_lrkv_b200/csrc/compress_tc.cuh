@@ -171,7 +171,6 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   const lrkv_bf16* Uqg = tensor == 0 && p.C.U_kq ? p.C.U_kq + (size_t)h * kD * R : nullptr;
   const float* mug = tensor == 0 && p.C.mu_k ? p.C.mu_k + (size_t)h * kD : nullptr;
   unsigned char* coef = static_cast<unsigned char*>(tensor == 0 ? p.C.coef_k : p.C.coef_v);
-  constexpr int bits = CB;                        // 16: bf16; 8, 4: codes + per-row scales
   float* scales = tensor == 0 ? p.C.scale_k : p.C.scale_v;
   float* errs = p.errs + (size_t)tensor * D.B * D.Hkv * D.T_cap;
 

@@ -52,7 +52,6 @@ namespace lrkv {
 namespace ds {
 
 constexpr int kTileC = 32;                       // positions per compressed tile (one mask word)
-constexpr int kAppendTail = 256;                 // positions the fused append's split gives up
 constexpr int kTileF = 16;                       // rows per full-rank tile
 constexpr int kMaxChunk = kMaxDecodeChunk;       // positions per split (mask words in smem)
 constexpr unsigned kFull = 0xffffffffu;
@@ -132,7 +131,7 @@ struct Shape {
                 "both key bases and the append scratch fit in a stage");
 };
 
-// The owner CTA's share of a fused decode-time append: one new token of row b,
+// The append CTA's work in a fused decode-time append: one new token of row b,
 // kv head h, at position pos, with every thread of the CTA (the StaticPCA
 // write path and the OjaKV hybrid policy, as in the append kernel):
 //   c_k = U_k^T k and c_v = U_v^T v on the tensor cores (x as an A row,
@@ -342,7 +341,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       }
     };
     load_uk(p.C.U_kq ? p.C.U_kq : p.C.U_k, uk);
-    if (APP && p.C.U_kq) load_uk(p.C.U_k, sm + S::OFF_UK2);
+    if (APP && p.C.U_kq && blockIdx.x == gridDim.x - 1) load_uk(p.C.U_k, sm + S::OFF_UK2);   // the append CTA
     cp_async_commit();
   }
   auto load_uv = [&]() {   // U_v into padded rows, 16-byte pieces over every thread
@@ -382,7 +381,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     }
   }
   // fused append: does row b have a new token; one element of its new key
-  // (threads < d) or value (threads >= d) row per thread, for the owner
+  // (threads < d) or value (threads >= d) row per thread, for the append CTA
   int n_b = 0;
   uint32_t st_new = 0;
   uint16_t xe = 0;
@@ -396,7 +395,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   const int F_raw = p.C.full_cnt[bh];
   T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
   // fused append: the new token (if the row has one and there is room) takes
-  // position T_old; the split holding it (the last one) is its owner
+  // position T_old
   int n_eff = 0;
   if constexpr (APP) {
     n_eff = n_b > 0 && T < D.T_cap ? 1 : 0;
@@ -404,12 +403,17 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   }
   const int T_old = T;
   T += n_eff;
-  // splits from the live length (every CTA of the (b, kv head) finds the same);
-  // with a fused append the owner's split is kept shorter by the append's cost
+  // splits from the live length (every CTA of the (b, kv head) finds the same).
+  // With a fused append the grid's last CTA does the append and nothing else
+  // (its record joins the merge), so the stream never waits for it: the other
+  // CTAs split the T_old cached positions among the remaining n_chunk_max - 1.
   int chunk;
-  const int n_chunks = decode_split(T, p.n_chunk_max, (long long)D.B * D.Hkv, p.num_sms, &chunk,
-                                    APP && n_eff > 0 ? kAppendTail : 0);
-  const bool active = c < n_chunks;
+  const int n_chunks = APP ? decode_split(T_old, p.n_chunk_max - 1, (long long)D.B * D.Hkv, p.num_sms, &chunk)
+                           : decode_split(T, p.n_chunk_max, (long long)D.B * D.Hkv, p.num_sms, &chunk);
+  const bool is_app = APP && c == (int)gridDim.x - 1;   // the append CTA
+  const bool streams = !is_app && c < n_chunks;
+  const bool active = streams || is_app;
+  const int n_rec = n_chunks + (APP ? 1 : 0);            // records merged: the splits', then the append's
   const int c0 = c * chunk;
   // this split's mask words (words past the sequence end are never used): the
   // loads go out now and land while q~ is formed
@@ -418,18 +422,18 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
 #pragma unroll
   for (int u = 0; u < kMW; ++u) {
     const int wl = tid + u * kThreads, wi = c0 / 32 + wl;
-    mw[u] = active && wl < chunk / 32 && wi < D.T_cap / 32 ? p.C.route_mask[bh * (D.T_cap / 32) + wi] : 0u;
+    mw[u] = streams && wl < chunk / 32 && wi < D.T_cap / 32 ? p.C.route_mask[bh * (D.T_cap / 32) + wi] : 0u;
   }
 
   // ---- this warp's tiles; the first ones are issued before the mask words and
   // the query projection, so their copies overlap both ------------------------------
   const int c1 = min(T_old, c0 + chunk);   // the new position is not read from the cache
-  const int n_pos = active && c1 > c0 ? c1 - c0 : 0;
+  const int n_pos = streams && c1 > c0 ? c1 - c0 : 0;
   // this split's share of the full-rank list
   const int F = min(max(F_raw, 0), D.F_cap);
   const int share = (F + n_chunks - 1) / n_chunks;
   const int f0 = min(F, c * share), f1 = min(F, f0 + share);
-  const int n_full = f1 - f0;
+  const int n_full = streams ? f1 - f0 : 0;
   const unsigned char* ck = static_cast<const unsigned char*>(p.C.coef_k) + (bh * D.T_cap + c0) * S::TKB;
   const unsigned char* cv = static_cast<const unsigned char*>(p.C.coef_v) + (bh * D.T_cap + c0) * S::TVB;
   const float* sck = CB < 16 ? p.C.scale_k + bh * D.T_cap + c0 : nullptr;   // code scales
@@ -530,7 +534,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   };
 #pragma unroll
   for (int s = 0; s < NST - 1; ++s) {
-    if (active && s < n_tiles) issue(s, false);
+    if (streams && s < n_tiles) issue(s, false);
     cp_async_commit();
   }
 
@@ -601,7 +605,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     sb = warp_sum(sb);
     if (lane == 0) s_bias[gi] = sb * scale;
   }
-  const bool owner = APP && n_eff > 0 && c == n_chunks - 1;
+  const bool owner = is_app && n_eff > 0;   // the append CTA has a token to append
   // Every thread of this CTA has read seq_len[b] (the barrier above): each CTA
   // takes the row's ticket once (release only) and looks at it later; the last
   // CTA of the grid for row b advances its length.
@@ -629,8 +633,8 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   for (int u = 0; u < kMW; ++u)
     if (tid + u * kThreads < kMaxChunk / 32) maskw[tid + u * kThreads] = mw[u];
   cp_async_wait<NST - 1>();   // U_v in (only the prologue's tiles may be in flight)
-  // the new token for the fold after the stream: its logit per head, whether
-  // it went to the full-rank list, and its value row (v, or c_v as stored)
+  // the append CTA's new token: its logit per head, whether it went to the
+  // full-rank list, and its value row (v, or c_v as stored)
   __shared__ float s_new[G];
   __shared__ float s_vals[kD];
   __shared__ int s_keep;
@@ -639,387 +643,384 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
 #pragma unroll
   for (int ks2 = 0; ks2 < KST; ++ks2) qb0[ks2] = s_qb[ks2][0][lane], qb1[ks2] = s_qb[ks2][1][lane];
   const float bias = live_t ? s_bias[t] : 0.f;   // this lane's head
-  // the owner of a fused append does it while its first tiles are in flight
-  // (U_k and the scratch sit in the last stage, which the stream refills only
-  // from its first step on)
+  // ---- the append CTA: the new token's compress and its record ------------------------
+  // (its U_k copy and scratch sit in the last stage; it streams no tiles)
   if constexpr (APP) {
-    if (owner) {
-      append_token<S, G, RK, RV, CB>(p, app, p.C.U_kq ? sm + S::OFF_UK2 : uk, uk, sm + S::OFF_UV, s_bias,
-                                 b, h, bh, T_old, F, scale, xe, s_new, s_vals, &s_keep);
-      __syncthreads();   // the token's logits and value row in for warp 0
+    if (is_app) {
+      if (owner)
+        append_token<S, G, RK, RV, CB>(p, app, p.C.U_kq ? sm + S::OFF_UK2 : uk, uk, sm + S::OFF_UV, s_bias,
+                                       b, h, bh, T_old, F, scale, xe, s_new, s_vals, &s_keep);
+      __syncthreads();   // the token's logits and value row in
+      // record n_chunks: per query head m = the token's logit, l = 1 and o = its
+      // value row in d-space (v, or U_v c_v as stored); an empty record
+      // (m = -inf) when the row has no token
+      float* recA = p.partials + (bh * p.n_chunk_max + n_chunks) * G * (size_t)S::REC;
+      const unsigned char* uv = sm + S::OFF_UV;
+      for (int o = tid; o < G * kD; o += kThreads) {
+        const int gi = o / kD, i = o - gi * kD;
+        float x = 0.f;
+        if (owner) {
+          if (s_keep) {
+            x = s_vals[i];
+          } else {
+            const lrkv_bf16* urow = reinterpret_cast<const lrkv_bf16*>(uv + i * S::VS);
+            for (int j = 0; j < RV; ++j) x = fmaf(bf2f(urow[j]), s_vals[j], x);
+          }
+        }
+        recA[gi * S::REC + 4 + i] = x;
+      }
+      if (tid < G) {
+        recA[tid * S::REC] = owner ? s_new[tid] : -INFINITY;
+        recA[tid * S::REC + 1] = owner ? 1.f : 0.f;
+        if (tid == 0) recA[2] = owner && s_keep ? 1.f : 0.f;
+      }
+      if (tid == tk) seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
     }
   }
 
-  // ---- stream the tiles ------------------------------------------------------------
-  // lane state: running max and sum of head t; accumulators O^T (rows = value
-  // columns, columns = head parts: all four fragment entries are head t) for
-  // the compressed and full-rank sums
-  float m_run = -INFINITY, l_run = 0.f;
-  float oc[MVT][4], of[8][4];
-#pragma unroll
-  for (int mt = 0; mt < MVT; ++mt) oc[mt][0] = oc[mt][1] = oc[mt][2] = oc[mt][3] = 0.f;
-#pragma unroll
-  for (int mt = 0; mt < 8; ++mt) of[mt][0] = of[mt][1] = of[mt][2] = of[mt][3] = 0.f;
+  if (!is_app) {
+    // ---- stream the tiles ------------------------------------------------------------
+    // lane state: running max and sum of head t; accumulators O^T (rows = value
+    // columns, columns = head parts: all four fragment entries are head t) for
+    // the compressed and full-rank sums
+    float m_run = -INFINITY, l_run = 0.f;
+    float oc[MVT][4], of[8][4];
+  #pragma unroll
+    for (int mt = 0; mt < MVT; ++mt) oc[mt][0] = oc[mt][1] = oc[mt][2] = oc[mt][3] = 0.f;
+  #pragma unroll
+    for (int mt = 0; mt < 8; ++mt) of[mt][0] = of[mt][1] = of[mt][2] = of[mt][3] = 0.f;
 
-  // Online softmax over NB 16-row blocks: s[nb] = {row g, row g + 8} of head t
-  // (-inf = no token).  Rescales this lane's accumulators when the max grows,
-  // and returns the probabilities packed as the P^T B fragments of each block
-  // (column 2t = bf16 high part, 2t + 1 = low part); with value weights wv
-  // (the rows' code scales) the packed entries are p * wv, the sum l takes p.
-  auto softmax_pack_w = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag, const float (*wv)[2]) {
-    constexpr int NB = decltype(nb_tag)::value;
-    float x = -INFINITY;
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) x = fmaxf(x, fmaxf(s[nb][0], s[nb][1]));
-    // the running max only grows: the reduction over the rows is needed only
-    // when some lane holds a score above it (rare after the first tiles)
-    if (__any_sync(kFull, x > m_run)) {
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
-      if (x > m_run) {
-        const float sc = m_run == -INFINITY ? 0.f : exp2f(m_run - x);
-        l_run *= sc;
-#pragma unroll
-        for (int mt = 0; mt < MVT; ++mt) oc[mt][0] *= sc, oc[mt][1] *= sc, oc[mt][2] *= sc, oc[mt][3] *= sc;
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt) of[mt][0] *= sc, of[mt][1] *= sc, of[mt][2] *= sc, of[mt][3] *= sc;
-        m_run = x;
+    // Online softmax over NB 16-row blocks: s[nb] = {row g, row g + 8} of head t
+    // (-inf = no token).  Rescales this lane's accumulators when the max grows,
+    // and returns the probabilities packed as the P^T B fragments of each block
+    // (column 2t = bf16 high part, 2t + 1 = low part); with value weights wv
+    // (the rows' code scales) the packed entries are p * wv, the sum l takes p.
+    auto softmax_pack_w = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag, const float (*wv)[2]) {
+      constexpr int NB = decltype(nb_tag)::value;
+      float x = -INFINITY;
+  #pragma unroll
+      for (int nb = 0; nb < NB; ++nb) x = fmaxf(x, fmaxf(s[nb][0], s[nb][1]));
+      // the running max only grows: the reduction over the rows is needed only
+      // when some lane holds a score above it (rare after the first tiles)
+      if (__any_sync(kFull, x > m_run)) {
+  #pragma unroll
+        for (int o = 4; o < 32; o <<= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, o));
+        if (x > m_run) {
+          const float sc = m_run == -INFINITY ? 0.f : exp2f(m_run - x);
+          l_run *= sc;
+  #pragma unroll
+          for (int mt = 0; mt < MVT; ++mt) oc[mt][0] *= sc, oc[mt][1] *= sc, oc[mt][2] *= sc, oc[mt][3] *= sc;
+  #pragma unroll
+          for (int mt = 0; mt < 8; ++mt) of[mt][0] *= sc, of[mt][1] *= sc, of[mt][2] *= sc, of[mt][3] *= sc;
+          m_run = x;
+        }
       }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-      float p0 = s[nb][0] == -INFINITY ? 0.f : exp2f(s[nb][0] - m_run);
-      float p1 = s[nb][1] == -INFINITY ? 0.f : exp2f(s[nb][1] - m_run);
-      l_run += p0 + p1;
-      if (wv) p0 *= wv[nb][0], p1 *= wv[nb][1];
-      // (high part, low part) of p: bf16(p) and bf16(p - bf16(p))
-      const float h0 = __uint_as_float(cvt_bf16x2(p0, p0) << 16);
-      const float h1 = __uint_as_float(cvt_bf16x2(p1, p1) << 16);
-      pb0[nb] = movmatrix_t(cvt_bf16x2(p0, p0 - h0));
-      pb1[nb] = movmatrix_t(cvt_bf16x2(p1, p1 - h1));
-    }
-  };
-  auto softmax_pack = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag) {
-    softmax_pack_w(s, pb0, pb1, nb_tag, static_cast<const float (*)[2]>(nullptr));
-  };
+      __syncwarp();
+  #pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        float p0 = s[nb][0] == -INFINITY ? 0.f : exp2f(s[nb][0] - m_run);
+        float p1 = s[nb][1] == -INFINITY ? 0.f : exp2f(s[nb][1] - m_run);
+        l_run += p0 + p1;
+        if (wv) p0 *= wv[nb][0], p1 *= wv[nb][1];
+        // (high part, low part) of p: bf16(p) and bf16(p - bf16(p))
+        const float h0 = __uint_as_float(cvt_bf16x2(p0, p0) << 16);
+        const float h1 = __uint_as_float(cvt_bf16x2(p1, p1) << 16);
+        pb0[nb] = movmatrix_t(cvt_bf16x2(p0, p0 - h0));
+        pb1[nb] = movmatrix_t(cvt_bf16x2(p1, p1 - h1));
+      }
+    };
+    auto softmax_pack = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag) {
+      softmax_pack_w(s, pb0, pb1, nb_tag, static_cast<const float (*)[2]>(nullptr));
+    };
 
-  for (int i = 0; i < n_tiles; ++i) {
-    if (i + NST - 1 < n_tiles) issue(i + NST - 1, true);
-    cp_async_commit();
-    cp_async_wait<NST - 1>();
-    __syncwarp();
-    const unsigned char* slot = slot_of(i % NST, warp);
-    int kw;
-    if (wi_comp.next(nct_w, n_tiles, kw)) {
-      // compressed tile: S^T[token][head part] = C_k q~^T, then O^T += C_v^T P^T
-      const uint32_t bits = tile_bits(warp + kWarps * kw);
-      float st[2][4];
-      if constexpr (CB == 16) {
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-          st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
-#pragma unroll
-          for (int ks = 0; ks < KST; ++ks) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(a0, a1, a2, a3,
-                    slot + (16 * nb + (lm & 1) * 8 + lr) * S::TKS + (ks * 16 + (lm >> 1) * 8) * 2);
-            mma_16816(st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
-          }
-        }
-        float s[2][2];
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {   // rows g, g + 8: high + low part of head t
-            const float v = st[nb][2 * x] + st[nb][2 * x + 1] + bias;
-            s[nb][x] = live_t && ((bits >> (16 * nb + g + x * 8)) & 1u) ? v : -INFINITY;
-          }
-        uint32_t pb0[2], pb1[2];
-        softmax_pack(s, pb0, pb1, std::integral_constant<int, 2>{});
-        const unsigned char* vrows = slot + kTileC * S::TKS;
-#pragma unroll
-        for (int mt = 0; mt < MVT; ++mt)
-#pragma unroll
+    for (int i = 0; i < n_tiles; ++i) {
+      if (i + NST - 1 < n_tiles) issue(i + NST - 1, true);
+      cp_async_commit();
+      cp_async_wait<NST - 1>();
+      __syncwarp();
+      const unsigned char* slot = slot_of(i % NST, warp);
+      int kw;
+      if (wi_comp.next(nct_w, n_tiles, kw)) {
+        // compressed tile: S^T[token][head part] = C_k q~^T, then O^T += C_v^T P^T
+        const uint32_t bits = tile_bits(warp + kWarps * kw);
+        float st[2][4];
+        if constexpr (CB == 16) {
+  #pragma unroll
           for (int nb = 0; nb < 2; ++nb) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4_t(a0, a1, a2, a3,
-                      vrows + (16 * nb + (lm >> 1) * 8 + lr) * S::TVS + (mt * 16 + (lm & 1) * 8) * 2);
-            mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
-          }
-      } else if constexpr (CB == 4) {
-        // int4 codes, converted to bf16 in registers (exact): a nibble n with
-        // its sign bit flipped is u = n + 8, the bf16 0x4300 | u is 128 + u, and
-        // subtracting 136 gives n.  Logits: a 16-bit load of a row gives a
-        // thread the k-step's codes 4t..4t+3 (k = 2t, 2t+1 | 2t+8, 2t+9, the
-        // order of q~'s B fragments, as for int8).  Values: a byte of a row holds
-        // columns 2g, 2g+1 of a 16-column block (accumulator rows g, g + 8).
-        const float* scl = reinterpret_cast<const float*>(slot + S::T_SC);   // [2][32]
-        const uint32_t k136 = 0xC308C308u, k1 = 0x3F803F80u;                 // bf16x2 (-136, -136), (1, 1)
-        auto nib_pairs = [&](uint32_t x16, uint32_t& lo01, uint32_t& lo23) {
-          // x16: four nibbles (codes c0..c3 from the low end) -> bf16x2 (c0, c1), (c2, c3)
-          const uint32_t u = x16 ^ 0x8888u;
-          lo01 = 0x43004300u | (u & 0xFu) | ((u & 0xF0u) << 12);
-          lo23 = 0x43004300u | ((u >> 8) & 0xFu) | ((u & 0xF000u) << 4);
-          asm("fma.rn.bf16x2 %0, %0, %1, %2;" : "+r"(lo01) : "r"(k1), "r"(k136));
-          asm("fma.rn.bf16x2 %0, %0, %1, %2;" : "+r"(lo23) : "r"(k1), "r"(k136));
-        };
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-          st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
-          const unsigned char* r_lo = slot + (16 * nb + g) * S::TKS + 2 * t;
-          const unsigned char* r_hi = r_lo + 8 * S::TKS;
-#pragma unroll
-          for (int ks = 0; ks < KST; ++ks) {
-            uint32_t a0, a1, a2, a3;
-            nib_pairs(*reinterpret_cast<const uint16_t*>(r_lo + 8 * ks), a0, a2);
-            nib_pairs(*reinterpret_cast<const uint16_t*>(r_hi + 8 * ks), a1, a3);
-            mma_16816(st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
-          }
-        }
-        float s[2][2], wv[2][2];
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            const int row = 16 * nb + g + x * 8;
-            const bool on = live_t && ((bits >> row) & 1u);
-            const float v = st[nb][2 * x] + st[nb][2 * x + 1];
-            s[nb][x] = on ? fmaf(v, scl[row], bias) : -INFINITY;
-            wv[nb][x] = on ? scl[kTileC + row] : 0.f;
-          }
-        uint32_t pb0[2], pb1[2];
-        softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv);
-        const unsigned char* vrows = slot + kTileC * S::TKS;
-#pragma unroll
-        for (int mt = 0; mt < MVT; ++mt)
-#pragma unroll
-          for (int nb = 0; nb < 2; ++nb) {
-            // tokens 16 nb + 2t, 2t+1 (a0, a1) and 2t+8, 2t+9 (a2, a3), byte g of the block
-            const unsigned char* c0p = vrows + (16 * nb + 2 * t) * S::TVS + 8 * mt + g;
-            const uint32_t x01 = (uint32_t)c0p[0] | ((uint32_t)c0p[S::TVS] << 8);
-            const uint32_t x89 = (uint32_t)c0p[8 * S::TVS] | ((uint32_t)c0p[9 * S::TVS] << 8);
-            // nibbles of x01: (token 2t: col 2g, 2g+1), (token 2t+1: col 2g, 2g+1)
-            uint32_t a0, a1, a2, a3, e, o;
-            nib_pairs(x01, e, o);   // e = (2t:2g, 2t:2g+1), o = (2t+1:2g, 2t+1:2g+1)
-            a0 = __byte_perm(e, o, 0x5410);   // (2t:2g, 2t+1:2g)
-            a1 = __byte_perm(e, o, 0x7632);   // (2t:2g+1, 2t+1:2g+1)
-            nib_pairs(x89, e, o);
-            a2 = __byte_perm(e, o, 0x5410);
-            a3 = __byte_perm(e, o, 0x7632);
-            mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
-          }
-      } else {
-        // int8 codes, converted to bf16 in registers (exact).  Logits: an
-        // ldmatrix of a k-step's 16 code bytes gives a thread bytes 4t..4t+3 of
-        // its row, k = 2t, 2t+1 (a0/a1) and 2t+8, 2t+9 (a2/a3) in the order q~'s
-        // B fragments were built in; the row's key scale multiplies the logit.
-        const float* scl = reinterpret_cast<const float*>(slot + S::T_SC);   // [2][32]
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-          st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
-          const unsigned char* rows = slot + (16 * nb + (lm & 1) * 8 + lr) * S::TKS;
-#pragma unroll
-          for (int kp = 0; kp < KST; kp += 2) {
-            uint32_t r0, r1, r2 = 0u, r3 = 0u, e0, e1, f0, f1;
-            if (kp + 1 < KST) ldsm_x4(r0, r1, r2, r3, rows + kp * 16 + (lm >> 1) * 16);
-            else ldsm_x2(r0, r1, rows + kp * 16);
-            s8x4_pairs(r0, e0, f0);
-            s8x4_pairs(r1, e1, f1);
-            mma_16816(st[nb], e0, e1, f0, f1, qb0[kp], qb1[kp]);
-            if (kp + 1 < KST) {
-              s8x4_pairs(r2, e0, f0);
-              s8x4_pairs(r3, e1, f1);
-              mma_16816(st[nb], e0, e1, f0, f1, qb0[kp + 1], qb1[kp + 1]);
+            st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
+  #pragma unroll
+            for (int ks = 0; ks < KST; ++ks) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4(a0, a1, a2, a3,
+                      slot + (16 * nb + (lm & 1) * 8 + lr) * S::TKS + (ks * 16 + (lm >> 1) * 8) * 2);
+              mma_16816(st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
             }
           }
-        }
-        float s[2][2], wv[2][2];
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {   // rows g, g + 8: high + low part of head t
-            const int row = 16 * nb + g + x * 8;
-            const bool on = live_t && ((bits >> row) & 1u);
-            const float v = st[nb][2 * x] + st[nb][2 * x + 1];
-            s[nb][x] = on ? fmaf(v, scl[row], bias) : -INFINITY;
-            wv[nb][x] = on ? scl[kTileC + row] : 0.f;   // scales of unread rows are never used
+          float s[2][2];
+  #pragma unroll
+          for (int nb = 0; nb < 2; ++nb)
+  #pragma unroll
+            for (int x = 0; x < 2; ++x) {   // rows g, g + 8: high + low part of head t
+              const float v = st[nb][2 * x] + st[nb][2 * x + 1] + bias;
+              s[nb][x] = live_t && ((bits >> (16 * nb + g + x * 8)) & 1u) ? v : -INFINITY;
+            }
+          uint32_t pb0[2], pb1[2];
+          softmax_pack(s, pb0, pb1, std::integral_constant<int, 2>{});
+          const unsigned char* vrows = slot + kTileC * S::TKS;
+  #pragma unroll
+          for (int mt = 0; mt < MVT; ++mt)
+  #pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4_t(a0, a1, a2, a3,
+                        vrows + (16 * nb + (lm >> 1) * 8 + lr) * S::TVS + (mt * 16 + (lm & 1) * 8) * 2);
+              mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
+            }
+        } else if constexpr (CB == 4) {
+          // int4 codes, converted to bf16 in registers (exact): a nibble n with
+          // its sign bit flipped is u = n + 8, the bf16 0x4300 | u is 128 + u, and
+          // subtracting 136 gives n.  Logits: a 16-bit load of a row gives a
+          // thread the k-step's codes 4t..4t+3 (k = 2t, 2t+1 | 2t+8, 2t+9, the
+          // order of q~'s B fragments, as for int8).  Values: a byte of a row holds
+          // columns 2g, 2g+1 of a 16-column block (accumulator rows g, g + 8).
+          const float* scl = reinterpret_cast<const float*>(slot + S::T_SC);   // [2][32]
+          const uint32_t k136 = 0xC308C308u, k1 = 0x3F803F80u;                 // bf16x2 (-136, -136), (1, 1)
+          auto nib_pairs = [&](uint32_t x16, uint32_t& lo01, uint32_t& lo23) {
+            // x16: four nibbles (codes c0..c3 from the low end) -> bf16x2 (c0, c1), (c2, c3)
+            const uint32_t u = x16 ^ 0x8888u;
+            lo01 = 0x43004300u | (u & 0xFu) | ((u & 0xF0u) << 12);
+            lo23 = 0x43004300u | ((u >> 8) & 0xFu) | ((u & 0xF000u) << 4);
+            asm("fma.rn.bf16x2 %0, %0, %1, %2;" : "+r"(lo01) : "r"(k1), "r"(k136));
+            asm("fma.rn.bf16x2 %0, %0, %1, %2;" : "+r"(lo23) : "r"(k1), "r"(k136));
+          };
+  #pragma unroll
+          for (int nb = 0; nb < 2; ++nb) {
+            st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
+            const unsigned char* r_lo = slot + (16 * nb + g) * S::TKS + 2 * t;
+            const unsigned char* r_hi = r_lo + 8 * S::TKS;
+  #pragma unroll
+            for (int ks = 0; ks < KST; ++ks) {
+              uint32_t a0, a1, a2, a3;
+              nib_pairs(*reinterpret_cast<const uint16_t*>(r_lo + 8 * ks), a0, a2);
+              nib_pairs(*reinterpret_cast<const uint16_t*>(r_hi + 8 * ks), a1, a3);
+              mma_16816(st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
+            }
           }
-        uint32_t pb0[2], pb1[2];
-        softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv);
-        // values: one transposing ldmatrix per 16 value columns covers the 32
-        // tokens; a thread's bytes are (token 2t | 2t+1) x (column 2g | 2g+1), so
-        // accumulator row g is column 2g of the block and row g + 8 column 2g + 1
-        const unsigned char* vrows = slot + kTileC * S::TKS;
-#pragma unroll
-        for (int mt = 0; mt < MVT; ++mt) {
-          uint32_t r0, r1, r2, r3, a0, a1, a2, a3;
-          ldsm_x4_t(r0, r1, r2, r3, vrows + (8 * lm + lr) * S::TVS + mt * 16);
-          s8x4_evenodd(r0, a0, a1);
-          s8x4_evenodd(r1, a2, a3);
-          mma_16816(oc[mt], a0, a1, a2, a3, pb0[0], pb1[0]);
-          s8x4_evenodd(r2, a0, a1);
-          s8x4_evenodd(r3, a2, a3);
-          mma_16816(oc[mt], a0, a1, a2, a3, pb0[1], pb1[1]);
-        }
-      }
-    } else {
-      // full-rank tile: 16 list rows
-      const int k = warp + kWarps * kw;
-      const int nrows = min(kTileF, n_full - k * kTileF);
-      float st[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(a0, a1, a2, a3, slot + ((lm & 1) * 8 + lr) * S::FS + (ks * 16 + (lm >> 1) * 8) * 2);
-        mma_16816(st, a0, a1, a2, a3, qf0[ks], qf1[ks]);
-      }
-      float s[1][2];
-#pragma unroll
-      for (int x = 0; x < 2; ++x) {   // rows g, g + 8 (the low-part column is 0 for q)
-        const float v = (st[2 * x] + st[2 * x + 1]) * scale;
-        s[0][x] = live_t && g + x * 8 < nrows ? v : -INFINITY;
-      }
-      uint32_t pb0[1], pb1[1];
-      softmax_pack(s, pb0, pb1, std::integral_constant<int, 1>{});
-      const unsigned char* vrows = slot + kTileF * S::FS;
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(a0, a1, a2, a3, vrows + ((lm >> 1) * 8 + lr) * S::FS + (mt * 16 + (lm & 1) * 8) * 2);
-        mma_16816(of[mt], a0, a1, a2, a3, pb0[0], pb1[0]);
-      }
-    }
-    __syncwarp();
-  }
-  cp_async_wait<0>();
-  // the row's length ticket: release-only, taken now that this thread has no
-  // copy in flight (a release waits for them); looked at after the record
-  if (APP && tid == tk) seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
-  __syncwarp();
-  griddep_launch_dependents();
-
-  // ---- fused append: fold the new token into warp 0's state ---------------------
-  if (owner && warp == 0 && live_t) {
-    const float sv = s_new[t];
-    if (sv > m_run) {
-      const float sc = m_run == -INFINITY ? 0.f : exp2f(m_run - sv);
-      l_run *= sc;
-#pragma unroll
-      for (int mt = 0; mt < MVT; ++mt) oc[mt][0] *= sc, oc[mt][1] *= sc, oc[mt][2] *= sc, oc[mt][3] *= sc;
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) of[mt][0] *= sc, of[mt][1] *= sc, of[mt][2] *= sc, of[mt][3] *= sc;
-      m_run = sv;
-    }
-    const float pn = exp2f(sv - m_run);
-    if (g == 0) l_run += pn;
-    if (s_keep) {
-#pragma unroll
-      for (int mi = 0; mi < 8; ++mi) {
-        of[mi][0] = fmaf(pn, s_vals[16 * mi + g], of[mi][0]);
-        of[mi][2] = fmaf(pn, s_vals[16 * mi + g + 8], of[mi][2]);
-      }
-    } else {   // accumulator rows g, g + 8 are value columns g, g + 8 (bf16) or 2g, 2g + 1 (codes)
-#pragma unroll
-      for (int mt = 0; mt < MVT; ++mt) {
-        oc[mt][0] = fmaf(pn, s_vals[16 * mt + (CB == 16 ? g : 2 * g)], oc[mt][0]);
-        oc[mt][2] = fmaf(pn, s_vals[16 * mt + (CB == 16 ? g + 8 : 2 * g + 1)], oc[mt][2]);
-      }
-    }
-  }
-
-  // ---- lift: of += U_v acc_c^T on the tensor cores --------------------------------
-  // acc_c^T (rows = r_v, columns = head parts) becomes the B operand: lane
-  // (g, t) holds acc_c[head t][16 mt + g (+8)] (high + low part columns), packs
-  // it as bf16 high and low parts (columns 2t, 2t + 1 of an 8x8 tile) and one
-  // transpose gives the fragment (k = 2t, 2t + 1; n = g).  The product lands in
-  // the full-rank accumulators, whose layout is the same: o = both parts summed.
-  {
-    const unsigned char* uv = sm + S::OFF_UV;
-    uint32_t lb0[MVT], lb1[MVT];
-#pragma unroll
-    for (int mt = 0; mt < MVT; ++mt) {
-      const float x0 = oc[mt][0] + oc[mt][1], x1 = oc[mt][2] + oc[mt][3];
-      const float h0 = __uint_as_float(cvt_bf16x2(x0, x0) << 16);
-      const float h1 = __uint_as_float(cvt_bf16x2(x1, x1) << 16);
-      lb0[mt] = movmatrix_t(cvt_bf16x2(x0, x0 - h0));
-      lb1[mt] = movmatrix_t(cvt_bf16x2(x1, x1 - h1));
-    }
-#pragma unroll
-    for (int mi = 0; mi < 8; ++mi)
-#pragma unroll
-      for (int mt = 0; mt < MVT; ++mt) {
-        uint32_t a0, a1, a2, a3;
-        if constexpr (CB == 16) {
-          ldsm_x4(a0, a1, a2, a3, uv + (16 * mi + (lm & 1) * 8 + lr) * S::VS + (mt * 16 + (lm >> 1) * 8) * 2);
+          float s[2][2], wv[2][2];
+  #pragma unroll
+          for (int nb = 0; nb < 2; ++nb)
+  #pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const int row = 16 * nb + g + x * 8;
+              const bool on = live_t && ((bits >> row) & 1u);
+              const float v = st[nb][2 * x] + st[nb][2 * x + 1];
+              s[nb][x] = on ? fmaf(v, scl[row], bias) : -INFINITY;
+              wv[nb][x] = on ? scl[kTileC + row] : 0.f;
+            }
+          uint32_t pb0[2], pb1[2];
+          softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv);
+          const unsigned char* vrows = slot + kTileC * S::TKS;
+  #pragma unroll
+          for (int mt = 0; mt < MVT; ++mt)
+  #pragma unroll
+            for (int nb = 0; nb < 2; ++nb) {
+              // tokens 16 nb + 2t, 2t+1 (a0, a1) and 2t+8, 2t+9 (a2, a3), byte g of the block
+              const unsigned char* c0p = vrows + (16 * nb + 2 * t) * S::TVS + 8 * mt + g;
+              const uint32_t x01 = (uint32_t)c0p[0] | ((uint32_t)c0p[S::TVS] << 8);
+              const uint32_t x89 = (uint32_t)c0p[8 * S::TVS] | ((uint32_t)c0p[9 * S::TVS] << 8);
+              // nibbles of x01: (token 2t: col 2g, 2g+1), (token 2t+1: col 2g, 2g+1)
+              uint32_t a0, a1, a2, a3, e, o;
+              nib_pairs(x01, e, o);   // e = (2t:2g, 2t:2g+1), o = (2t+1:2g, 2t+1:2g+1)
+              a0 = __byte_perm(e, o, 0x5410);   // (2t:2g, 2t+1:2g)
+              a1 = __byte_perm(e, o, 0x7632);   // (2t:2g+1, 2t+1:2g+1)
+              nib_pairs(x89, e, o);
+              a2 = __byte_perm(e, o, 0x5410);
+              a3 = __byte_perm(e, o, 0x7632);
+              mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
+            }
         } else {
-          // accumulator row k of the block is value column 2k (k < 8) or
-          // 2(k - 8) + 1: A[i][k] = U_v[i][that column], so a thread's k = 2t,
-          // 2t+1 are columns 4t, 4t+2 and k = 2t+8, 2t+9 columns 4t+1, 4t+3
-          const uint2 w0 = *reinterpret_cast<const uint2*>(uv + (16 * mi + g) * S::VS + (mt * 16 + 4 * t) * 2);
-          const uint2 w1 = *reinterpret_cast<const uint2*>(uv + (16 * mi + g + 8) * S::VS + (mt * 16 + 4 * t) * 2);
-          a0 = __byte_perm(w0.x, w0.y, 0x5410);
-          a2 = __byte_perm(w0.x, w0.y, 0x7632);
-          a1 = __byte_perm(w1.x, w1.y, 0x5410);
-          a3 = __byte_perm(w1.x, w1.y, 0x7632);
+          // int8 codes, converted to bf16 in registers (exact).  Logits: an
+          // ldmatrix of a k-step's 16 code bytes gives a thread bytes 4t..4t+3 of
+          // its row, k = 2t, 2t+1 (a0/a1) and 2t+8, 2t+9 (a2/a3) in the order q~'s
+          // B fragments were built in; the row's key scale multiplies the logit.
+          const float* scl = reinterpret_cast<const float*>(slot + S::T_SC);   // [2][32]
+  #pragma unroll
+          for (int nb = 0; nb < 2; ++nb) {
+            st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
+            const unsigned char* rows = slot + (16 * nb + (lm & 1) * 8 + lr) * S::TKS;
+  #pragma unroll
+            for (int kp = 0; kp < KST; kp += 2) {
+              uint32_t r0, r1, r2 = 0u, r3 = 0u, e0, e1, f0, f1;
+              if (kp + 1 < KST) ldsm_x4(r0, r1, r2, r3, rows + kp * 16 + (lm >> 1) * 16);
+              else ldsm_x2(r0, r1, rows + kp * 16);
+              s8x4_pairs(r0, e0, f0);
+              s8x4_pairs(r1, e1, f1);
+              mma_16816(st[nb], e0, e1, f0, f1, qb0[kp], qb1[kp]);
+              if (kp + 1 < KST) {
+                s8x4_pairs(r2, e0, f0);
+                s8x4_pairs(r3, e1, f1);
+                mma_16816(st[nb], e0, e1, f0, f1, qb0[kp + 1], qb1[kp + 1]);
+              }
+            }
+          }
+          float s[2][2], wv[2][2];
+  #pragma unroll
+          for (int nb = 0; nb < 2; ++nb)
+  #pragma unroll
+            for (int x = 0; x < 2; ++x) {   // rows g, g + 8: high + low part of head t
+              const int row = 16 * nb + g + x * 8;
+              const bool on = live_t && ((bits >> row) & 1u);
+              const float v = st[nb][2 * x] + st[nb][2 * x + 1];
+              s[nb][x] = on ? fmaf(v, scl[row], bias) : -INFINITY;
+              wv[nb][x] = on ? scl[kTileC + row] : 0.f;   // scales of unread rows are never used
+            }
+          uint32_t pb0[2], pb1[2];
+          softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv);
+          // values: one transposing ldmatrix per 16 value columns covers the 32
+          // tokens; a thread's bytes are (token 2t | 2t+1) x (column 2g | 2g+1), so
+          // accumulator row g is column 2g of the block and row g + 8 column 2g + 1
+          const unsigned char* vrows = slot + kTileC * S::TKS;
+  #pragma unroll
+          for (int mt = 0; mt < MVT; ++mt) {
+            uint32_t r0, r1, r2, r3, a0, a1, a2, a3;
+            ldsm_x4_t(r0, r1, r2, r3, vrows + (8 * lm + lr) * S::TVS + mt * 16);
+            s8x4_evenodd(r0, a0, a1);
+            s8x4_evenodd(r1, a2, a3);
+            mma_16816(oc[mt], a0, a1, a2, a3, pb0[0], pb1[0]);
+            s8x4_evenodd(r2, a0, a1);
+            s8x4_evenodd(r3, a2, a3);
+            mma_16816(oc[mt], a0, a1, a2, a3, pb0[1], pb1[1]);
+          }
         }
-        mma_16816(of[mi], a0, a1, a2, a3, lb0[mt], lb1[mt]);
+      } else {
+        // full-rank tile: 16 list rows
+        const int k = warp + kWarps * kw;
+        const int nrows = min(kTileF, n_full - k * kTileF);
+        float st[4] = {0.f, 0.f, 0.f, 0.f};
+  #pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(a0, a1, a2, a3, slot + ((lm & 1) * 8 + lr) * S::FS + (ks * 16 + (lm >> 1) * 8) * 2);
+          mma_16816(st, a0, a1, a2, a3, qf0[ks], qf1[ks]);
+        }
+        float s[1][2];
+  #pragma unroll
+        for (int x = 0; x < 2; ++x) {   // rows g, g + 8 (the low-part column is 0 for q)
+          const float v = (st[2 * x] + st[2 * x + 1]) * scale;
+          s[0][x] = live_t && g + x * 8 < nrows ? v : -INFINITY;
+        }
+        uint32_t pb0[1], pb1[1];
+        softmax_pack(s, pb0, pb1, std::integral_constant<int, 1>{});
+        const unsigned char* vrows = slot + kTileF * S::FS;
+  #pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(a0, a1, a2, a3, vrows + ((lm >> 1) * 8 + lr) * S::FS + (mt * 16 + (lm & 1) * 8) * 2);
+          mma_16816(of[mt], a0, a1, a2, a3, pb0[0], pb1[0]);
+        }
       }
-  }
+      __syncwarp();
+    }
+    cp_async_wait<0>();
+    // the row's length ticket: release-only, taken now that this thread has no
+    // copy in flight (a release waits for them); looked at after the record
+    if (APP && tid == tk) seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
+    __syncwarp();
+    griddep_launch_dependents();
 
-  // ---- this warp's partial state into its stage-0 slot -------------------------------
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) l_run += __shfl_xor_sync(kFull, l_run, o);
-  {
-    float* Wp = reinterpret_cast<float*>(slot_of(0, warp));
-    if (live_t) {
-      // lane (g, t): head t, output rows mi*16 + g and mi*16 + g + 8, high + low part
-      float* pf = Wp + S::W_PF + t * kD;
-#pragma unroll
-      for (int mi = 0; mi < 8; ++mi) {
-        pf[mi * 16 + g] = of[mi][0] + of[mi][1];
-        pf[mi * 16 + g + 8] = of[mi][2] + of[mi][3];
+    // ---- lift: of += U_v acc_c^T on the tensor cores --------------------------------
+    // acc_c^T (rows = r_v, columns = head parts) becomes the B operand: lane
+    // (g, t) holds acc_c[head t][16 mt + g (+8)] (high + low part columns), packs
+    // it as bf16 high and low parts (columns 2t, 2t + 1 of an 8x8 tile) and one
+    // transpose gives the fragment (k = 2t, 2t + 1; n = g).  The product lands in
+    // the full-rank accumulators, whose layout is the same: o = both parts summed.
+    {
+      const unsigned char* uv = sm + S::OFF_UV;
+      uint32_t lb0[MVT], lb1[MVT];
+  #pragma unroll
+      for (int mt = 0; mt < MVT; ++mt) {
+        const float x0 = oc[mt][0] + oc[mt][1], x1 = oc[mt][2] + oc[mt][3];
+        const float h0 = __uint_as_float(cvt_bf16x2(x0, x0) << 16);
+        const float h1 = __uint_as_float(cvt_bf16x2(x1, x1) << 16);
+        lb0[mt] = movmatrix_t(cvt_bf16x2(x0, x0 - h0));
+        lb1[mt] = movmatrix_t(cvt_bf16x2(x1, x1 - h1));
       }
-      if (g == 0) {
-        Wp[S::W_M + t] = m_run;
-        Wp[S::W_L + t] = l_run;
+  #pragma unroll
+      for (int mi = 0; mi < 8; ++mi)
+  #pragma unroll
+        for (int mt = 0; mt < MVT; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          if constexpr (CB == 16) {
+            ldsm_x4(a0, a1, a2, a3, uv + (16 * mi + (lm & 1) * 8 + lr) * S::VS + (mt * 16 + (lm >> 1) * 8) * 2);
+          } else {
+            // accumulator row k of the block is value column 2k (k < 8) or
+            // 2(k - 8) + 1: A[i][k] = U_v[i][that column], so a thread's k = 2t,
+            // 2t+1 are columns 4t, 4t+2 and k = 2t+8, 2t+9 columns 4t+1, 4t+3
+            const uint2 w0 = *reinterpret_cast<const uint2*>(uv + (16 * mi + g) * S::VS + (mt * 16 + 4 * t) * 2);
+            const uint2 w1 = *reinterpret_cast<const uint2*>(uv + (16 * mi + g + 8) * S::VS + (mt * 16 + 4 * t) * 2);
+            a0 = __byte_perm(w0.x, w0.y, 0x5410);
+            a2 = __byte_perm(w0.x, w0.y, 0x7632);
+            a1 = __byte_perm(w1.x, w1.y, 0x5410);
+            a3 = __byte_perm(w1.x, w1.y, 0x7632);
+          }
+          mma_16816(of[mi], a0, a1, a2, a3, lb0[mt], lb1[mt]);
+        }
+    }
+
+    // ---- this warp's partial state into its stage-0 slot -------------------------------
+  #pragma unroll
+    for (int o = 4; o < 32; o <<= 1) l_run += __shfl_xor_sync(kFull, l_run, o);
+    {
+      float* Wp = reinterpret_cast<float*>(slot_of(0, warp));
+      if (live_t) {
+        // lane (g, t): head t, output rows mi*16 + g and mi*16 + g + 8, high + low part
+        float* pf = Wp + S::W_PF + t * kD;
+  #pragma unroll
+        for (int mi = 0; mi < 8; ++mi) {
+          pf[mi * 16 + g] = of[mi][0] + of[mi][1];
+          pf[mi * 16 + g + 8] = of[mi][2] + of[mi][3];
+        }
+        if (g == 0) {
+          Wp[S::W_M + t] = m_run;
+          Wp[S::W_L + t] = l_run;
+        }
       }
     }
-  }
-  __syncthreads();
+    __syncthreads();
 
-  // ---- merge the warps into this split's record ---------------------------------
-  auto wpart = [&](int w) { return reinterpret_cast<const float*>(slot_of(0, w)); };
-  __shared__ float s_we[kWarps][G];
-  float* rec0 = p.partials + (bh * p.n_chunk_max + c) * G * (size_t)S::REC;
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wpart(w)[S::W_M + tid]);
-    float Ls = 0.f;
-    for (int w = 0; w < kWarps; ++w) {
-      const float mw = wpart(w)[S::W_M + tid];
-      const float e = mw == -INFINITY ? 0.f : exp2f(mw - M);
-      s_we[w][tid] = e;
-      Ls = fmaf(wpart(w)[S::W_L + tid], e, Ls);
+    // ---- merge the warps into this split's record ---------------------------------
+    auto wpart = [&](int w) { return reinterpret_cast<const float*>(slot_of(0, w)); };
+    __shared__ float s_we[kWarps][G];
+    float* rec0 = p.partials + (bh * p.n_chunk_max + c) * G * (size_t)S::REC;
+    if (tid < G) {
+      float M = -INFINITY;
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wpart(w)[S::W_M + tid]);
+      float Ls = 0.f;
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = wpart(w)[S::W_M + tid];
+        const float e = mw == -INFINITY ? 0.f : exp2f(mw - M);
+        s_we[w][tid] = e;
+        Ls = fmaf(wpart(w)[S::W_L + tid], e, Ls);
+      }
+      rec0[tid * S::REC] = M;
+      rec0[tid * S::REC + 1] = Ls;
+      if (APP && tid == 0) rec0[2] = 0.f;
     }
-    rec0[tid * S::REC] = M;
-    rec0[tid * S::REC + 1] = Ls;
-    if (APP && tid == 0) rec0[2] = owner && s_keep ? 1.f : 0.f;
-  }
-  __syncthreads();
-  for (int o = tid; o < G * kD; o += kThreads) {
-    const int gi = o / kD, i = o - gi * kD;
-    float x = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[S::W_PF + o], s_we[w][gi], x);
-    rec0[gi * S::REC + 4 + i] = x;
+    __syncthreads();
+    for (int o = tid; o < G * kD; o += kThreads) {
+      const int gi = o / kD, i = o - gi * kD;
+      float x = 0.f;
+  #pragma unroll
+      for (int w = 0; w < kWarps; ++w) x = fmaf(wpart(w)[S::W_PF + o], s_we[w][gi], x);
+      rec0[gi * S::REC + 4 + i] = x;
+    }
   }
 
   if (APP && tid == tk) advance_len();
 
   // ---- the last split of this (batch row, kv head) merges every record ------------
   __syncthreads();
-  if (tid == 0) s_last = atom_add_acq_rel_gpu(p.tickets + bh, 1) == n_chunks - 1;
+  if (tid == 0) s_last = atom_add_acq_rel_gpu(p.tickets + bh, 1) == n_rec - 1;
   __syncthreads();
   if (!s_last) return;
   // Warp w < 8 serves query head w / (8 / G) and a block of its columns; each
@@ -1042,7 +1043,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     // one batch of up to 32 records: every load is issued before the first use
     auto batch = [&](int k0, float M) {
       const int k = k0 + lane;
-      const int nk = min(32, n_chunks - k0);
+      const int nk = min(32, n_rec - k0);
       float vals[32][CPL];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
@@ -1055,8 +1056,8 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
           vals[j][0] = j < nk && on ? __ldcg(v) : 0.f;
         }
       }
-      const float m = k < n_chunks ? __ldcg(recs + (size_t)k * kStride) : -INFINITY;
-      const float l = k < n_chunks ? __ldcg(recs + (size_t)k * kStride + 1) : 0.f;
+      const float m = k < n_rec ? __ldcg(recs + (size_t)k * kStride) : -INFINITY;
+      const float l = k < n_rec ? __ldcg(recs + (size_t)k * kStride + 1) : 0.f;
       if (M == -INFINITY) M = warp_max(m);      // a single batch: its own max is the max
       const float w = m == -INFINITY ? 0.f : exp2f(m - M);
       Lsum = fmaf(w, l, Lsum);
@@ -1067,13 +1068,13 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
         for (int u = 0; u < CPL; ++u) acc[u] = fmaf(wj, vals[j][u], acc[u]);
       }
     };
-    if (n_chunks <= 32) {
+    if (n_rec <= 32) {
       batch(0, -INFINITY);
     } else {
       float M = -INFINITY;
-      for (int k = lane; k < n_chunks; k += 32) M = fmaxf(M, __ldcg(recs + (size_t)k * kStride));
+      for (int k = lane; k < n_rec; k += 32) M = fmaxf(M, __ldcg(recs + (size_t)k * kStride));
       M = warp_max(M);
-      for (int k0 = 0; k0 < n_chunks; k0 += 32) batch(k0, M);
+      for (int k0 = 0; k0 < n_rec; k0 += 32) batch(k0, M);
     }
     Lsum = warp_sum(Lsum);
     if (on) {
@@ -1085,8 +1086,8 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   if (tid == 0) {
     p.tickets[bh] = 0;
     // fused append: every CTA of this (b, kv head) has read the list length;
-    // the new full-rank row (if the owner appended one) now counts
-    if (APP && __ldcg(p.partials + (bh * p.n_chunk_max + n_chunks - 1) * G * (size_t)S::REC + 2) != 0.f)
+    // the new full-rank row (if the append CTA added one) now counts
+    if (APP && __ldcg(p.partials + (bh * p.n_chunk_max + n_chunks) * G * (size_t)S::REC + 2) != 0.f)
       p.C.full_cnt[bh] = F + 1;
   }
 }

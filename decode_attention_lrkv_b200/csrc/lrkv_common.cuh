@@ -224,9 +224,11 @@ inline WsLayout ws_layout(const lrkv_dims& D) {
   off = align_up(off + sizeof(int32_t) * (size_t)D.B * D.Hkv * L.n_tiles, 256);
   L.tile_bits = off;
   off = align_up(off + sizeof(uint32_t) * 4 * (size_t)D.B * D.Hkv * L.n_tiles, 256);
-  // decode: the grid has the splits of a full cache; each CTA re-splits the
-  // live length (decode_split) within them
+  // decode: the grid has the splits of a full cache (at least two: a fused
+  // append takes the last CTA); each CTA re-splits the live length
+  // (decode_split) within them
   L.n_chunk_max = decode_split(D.T_cap, 1024, (long long)D.B * D.Hkv, num_sms(), &L.chunk);
+  if (L.n_chunk_max < 2) L.n_chunk_max = 2;
   L.partial_floats = 4 + D.r_v + D.d;   // m, l, pad, pad, acc_c[r_v], acc_f[d]
   L.partials = off;
   int g = D.Hkv > 0 ? D.Hq / D.Hkv : 0;
