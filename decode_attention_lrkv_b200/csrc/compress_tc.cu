@@ -2,6 +2,7 @@
 // passes, in their own translation unit (declared in compress_tc.h).
 #include <cuda.h>
 
+#include <algorithm>
 #include <cstdlib>
 
 #include "compress_tc.cuh"
@@ -62,6 +63,42 @@ bool rows_map(CUtensorMap* map, const lrkv_bf16* base, const lrkv_dims& D, int t
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The projection's grid over `groups` (kv head, K or V) groups of `n_units`
+// tiles each (Params::per_group): k CTAs per group, or one range per SM over
+// the groups' tiles laid end to end, a range that crosses into the next group
+// finishing there as a second CTA.  The modelled makespan in tiles (with
+// kCtaSetupTiles for each CTA on an SM: basis layouts, U U^T, the pipeline's
+// fill and drain) picks one: 64 groups on 148 SMs leave 20 SMs idle in the
+// first form.
+int projection_grid(int groups, int n_units, int sms, ptc::Params* pp) {
+  constexpr long long kCtaSetupTiles = 8;
+  const long long total = (long long)groups * n_units;
+  int k = sms / groups;
+  if (k < 1) k = 1;
+  if (k > n_units) k = n_units;
+  const long long grid_a = (long long)k * groups;
+  const long long cost_a = (grid_a + sms - 1) / sms * ((n_units + k - 1) / k + kCtaSetupTiles);
+  const int n_ranges = (int)(total < sms ? total : sms);
+  const long long per = (total + n_ranges - 1) / n_ranges;
+  const long long cost_b = per + 2 * kCtaSetupTiles;
+  pp->per_group = k;
+  pp->n_ranges = 0;
+  if (per > n_units || n_ranges > ptc::kMaxRanges || cost_b >= cost_a) return (int)grid_a;
+  // ranges split at a group end: their second parts, longest first
+  const int q = (int)(total / n_ranges), r = (int)(total % n_ranges);
+  int order[ptc::kMaxRanges], rest[ptc::kMaxRanges], n2 = 0;
+  for (int x = 0; x < n_ranges; ++x) {
+    const int l0 = x * q + (x < r ? x : r), l1 = l0 + q + (x < r ? 1 : 0);
+    const int end = (l0 / n_units + 1) * n_units;
+    if (l1 > end) order[n2] = x, rest[x] = l1 - end, ++n2;
+  }
+  std::stable_sort(order, order + n2, [&](int a, int b) { return rest[a] > rest[b]; });
+  for (int j = 0; j < n2; ++j) pp->second[j] = (uint16_t)order[j];
+  pp->per_group = 0;
+  pp->n_ranges = n_ranges;
+  return n_ranges + n2;
+}
+
 // Prefill-sized compress: tensor-core projection, then the two routing passes.
 }  // namespace
 
@@ -69,6 +106,9 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
                         const lrkv_bf16* v_new, int t_new, const int32_t* t_new_b, float tau,
                         float* err_out, char* w, const WsLayout& L, cudaStream_t s) {
   ptc::Params pp = {};
+  const int tmax0 = t_new < D.T_cap ? t_new : D.T_cap;
+  // the projection counts its tiles over every (kv head, K or V) group in 32 bits
+  if (2LL * D.Hkv * D.B * ((tmax0 + ptc::kTile - 1) / ptc::kTile) >= (1LL << 31)) return LRKV_ERR_UNSUPPORTED;
   if (!rows_map(&pp.map_k, k_new, D, t_new) || !rows_map(&pp.map_v, v_new, D, t_new))
     return LRKV_ERR_CUDA;
   const int tmax = t_new < D.T_cap ? t_new : D.T_cap;
@@ -81,11 +121,7 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
   pp.r_max = D.r_k > D.r_v ? D.r_k : D.r_v;
   pp.n_stages = ptc::stages_for(pp.r_max);
   pp.wait_iters = main_wait_iters();
-  const int groups = 2 * D.Hkv;
-  const int n_units = D.B * pp.tiles_per_b;
-  int per_group = num_sms() / groups;
-  if (per_group < 1) per_group = 1;
-  if (per_group > n_units) per_group = n_units;
+  const int n_ctas = projection_grid(2 * D.Hkv, D.B * pp.tiles_per_b, num_sms(), &pp);
   const size_t smem = ptc::Layout(pp.r_max, pp.n_stages).bytes;
   const int bits = coef_bits_of(D);
   auto kern = bits == 8 ? ptc::project_tc_kernel<8> : bits == 4 ? ptc::project_tc_kernel<4>
@@ -93,7 +129,7 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
   if (!set_smem(kern, smem) || !set_smem(ptc::route_count_kernel, 0) ||
       !set_smem(ptc::route_scatter_kernel, 0))
     return LRKV_ERR_CUDA;
-  kern<<<dim3(per_group, groups), ptc::kThreads, smem, s>>>(pp);
+  kern<<<n_ctas, ptc::kThreads, smem, s>>>(pp);
   lrkv_status st = launched();
   if (st != LRKV_OK) return st;
   ptc::RouteParams rp = {};

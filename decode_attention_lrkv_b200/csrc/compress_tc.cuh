@@ -10,9 +10,10 @@
 // same quantity computed in one product; U is bf16 and not exactly
 // orthonormal, so P is not a projector and no norm identity is used.
 //
-// Kernel 1, project_tc_kernel: one CTA per SM works on one (kv head, K or V)
-// stream of 128-token tiles.  Per CTA, P is formed once on the tensor cores
-// (U U^T) and split into bf16 high and low parts (P = P_hi + P_lo to 2^-17).
+// Kernel 1, project_tc_kernel: each CTA works on a contiguous run of the
+// 128-token tiles of one (kv head, K or V) group.  Per CTA, P is formed once
+// on the tensor cores (U U^T) and split into bf16 high and low parts (P =
+// P_hi + P_lo to 2^-17).
 // Per tile, TMA brings the 128 x 128 input rows (128-byte swizzle); one
 // thread issues
 //     [D2 | D1] = X [P_hi | U]   (M 128, N 128 + r, K 128)
@@ -58,6 +59,7 @@ constexpr int kBoxBytes = kStageBytes / 2;
 constexpr uint32_t kTmemCols = 512;                  // two buffers of [D1 | D2]
 constexpr uint32_t kWaitIters = 1u << 22;
 constexpr size_t kSmemLimit = 227 * 1024;
+constexpr int kMaxRanges = 256;                      // tile ranges of the end-to-end split
 
 // Shared memory (bytes) for rank rm (the larger rank of the launch: both
 // tensors share one layout) and ns input stages; operand regions 1024-aligned.
@@ -103,7 +105,37 @@ struct Params {
   int r_max;             // max(r_k, r_v): the shared-memory layout
   int n_stages;          // input stages: stages_for(r_max)
   uint32_t wait_iters;   // limit of the MMA issuer's wait for each input tile (kWaitIters)
+  // Which tiles a CTA takes.  per_group > 0: that many CTAs per group, CTA x
+  // on group x / per_group.  per_group = 0: the groups' tiles laid end to end
+  // are cut into n_ranges equal ranges (one per SM, each within two groups);
+  // CTA x < n_ranges takes range x up to its group's end, and CTA n_ranges + k
+  // the rest of range second[k] (those rests in decreasing length, so that the
+  // SM that finishes its first part soonest picks up the longest rest).
+  int per_group;
+  int n_ranges;
+  uint16_t second[kMaxRanges];
 };
+
+// This CTA's group and tiles [u_begin, u_end) of it (Params: per_group).
+__device__ __forceinline__ int cta_tiles(const Params& p, int n_units, int* u_begin, int* u_end) {
+  const int x = (int)blockIdx.x;
+  if (p.per_group > 0) {
+    const int grp = x / p.per_group, sub = x - grp * p.per_group;
+    const int q = n_units / p.per_group, r = n_units - q * p.per_group;
+    *u_begin = sub * q + min(sub, r);
+    *u_end = *u_begin + q + (sub < r ? 1 : 0);
+    return grp;
+  }
+  const int total = 2 * p.D.Hkv * n_units;
+  const int q = total / p.n_ranges, r = total - q * p.n_ranges;
+  const bool first = x < p.n_ranges;
+  const int rg = first ? x : p.second[x - p.n_ranges];
+  const int l0 = rg * q + min(rg, r), l1 = l0 + q + (rg < r ? 1 : 0);
+  const int grp = l0 / n_units + (first ? 0 : 1);
+  *u_begin = first ? l0 - grp * n_units : 0;
+  *u_end = min(l1 - grp * n_units, n_units);
+  return grp;
+}
 
 // Byte offset of element (row n, column k) in a no-swizzle K-major operand:
 // 8x8 core matrices of 128 contiguous bytes, K-adjacent ones 128 B apart and
@@ -151,7 +183,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
   return false;
 }
 
-// grid (CTAs per group, 2 * Hkv): group = 2 h + tensor (0 keys, 1 values).
+// 1-d grid (Params: per_group); group = 2 h + tensor (0 keys, 1 values).
 // CB: stored coefficient format, 16 (bf16) or 8, 4 (codes with per-row scales).
 template <int CB>
 __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_constant__ Params p) {
@@ -161,7 +193,9 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const lrkv_dims& D = p.D;
-  const int group = blockIdx.y, tensor = group & 1, h = group >> 1;
+  const int n_units = D.B * p.tiles_per_b;
+  int u_begin, u_end;
+  const int group = cta_tiles(p, n_units, &u_begin, &u_end), tensor = group & 1, h = group >> 1;
   const CUtensorMap* map = tensor == 0 ? &p.map_k : &p.map_v;
   const int R = tensor == 0 ? D.r_k : D.r_v;
   const int NS = p.n_stages;
@@ -183,11 +217,6 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   uint64_t* drain = pready + 1;          // final MMA drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  // this CTA's units: a contiguous range of the (b, tile) list of its group
-  const int n_units = D.B * p.tiles_per_b;
-  const int u_begin = (int)((long long)blockIdx.x * n_units / gridDim.x);
-  const int u_end = (int)((long long)(blockIdx.x + 1) * n_units / gridDim.x);
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {

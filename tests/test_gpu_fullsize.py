@@ -197,3 +197,99 @@ def test_long_capacity_holding_8k():
         gc = _gpu_head(D, cache, 0, h)
         ref = O.decode_attn(gc, q[0:1, h * g:(h + 1) * g])
         assert U.out_rel_err(o2[0, h * g:(h + 1) * g], ref[0]) <= U.OUT_RTOL, h
+
+
+@pytest.mark.parametrize("wi,bits", [(4, 8), (1, 4)], ids=["mha131072_int8", "llama8k_int4"])
+def test_full_size_quantised(wi, bits):
+    """A quantised cache at full context beside a bf16 cache fed the same calls
+    (prefill, one append, one fused append + decode): on sampled heads the codes
+    and scales equal the oracle's quantiser applied to the bf16 rows the same
+    calls stored (bit for bit), the routing state is the bf16 cache's, and the
+    decode matches the oracle's decode over the dequantised rows."""
+    w = synth.workload(wi, layers=1)
+    seed = 51 + wi
+    layer = synth.make_layer(w, 0, seed, device=DEV)
+    T_cap = synth.pad_to(w.T + BENCH_EXTRA, 32)
+    Db = U.dims_of(w, T_cap, bench_f_cap(wi, T_cap))
+    Dq = U.dims_of(w, T_cap, bench_f_cap(wi, T_cap), coef_bits=bits)
+    cb = L.LayerCache(Db, layer["U_k"], layer["U_v"], device=DEV)
+    cq = L.LayerCache(Dq, layer["U_k"], layer["U_v"], device=DEV)
+    wsb, wsq = L.make_workspace(Db, DEV), L.make_workspace(Dq, DEV)
+    Ka, Va = synth.decode_tokens(w, layer["Qk"], layer["Qv"], 2, seed, 0, DEV)
+    qf = synth.decode_queries(w, 1, seed, 0, DEV)
+    outs = []
+    for D, c, ws in ((Db, cb, wsb), (Dq, cq, wsq)):
+        L.lrkv_compress(D, c, layer["K"], layer["V"], w.tau, ws=ws)
+        L.lrkv_compress(D, c, Ka[:, :1].contiguous(), Va[:, :1].contiguous(), w.tau, ws=ws)
+        o = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=DEV)
+        L.lrkv_append_decode_attn(D, c, Ka[:, 1:2].contiguous(), Va[:, 1:2].contiguous(), w.tau, qf[0], o, ws=ws)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert int(cq.dev_status[0]) == 0 and int(cb.dev_status[0]) == 0
+    for f in ("route_mask", "full_idx", "full_cnt", "seq_len"):
+        assert torch.equal(getattr(cq, f), getattr(cb, f)), f
+    out = U.f64(outs[1])
+    q = U.f64(qf[0])
+    g = w.Hq // w.Hkv
+    T = int(cq.seq_len[0])
+    rng = np.random.default_rng(seed)
+    for h in sorted({0, w.Hkv - 1, int(rng.integers(w.Hkv))}):
+        gb = _gpu_head(Db, cb, 0, h)
+        want = O.quantize_cache(gb, bits)
+        codes = lambda t: t.cpu().numpy().view(np.int8) if bits == 8 else O.unpack_int4(t.cpu().numpy())
+        qk, qv = codes(cq.coef_k[0, h, :T]), codes(cq.coef_v[0, h, :T])
+        sk, sv = cq.scale_k[0, h, :T].cpu().numpy(), cq.scale_v[0, h, :T].cpu().numpy()
+        assert np.array_equal(qk, want["qk"][0, 0, :T]) and np.array_equal(sk, want["sk"][0, 0, :T]), h
+        assert np.array_equal(qv, want["qv"][0, 0, :T]) and np.array_equal(sv, want["sv"][0, 0, :T]), h
+        gq = gb
+        gq.coef_k[0, 0, :T] = O.dequantize_coef(qk, sk)
+        gq.coef_v[0, 0, :T] = O.dequantize_coef(qv, sv)
+        ref = O.decode_attn(gq, q[0:1, h * g:(h + 1) * g])
+        assert U.out_rel_err(out[0, h * g:(h + 1) * g], ref[0]) <= U.OUT_RTOL, h
+
+
+def test_full_size_attention_aware():
+    """The 8K workload with an attention-aware key basis (Theorem 1 from seeded
+    calibration queries and the head's keys): sampled heads' coefficients,
+    routing and decode against the oracle's aware cache."""
+    from tests.test_gpu_aware import _aware_bases
+    w = synth.workload(1, layers=1)
+    seed = 57
+    layer = synth.make_layer(w, 0, seed, device=DEV)
+    T_cap = synth.pad_to(w.T + BENCH_EXTRA, 32)
+    # the aware key basis routes far more than the orthonormal one here (its
+    # mean is not in the span): a list for every position
+    D = U.dims_of(w, T_cap, T_cap)
+    K64 = U.f64(layer["K"])
+    Wk, Wq, mu = _aware_bases(K64, w.r_k, seed)
+    t = lambda a, dt: torch.from_numpy(a).to(dt).to(DEV)
+    cache = L.LayerCache(D, t(Wk, torch.bfloat16), layer["U_v"], device=DEV,
+                         U_kq=t(Wq, torch.bfloat16), mu_k=t(mu, torch.float32))
+    ws = L.make_workspace(D, DEV)
+    L.lrkv_compress(D, cache, layer["K"], layer["V"], w.tau, ws=ws)
+    Ka, Va = synth.decode_tokens(w, layer["Qk"], layer["Qv"], 1, seed, 0, DEV)
+    o = torch.empty(w.B, w.Hq, w.d, dtype=torch.float32, device=DEV)
+    L.lrkv_append_decode_attn(D, cache, Ka.contiguous(), Va.contiguous(), w.tau, layer["q"], o, ws=ws)
+    torch.cuda.synchronize()
+    assert int(cache.dev_status[0]) == 0
+    out, q = U.f64(o), U.f64(layer["q"])
+    g = w.Hq // w.Hkv
+    V64, Uv = U.f64(layer["V"]), U.f64(layer["U_v"])
+    for h in (0, 3, 7):
+        od = O.Dims(B=1, Hq=g, Hkv=1, d=w.d, r_k=w.r_k, r_v=w.r_v, T_cap=T_cap, F_cap=D.F_cap)
+        oc = O.Cache.empty(od, Wk[h:h + 1], Uv[h:h + 1], U_kq=Wq[h:h + 1], mu_k=mu[h:h + 1])
+        e0, _, _ = O.compress(oc, K64[:, :, h:h + 1], V64[:, :, h:h + 1], w.tau)
+        e1, _, _ = O.compress(oc, U.f64(Ka)[:, :, h:h + 1], U.f64(Va)[:, :, h:h + 1], w.tau)
+        e_ref = np.concatenate([e0[0, 0], e1[0, 0]])
+        gc = _gpu_head(D, cache, 0, h)
+        gc.U_kq, gc.mu_k = oc.U_kq, oc.mu_k
+        T = int(oc.seq_len[0])
+        X = np.concatenate([K64[0, :, h], U.f64(Ka)[0, :, h]])
+        tol = O.bf16_ulp(np.maximum(np.abs(gc.coef_k[0, 0, :T]), np.abs(oc.coef_k[0, 0, :T])))
+        tol = tol + U.COEF_ABS_SAFETY * U.GAMMA_128 * ((np.abs(X) + np.abs(mu[h])) @ np.abs(Wk[h]))
+        assert (np.abs(gc.coef_k[0, 0, :T] - oc.coef_k[0, 0, :T]) <= tol).all(), h
+        band = set(np.flatnonzero(np.abs(e_ref - w.tau) < U.BAND).tolist())
+        rg, ro = set(U.routed_positions(gc, 0, 0)), set(U.routed_positions(oc, 0, 0))
+        assert (rg ^ ro) <= band, h
+        ref = O.decode_attn(gc, q[0:1, h * g:(h + 1) * g])
+        assert U.out_rel_err(out[0, h * g:(h + 1) * g], ref[0]) <= U.OUT_RTOL, h
