@@ -589,8 +589,15 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     }
     const bool lo_n = g & 1;
     const bool live = (g >> 1) < G;
-    s_qb[ks2][0][lane] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
-    s_qb[ks2][1][lane] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
+    if constexpr (CB == 8) {
+      // int8 codes meet q~ as f16 (high and low parts): a code widens to f16
+      // in half the instructions it takes to reach bf16
+      s_qb[ks2][0][lane] = live ? f16_part_bits(x0 * scale, lo_n) | (f16_part_bits(x1 * scale, lo_n) << 16) : 0u;
+      s_qb[ks2][1][lane] = live ? f16_part_bits(y0 * scale, lo_n) | (f16_part_bits(y1 * scale, lo_n) << 16) : 0u;
+    } else {
+      s_qb[ks2][0][lane] = live ? pack_bf16(bf16_part(x0 * scale, lo_n), bf16_part(x1 * scale, lo_n)) : 0u;
+      s_qb[ks2][1][lane] = live ? pack_bf16(bf16_part(y0 * scale, lo_n), bf16_part(y1 * scale, lo_n)) : 0u;
+    }
   }
   // q . mu_k per query head (scaled), added to every compressed logit: 0 unless
   // the cache has an attention-aware key basis with a mean
@@ -839,10 +846,12 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
               mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
             }
         } else {
-          // int8 codes, converted to bf16 in registers (exact).  Logits: an
-          // ldmatrix of a k-step's 16 code bytes gives a thread bytes 4t..4t+3 of
-          // its row, k = 2t, 2t+1 (a0/a1) and 2t+8, 2t+9 (a2/a3) in the order q~'s
-          // B fragments were built in; the row's key scale multiplies the logit.
+          // int8 codes, converted in registers (exact): to f16 for the logits
+          // (against q~'s f16 high and low parts), to bf16 for the value sums.
+          // Logits: an ldmatrix of a k-step's 16 code bytes gives a thread bytes
+          // 4t..4t+3 of its row, k = 2t, 2t+1 (a0/a1) and 2t+8, 2t+9 (a2/a3) in
+          // the order q~'s B fragments were built in; the row's key scale
+          // multiplies the logit.
           const float* scl = reinterpret_cast<const float*>(slot + S::T_SC);   // [2][32]
   #pragma unroll
           for (int nb = 0; nb < 2; ++nb) {
@@ -853,13 +862,13 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
               uint32_t r0, r1, r2 = 0u, r3 = 0u, e0, e1, f0, f1;
               if (kp + 1 < KST) ldsm_x4(r0, r1, r2, r3, rows + kp * 16 + (lm >> 1) * 16);
               else ldsm_x2(r0, r1, rows + kp * 16);
-              s8x4_pairs(r0, e0, f0);
-              s8x4_pairs(r1, e1, f1);
-              mma_16816(st[nb], e0, e1, f0, f1, qb0[kp], qb1[kp]);
+              s8x4_f16pairs(r0, e0, f0);
+              s8x4_f16pairs(r1, e1, f1);
+              mma_16816_f16(st[nb], e0, e1, f0, f1, qb0[kp], qb1[kp]);
               if (kp + 1 < KST) {
-                s8x4_pairs(r2, e0, f0);
-                s8x4_pairs(r3, e1, f1);
-                mma_16816(st[nb], e0, e1, f0, f1, qb0[kp + 1], qb1[kp + 1]);
+                s8x4_f16pairs(r2, e0, f0);
+                s8x4_f16pairs(r3, e1, f1);
+                mma_16816_f16(st[nb], e0, e1, f0, f1, qb0[kp + 1], qb1[kp + 1]);
               }
             }
           }

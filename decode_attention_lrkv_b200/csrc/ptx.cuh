@@ -2,6 +2,7 @@
 // bulk (TMA) global->shared copies.  Every wait is bounded by the caller.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace lrkv {
@@ -144,6 +145,15 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+// The same shape with f16 operands: D = A(16x16 f16, row) * B(16x8 f16, col) + D.
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 // D = A(16x8 bf16, row) * B(8x8 bf16, col) + D, fp32 accumulate.
 __device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
   asm volatile(
@@ -206,6 +216,12 @@ __device__ __forceinline__ float bf16_part(float x, bool lo_part) {
   const float h = __bfloat162float(__float2bfloat16_rn(x));
   return lo_part ? x - h : h;
 }
+// The f16 high part of x (round to nearest even), or the low part x - high,
+// each as an f16 bit pattern.
+__device__ __forceinline__ uint32_t f16_part_bits(float x, bool lo_part) {
+  const __half h = __float2half_rn(x);
+  return __half_as_ushort(lo_part ? __float2half_rn(x - __half2float(h)) : h);
+}
 
 }  // namespace lrkv
 
@@ -238,6 +254,18 @@ __device__ __forceinline__ void s8x4_pairs(uint32_t w, uint32_t& b01, uint32_t& 
   const uint32_t u = w ^ 0x80808080u;
   b01 = bf16x2_upper(s8_byte_f32(u, 0x7440), s8_byte_f32(u, 0x7441));
   b23 = bf16x2_upper(s8_byte_f32(u, 0x7442), s8_byte_f32(u, 0x7443));
+}
+// Four int8 codes in w: f16x2 of bytes (0, 1) and of bytes (2, 3), exactly.
+// With the sign bit flipped a byte is u = b + 128 in [0, 255]; the f16 with
+// high byte 0x64 and low byte u is 1024 + u (f16 spacing is 1 on [1024,
+// 2048)), and subtracting 1152 leaves b.
+__device__ __forceinline__ void s8x4_f16pairs(uint32_t w, uint32_t& h01, uint32_t& h23) {
+  const uint32_t u = w ^ 0x80808080u;
+  h01 = __byte_perm(u, 0x64646464u, 0x4140);
+  h23 = __byte_perm(u, 0x64646464u, 0x4342);
+  const uint32_t k1 = 0x3C003C00u, km = 0xE480E480u;   // f16x2 (1, 1), (-1152, -1152)
+  asm("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(h01) : "r"(k1), "r"(km));
+  asm("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(h23) : "r"(k1), "r"(km));
 }
 // Four int8 codes in w: bf16x2 of bytes (0, 2) and of bytes (1, 3).
 __device__ __forceinline__ void s8x4_evenodd(uint32_t w, uint32_t& b02, uint32_t& b13) {
