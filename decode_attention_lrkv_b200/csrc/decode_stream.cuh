@@ -697,13 +697,26 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   #pragma unroll
     for (int mt = 0; mt < 8; ++mt) of[mt][0] = of[mt][1] = of[mt][2] = of[mt][3] = 0.f;
 
+    // int8 codes: the value sums run on f16 operands, p * w (w the row's code
+    // scale) times 2^e_v, so the largest row scale seen sits near 2^9..2^10:
+    // far from f16 overflow, and the smallest weights that matter stay normal.
+    // e_v is set by the first tile with a code row and only lowered when a
+    // later tile would come within 2^15; the accumulators then scale by the
+    // power of two (exact).  The lift divides them by 2^e_v.
+    int e_v = 0;
+    bool e_set = false;
+    float v_scale = 1.f;
+
     // Online softmax over NB 16-row blocks: s[nb] = {row g, row g + 8} of head t
     // (-inf = no token).  Rescales this lane's accumulators when the max grows,
     // and returns the probabilities packed as the P^T B fragments of each block
-    // (column 2t = bf16 high part, 2t + 1 = low part); with value weights wv
-    // (the rows' code scales) the packed entries are p * wv, the sum l takes p.
-    auto softmax_pack_w = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag, const float (*wv)[2]) {
+    // (column 2t = high part, 2t + 1 = low part; bf16, or f16 with F16); with
+    // value weights wv (the rows' code scales) the packed entries are p * wv,
+    // the sum l takes p.
+    auto softmax_pack_w = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag, const float (*wv)[2],
+                              auto f16_tag) {
       constexpr int NB = decltype(nb_tag)::value;
+      constexpr bool F16 = decltype(f16_tag)::value;
       float x = -INFINITY;
   #pragma unroll
       for (int nb = 0; nb < NB; ++nb) x = fmaxf(x, fmaxf(s[nb][0], s[nb][1]));
@@ -729,6 +742,13 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
         float p1 = s[nb][1] == -INFINITY ? 0.f : exp2f(s[nb][1] - m_run);
         l_run += p0 + p1;
         if (wv) p0 *= wv[nb][0], p1 *= wv[nb][1];
+        if constexpr (F16) {   // (high part, low part): f16(p) and f16(p - f16(p))
+          const float h0 = __half2float(__float2half_rn(p0));
+          const float h1 = __half2float(__float2half_rn(p1));
+          pb0[nb] = movmatrix_t(cvt_f16x2(p0, p0 - h0));
+          pb1[nb] = movmatrix_t(cvt_f16x2(p1, p1 - h1));
+          continue;
+        }
         // (high part, low part) of p: bf16(p) and bf16(p - bf16(p))
         const float h0 = __uint_as_float(cvt_bf16x2(p0, p0) << 16);
         const float h1 = __uint_as_float(cvt_bf16x2(p1, p1) << 16);
@@ -737,7 +757,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       }
     };
     auto softmax_pack = [&](auto& s, auto& pb0, auto& pb1, auto nb_tag) {
-      softmax_pack_w(s, pb0, pb1, nb_tag, static_cast<const float (*)[2]>(nullptr));
+      softmax_pack_w(s, pb0, pb1, nb_tag, static_cast<const float (*)[2]>(nullptr), std::false_type{});
     };
 
     for (int i = 0; i < n_tiles; ++i) {
@@ -825,7 +845,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
               wv[nb][x] = on ? scl[kTileC + row] : 0.f;
             }
           uint32_t pb0[2], pb1[2];
-          softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv);
+          softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv, std::false_type{});
           const unsigned char* vrows = slot + kTileC * S::TKS;
   #pragma unroll
           for (int mt = 0; mt < MVT; ++mt)
@@ -873,18 +893,41 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
             }
           }
           float s[2][2], wv[2][2];
+          float wmax = 0.f;   // the largest code scale of the tile's read rows
   #pragma unroll
           for (int nb = 0; nb < 2; ++nb)
   #pragma unroll
             for (int x = 0; x < 2; ++x) {   // rows g, g + 8: high + low part of head t
               const int row = 16 * nb + g + x * 8;
-              const bool on = live_t && ((bits >> row) & 1u);
+              const bool read = (bits >> row) & 1u;
+              const bool on = live_t && read;
               const float v = st[nb][2 * x] + st[nb][2 * x + 1];
               s[nb][x] = on ? fmaf(v, scl[row], bias) : -INFINITY;
-              wv[nb][x] = on ? scl[kTileC + row] : 0.f;   // scales of unread rows are never used
+              const float w = read ? scl[kTileC + row] : 0.f;   // scales of unread rows are never used
+              wmax = fmaxf(wmax, w);
+              wv[nb][x] = on ? w : 0.f;
             }
+  #pragma unroll
+          for (int o = 4; o < 32; o <<= 1) wmax = fmaxf(wmax, __shfl_xor_sync(kFull, wmax, o));
+          if (wmax > 0.f) {   // warp-uniform
+            const int ew = (int)((__float_as_uint(wmax) >> 23) & 0xff) - 127;   // wmax in [2^ew, 2^(ew+1))
+            if (!e_set || ew + e_v >= 15) {
+              const int e_new = min(max(9 - ew, -126), 126);
+              if (e_set) {   // lower the scale of what is summed so far (e_new < e_v)
+                const int d = e_new - e_v;
+                const float f = d < -126 ? 0.f : __uint_as_float((uint32_t)(d + 127) << 23);
+  #pragma unroll
+                for (int mt = 0; mt < MVT; ++mt) oc[mt][0] *= f, oc[mt][1] *= f, oc[mt][2] *= f, oc[mt][3] *= f;
+              }
+              e_v = e_new;
+              e_set = true;
+              v_scale = __uint_as_float((uint32_t)(e_v + 127) << 23);
+            }
+          }
+  #pragma unroll
+          for (int nb = 0; nb < 2; ++nb) wv[nb][0] *= v_scale, wv[nb][1] *= v_scale;
           uint32_t pb0[2], pb1[2];
-          softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv);
+          softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv, std::true_type{});
           // values: one transposing ldmatrix per 16 value columns covers the 32
           // tokens; a thread's bytes are (token 2t | 2t+1) x (column 2g | 2g+1), so
           // accumulator row g is column 2g of the block and row g + 8 column 2g + 1
@@ -893,12 +936,12 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
           for (int mt = 0; mt < MVT; ++mt) {
             uint32_t r0, r1, r2, r3, a0, a1, a2, a3;
             ldsm_x4_t(r0, r1, r2, r3, vrows + (8 * lm + lr) * S::TVS + mt * 16);
-            s8x4_evenodd(r0, a0, a1);
-            s8x4_evenodd(r1, a2, a3);
-            mma_16816(oc[mt], a0, a1, a2, a3, pb0[0], pb1[0]);
-            s8x4_evenodd(r2, a0, a1);
-            s8x4_evenodd(r3, a2, a3);
-            mma_16816(oc[mt], a0, a1, a2, a3, pb0[1], pb1[1]);
+            s8x4_f16evenodd(r0, a0, a1);
+            s8x4_f16evenodd(r1, a2, a3);
+            mma_16816_f16(oc[mt], a0, a1, a2, a3, pb0[0], pb1[0]);
+            s8x4_f16evenodd(r2, a0, a1);
+            s8x4_f16evenodd(r3, a2, a3);
+            mma_16816_f16(oc[mt], a0, a1, a2, a3, pb0[1], pb1[1]);
           }
         }
       } else {
@@ -948,7 +991,11 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       uint32_t lb0[MVT], lb1[MVT];
   #pragma unroll
       for (int mt = 0; mt < MVT; ++mt) {
-        const float x0 = oc[mt][0] + oc[mt][1], x1 = oc[mt][2] + oc[mt][3];
+        float x0 = oc[mt][0] + oc[mt][1], x1 = oc[mt][2] + oc[mt][3];
+        if constexpr (CB == 8) {   // back from the 2^e_v scale of the value sums (exact)
+          const float inv = __uint_as_float((uint32_t)(127 - e_v) << 23);
+          x0 *= inv, x1 *= inv;
+        }
         const float h0 = __uint_as_float(cvt_bf16x2(x0, x0) << 16);
         const float h1 = __uint_as_float(cvt_bf16x2(x1, x1) << 16);
         lb0[mt] = movmatrix_t(cvt_bf16x2(x0, x0 - h0));

@@ -267,6 +267,21 @@ __device__ __forceinline__ void s8x4_f16pairs(uint32_t w, uint32_t& h01, uint32_
   asm("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(h01) : "r"(k1), "r"(km));
   asm("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(h23) : "r"(k1), "r"(km));
 }
+// Four int8 codes in w: f16x2 of bytes (0, 2) and of bytes (1, 3), exactly.
+__device__ __forceinline__ void s8x4_f16evenodd(uint32_t w, uint32_t& h02, uint32_t& h13) {
+  const uint32_t u = w ^ 0x80808080u;
+  h02 = __byte_perm(u, 0x64646464u, 0x4240);
+  h13 = __byte_perm(u, 0x64646464u, 0x4341);
+  const uint32_t k1 = 0x3C003C00u, km = 0xE480E480u;   // f16x2 (1, 1), (-1152, -1152)
+  asm("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(h02) : "r"(k1), "r"(km));
+  asm("fma.rn.f16x2 %0, %0, %1, %2;" : "+r"(h13) : "r"(k1), "r"(km));
+}
+// Two floats -> f16x2 in one conversion (round to nearest even), `lo` in the low half.
+__device__ __forceinline__ uint32_t cvt_f16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
 // Four int8 codes in w: bf16x2 of bytes (0, 2) and of bytes (1, 3).
 __device__ __forceinline__ void s8x4_evenodd(uint32_t w, uint32_t& b02, uint32_t& b13) {
   const uint32_t u = w ^ 0x80808080u;

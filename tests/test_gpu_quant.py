@@ -156,3 +156,38 @@ def test_decode_on_oracle_quantised_cache(bits):
     assert U.out_rel_err(out, ref) <= U.OUT_RTOL
     # the code-space form of the oracle agrees with its plain form
     assert U.out_rel_err(O.decode_attn_quant_coef(oc, ocd, U.f64(layer["q"])), ref) <= 1e-12
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_value_scales_spanning_many_octaves(bits):
+    """Row value scales that jump by tens of octaves along the sequence (2^-40,
+    then 1, then 2^20 times the quantiser's): the int8 value sums run on f16
+    operands under a per-warp power-of-two scale that later tiles must lower.
+    The decode still matches the oracle's over the same codes and scales."""
+    w = synth.workload(1, T=2100, layers=1)
+    layer = synth.make_layer(w, 0, 75, device=DEV)
+    D = U.dims_of(w, synth.pad_to(w.T, 32), coef_bits=bits)
+    oc = O.Cache.empty(U.oracle_dims(D), U.f64(layer["U_k"]), U.f64(layer["U_v"]))
+    O.compress(oc, U.f64(layer["K"]), U.f64(layer["V"]), w.tau)
+    ocd = O.quantize_cache(oc, bits)
+    sv = ocd["sv"].astype(np.float64)
+    sv[:, :, :700] *= 2.0 ** -40
+    sv[:, :, 1400:] *= 2.0 ** 20
+    ocd["sv"] = sv.astype(np.float32)
+    _, bf = U.oracle_to_gpu(oc)
+    cache = L.LayerCache(D, layer["U_k"], layer["U_v"], device=DEV)
+    for f in ("route_mask", "full_idx", "full_k", "full_v", "full_cnt", "seq_len"):
+        getattr(cache, f).copy_(getattr(bf, f))
+    pack = (lambda a: a.view(np.uint8)) if bits == 8 else O.pack_int4
+    cache.coef_k.copy_(torch.from_numpy(np.ascontiguousarray(pack(ocd["qk"]))))
+    cache.coef_v.copy_(torch.from_numpy(np.ascontiguousarray(pack(ocd["qv"]))))
+    cache.scale_k.copy_(torch.from_numpy(ocd["sk"]))
+    cache.scale_v.copy_(torch.from_numpy(ocd["sv"]))
+    ws = L.make_workspace(D, DEV)
+    # queries that weight the sequence's three parts alike: mostly the
+    # full-rank rows and the 2^20-scaled part matter, yet the first part's
+    # tiles (scale 2^-40) come first for most warps
+    out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
+    ref = O.decode_attn_quant(oc, ocd, U.f64(layer["q"]))
+    assert np.isfinite(out).all()
+    assert U.out_rel_err(out, ref) <= U.OUT_RTOL
