@@ -188,15 +188,29 @@ __host__ __device__ inline int decode_split(int T, int n_max_grid, long long BH,
   int n_max = (int)((uT + kMinDecodeChunk - 1) / kMinDecodeChunk);
   if (n_max > n_max_grid) n_max = n_max_grid;
   if (n_max < n_min) n_max = n_min;
+  // The model only ranks candidates (the chunk itself is computed exactly
+  // below), so on the device its quotients use the fast approximate divide
+  // (relative error ~2.4e-7): every CTA runs this on its critical path, and
+  // 21 IEEE divisions in a chain took ~1 us there.  Floor and ceil take the
+  // quotient nudged by 1e-6 of itself, which keeps exact integers where the
+  // exact model puts them (the smallest relative gap to an integer here is
+  // above 1e-6 for T below a million positions).
+#ifdef __CUDA_ARCH__
+  auto q = [](float a, float b) { return __fdividef(a, b); };
+#else
+  auto q = [](float a, float b) { return a / b; };
+#endif
+  auto fl = [](float x) { return floorf(x * (1.f + 1e-6f)); };
+  auto ce = [](float x) { return ceilf(x * (1.f - 1e-6f)); };
   const float fbh = (float)BH, fsm = (float)sms, ft = (float)T;
-  const float w0 = ceilf(fbh * (float)n_min / fsm);   // waves at n_min
+  const float w0 = ce(q(fbh * (float)n_min, fsm));   // waves at n_min
   float best_cost = -1.f;
   int best_n = n_min;
   for (int k = 0; k <= 4; ++k) {
-    float nf = k < 4 ? floorf((w0 + (float)k) * fsm / fbh) : (float)n_max;
+    float nf = k < 4 ? fl(q((w0 + (float)k) * fsm, fbh)) : (float)n_max;
     nf = fminf(fmaxf(nf, (float)n_min), (float)n_max);
-    const float ch = ceilf(ft / (32.f * nf)) * 32.f;
-    const float waves = ceilf(fbh * ceilf(ft / ch) / fsm);
+    const float ch = ce(q(ft, 32.f * nf)) * 32.f;
+    const float waves = ce(q(fbh * ce(q(ft, ch)), fsm));
     const float cost = waves * (ch + (float)kDecodeOverhead);
     if (best_cost < 0.f || cost < best_cost) best_cost = cost, best_n = (int)nf;
   }
