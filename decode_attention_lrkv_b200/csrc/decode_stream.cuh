@@ -309,6 +309,9 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   constexpr int kWarps = S::kWarps, kThreads = S::kThreads;
   constexpr int KST = RK / 16;                   // k-steps of the compressed logits
   constexpr int MVT = RV / 16;                   // m-tiles of the compressed value sum
+  // int4 value rows that are whole 16-byte pieces (r_v a multiple of 32) are
+  // read with transposing ldmatrix (value columns in the order noted there)
+  constexpr bool kInt4Ldsm = CB == 4 && RV % 32 == 0;
   constexpr int KP = S::KP, VP = S::VP;          // 16-byte pieces per stored row
   constexpr int UKP = S::UKP, UVP = S::UVP;      // 16-byte pieces per basis row
   constexpr int NST = S::STAGES;
@@ -812,6 +815,13 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
           // columns 2g, 2g+1 of a 16-column block (accumulator rows g, g + 8).
           const float* scl = reinterpret_cast<const float*>(slot + S::T_SC);   // [2][32]
           const uint32_t k136 = 0xC308C308u, k1 = 0x3F803F80u;                 // bf16x2 (-136, -136), (1, 1)
+          // nibble i (bits 4i..4i+3) of both 16-bit halves of u (sign bits
+          // already flipped) -> bf16x2 of the two codes
+          auto nib_col = [&](uint32_t u, int i) {
+            uint32_t x = ((u >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+            asm("fma.rn.bf16x2 %0, %0, %1, %2;" : "+r"(x) : "r"(k1), "r"(k136));
+            return x;
+          };
           auto nib_pairs = [&](uint32_t x16, uint32_t& lo01, uint32_t& lo23) {
             // x16: four nibbles (codes c0..c3 from the low end) -> bf16x2 (c0, c1), (c2, c3)
             const uint32_t u = x16 ^ 0x8888u;
@@ -847,6 +857,28 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
           uint32_t pb0[2], pb1[2];
           softmax_pack_w(s, pb0, pb1, std::integral_constant<int, 2>{}, wv, std::false_type{});
           const unsigned char* vrows = slot + kTileC * S::TKS;
+          if constexpr (kInt4Ldsm) {
+            // value rows of 16-byte multiples: one transposing ldmatrix per 32
+            // value columns (16 bytes of 8 token rows per matrix; matrices =
+            // tokens 0-7, 8-15, 16-23, 24-31) gives thread (g, t) the 16-bit
+            // element g (columns 4g..4g+3, one nibble each) of tokens 2t, 2t+1.
+            // Accumulator block 2 qc + sb: row g is value column 32 qc + 4g + 2 sb,
+            // row g + 8 the next one; nibble 2 sb (2 sb + 1) of both tokens makes a
+            // bf16 pair through 0x4300 | u and one packed fma.
+  #pragma unroll
+            for (int qc = 0; qc < RV / 32; ++qc) {
+              uint32_t r[4];
+              ldsm_x4_t(r[0], r[1], r[2], r[3], vrows + (8 * lm + lr) * S::TVS + qc * 16);
+  #pragma unroll
+              for (int nb = 0; nb < 2; ++nb) {
+                const uint32_t lo = r[2 * nb] ^ 0x88888888u, hi = r[2 * nb + 1] ^ 0x88888888u;
+  #pragma unroll
+                for (int sb = 0; sb < 2; ++sb)
+                  mma_16816(oc[2 * qc + sb], nib_col(lo, 2 * sb), nib_col(lo, 2 * sb + 1), nib_col(hi, 2 * sb),
+                            nib_col(hi, 2 * sb + 1), pb0[nb], pb1[nb]);
+              }
+            }
+          } else {
   #pragma unroll
           for (int mt = 0; mt < MVT; ++mt)
   #pragma unroll
@@ -865,6 +897,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
               a3 = __byte_perm(e, o, 0x7632);
               mma_16816(oc[mt], a0, a1, a2, a3, pb0[nb], pb1[nb]);
             }
+          }
         } else {
           // int8 codes, converted in registers (exact): to f16 for the logits
           // (against q~'s f16 high and low parts), to bf16 for the value sums.
@@ -1008,6 +1041,20 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
           uint32_t a0, a1, a2, a3;
           if constexpr (CB == 16) {
             ldsm_x4(a0, a1, a2, a3, uv + (16 * mi + (lm & 1) * 8 + lr) * S::VS + (mt * 16 + (lm >> 1) * 8) * 2);
+          } else if constexpr (kInt4Ldsm) {
+            // block mt = 2 qc + sb: accumulator row k < 8 is value column 32 qc +
+            // 4k + 2 sb, row k >= 8 the one after 32 qc + 4(k - 8) + 2 sb; a
+            // thread's k = 2t, 2t+1 are columns 8t + 2 sb, 8t + 4 + 2 sb of the
+            // 32 and k = 2t+8, 2t+9 the next ones: columns 8t..8t+7 in one load
+            const int qc = mt >> 1, sb = mt & 1;
+            const uint4 w0 = *reinterpret_cast<const uint4*>(uv + (16 * mi + g) * S::VS + (32 * qc + 8 * t) * 2);
+            const uint4 w1 = *reinterpret_cast<const uint4*>(uv + (16 * mi + g + 8) * S::VS + (32 * qc + 8 * t) * 2);
+            const uint32_t p0 = sb ? w0.y : w0.x, q0 = sb ? w0.w : w0.z;
+            const uint32_t p1 = sb ? w1.y : w1.x, q1 = sb ? w1.w : w1.z;
+            a0 = __byte_perm(p0, q0, 0x5410);
+            a2 = __byte_perm(p0, q0, 0x7632);
+            a1 = __byte_perm(p1, q1, 0x5410);
+            a3 = __byte_perm(p1, q1, 0x7632);
           } else {
             // accumulator row k of the block is value column 2k (k < 8) or
             // 2(k - 8) + 1: A[i][k] = U_v[i][that column], so a thread's k = 2t,
