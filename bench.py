@@ -568,9 +568,10 @@ def _event_time_ms(fn, reps, warm=3):
 def side_measurements(L, w, dims, layers, dev, pk):
     """Timings of the calls the step does not use, on this workload's geometry:
     the online basis update (one Oja batch step of every kv head's key basis
-    over 4096 rows) and the CUDA-core decode kernel, which serves query groups
-    the streaming kernel has no instantiation for (GQA 3 and 8 on layer 0's
-    cache; the cache does not depend on the query heads)."""
+    over 4096 rows) and the decode with other query groups on layer 0's cache
+    (the cache does not depend on the query heads): GQA 3 (one launch of the
+    streaming kernel, 4 heads with one idle) and GQA 8 (two launches of 4
+    heads, each streaming the cache)."""
     out = {}
     g = torch.Generator(device=dev).manual_seed(99)
     n_rows = 4096
@@ -595,10 +596,10 @@ def side_measurements(L, w, dims, layers, dev, pk):
         fc = lay["cache"].full_cnt.cpu().numpy()
         nb = A.decode_bytes(Dg.B, Dg.Hq, Dg.Hkv, Dg.d, Dg.r_k, Dg.r_v, lay["cache"].seq_len.cpu().tolist(), fc,
                             coef_bits=dims.bits)
-        fb[f"gqa{gg}"] = {"us_per_launch": round(ms * 1e3, 2), "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+        fb[f"gqa{gg}"] = {"us_per_call": round(ms * 1e3, 2), "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
                           "frac_of_measured_hbm": round(nb / (ms * 1e-3) / 1e9 / pk.get("hbm_gbs", 6549.1), 4)}
         del wsg
-    out["cuda_core_decode"] = fb
+    out["gqa_decode"] = fb
     return out
 
 

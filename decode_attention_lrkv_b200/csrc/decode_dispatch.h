@@ -10,12 +10,15 @@
 
 namespace lrkv {
 
-// Whether the streaming (tensor-core) kernel covers these sizes.
+// Whether the streaming (tensor-core) kernel covers these sizes: the rank
+// pairs it is instantiated for, any number of query heads per kv head.
 bool stream_decode_supported(const lrkv_dims& D);
 
-// The tensor-core streaming kernel for the shapes it is instantiated for, the
-// CUDA-core kernel for every other valid shape.  p.k_new set: the fused
-// append + decode, which only the streaming kernel has.
+// The tensor-core streaming kernel for the shapes it is instantiated for (1
+// or 2 query heads per kv head in one launch, more in launches of 4 heads,
+// each streaming the cache), the CUDA-core kernel for every other valid
+// shape.  p.k_new set: the fused append + decode, which only the streaming
+// kernel has (its first launch appends).
 lrkv_status launch_decode(const DecodeParams& p, cudaStream_t s);
 
 // Per query-group launchers of the streaming kernel (*done = false: no

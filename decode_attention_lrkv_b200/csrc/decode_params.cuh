@@ -14,6 +14,10 @@ struct DecodeParams {
   int32_t* tickets;   // [B][Hkv]
   float* partials;    // [B][Hkv][n_chunk_max][g][2 + r_v + d]
   int n_chunk_max;    // splits per (b, kv head) in the grid (those of a full cache)
+  // query heads per kv head (Hq / Hkv), and the first of this launch's: the
+  // streaming kernel serves up to its template's G of them per launch
+  int g_all;
+  int g_off;
   int num_sms;        // SMs of the device: each CTA sizes its split from the live length
   // fused decode-time append (lrkv_append_decode_attn); k_new null: plain decode
   const lrkv_bf16* k_new;   // [B][1][Hkv][d]

@@ -20,26 +20,42 @@ lrkv_status launch_simple_any(const DecodeParams& p, dim3 grid, cudaStream_t s) 
 }
 
 bool stream_decode_supported(const lrkv_dims& D) {
-  const int g = D.Hq / D.Hkv;
-  if (g != 1 && g != 2 && g != 4) return false;
+  if (D.Hkv < 1 || D.Hq < D.Hkv) return false;
   const int rk = D.r_k, rv = D.r_v;
   return (rk == 32 && rv == 32) || (rk == 48 && rv == 64) || (rk == 48 && rv == 80) ||
          (rk == 64 && rv == 64) || (rk == 64 && rv == 96);
 }
 
-lrkv_status launch_decode(const DecodeParams& p, cudaStream_t s) {
-  const dim3 grid(p.n_chunk_max, p.D.Hkv, p.D.B);
-  const int g = p.D.Hq / p.D.Hkv;
-  if (stream_decode_supported(p.D)) {
-    bool done = false;
-    lrkv_status st = LRKV_OK;
-    if (g == 1) st = launch_stream_g1(p, grid, s, &done);
-    else if (g == 2) st = launch_stream_g2(p, grid, s, &done);
-    else st = launch_stream_g4(p, grid, s, &done);
-    if (done) return st;
+// Query heads per launch of the streaming kernel: 1 or 2 as they are, else
+// passes of 4 (the last one partly empty), each streaming the cache once.
+int stream_heads_per_pass(int g) { return g <= 2 ? g : 4; }
+
+lrkv_status launch_decode(const DecodeParams& p0, cudaStream_t s) {
+  const dim3 grid(p0.n_chunk_max, p0.D.Hkv, p0.D.B);
+  const int g = p0.D.Hq / p0.D.Hkv;
+  if (stream_decode_supported(p0.D)) {
+    DecodeParams p = p0;
+    p.g_all = g;
+    const int per = stream_heads_per_pass(g);
+    for (int off = 0; off < g; off += per) {
+      p.g_off = off;
+      if (off > 0) {   // a fused append happens once, in the first pass; later passes read its result
+        p.k_new = p.v_new = nullptr;
+        p.t_new_b = nullptr;
+        p.err_out = nullptr;
+      }
+      bool done = false;
+      lrkv_status st = LRKV_OK;
+      if (per == 1) st = launch_stream_g1(p, grid, s, &done);
+      else if (per == 2) st = launch_stream_g2(p, grid, s, &done);
+      else st = launch_stream_g4(p, grid, s, &done);
+      if (st != LRKV_OK) return st;
+      if (!done) return LRKV_ERR_UNSUPPORTED;   // not reached: the rank pairs above are instantiated
+    }
+    return LRKV_OK;
   }
-  if (p.k_new) return LRKV_ERR_UNSUPPORTED;
-  return launch_simple_any(p, grid, s);
+  if (p0.k_new) return LRKV_ERR_UNSUPPORTED;
+  return launch_simple_any(p0, grid, s);
 }
 
 }  // namespace lrkv

@@ -287,10 +287,11 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
     if (p.err_out) p.err_out[bh] = e;
     *s_keep = keep;
   }
-  if (warp < G) {   // the token's logit for query head `warp`, base 2
+  if (warp < G && warp < p.g_all - p.g_off) {   // the token's logit for query head `warp`, base 2
     float sd = 0.f;
     if (keep) {     // full rank: q . k / sqrt(d)
-      const uint16_t* qrow = reinterpret_cast<const uint16_t*>(p.q) + ((size_t)b * D.Hq + (size_t)h * G + warp) * kD;
+      const uint16_t* qrow = reinterpret_cast<const uint16_t*>(p.q) +
+                             ((size_t)b * D.Hq + (size_t)h * p.g_all + p.g_off + warp) * kD;
       for (int i = lane; i < kD; i += 32) sd = fmaf(bf2f(qrow[i]), app[S::A_X + i], sd);
       sd = warp_sum(sd) * scale;
     } else {        // compressed: q . mu_k + q~ . c_k as stored, both already scaled
@@ -298,6 +299,8 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
       sd = warp_sum(sd) + s_bias[warp];
     }
     if (lane == 0) s_new[warp] = sd;
+  } else if (warp < G && lane == 0) {
+    s_new[warp] = -INFINITY;   // no such query head in this pass
   }
   if (tid < kD) s_vals[tid] = keep ? app[S::A_X + kD + tid] : (tid < RV ? app[S::A_CV + tid] : 0.f);
 }
@@ -323,7 +326,11 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   // N columns of the token-side MMAs: column 2h = bf16 high part of query head
   // h, column 2h + 1 = its low part.  A lane's accumulator fragment (columns
   // 2t, 2t + 1) therefore holds both parts of head t: one head per lane.
-  const bool live_t = t < G;                     // this lane's head exists
+  // query heads of this pass: q_head(x) is the x-th of the kv head's group;
+  // heads x >= g_live of the template's G do not exist in this pass
+  const int g_live = min(G, p.g_all - p.g_off);
+  auto q_head = [&](int x) { return (size_t)b * D.Hq + (size_t)h * p.g_all + p.g_off + x; };
+  const bool live_t = t < g_live;                // this lane's head exists
   const int lm = lane >> 3, lr = lane & 7;       // ldmatrix address roles
   const size_t bh = (size_t)b * D.Hkv + h;
 
@@ -366,8 +373,8 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   uint32_t qf0[8], qf1[8];
   {
     const int hq = g >> 1;                                    // B column g: head g / 2
-    const bool on = (g & 1) == 0 && hq < G;
-    const lrkv_bf16* qrow = p.q + ((size_t)b * D.Hq + (size_t)h * G + (hq < G ? hq : 0)) * kD;
+    const bool on = (g & 1) == 0 && hq < g_live;
+    const lrkv_bf16* qrow = p.q + q_head(hq < g_live ? hq : 0) * kD;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       qf0[ks] = on ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
@@ -376,11 +383,11 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   }
   uint32_t qa0[8], qa1[8];   // q as the A operand: row m = head m < G
   {
-    const lrkv_bf16* qrow = p.q + ((size_t)b * D.Hq + (size_t)h * G + (g < G ? g : 0)) * kD;
+    const lrkv_bf16* qrow = p.q + q_head(g < g_live ? g : 0) * kD;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      qa0[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
-      qa1[ks] = g < G ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
+      qa0[ks] = g < g_live ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * t) : 0u;
+      qa1[ks] = g < g_live ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * t) : 0u;
     }
   }
   // fused append: does row b have a new token; one element of its new key
@@ -591,7 +598,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       y0 = from_a1 ? qb0_ : pb0, y1 = from_a1 ? qb1_ : pb1;
     }
     const bool lo_n = g & 1;
-    const bool live = (g >> 1) < G;
+    const bool live = (g >> 1) < g_live;
     if constexpr (CB == 8) {
       // int8 codes meet q~ as f16 (high and low parts): a code widens to f16
       // in half the instructions it takes to reach bf16
@@ -608,8 +615,8 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   if (warp >= kWarps - G) {
     const int gi = warp - (kWarps - G);
     float sb = 0.f;
-    if (p.C.mu_k) {
-      const lrkv_bf16* qrow = p.q + ((size_t)b * D.Hq + (size_t)h * G + gi) * kD;
+    if (p.C.mu_k && gi < g_live) {
+      const lrkv_bf16* qrow = p.q + q_head(gi) * kD;
       for (int i = lane; i < kD; i += 32) sb = fmaf(bf2f(qrow[i]), p.C.mu_k[(size_t)h * kD + i], sb);
     }
     sb = warp_sum(sb);
@@ -1180,8 +1187,8 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       for (int k0 = 0; k0 < n_rec; k0 += 32) batch(k0, M);
     }
     Lsum = warp_sum(Lsum);
-    if (on) {
-      float* out = p.out + ((size_t)b * D.Hq + (size_t)h * G + gi) * kD + col;
+    if (on && gi < g_live) {
+      float* out = p.out + q_head(gi) * kD + col;
 #pragma unroll
       for (int u = 0; u < CPL; ++u) out[u] = Lsum > 0.f ? acc[u] / Lsum : 0.f;
     }

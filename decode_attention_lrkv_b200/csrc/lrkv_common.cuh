@@ -245,7 +245,10 @@ inline WsLayout ws_layout(const lrkv_dims& D) {
   if (L.n_chunk_max < 2) L.n_chunk_max = 2;
   L.partial_floats = 4 + D.r_v + D.d;   // m, l, pad, pad, acc_c[r_v], acc_f[d]
   L.partials = off;
+  // records per split: the query heads of a launch (the CUDA-core kernel
+  // takes all g at once, the streaming kernel passes of up to 4)
   int g = D.Hkv > 0 ? D.Hq / D.Hkv : 0;
+  if (g > 2 && g < 4) g = 4;
   off = align_up(off + sizeof(float) * (size_t)D.B * D.Hkv * L.n_chunk_max * g *
                            L.partial_floats, 256);
   L.total = off;

@@ -205,10 +205,12 @@ LRKV_API lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* c
  * issued back to back on `stream` (append-then-attend: the new token is
  * attended).  k_new, v_new: [B][1][Hkv][d] bf16; t_new_b: nullable device [B]
  * int32, each 0 or 1 (a row with 0 only attends); err_out: nullable device
- * [B][Hkv][1] fp32.  The append is done inside the decode kernel by the CTA
- * that holds the new position; the list length and seq_len are advanced on
- * the device once every CTA has read them.  Shapes the streaming decode kernel
- * does not cover run the two calls above instead (two launches).
+ * [B][Hkv][1] fp32.  The append is done inside the decode kernel by one extra
+ * CTA per (batch row, kv head); the list length and seq_len are advanced on
+ * the device once every CTA has read them.  With more than 4 query heads per
+ * kv head (or 3) the streaming kernel runs in launches of 4 heads, the first
+ * of which appends.  Rank pairs the streaming kernel has no instantiation for
+ * run the two calls above instead (two launches).
  * Arguments, layouts and errors otherwise as lrkv_compress / lrkv_decode_attn.
  */
 LRKV_API lrkv_status lrkv_append_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache,

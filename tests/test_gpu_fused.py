@@ -150,12 +150,17 @@ def test_fused_on_an_empty_cache():
                                  band=band)
 
 
-def test_fused_shape_without_streaming_kernel():
-    """g = 3 has no streaming kernel: the call runs the two launches it fuses."""
-    w = synth.workload(1, T=300, layers=1)
+@pytest.mark.parametrize("Hq,r_k,r_v", [(6, 32, 48), (6, 64, 96), (16, 64, 96), (10, 48, 64)],
+                         ids=["g3_no_streaming_kernel", "g3_one_launch", "g8_two_launches", "g5_two_launches"])
+def test_fused_other_group_sizes(Hq, r_k, r_v):
+    """Groups of 3, 5 and 8 query heads per kv head: the streaming kernel runs
+    the fused step in launches of 4 heads, the first of which appends (later
+    launches read the appended token); a rank pair it has no instantiation for
+    (32/48) runs the two launches the call fuses."""
+    w = synth.workload(1, T=300, layers=1, r_k=r_k, r_v=r_v)
     layer = synth.make_layer(w, 0, 47, device=DEV)
-    Hkv, Hq = 2, 6
-    D = L.Dims(B=1, Hq=Hq, Hkv=Hkv, d=128, r_k=64, r_v=96, T_cap=320, F_cap=320)
+    Hkv = 2
+    D = L.Dims(B=1, Hq=Hq, Hkv=Hkv, d=128, r_k=r_k, r_v=r_v, T_cap=320, F_cap=320)
     U_k, U_v = layer["U_k"][:Hkv].contiguous(), layer["U_v"][:Hkv].contiguous()
     cache = L.LayerCache(D, U_k, U_v, device=DEV)
     oc = O.Cache.empty(U.oracle_dims(D), U.f64(U_k), U.f64(U_v))

@@ -230,11 +230,15 @@ def test_prefill_in_two_parts_unaligned_start():
 
 
 @pytest.mark.parametrize("Hq,Hkv,r_k,r_v", [(16, 8, 48, 80), (4, 2, 64, 64), (6, 2, 48, 64),
-                                            (16, 2, 32, 32), (8, 8, 32, 48)],
-                         ids=["g2_48_80", "g2_64_64", "g3_simple", "g8_simple", "g1_rank_pair_simple"])
+                                            (16, 2, 32, 32), (20, 4, 64, 96), (8, 8, 32, 48),
+                                            (6, 2, 32, 48), (16, 2, 32, 48)],
+                         ids=["g2_48_80", "g2_64_64", "g3_stream", "g8_stream_two_passes",
+                              "g5_stream_two_passes", "g1_rank_pair_simple", "g3_simple", "g8_simple"])
 def test_group_sizes_and_rank_pairs(Hq, Hkv, r_k, r_v):
-    """GQA groups of 1, 2, 3 and 8 query heads and a rank pair outside the
-    streaming kernel's instantiations (served by the CUDA-core kernel)."""
+    """GQA groups of 1, 2, 3, 5 and 8 query heads: the streaming kernel takes
+    any group in launches of up to 4 heads (3: one launch with an idle head;
+    5, 8: two launches); a rank pair outside its instantiations (32/48) goes to
+    the CUDA-core kernel, at groups of 1, 3 and 8."""
     w = synth.workload(1, Hq=Hq, Hkv=Hkv, r_k=r_k, r_v=r_v, T=900, layers=1)
     layer, D, cache, oc, ws = _setup(w, seed=13)
     gc, band = _compress_both(D, cache, oc, layer["K"], layer["V"], w.tau, ws)
@@ -249,8 +253,8 @@ def test_group_sizes_and_rank_pairs(Hq, Hkv, r_k, r_v):
 def test_capacity_far_above_the_live_length(Hq, Hkv, r_k, r_v):
     """A cache allocated for 16384 positions that holds 600: the decode splits
     follow the live length (the grid is sized for the capacity), with the
-    streaming kernel (GQA 4, MHA) and the CUDA-core kernel (GQA 3); then a
-    fused append + decode step on the same cache."""
+    streaming kernel at GQA 4, MHA and GQA 3 (a launch of 4 heads, one idle);
+    then a fused append + decode step on the same cache."""
     w = synth.workload(1, Hq=Hq, Hkv=Hkv, r_k=r_k, r_v=r_v, T=600, layers=1)
     layer, D, cache, oc, ws = _setup(w, seed=19, T_cap=16384, F_cap=4096)
     gc, band = _compress_both(D, cache, oc, layer["K"], layer["V"], w.tau, ws)
