@@ -159,73 +159,126 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
   // c = U^T (x - mu) on the tensor cores: x (bf16, exact) is row 8 of the A
   // operand; a key mean (fp32) enters as its bf16 high and low parts in rows 9
   // and 10, so U^T mu is fp32-accurate and c = row 8 - (row 9 + row 10).  Warp
-  // w forms columns [16w, 16w + 16) of c_k (w < r_k / 16) and of c_v (w < r_v / 16).
-  auto coef_block = [&](const unsigned char* U, int stride, const float* x, const float* mu,
-                        float* cdst) {
-    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+  // w forms columns [16w, 16w + 16) of c_k (w < r_k / 16) and of c_v (w < r_v / 16),
+  // the two products interleaved and the even and odd k-steps in separate
+  // accumulators (short chains of dependent MMAs).
+  const float* mu_h = p.C.mu_k ? p.C.mu_k + (size_t)h * kD : nullptr;
+  {
+    const bool do_k = warp < KST, do_v = warp < MVT;
+    float ak[2][2][4], av[2][2][4];   // [k-step parity][column half][fragment]
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ak[q][u][e] = av[q][u][e] = 0.f;
+    const float* xk = app + S::A_X;
+    const float* xv = app + S::A_X + kD;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       const int i0 = ks * 16 + 2 * t, i1 = i0 + 8;
-      uint32_t x0 = 0u, x1 = 0u;
-      if (g == 0) {
-        x0 = pack_bf16(x[i0], x[i0 + 1]);
-        x1 = pack_bf16(x[i1], x[i1 + 1]);
-      } else if (mu && g <= 2) {
-        const bool lo = g == 2;
-        x0 = pack_bf16(bf16_part(mu[i0], lo), bf16_part(mu[i0 + 1], lo));
-        x1 = pack_bf16(bf16_part(mu[i1], lo), bf16_part(mu[i1 + 1], lo));
+      if (do_k) {
+        uint32_t x0 = 0u, x1 = 0u;
+        if (g == 0) {
+          x0 = pack_bf16(xk[i0], xk[i0 + 1]);
+          x1 = pack_bf16(xk[i1], xk[i1 + 1]);
+        } else if (mu_h && g <= 2) {
+          const bool lo = g == 2;
+          x0 = pack_bf16(bf16_part(mu_h[i0], lo), bf16_part(mu_h[i0 + 1], lo));
+          x1 = pack_bf16(bf16_part(mu_h[i1], lo), bf16_part(mu_h[i1 + 1], lo));
+        }
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(b0, b1, b2, b3, uk + (ks * 16 + (lm & 1) * 8 + lr) * S::KS + (16 * warp + (lm >> 1) * 8) * 2);
+        mma_16816(ak[ks & 1][0], 0u, x0, 0u, x1, b0, b1);
+        mma_16816(ak[ks & 1][1], 0u, x0, 0u, x1, b2, b3);
       }
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(b0, b1, b2, b3, U + (ks * 16 + (lm & 1) * 8 + lr) * stride + (16 * warp + (lm >> 1) * 8) * 2);
-      mma_16816(a0, 0u, x0, 0u, x1, b0, b1);
-      mma_16816(a1, 0u, x0, 0u, x1, b2, b3);
+      if (do_v) {
+        const uint32_t x0 = g == 0 ? pack_bf16(xv[i0], xv[i0 + 1]) : 0u;
+        const uint32_t x1 = g == 0 ? pack_bf16(xv[i1], xv[i1 + 1]) : 0u;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(b0, b1, b2, b3, uv + (ks * 16 + (lm & 1) * 8 + lr) * S::VS + (16 * warp + (lm >> 1) * 8) * 2);
+        mma_16816(av[ks & 1][0], 0u, x0, 0u, x1, b0, b1);
+        mma_16816(av[ks & 1][1], 0u, x0, 0u, x1, b2, b3);
+      }
     }
-    float m[4] = {0.f, 0.f, 0.f, 0.f};   // U^T mu: rows 9 and 10, from lanes 4 + t and 8 + t
-    if (mu) {
-      const float v[4] = {a0[2], a0[3], a1[2], a1[3]};
+    if (do_k) {
+      float m[4] = {0.f, 0.f, 0.f, 0.f};   // U^T mu: rows 9 and 10, from lanes 4 + t and 8 + t
+      const float v[4] = {ak[0][0][2] + ak[1][0][2], ak[0][0][3] + ak[1][0][3],
+                          ak[0][1][2] + ak[1][1][2], ak[0][1][3] + ak[1][1][3]};
+      if (mu_h) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        m[e] = __shfl_sync(kFull, v[e], (lane + 4) & 31) + __shfl_sync(kFull, v[e], (lane + 8) & 31);
+        for (int e = 0; e < 4; ++e)
+          m[e] = __shfl_sync(kFull, v[e], (lane + 4) & 31) + __shfl_sync(kFull, v[e], (lane + 8) & 31);
+      }
+      if (g == 0) {
+        float* cdst = app + S::A_CK;
+        cdst[16 * warp + 2 * t] = v[0] - m[0];
+        cdst[16 * warp + 2 * t + 1] = v[1] - m[1];
+        cdst[16 * warp + 8 + 2 * t] = v[2] - m[2];
+        cdst[16 * warp + 8 + 2 * t + 1] = v[3] - m[3];
+      }
     }
-    if (g == 0) {
-      cdst[16 * warp + 2 * t] = a0[2] - m[0];
-      cdst[16 * warp + 2 * t + 1] = a0[3] - m[1];
-      cdst[16 * warp + 8 + 2 * t] = a1[2] - m[2];
-      cdst[16 * warp + 8 + 2 * t + 1] = a1[3] - m[3];
+    if (do_v && g == 0) {
+      float* cdst = app + S::A_CV;
+      cdst[16 * warp + 2 * t] = av[0][0][2] + av[1][0][2];
+      cdst[16 * warp + 2 * t + 1] = av[0][0][3] + av[1][0][3];
+      cdst[16 * warp + 8 + 2 * t] = av[0][1][2] + av[1][1][2];
+      cdst[16 * warp + 8 + 2 * t + 1] = av[0][1][3] + av[1][1][3];
     }
-  };
-  const float* mu_h = p.C.mu_k ? p.C.mu_k + (size_t)h * kD : nullptr;
-  if (warp < KST) coef_block(uk, S::KS, app + S::A_X, mu_h, app + S::A_CK);
-  if (warp < MVT) coef_block(uv, S::VS, app + S::A_X + kD, nullptr, app + S::A_CV);
+  }
   __syncthreads();
   // direct reconstruction x_hat = U c on the tensor cores: A = U's rows
-  // [16w, 16w + 16) (warp w, keys then values), B = c split into bf16 high
-  // (column 0) and low (column 1) parts; lane (g, t = 0) gets x_hat of rows
-  // 16w + g and 16w + g + 8 as the sum of its two columns
-  auto recon_sq = [&](const unsigned char* U, int stride, int r, const float* cc, const float* x) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int ks = 0; ks < r / 16; ++ks) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(a0, a1, a2, a3, U + (16 * warp + (lm & 1) * 8 + lr) * stride + (ks * 16 + (lm >> 1) * 8) * 2);
-      const bool lo = g & 1;
-      const float* c2 = cc + ks * 16 + 2 * t;
-      const uint32_t b0 = g < 2 ? pack_bf16(bf16_part(c2[0], lo), bf16_part(c2[1], lo)) : 0u;
-      const uint32_t b1 = g < 2 ? pack_bf16(bf16_part(c2[8], lo), bf16_part(c2[9], lo)) : 0u;
-      mma_16816(acc, a0, a1, a2, a3, b0, b1);
-    }
-    float rr = 0.f;
-    if (t == 0) {
-      const float d0 = x[16 * warp + g] - (acc[0] + acc[1]);
-      const float d1 = x[16 * warp + g + 8] - (acc[2] + acc[3]);
-      rr = d0 * d0 + d1 * d1;
-    }
-    return warp_sum(rr);
-  };
+  // [16w, 16w + 16) (warp w), B = c split into bf16 high (column 0) and low
+  // (column 1) parts; lane (g, t = 0) gets x_hat of rows 16w + g and 16w + g + 8
+  // as the sum of its two columns.  Keys and values interleaved, even and odd
+  // k-steps in separate accumulators.
   {
-    const float rk = recon_sq(ukq, S::KS, RK, app + S::A_CK, app + S::A_XC);
-    const float rv = recon_sq(uv, S::VS, RV, app + S::A_CV, app + S::A_X + kD);
+    float rk_acc[2][4], rv_acc[2][4];
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) rk_acc[q][e] = rv_acc[q][e] = 0.f;
+    const bool lo = g & 1;
+    auto bfrag = [&](const float* c2, uint32_t& b0, uint32_t& b1) {
+      b0 = g < 2 ? pack_bf16(bf16_part(c2[0], lo), bf16_part(c2[1], lo)) : 0u;
+      b1 = g < 2 ? pack_bf16(bf16_part(c2[8], lo), bf16_part(c2[9], lo)) : 0u;
+    };
+    constexpr int KS_MAX = KST > MVT ? KST : MVT;
+#pragma unroll
+    for (int ks = 0; ks < KS_MAX; ++ks) {
+      if (ks < KST) {
+        uint32_t a0, a1, a2, a3, b0, b1;
+        ldsm_x4(a0, a1, a2, a3, ukq + (16 * warp + (lm & 1) * 8 + lr) * S::KS + (ks * 16 + (lm >> 1) * 8) * 2);
+        bfrag(app + S::A_CK + ks * 16 + 2 * t, b0, b1);
+        mma_16816(rk_acc[ks & 1], a0, a1, a2, a3, b0, b1);
+      }
+      if (ks < MVT) {
+        uint32_t a0, a1, a2, a3, b0, b1;
+        ldsm_x4(a0, a1, a2, a3, uv + (16 * warp + (lm & 1) * 8 + lr) * S::VS + (ks * 16 + (lm >> 1) * 8) * 2);
+        bfrag(app + S::A_CV + ks * 16 + 2 * t, b0, b1);
+        mma_16816(rv_acc[ks & 1], a0, a1, a2, a3, b0, b1);
+      }
+    }
+    float rk = 0.f, rv = 0.f;
+    if (t == 0) {
+      const float* xk = app + S::A_XC;
+      const float* xv = app + S::A_X + kD;
+      const float k0 = xk[16 * warp + g] - ((rk_acc[0][0] + rk_acc[1][0]) + (rk_acc[0][1] + rk_acc[1][1]));
+      const float k1 = xk[16 * warp + g + 8] - ((rk_acc[0][2] + rk_acc[1][2]) + (rk_acc[0][3] + rk_acc[1][3]));
+      const float v0 = xv[16 * warp + g] - ((rv_acc[0][0] + rv_acc[1][0]) + (rv_acc[0][1] + rv_acc[1][1]));
+      const float v1 = xv[16 * warp + g + 8] - ((rv_acc[0][2] + rv_acc[1][2]) + (rv_acc[0][3] + rv_acc[1][3]));
+      rk = k0 * k0 + k1 * k1;
+      rv = v0 * v0 + v1 * v1;
+    }
     const float x = app[S::A_X + tid];
-    const float ns = warp_sum(x * x);   // warps < 4: the key's squares, else the value's
+    float ns = x * x;   // warps < 4: the key's squares, else the value's
+    // the three warp sums together (independent shuffles)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      rk += __shfl_xor_sync(kFull, rk, o);
+      rv += __shfl_xor_sync(kFull, rv, o);
+      ns += __shfl_xor_sync(kFull, ns, o);
+    }
     if (lane == 0) {
       app[S::A_RED + warp] = rk;
       app[S::A_RED + 8 + warp] = rv;
@@ -302,7 +355,30 @@ __device__ __forceinline__ void append_token(const DecodeParams& p, float* app,
   } else if (warp < G && lane == 0) {
     s_new[warp] = -INFINITY;   // no such query head in this pass
   }
-  if (tid < kD) s_vals[tid] = keep ? app[S::A_X + kD + tid] : (tid < RV ? app[S::A_CV + tid] : 0.f);
+  // the token's value row in d-space: v itself when it went to the list, else
+  // U_v c_v as stored, on the tensor cores (warp w: rows [16w, 16w + 16), c_v
+  // as bf16 high and low parts in columns 0 and 1, even and odd k-steps apart)
+  if (keep) {
+    if (tid < kD) s_vals[tid] = app[S::A_X + kD + tid];
+  } else {
+    float acc[2][4];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
+    const bool lo = g & 1;
+#pragma unroll
+    for (int ks = 0; ks < MVT; ++ks) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(a0, a1, a2, a3, uv + (16 * warp + (lm & 1) * 8 + lr) * S::VS + (ks * 16 + (lm >> 1) * 8) * 2);
+      const float* c2 = app + S::A_CV + ks * 16 + 2 * t;
+      const uint32_t b0 = g < 2 ? pack_bf16(bf16_part(c2[0], lo), bf16_part(c2[1], lo)) : 0u;
+      const uint32_t b1 = g < 2 ? pack_bf16(bf16_part(c2[8], lo), bf16_part(c2[9], lo)) : 0u;
+      mma_16816(acc[ks & 1], a0, a1, a2, a3, b0, b1);
+    }
+    if (t == 0) {
+      s_vals[16 * warp + g] = (acc[0][0] + acc[1][0]) + (acc[0][1] + acc[1][1]);
+      s_vals[16 * warp + g + 8] = (acc[0][2] + acc[1][2]) + (acc[0][3] + acc[1][3]);
+    }
+  }
 }
 
 template <int G, int RK, int RV, int W, int NS, bool APP, int CB>
@@ -672,19 +748,9 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
       // value row in d-space (v, or U_v c_v as stored); an empty record
       // (m = -inf) when the row has no token
       float* recA = p.partials + (bh * p.n_chunk_max + n_chunks) * G * (size_t)S::REC;
-      const unsigned char* uv = sm + S::OFF_UV;
       for (int o = tid; o < G * kD; o += kThreads) {
         const int gi = o / kD, i = o - gi * kD;
-        float x = 0.f;
-        if (owner) {
-          if (s_keep) {
-            x = s_vals[i];
-          } else {
-            const lrkv_bf16* urow = reinterpret_cast<const lrkv_bf16*>(uv + i * S::VS);
-            for (int j = 0; j < RV; ++j) x = fmaf(bf2f(urow[j]), s_vals[j], x);
-          }
-        }
-        recA[gi * S::REC + 4 + i] = x;
+        recA[gi * S::REC + 4 + i] = owner ? s_vals[i] : 0.f;
       }
       if (tid < G) {
         recA[tid * S::REC] = owner ? s_new[tid] : -INFINITY;
@@ -782,16 +848,22 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
         const uint32_t bits = tile_bits(warp + kWarps * kw);
         float st[2][4];
         if constexpr (CB == 16) {
+          // even and odd k-steps into separate accumulators: shorter chains of
+          // dependent MMAs
+          float so[2][4];
   #pragma unroll
           for (int nb = 0; nb < 2; ++nb) {
             st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
+            so[nb][0] = so[nb][1] = so[nb][2] = so[nb][3] = 0.f;
   #pragma unroll
             for (int ks = 0; ks < KST; ++ks) {
               uint32_t a0, a1, a2, a3;
               ldsm_x4(a0, a1, a2, a3,
                       slot + (16 * nb + (lm & 1) * 8 + lr) * S::TKS + (ks * 16 + (lm >> 1) * 8) * 2);
-              mma_16816(st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
+              mma_16816(ks & 1 ? so[nb] : st[nb], a0, a1, a2, a3, qb0[ks], qb1[ks]);
             }
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) st[nb][e] += so[nb][e];
           }
           float s[2][2];
   #pragma unroll
@@ -913,9 +985,11 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
           // the order q~'s B fragments were built in; the row's key scale
           // multiplies the logit.
           const float* scl = reinterpret_cast<const float*>(slot + S::T_SC);   // [2][32]
+          float so8[2][4];
   #pragma unroll
           for (int nb = 0; nb < 2; ++nb) {
             st[nb][0] = st[nb][1] = st[nb][2] = st[nb][3] = 0.f;
+            so8[nb][0] = so8[nb][1] = so8[nb][2] = so8[nb][3] = 0.f;
             const unsigned char* rows = slot + (16 * nb + (lm & 1) * 8 + lr) * S::TKS;
   #pragma unroll
             for (int kp = 0; kp < KST; kp += 2) {
@@ -925,12 +999,14 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
               s8x4_f16pairs(r0, e0, f0);
               s8x4_f16pairs(r1, e1, f1);
               mma_16816_f16(st[nb], e0, e1, f0, f1, qb0[kp], qb1[kp]);
-              if (kp + 1 < KST) {
+              if (kp + 1 < KST) {   // odd k-steps in their own accumulator
                 s8x4_f16pairs(r2, e0, f0);
                 s8x4_f16pairs(r3, e1, f1);
-                mma_16816_f16(st[nb], e0, e1, f0, f1, qb0[kp + 1], qb1[kp + 1]);
+                mma_16816_f16(so8[nb], e0, e1, f0, f1, qb0[kp + 1], qb1[kp + 1]);
               }
             }
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) st[nb][e] += so8[nb][e];
           }
           float s[2][2], wv[2][2];
           float wmax = 0.f;   // the largest code scale of the tile's read rows
@@ -988,13 +1064,20 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
         // full-rank tile: 16 list rows
         const int k = warp + kWarps * kw;
         const int nrows = min(kTileF, n_full - k * kTileF);
-        float st[4] = {0.f, 0.f, 0.f, 0.f};
+        // the 8 k-steps into 4 accumulators: chains of 2 dependent MMAs, not 8
+        // (a dependent mma.sync waits for the previous one's result)
+        float sq[4][4];
+  #pragma unroll
+        for (int u = 0; u < 4; ++u) sq[u][0] = sq[u][1] = sq[u][2] = sq[u][3] = 0.f;
   #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           uint32_t a0, a1, a2, a3;
           ldsm_x4(a0, a1, a2, a3, slot + ((lm & 1) * 8 + lr) * S::FS + (ks * 16 + (lm >> 1) * 8) * 2);
-          mma_16816(st, a0, a1, a2, a3, qf0[ks], qf1[ks]);
+          mma_16816(sq[ks & 3], a0, a1, a2, a3, qf0[ks], qf1[ks]);
         }
+        float st[4];
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) st[e] = (sq[0][e] + sq[1][e]) + (sq[2][e] + sq[3][e]);
         float s[1][2];
   #pragma unroll
         for (int x = 0; x < 2; ++x) {   // rows g, g + 8 (the low-part column is 0 for q)
