@@ -147,11 +147,11 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
   rp.n_tiles = L.n_tiles;
   rp.bh_tickets = reinterpret_cast<int32_t*>(w + L.decode_tickets);
   rp.ticket = reinterpret_cast<int32_t*>(w + L.compress_ticket);
+  // the routing passes launch as dependents (programmatic dependent launch):
+  // their launch overlaps the preceding kernel's tail, and each waits for it
   const dim3 grid(pp.tiles_per_b, D.Hkv, D.B);
-  ptc::route_count_kernel<<<grid, 128, 0, s>>>(rp);
-  if ((st = launched()) != LRKV_OK) return st;
-  ptc::route_scatter_kernel<<<grid, 128, 0, s>>>(rp);
-  return launched();
+  if ((st = launch_pdl(ptc::route_count_kernel, grid, dim3(128), 0, s, rp)) != LRKV_OK) return st;
+  return launch_pdl(ptc::route_scatter_kernel, grid, dim3(128), 0, s, rp);
 }
 
 

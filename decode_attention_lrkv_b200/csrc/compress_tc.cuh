@@ -193,6 +193,8 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const lrkv_dims& D = p.D;
+  // the routing passes may launch now: they wait for this grid to finish
+  griddep_launch_dependents();
   const int n_units = D.B * p.tiles_per_b;
   int u_begin, u_end;
   const int group = cta_tiles(p, n_units, &u_begin, &u_end), tensor = group & 1, h = group >> 1;
@@ -622,6 +624,9 @@ __device__ __forceinline__ int route_eff(const RouteParams& p, int b, int* start
 
 // grid (tiles_per_b, Hkv, B), 128 threads
 __global__ void __launch_bounds__(128) route_count_kernel(RouteParams p) {
+  // launched as a dependent of the projection: nothing is read before it is done
+  griddep_wait();
+  griddep_launch_dependents();
   const lrkv_dims& D = p.D;
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -650,6 +655,7 @@ __global__ void __launch_bounds__(128) route_count_kernel(RouteParams p) {
 
 // grid (tiles_per_b, Hkv, B), 128 threads
 __global__ void __launch_bounds__(128) route_scatter_kernel(RouteParams p) {
+  griddep_wait();   // a dependent of the count pass
   const lrkv_dims& D = p.D;
   const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

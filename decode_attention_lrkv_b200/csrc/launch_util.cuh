@@ -24,6 +24,16 @@ inline bool set_smem(Kernel kern, size_t smem) {
   return true;
 }
 
+// An empty kernel, launched without programmatic dependent launch after a
+// call that writes bases: the decode kernels read the bases before waiting on
+// the preceding kernel of the stream, so that kernel must be one that writes
+// none of them.
+__global__ void stream_fence_kernel();
+inline lrkv_status launch_stream_fence(cudaStream_t s) {
+  stream_fence_kernel<<<1, 32, 0, s>>>();
+  return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+}
+
 template <typename Params>
 inline lrkv_status launch_pdl(void (*kern)(Params), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t s, const Params& p) {

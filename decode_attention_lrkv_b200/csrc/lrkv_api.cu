@@ -15,6 +15,10 @@
 #include "lrkv_common.cuh"
 #include "lrkv_host.cuh"
 
+namespace lrkv {
+__global__ void stream_fence_kernel() {}
+}  // namespace lrkv
+
 namespace {
 
 using namespace lrkv;
@@ -185,7 +189,8 @@ lrkv_status lrkv_fit_basis(const lrkv_dims* dims, const lrkv_bf16* X, int32_t n_
   const size_t esmem = fit::eig_smem_bytes();
   if (!set_smem(fit::eig_kernel, esmem)) return LRKV_ERR_CUDA;
   fit::eig_kernel<<<dims->Hkv, fit::kEigThreads, esmem, s>>>(ep);
-  return launched();
+  if ((st = launched()) != LRKV_OK) return st;
+  return launch_stream_fence(s);   // the bases are written: a decode may follow
 }
 
 lrkv_status lrkv_rank_for_budget(const float* eigvals, int32_t n_heads, int32_t d, double budget,

@@ -88,7 +88,8 @@ lrkv_status lrkv_oja_update(const lrkv_dims* dims, const lrkv_bf16* X, int32_t n
   const size_t smem = oja::finish_smem_bytes(r);
   if (!set_smem(oja::oja_finish_kernel, smem)) return LRKV_ERR_CUDA;
   oja::oja_finish_kernel<<<dims->Hkv, oja::kFinishThreads, smem, s>>>(fp);
-  return cudaGetLastError() == cudaSuccess ? LRKV_OK : LRKV_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return LRKV_ERR_CUDA;
+  return launch_stream_fence(s);   // the bases are written: a decode may follow
 }
 
 }  // extern "C"

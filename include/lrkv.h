@@ -237,7 +237,8 @@ LRKV_API lrkv_status lrkv_append_decode_attn(const lrkv_dims* dims, const lrkv_c
  * eigvals_out: nullable [Hkv][d] fp32, every eigenvalue of G_h, descending (the
  *           discarded mass of a rank-r basis is the sum past index r).
  * ws:       lrkv_fit_workspace_size(dims, n_rows) bytes (any contents).
- * Returns LRKV_OK when the work was enqueued (two kernels on `stream`).
+ * Returns LRKV_OK when the work was enqueued (two kernels on `stream`, then an
+ * empty one, so that a decode issued next finds the bases written).
  */
 LRKV_API size_t lrkv_fit_workspace_size(const lrkv_dims* dims, int32_t n_rows);
 LRKV_API lrkv_status lrkv_fit_basis(const lrkv_dims* dims, const lrkv_bf16* X, int32_t n_rows,
@@ -288,7 +289,9 @@ LRKV_API lrkv_status lrkv_rank_for_budget(const float* eigvals, int32_t n_heads,
  * ws:    lrkv_oja_workspace_size(dims, n_rows, r) bytes (any contents).
  * A cache keeps one basis per kv head: after an update, compressed rows stored
  * earlier are read with the new basis (the library does not rewrite them).
- * Returns LRKV_OK when the work was enqueued (two kernels on `stream`). */
+ * Returns LRKV_OK when the work was enqueued (two kernels on `stream`, then an
+ * empty one, so that a decode issued next, which reads the bases before
+ * waiting on the preceding kernel, finds them written). */
 LRKV_API size_t lrkv_oja_workspace_size(const lrkv_dims* dims, int32_t n_rows, int32_t r);
 LRKV_API lrkv_status lrkv_oja_update(const lrkv_dims* dims, const lrkv_bf16* X, int32_t n_rows,
                                      int32_t r, float eta, float* U, lrkv_bf16* U_out, void* ws,

@@ -79,3 +79,27 @@ def test_zero_step_keeps_the_basis():
     L.lrkv_oja_update(D, layer["K"], Ug, 0.0)
     torch.cuda.synchronize()
     assert (Ug - U0).abs().max().item() <= 1e-6
+
+
+def test_update_then_decode_reads_the_new_basis():
+    """An update that writes a cache's value basis in place (U_out = the
+    cache's U_v), then a decode issued right after it on the same stream: the
+    decode (which loads the bases before waiting on the preceding kernel)
+    attends with the updated basis.  Checked against the oracle's decode over
+    the same cache contents with that basis."""
+    w = synth.workload(1, T=700, layers=1)
+    layer = synth.make_layer(w, 0, 87, device=DEV)
+    D = U.dims_of(w, synth.pad_to(w.T, 32))
+    cache = L.LayerCache(D, layer["U_k"], layer["U_v"].clone(), device=DEV)
+    ws = L.make_workspace(D, DEV)
+    L.lrkv_compress(D, cache, layer["K"], layer["V"], w.tau, ws=ws)
+    Uf = layer["Qv"][:, :, :w.r_v].contiguous()          # fp32 orthonormal start
+    X = layer["V"][0, :256].contiguous()                  # [256, Hkv, d]
+    torch.cuda.synchronize()
+    L.lrkv_oja_update(D, X.unsqueeze(0), Uf, 0.5, U_out=cache.U_v)
+    out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
+    torch.cuda.synchronize()
+    gc = U.gpu_to_oracle(D, cache)                        # holds the updated U_v
+    assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
+    # the basis did change
+    assert (cache.U_v.float() - layer["U_v"].float()).abs().max().item() > 1e-3
