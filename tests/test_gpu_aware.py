@@ -89,7 +89,8 @@ def _compress_both(D, cache, oc, K, V, tau, ws, t_new_b=None, band=None):
 WORKLOADS = [
     ("llama8k_small", synth.workload(1, T=1000, layers=1)),
     ("mha_small", synth.workload(4, T=700, layers=1)),
-    ("gqa3_cuda_cores", synth.workload(1, Hq=24, T=600, layers=1)),
+    ("gqa3", synth.workload(1, Hq=24, T=600, layers=1)),
+    ("cuda_cores_32_48", synth.workload(1, r_k=32, r_v=48, T=600, layers=1)),
 ]
 
 

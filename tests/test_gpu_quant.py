@@ -98,7 +98,8 @@ WORKLOADS = [
     ("llama32k_small", synth.workload(2, T=900, layers=1)),
     ("ragged_small", synth.workload(3, B=3, T=600, ragged_min=250, layers=1)),
     ("tiny", synth.workload(0)),
-    ("gqa3_cuda_cores", synth.workload(1, Hq=24, T=500, layers=1)),
+    ("gqa3", synth.workload(1, Hq=24, T=500, layers=1)),
+    ("cuda_cores_32_48", synth.workload(1, r_k=32, r_v=48, T=500, layers=1)),
 ]
 
 

@@ -8,8 +8,9 @@ scratch from a device array the library holds instead of a workspace.  Its
 output must match lrkv_decode_attn's, within the parity tolerance, call
 after call: the shared array keeps the previous call's contents, so each
 call has to start from cleared tickets.  Shapes of both decode kernels are
-covered (the streaming kernel, GQA 4; the CUDA-core kernel, GQA 3), and one
-call is checked against the fp64 oracle as well.  This file is collected last.
+covered (the streaming kernel at GQA 4 and 3; the CUDA-core kernel, ranks
+32/48), and one call is checked against the fp64 oracle as well.  This file is
+collected last.
 """
 import ctypes
 
@@ -38,10 +39,11 @@ def _noalloc(lib, D, cache, q, out, stream):
                                         ctypes.c_void_p(stream.cuda_stream))
 
 
-@pytest.mark.parametrize("Hq", [32, 24], ids=["gqa4_streaming", "gqa3_cuda_cores"])
-def test_noalloc_matches_workspace_decode_on_consecutive_calls(Hq):
+@pytest.mark.parametrize("Hq,r_k,r_v", [(32, 64, 96), (24, 64, 96), (24, 32, 48)],
+                         ids=["gqa4_streaming", "gqa3_streaming", "gqa3_cuda_cores"])
+def test_noalloc_matches_workspace_decode_on_consecutive_calls(Hq, r_k, r_v):
     dev = torch.device("cuda", 0)
-    w = synth.workload(1, Hq=Hq, T=3000, layers=1)
+    w = synth.workload(1, Hq=Hq, r_k=r_k, r_v=r_v, T=3000, layers=1)
     lay = synth.make_layer(w, 0, 77, device=dev)
     D = L.Dims(B=w.B, Hq=w.Hq, Hkv=w.Hkv, d=w.d, r_k=w.r_k, r_v=w.r_v, T_cap=3008, F_cap=3008)
     cache = L.LayerCache(D, lay["U_k"], lay["U_v"], device=dev)
