@@ -451,7 +451,9 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
         // (c = U^T x - U^T mu with a key mean), 32 columns per wait: the row's
         // amax of bf16(c), then its codes and scale
         const size_t row = bh * D.T_cap + start + t;
-        float amax = 0.f;
+        // amax of the bf16 magnitudes, as a packed 16-bit unsigned max of their
+        // bit patterns (the order of non-negative bf16 values)
+        uint32_t am2 = 0u;
 #pragma unroll 1
         for (int c0 = 0; c0 < R; c0 += 32) {
           float v[2][16];
@@ -467,10 +469,10 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
                 const float m0 = mug ? cmu[(c0 + 16 * q + k) & (kD - 1)] : 0.f;
                 const float m1 = mug ? cmu[(c0 + 16 * q + k + 1) & (kD - 1)] : 0.f;
                 const uint32_t pr = cvt_bf16x2(v[q][k] - m0, v[q][k + 1] - m1);   // bf16 pair
-                amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(pr << 16)),
-                                         fabsf(__uint_as_float(pr & 0xffff0000u))));
+                am2 = __vmaxu2(am2, pr & 0x7fff7fffu);
               }
         }
+        const float amax = __uint_as_float(max(am2 & 0xffffu, am2 >> 16) << 16);
         const float qs = quant_scale(amax, CB);
         const float qinv = qs > 0.f ? 1.f / qs : 0.f;
         if (valid) scales[row] = qs;

@@ -79,34 +79,44 @@ __device__ __forceinline__ int quant_code_fast(float cb, float s, float inv, int
   return qv > Q ? Q : (qv < -Q ? -Q : qv);
 }
 
-// The codes of 16 values w (fp32, rounded to bf16 here) of a row with scale s
-// and inv = 1/s (any rounding), packed: 8-bit codes into cw[0..3] (byte k),
-// 4-bit codes into cw[0..1] (nibble k).  The same decisions as quant_code,
-// with plain ALU/FMA steps: the nearest integer (half to even) of t = bf16(w) *
-// inv comes from adding 1.5 * 2^23 (|t| < 2^22), and t is within 2^-15 of the
-// correctly rounded quotient bf16(w) / s (|t| <= 128), so only a t that close
-// to a half-integer redoes the correctly rounded division.
-// bw: the 16 values already rounded, as bf16 pairs (element 2i in the low half of bw[i]).
+// The codes of 16 values of a row with scale s and inv = 1/s (any rounding),
+// packed: 8-bit codes into cw[0..3] (byte k), 4-bit codes into cw[0..1]
+// (nibble k).  The same decisions as quant_code, with plain ALU/FMA steps:
+// rr = t + 1.5 * 2^23 for t = w * inv holds the nearest integer of t (half to
+// even) in its low mantissa bits, so the code's two's-complement byte (nibble)
+// is the low byte (nibble) of rr's bits; t is within 2^-15 of the correctly
+// rounded quotient w / s (|t| <= Q + 2^-16 since s is the row's amax / Q, so
+// no clamp is needed), and only a t that close to a half-integer redoes the
+// correctly rounded division.
+// bw: the 16 values, bf16, as pairs (element 2i in the low half of bw[i]).
 __device__ __forceinline__ void quant_pack16_bf(const uint32_t (&bw)[8], float s, float inv, int bits,
                                                 uint32_t (&cw)[4]) {
-  const int Q = bits == 8 ? 127 : 7;
-  cw[0] = cw[1] = cw[2] = cw[3] = 0u;
+  uint32_t r[16];
 #pragma unroll
-  for (int k = 0; k < 16; k += 2) {
+  for (int k = 0; k < 16; ++k) {
     const uint32_t pr = bw[k >> 1];
-    const float b[2] = {__uint_as_float(pr << 16), __uint_as_float(pr & 0xffff0000u)};
+    const float b = (k & 1) ? __uint_as_float(pr & 0xffff0000u) : __uint_as_float(pr << 16);
+    const float t = b * inv;
+    float rr = t + 12582912.f;
+    if (fabsf(t - (rr - 12582912.f)) >= 0.49996948f)   // within 2^-15 of a half-integer: rare
+      rr = __int_as_float(0x4B400000 + (s > 0.f ? __float2int_rn(__fdiv_rn(b, s)) : 0));
+    r[k] = __float_as_uint(rr);
+  }
+  if (bits == 8) {
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float t = b[e] * inv;
-      const float rr = t + 12582912.f;
-      int qi = __float_as_int(rr) - 0x4B400000;
-      if (fabsf(fabsf(t - (rr - 12582912.f)) - 0.5f) <= 3.0517578125e-05f || fabsf(t) > 128.f)
-        qi = s > 0.f ? __float2int_rn(__fdiv_rn(b[e], s)) : 0;   // rare
-      qi = qi > Q ? Q : (qi < -Q ? -Q : qi);
-      const int kk = k + e;
-      if (bits == 8) cw[kk >> 2] |= ((uint32_t)qi & 0xffu) << (8 * (kk & 3));
-      else cw[kk >> 3] |= ((uint32_t)qi & 0xfu) << (4 * (kk & 7));
+    for (int j = 0; j < 4; ++j)
+      cw[j] = __byte_perm(__byte_perm(r[4 * j], r[4 * j + 1], 0x0040), __byte_perm(r[4 * j + 2], r[4 * j + 3], 0x0040),
+                          0x5410);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {   // even codes' bytes, odd codes' bytes, then nibble pairs
+      const uint32_t ev = __byte_perm(__byte_perm(r[8 * j], r[8 * j + 2], 0x0040),
+                                      __byte_perm(r[8 * j + 4], r[8 * j + 6], 0x0040), 0x5410);
+      const uint32_t od = __byte_perm(__byte_perm(r[8 * j + 1], r[8 * j + 3], 0x0040),
+                                      __byte_perm(r[8 * j + 5], r[8 * j + 7], 0x0040), 0x5410);
+      cw[j] = (ev & 0x0f0f0f0fu) | ((od << 4) & 0xf0f0f0f0u);
     }
+    cw[2] = cw[3] = 0u;
   }
 }
 
