@@ -71,7 +71,7 @@ constexpr int kMaxRanges = 256;                      // tile ranges of the end-t
 // last input stage; the query-side key basis U_q of an attention-aware key
 // basis (P = I - U_q U^T) borrows the one before.
 struct Layout {
-  int x, phi, plo, ut, u, uq, bar, part, mu;
+  int x, phi, plo, ut, u, uq, bar, part, mu, amx;
   size_t bytes;
   __host__ __device__ Layout(int rm, int ns) {
     x = 0;
@@ -83,7 +83,8 @@ struct Layout {
     bar = plo + kD * kD * 2;
     part = bar + 128;
     mu = part + 2 * kTile * 8;
-    bytes = (size_t)mu + 2 * kD * 4 + 1024;   // + slack to align the base to 1024
+    amx = mu + 2 * kD * 4;                   // [2][2][128] u32: the two groups' row amax halves
+    bytes = (size_t)amx + 2 * 2 * kTile * 4 + 1024;   // + slack to align the base to 1024
   }
 };
 static_assert(kD * 128 * 2 <= kStageBytes, "U fits in one input stage");
@@ -446,24 +447,28 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
       const size_t bh = (size_t)b * D.Hkv + h;
       const uint32_t d2 = lane_base + buf * 256, d1 = d2 + 128;
       float rs = 0.f, xs = 0.f;
-      if (CB < 16 && grp_a) {
-        // quantised rows: group A takes two TMEM passes over the coefficients
-        // (c = U^T x - U^T mu with a key mean), 32 columns per wait: the row's
-        // amax of bf16(c), then its codes and scale
+      if (CB < 16) {
+        // quantised rows: each group takes half of the coefficient columns (A
+        // the first Rh, B the rest) in two TMEM passes, 32 columns per wait
+        // (c = U^T x - U^T mu with a key mean): its part of the row's amax of
+        // bf16(c), exchanged through shared memory, then its codes; A stores
+        // the scale
         const size_t row = bh * D.T_cap + start + t;
+        const int Rh = ((R / 16 + 1) / 2) * 16;
+        const int cb0 = grp_a ? 0 : Rh, cb1 = grp_a ? Rh : R;
         // amax of the bf16 magnitudes, as a packed 16-bit unsigned max of their
         // bit patterns (the order of non-negative bf16 values)
         uint32_t am2 = 0u;
 #pragma unroll 1
-        for (int c0 = 0; c0 < R; c0 += 32) {
+        for (int c0 = cb0; c0 < cb1; c0 += 32) {
           float v[2][16];
 #pragma unroll
           for (int q = 0; q < 2; ++q)
-            if (c0 + 16 * q < R) tc5::tmem_ld16(d1 + c0 + 16 * q, v[q]);
+            if (c0 + 16 * q < cb1) tc5::tmem_ld16(d1 + c0 + 16 * q, v[q]);
           tc5::tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 2; ++q)
-            if (c0 + 16 * q < R)
+            if (c0 + 16 * q < cb1)
 #pragma unroll
               for (int k = 0; k < 16; k += 2) {
                 const float m0 = mug ? cmu[(c0 + 16 * q + k) & (kD - 1)] : 0.f;
@@ -472,20 +477,23 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
                 am2 = __vmaxu2(am2, pr & 0x7fff7fffu);
               }
         }
-        const float amax = __uint_as_float(max(am2 & 0xffffu, am2 >> 16) << 16);
+        uint32_t* amx = reinterpret_cast<uint32_t*>(sm + Lo.amx) + (i & 1) * 2 * kTile;
+        amx[(grp_a ? 0 : kTile) + m] = max(am2 & 0xffffu, am2 >> 16);
+        tc5::named_bar_sync(1, kEpi);   // both halves of every row's amax in
+        const float amax = __uint_as_float(max(amx[m], amx[kTile + m]) << 16);
         const float qs = quant_scale(amax, CB);
         const float qinv = qs > 0.f ? 1.f / qs : 0.f;
-        if (valid) scales[row] = qs;
+        if (grp_a && valid) scales[row] = qs;
 #pragma unroll 1
-        for (int c0 = 0; c0 < R; c0 += 32) {
+        for (int c0 = cb0; c0 < cb1; c0 += 32) {
           float v[2][16];
 #pragma unroll
           for (int q = 0; q < 2; ++q)
-            if (c0 + 16 * q < R) tc5::tmem_ld16(d1 + c0 + 16 * q, v[q]);
+            if (c0 + 16 * q < cb1) tc5::tmem_ld16(d1 + c0 + 16 * q, v[q]);
           tc5::tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
-            if (!valid || c0 + 16 * q >= R) continue;
+            if (!valid || c0 + 16 * q >= cb1) continue;
             uint32_t bw[8];
 #pragma unroll
             for (int k = 0; k < 16; k += 2) {
