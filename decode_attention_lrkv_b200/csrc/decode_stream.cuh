@@ -40,6 +40,7 @@
 // waiting on the preceding kernel of the stream (they are not written by the
 // kernels around a decode); the query, produced upstream, and every piece of
 // cache state (an append to the same cache may precede) are read after it.
+// Every CTA lets the next kernel launch right after its own base loads.
 #pragma once
 
 #include <type_traits>
@@ -439,6 +440,10 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     cp_async_commit();
   };
   load_uv();
+  // The next kernel of the stream may be launched now: its CTAs take SMs as
+  // this grid's CTAs leave and load their bases, and its wait still covers all
+  // of this grid (every CTA of it has started once all have passed here).
+  griddep_launch_dependents();
 
   // ---- after the preceding kernel of the stream: the query (produced upstream)
   // and the cache state (an append may precede), all loaded in one batch ----------
@@ -1101,7 +1106,6 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
     // copy in flight (a release waits for them); looked at after the record
     if (APP && tid == tk) seq_ticket = atom_add_release_gpu(p.seq_tickets + b, 1);
     __syncwarp();
-    griddep_launch_dependents();
 
     // ---- lift: of += U_v acc_c^T on the tensor cores --------------------------------
     // acc_c^T (rows = r_v, columns = head parts) becomes the B operand: lane
