@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
   const lrkv_bf16* Uqg = tensor == 0 && p.C.U_kq ? p.C.U_kq + (size_t)h * kD * R : nullptr;
   const float* mug = tensor == 0 && p.C.mu_k ? p.C.mu_k + (size_t)h * kD : nullptr;
   unsigned char* coef = static_cast<unsigned char*>(tensor == 0 ? p.C.coef_k : p.C.coef_v);
+  const bool coef32 = (reinterpret_cast<uintptr_t>(coef) & 31u) == 0;   // 32-byte stores allowed
   float* scales = tensor == 0 ? p.C.scale_k : p.C.scale_v;
   float* errs = p.errs + (size_t)tensor * D.B * D.Hkv * D.T_cap;
 
@@ -533,12 +534,18 @@ __global__ void __launch_bounds__(kThreads, 1) project_tc_kernel(const __grid_co
             if (!valid || c0 + 16 * q >= R) continue;
             const float* w = v[q];
             lrkv_bf16* crow = reinterpret_cast<lrkv_bf16*>(coef) + row * R;
-            *reinterpret_cast<uint4*>(crow + c0 + 16 * q) =
-                make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]), pack_bf16(w[4], w[5]),
-                           pack_bf16(w[6], w[7]));
-            *reinterpret_cast<uint4*>(crow + c0 + 16 * q + 8) =
-                make_uint4(pack_bf16(w[8], w[9]), pack_bf16(w[10], w[11]),
-                           pack_bf16(w[12], w[13]), pack_bf16(w[14], w[15]));
+            uint32_t pk[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) pk[e] = pack_bf16(w[2 * e], w[2 * e + 1]);
+            if (coef32) {   // 16 columns = 32 bytes in one store (rows are 32-byte multiples)
+              asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                           ::"l"(crow + c0 + 16 * q), "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]),
+                           "r"(pk[4]), "r"(pk[5]), "r"(pk[6]), "r"(pk[7])
+                           : "memory");
+            } else {
+              *reinterpret_cast<uint4*>(crow + c0 + 16 * q) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              *reinterpret_cast<uint4*>(crow + c0 + 16 * q + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
           }
         }
       }
