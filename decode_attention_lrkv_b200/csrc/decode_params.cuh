@@ -12,8 +12,11 @@ struct DecodeParams {
   const lrkv_bf16* q;
   float* out;
   int32_t* tickets;   // [B][Hkv]
-  float* partials;    // [B][Hkv][n_chunk_max][g][2 + r_v + d]
-  int n_chunk_max;    // splits per (b, kv head) in the grid (those of a full cache)
+  float* partials;    // [B][Hkv][n_chunk_max][g][4 + r_v + d]
+  int n_split;        // splits per (b, kv head) in the plain decode's grid (those of a full cache)
+  // records per (b, kv head), and the fused call's grid: its last CTA appends,
+  // the others hold at least the fewest splits any cached length needs
+  int n_chunk_max;
   // query heads per kv head (Hq / Hkv), and the first of this launch's: the
   // streaming kernel serves up to its template's G of them per launch
   int g_all;

@@ -30,8 +30,12 @@ bool stream_decode_supported(const lrkv_dims& D) {
 // passes of 4 (the last one partly empty), each streaming the cache once.
 int stream_heads_per_pass(int g) { return g <= 2 ? g : 4; }
 
+// Grid: the plain decode's splits, or the fused call's (its last CTA appends).
+static dim3 decode_grid(const DecodeParams& p) {
+  return dim3(p.k_new ? p.n_chunk_max : p.n_split, p.D.Hkv, p.D.B);
+}
+
 lrkv_status launch_decode(const DecodeParams& p0, cudaStream_t s) {
-  const dim3 grid(p0.n_chunk_max, p0.D.Hkv, p0.D.B);
   const int g = p0.D.Hq / p0.D.Hkv;
   if (stream_decode_supported(p0.D)) {
     DecodeParams p = p0;
@@ -44,6 +48,7 @@ lrkv_status launch_decode(const DecodeParams& p0, cudaStream_t s) {
         p.t_new_b = nullptr;
         p.err_out = nullptr;
       }
+      const dim3 grid = decode_grid(p);
       bool done = false;
       lrkv_status st = LRKV_OK;
       if (per == 1) st = launch_stream_g1(p, grid, s, &done);
@@ -55,7 +60,7 @@ lrkv_status launch_decode(const DecodeParams& p0, cudaStream_t s) {
     return LRKV_OK;
   }
   if (p0.k_new) return LRKV_ERR_UNSUPPORTED;
-  return launch_simple_any(p0, grid, s);
+  return launch_simple_any(p0, decode_grid(p0), s);
 }
 
 }  // namespace lrkv

@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_simple_kernel(DecodeParams
   int T = p.C.seq_len[b];
   T = T < 0 ? 0 : (T > D.T_cap ? D.T_cap : T);
   int chunk;   // positions per split, from the live length
-  const int n_chunks = decode_split(T, p.n_chunk_max, (long long)D.B * D.Hkv, p.num_sms, &chunk);
+  const int n_chunks = decode_split(T, p.n_split, (long long)D.B * D.Hkv, p.num_sms, &chunk);
   if (c >= n_chunks) return;
   const int r_k = D.r_k, r_v = D.r_v;
   const size_t bh = (size_t)b * D.Hkv + h;

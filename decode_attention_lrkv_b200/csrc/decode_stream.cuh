@@ -497,10 +497,11 @@ __global__ void __launch_bounds__(W * 32, 1) decode_stream_kernel(DecodeParams p
   // splits from the live length (every CTA of the (b, kv head) finds the same).
   // With a fused append the grid's last CTA does the append and nothing else
   // (its record joins the merge), so the stream never waits for it: the other
-  // CTAs split the T_old cached positions among the remaining n_chunk_max - 1.
+  // CTAs split the T_old cached positions among the remaining n_chunk_max - 1
+  // (at least the ceil(T_cap / kMaxDecodeChunk) splits any cached length needs).
   int chunk;
   const int n_chunks = APP ? decode_split(T_old, p.n_chunk_max - 1, (long long)D.B * D.Hkv, p.num_sms, &chunk)
-                           : decode_split(T, p.n_chunk_max, (long long)D.B * D.Hkv, p.num_sms, &chunk);
+                           : decode_split(T, p.n_split, (long long)D.B * D.Hkv, p.num_sms, &chunk);
   const bool is_app = APP && c == (int)gridDim.x - 1;   // the append CTA
   const bool streams = !is_app && c < n_chunks;
   const bool active = streams || is_app;

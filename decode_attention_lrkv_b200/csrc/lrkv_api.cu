@@ -105,6 +105,7 @@ lrkv_status lrkv_decode_attn(const lrkv_dims* dims, const lrkv_cache* cache, con
   p.out = out;
   p.tickets = reinterpret_cast<int32_t*>(w + L.decode_tickets);
   p.partials = reinterpret_cast<float*>(w + L.partials);
+  p.n_split = L.n_split;
   p.n_chunk_max = L.n_chunk_max;
   p.num_sms = num_sms();
   return launch_decode(p, s);
@@ -138,6 +139,7 @@ lrkv_status lrkv_append_decode_attn(const lrkv_dims* dims, const lrkv_cache* cac
   p.out = out;
   p.tickets = reinterpret_cast<int32_t*>(w + L.decode_tickets);
   p.partials = reinterpret_cast<float*>(w + L.partials);
+  p.n_split = L.n_split;
   p.n_chunk_max = L.n_chunk_max;
   p.num_sms = num_sms();
   p.k_new = k_new;

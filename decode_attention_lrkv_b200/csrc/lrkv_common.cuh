@@ -146,7 +146,8 @@ struct WsLayout {
   size_t partials;         // float [B][Hkv][n_chunk_max][g][4 + r_v + d]
   size_t total;
   int chunk;               // decode: positions per split of a full cache
-  int n_chunk_max;         // decode: splits per (b, kv head) in the grid
+  int n_split;             // decode: splits per (b, kv head) in the plain decode's grid
+  int n_chunk_max;         // decode: records per (b, kv head), the fused call's grid
   int partial_floats;      // floats per (split, q head)
 };
 
@@ -248,10 +249,15 @@ inline WsLayout ws_layout(const lrkv_dims& D) {
   off = align_up(off + sizeof(int32_t) * (size_t)D.B * D.Hkv * L.n_tiles, 256);
   L.tile_bits = off;
   off = align_up(off + sizeof(uint32_t) * 4 * (size_t)D.B * D.Hkv * L.n_tiles, 256);
-  // decode: the grid has the splits of a full cache (at least two: a fused
-  // append takes the last CTA); each CTA re-splits the live length
-  // (decode_split) within them
-  L.n_chunk_max = decode_split(D.T_cap, 1024, (long long)D.B * D.Hkv, num_sms(), &L.chunk);
+  // decode: the plain decode's grid has the splits of a full cache; each CTA
+  // re-splits the live length (decode_split) within them.  A fused append
+  // takes the last CTA of its grid, and the other CTAs must still hold the
+  // fewest splits a cached length can need (ceil(T_cap / kMaxDecodeChunk)), so
+  // its grid, and the records per (b, kv head), are one more than that when
+  // the plain grid has no CTA to spare.
+  L.n_split = decode_split(D.T_cap, 1024, (long long)D.B * D.Hkv, num_sms(), &L.chunk);
+  const int n_least = (D.T_cap + kMaxDecodeChunk - 1) / kMaxDecodeChunk;
+  L.n_chunk_max = L.n_split > n_least ? L.n_split : n_least + 1;
   if (L.n_chunk_max < 2) L.n_chunk_max = 2;
   L.partial_floats = 4 + D.r_v + D.d;   // m, l, pad, pad, acc_c[r_v], acc_f[d]
   L.partials = off;

@@ -88,6 +88,7 @@ extern "C" LRKV_API lrkv_status lrkv_decode_attn_noalloc(const lrkv_dims* dims,
   p.out = out;
   p.tickets = reinterpret_cast<int32_t*>(base);
   p.partials = reinterpret_cast<float*>(base + ticket_bytes);
+  p.n_split = L.n_split;
   p.n_chunk_max = L.n_chunk_max;
   p.num_sms = num_sms();
   return launch_decode(p, s);

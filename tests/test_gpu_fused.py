@@ -7,8 +7,9 @@ tau, list rows exact and in position order, the error output within 5e-5,
 seq_len and status words equal, and each step's output within
 ||o - o_ref||_inf / ||o_ref||_inf <= 2e-3 of the oracle attending over the
 cache after the append.  Also: the fused call and the two separate calls
-leave the same cache, rows with no token, full sequences, a full list, and a
-shape the streaming kernel does not cover (two launches).
+leave the same cache, rows with no token, full sequences, a full list, a
+split grid with no CTA to spare for the append, and a shape the streaming
+kernel does not cover (two launches).
 """
 import numpy as np
 import pytest
@@ -138,6 +139,27 @@ def test_fused_at_split_boundaries(T):
     for s in range(2):
         _, band, _ = _fused_both(D, cache, oc, Ka[:, s:s + 1].contiguous(),
                                  Va[:, s:s + 1].contiguous(), qs[s], w.tau, ws, band=band)
+
+
+def test_fused_when_the_split_grid_has_no_spare_cta():
+    """B * Hkv = 64 sequences-heads with T_cap = 8224: the split model gives a
+    full cache two splits of at most 8192 positions, and a cached length past
+    8192 needs both of them as well, so the fused call's grid holds a third CTA
+    for the append.  Two steps at cached lengths 8222 and 8223 attend to every
+    position and keep each (b, kv head)'s records apart."""
+    w = synth.workload(1, B=8, T=8222, layers=1)
+    layer, D, cache, oc, ws = _setup(w, seed=47, T_cap=8224, F_cap=2048)
+    _, band = _compress_both(D, cache, oc, layer["K"], layer["V"], w.tau, ws)
+    Ka, Va = synth.decode_tokens(w, layer["Qk"], layer["Qv"], 2, 47, 0, DEV)
+    qs = synth.decode_queries(w, 2, 47, 0, DEV)
+    for s in range(2):
+        gc, band, _ = _fused_both(D, cache, oc, Ka[:, s:s + 1].contiguous(),
+                                  Va[:, s:s + 1].contiguous(), qs[s], w.tau, ws, band=band)
+    assert (gc.seq_len == 8224).all()
+    out = torch.empty(D.B, D.Hq, D.d, dtype=torch.float32, device=DEV)   # and a plain decode of the full cache
+    L.lrkv_decode_attn(D, cache, qs[0], out, ws=ws)
+    torch.cuda.synchronize()
+    assert U.out_rel_err(U.f64(out), O.decode_attn(oc, U.f64(qs[0]))) <= U.OUT_RTOL
 
 
 def test_fused_on_an_empty_cache():
