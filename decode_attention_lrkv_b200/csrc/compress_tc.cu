@@ -147,11 +147,17 @@ lrkv_status compress_tc(const lrkv_dims& D, const lrkv_cache& C, const lrkv_bf16
   rp.n_tiles = L.n_tiles;
   rp.bh_tickets = reinterpret_cast<int32_t*>(w + L.decode_tickets);
   rp.ticket = reinterpret_cast<int32_t*>(w + L.compress_ticket);
+  // the scatter pass takes runs of tiles per CTA once the grid holds more than
+  // 16 CTAs per SM (a wave of 128-thread CTAs) twice over
+  const long long n_tiles_all = (long long)pp.tiles_per_b * D.Hkv * D.B;
+  long long tpc = n_tiles_all / (16LL * num_sms());
+  rp.tiles_per_cta = (int)(tpc < 1 ? 1 : tpc > ptc::kMaxScatterTiles ? ptc::kMaxScatterTiles : tpc);
   // the routing passes launch as dependents (programmatic dependent launch):
   // their launch overlaps the preceding kernel's tail, and each waits for it
   const dim3 grid(pp.tiles_per_b, D.Hkv, D.B);
+  const dim3 grid_s((pp.tiles_per_b + rp.tiles_per_cta - 1) / rp.tiles_per_cta, D.Hkv, D.B);
   if ((st = launch_pdl(ptc::route_count_kernel, grid, dim3(128), 0, s, rp)) != LRKV_OK) return st;
-  return launch_pdl(ptc::route_scatter_kernel, grid, dim3(128), 0, s, rp);
+  return launch_pdl(ptc::route_scatter_kernel, grid_s, dim3(128), 0, s, rp);
 }
 
 

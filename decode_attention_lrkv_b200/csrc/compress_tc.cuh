@@ -34,8 +34,11 @@
 // Kernel 3, route_scatter_kernel: the list slot of a routed token is the
 // list length before the call + routed tokens of earlier tiles (a block sum
 // over the tile counts) + earlier routed tokens of its tile (ballot prefix),
-// so the list stays in position order.  Rows are copied warp-cooperatively;
-// mask words are updated with atomics where tiles share a word.  The last CTA
+// so the list stays in position order.  A CTA takes a run of up to 8 tiles of
+// one (b, kv head) when the grid is large (fewer CTAs, fewer same-address
+// tickets); their kept rows are listed in shared memory and copied
+// warp-cooperatively, 8 rows per warp with every load before the first store.
+// Mask words are updated with atomics where tiles share a word.  The last CTA
 // of each (b, kv head) sets full_cnt; the last CTA of the grid advances seq_len.
 #pragma once
 
@@ -625,6 +628,7 @@ struct RouteParams {
   int32_t* tile_cnt;       // [B][Hkv][n_tiles]
   uint32_t* tile_bits;     // [B][Hkv][n_tiles][4]
   int n_tiles;
+  int tiles_per_cta;       // route_scatter_kernel: consecutive tiles per CTA, 1..kMaxScatterTiles
   int32_t* bh_tickets;     // [B][Hkv], zero between calls
   int32_t* ticket;         // [1], zero between calls
 };
@@ -638,6 +642,8 @@ __device__ __forceinline__ int route_eff(const RouteParams& p, int b, int* start
   *start = s0;
   return ne;
 }
+
+constexpr int kMaxScatterTiles = 8;
 
 // grid (tiles_per_b, Hkv, B), 128 threads
 __global__ void __launch_bounds__(128) route_count_kernel(RouteParams p) {
@@ -670,14 +676,16 @@ __global__ void __launch_bounds__(128) route_count_kernel(RouteParams p) {
   if (tid == 0) p.tile_cnt[bh * p.n_tiles + tile] = (s_cnt[0] + s_cnt[1]) + (s_cnt[2] + s_cnt[3]);
 }
 
-// grid (tiles_per_b, Hkv, B), 128 threads
+// grid (ceil(tiles_per_b / tiles_per_cta), Hkv, B), 128 threads: tiles
+// [x * tiles_per_cta, (x + 1) * tiles_per_cta) of one (b, kv head) per CTA
 __global__ void __launch_bounds__(128) route_scatter_kernel(RouteParams p) {
   griddep_wait();   // a dependent of the count pass
   const lrkv_dims& D = p.D;
-  const int tile = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   __shared__ int s_red[4];
-  __shared__ int s_wcnt[4];
+  __shared__ uint32_t s_bits[kMaxScatterTiles][4];
+  __shared__ int2 s_rows[kMaxScatterTiles * 128];   // kept rows in list order: (slot, token)
   __shared__ bool s_last_bh, s_last;
   uint32_t st = 0;
   int start;
@@ -685,83 +693,88 @@ __global__ void __launch_bounds__(128) route_scatter_kernel(RouteParams p) {
   const size_t bh = (size_t)b * D.Hkv + h;
   const int32_t* cnt = p.tile_cnt + bh * p.n_tiles;
   const int old = min(max(p.C.full_cnt[bh], 0), D.F_cap);
-  const int t0 = tile * 128;
+  const int tile_a = blockIdx.x * p.tiles_per_cta;
+  const int n_tl = max(0, min(p.tiles_per_cta, (ne + 127) / 128 - tile_a));   // tiles with new tokens
   bool overflow = false;
-  if (t0 < ne) {
+  if (n_tl > 0) {
     // routed tokens of the earlier tiles of this (b, kv head)
     int before = 0;
-    for (int i = tid; i < tile; i += 128) before += cnt[i];
+    for (int i = tid; i < tile_a; i += 128) before += cnt[i];
     before = (int)warp_sum((float)before);   // counts < 2^24: exact in fp32
     if (lane == 0) s_red[warp] = before;
-    const uint32_t wbits = p.tile_bits[(bh * p.n_tiles + tile) * 4 + warp];
-    if (lane == 0) s_wcnt[warp] = __popc(wbits);
+    if (tid < 4 * n_tl) s_bits[tid >> 2][tid & 3] = p.tile_bits[(bh * p.n_tiles + tile_a + (tid >> 2)) * 4 + (tid & 3)];
     __syncthreads();
-    const int base = old + (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
-    int wbefore = 0;
-    for (int w = 0; w < warp; ++w) wbefore += s_wcnt[w];
-    const int t = t0 + tid;
-    const bool valid = t < ne;
-    const bool routed = (wbits >> lane) & 1u;
-    const int slot = base + wbefore + __popc(wbits & ((1u << lane) - 1u));
-    const bool keep = routed && slot < D.F_cap;
-    overflow = routed && !keep;
-    const int pos = start + t;
-    if (keep) p.C.full_idx[bh * D.F_cap + slot] = pos;
-    // mask words: this warp's 32 positions span at most two words
-    const uint32_t keep_b = __ballot_sync(0xffffffffu, keep);
-    const uint32_t valid_b = __ballot_sync(0xffffffffu, valid);
-    if (lane == 0 && valid_b) {
-      uint32_t* mrow = p.C.route_mask + bh * (D.T_cap / 32);
-      const int p0 = start + t0 + warp * 32;
-      const int w0 = p0 >> 5, sh = p0 & 31;
-      const uint32_t r0 = valid_b << sh, k0 = keep_b << sh;
-      if (r0) {
-        if (r0 == 0xffffffffu) mrow[w0] = k0;
-        else {
-          atomicAnd(&mrow[w0], ~r0);
-          if (k0) atomicOr(&mrow[w0], k0);
+    const int base = old + (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);   // this CTA's first slot
+    int off = 0;   // routed tokens of this CTA's earlier tiles
+    for (int j = 0; j < n_tl; ++j) {
+      const int t0 = (tile_a + j) * 128;
+      const uint32_t wbits = s_bits[j][warp];
+      int wbefore = 0;
+      for (int w = 0; w < warp; ++w) wbefore += __popc(s_bits[j][w]);
+      const int t = t0 + tid;
+      const bool valid = t < ne;
+      const bool routed = (wbits >> lane) & 1u;
+      const int idx = off + wbefore + __popc(wbits & ((1u << lane) - 1u));   // slot - base
+      const int slot = base + idx;
+      const bool keep = routed && slot < D.F_cap;
+      overflow |= routed && !keep;
+      if (keep) {
+        p.C.full_idx[bh * D.F_cap + slot] = start + t;
+        s_rows[idx] = make_int2(slot, t);
+      }
+      // mask words: this warp's 32 positions span at most two words
+      const uint32_t keep_b = __ballot_sync(0xffffffffu, keep);
+      const uint32_t valid_b = __ballot_sync(0xffffffffu, valid);
+      if (lane == 0 && valid_b) {
+        uint32_t* mrow = p.C.route_mask + bh * (D.T_cap / 32);
+        const int p0 = start + t0 + warp * 32;
+        const int w0 = p0 >> 5, sh = p0 & 31;
+        const uint32_t r0 = valid_b << sh, k0 = keep_b << sh;
+        if (r0) {
+          if (r0 == 0xffffffffu) mrow[w0] = k0;
+          else {
+            atomicAnd(&mrow[w0], ~r0);
+            if (k0) atomicOr(&mrow[w0], k0);
+          }
+        }
+        if (sh) {
+          const uint32_t r1 = valid_b >> (32 - sh), k1 = keep_b >> (32 - sh);
+          if (r1) {
+            atomicAnd(&mrow[w0 + 1], ~r1);
+            if (k1) atomicOr(&mrow[w0 + 1], k1);
+          }
         }
       }
-      if (sh) {
-        const uint32_t r1 = valid_b >> (32 - sh), k1 = keep_b >> (32 - sh);
-        if (r1) {
-          atomicAnd(&mrow[w0 + 1], ~r1);
-          if (k1) atomicOr(&mrow[w0 + 1], k1);
-        }
-      }
+      off += (__popc(s_bits[j][0]) + __popc(s_bits[j][1])) + (__popc(s_bits[j][2]) + __popc(s_bits[j][3]));
     }
-    // copy the kept rows (32 lanes x 8 bytes per row), up to kBatch rows per
-    // pass with every load of the pass issued before its first store
+    __syncthreads();   // the kept rows are listed
+    // the kept rows are list entries [0, n_keep): slots are consecutive from base
+    const int n_keep = max(0, min(off, D.F_cap - base));
+    // copy them (32 lanes x 8 bytes per row): warp w takes rows [c0, c0 + 8)
+    // for c0 = 8w, 8w + 32, ..., every load of a batch issued before its first store
     constexpr int kBatch = 8;
-    uint32_t todo = keep_b;
-    const int wslot0 = base + wbefore;
-    while (todo) {
+    for (int c0 = warp * kBatch; c0 < n_keep; c0 += 4 * kBatch) {
       uint2 kr[kBatch], vr[kBatch];
-      int sl[kBatch];
 #pragma unroll
       for (int q = 0; q < kBatch; ++q) {
-        sl[q] = -1;
-        if (todo) {
-          const int src = __ffs(todo) - 1;
-          todo &= todo - 1;
-          const int ts = t0 + warp * 32 + src;
-          sl[q] = wslot0 + __popc(wbits & ((1u << src) - 1u));
-          const size_t x = (((size_t)b * p.t_new + ts) * D.Hkv + h) * kD;
+        if (c0 + q < n_keep) {
+          const size_t x = (((size_t)b * p.t_new + s_rows[c0 + q].y) * D.Hkv + h) * kD;
           kr[q] = reinterpret_cast<const uint2*>(p.k_new + x)[lane];
           vr[q] = reinterpret_cast<const uint2*>(p.v_new + x)[lane];
         }
       }
 #pragma unroll
       for (int q = 0; q < kBatch; ++q) {
-        if (sl[q] >= 0) {
-          reinterpret_cast<uint2*>(p.C.full_k + (bh * D.F_cap + sl[q]) * kD)[lane] = kr[q];
-          reinterpret_cast<uint2*>(p.C.full_v + (bh * D.F_cap + sl[q]) * kD)[lane] = vr[q];
+        if (c0 + q < n_keep) {
+          const size_t y = (bh * D.F_cap + s_rows[c0 + q].x) * kD;
+          reinterpret_cast<uint2*>(p.C.full_k + y)[lane] = kr[q];
+          reinterpret_cast<uint2*>(p.C.full_v + y)[lane] = vr[q];
         }
       }
     }
   }
   if (__syncthreads_or(overflow)) st |= LRKV_DEV_FULL_OVERFLOW;
-  if (tile == 0 && h == 0) {
+  if (blockIdx.x == 0 && h == 0) {
     uint32_t dummy = 0;
     const int n = new_tokens(p.t_new_b, b, p.t_new, &dummy);
     if (ne < n) st |= LRKV_DEV_SEQ_OVERFLOW;

@@ -229,6 +229,25 @@ def test_prefill_in_two_parts_unaligned_start():
     assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
 
 
+def test_scatter_with_runs_of_tiles_per_cta():
+    """A prefill of 4 x 8 (b, kv head) pairs x 150 tiles of 128 tokens: more
+    than twice a wave of 128-thread CTAs on a 148-SM part, so the scatter pass
+    gives each CTA a run of tiles.  Ragged rows, a start mid mask word, and a
+    list that fills up partway through the runs (FULL_OVERFLOW)."""
+    w = synth.workload(1, B=4, T=19237, layers=1)
+    layer, D, cache, oc, ws = _setup(w, seed=53, T_cap=19264, F_cap=1200)
+    K, V = layer["K"], layer["V"]
+    cut = 37
+    gc, band = _compress_both(D, cache, oc, K[:, :cut].contiguous(), V[:, :cut].contiguous(),
+                              w.tau, ws)
+    gc, band = _compress_both(D, cache, oc, K[:, cut:].contiguous(), V[:, cut:].contiguous(),
+                              w.tau, ws, t_new_b=[19200, 18000, 19100, 17500], band=band)
+    assert gc.status & L.DEV_FULL_OVERFLOW
+    assert list(gc.seq_len) == [19237, 18037, 19137, 17537]
+    out = U.f64(U.gpu_decode(D, cache, layer["q"], ws))
+    assert U.out_rel_err(out, O.decode_attn(gc, U.f64(layer["q"]))) <= U.OUT_RTOL
+
+
 @pytest.mark.parametrize("Hq,Hkv,r_k,r_v", [(16, 8, 48, 80), (4, 2, 64, 64), (6, 2, 48, 64),
                                             (16, 2, 32, 32), (20, 4, 64, 96), (8, 8, 32, 48),
                                             (6, 2, 32, 48), (16, 2, 32, 48)],
