@@ -97,6 +97,37 @@ def _call_decode(lib, dims, cache, q=0x20000000, out=0x30000000, ws=0x40000000, 
                                 None)
 
 
+def _decode_records(D):
+    """Split records per (b, kv head) in lrkv_workspace_size(D): the decode's
+    region comes last, after the decode tickets, the compress ticket, the row
+    tickets, the prefill's per-token errors and its per-tile counts and bits
+    (each region rounded up to 256 bytes), and holds
+    [B][Hkv][records][g][4 + r_v + d] fp32, g raised to 4 for groups of 3."""
+    a = lambda x: (x + 255) // 256 * 256
+    bh = D.B * D.Hkv
+    n_tiles = (D.T_cap + 127) // 128
+    fixed = a(4 * bh) + a(4) + a(4 * D.B) + a(8 * bh * D.T_cap) + a(4 * bh * n_tiles) + a(16 * bh * n_tiles)
+    g = D.Hq // D.Hkv
+    g = 4 if 2 < g < 4 else g
+    return (L.lrkv_workspace_size(D) - fixed) // (4 * bh * g * (4 + D.r_v + D.d))
+
+
+def test_decode_records_hold_the_fewest_splits_and_the_append(lib):
+    """A fused append + decode streams the cached positions over at most
+    records - 1 splits of at most 8192 positions (its grid's last CTA appends),
+    so for any cached length up to T_cap the workspace must hold
+    ceil(T_cap / 8192) + 1 records per (b, kv head).  The cases include T_cap
+    just past a multiple of 8192 with many (b, kv head) pairs, where the split
+    model gives a full cache exactly ceil(T_cap / 8192) splits (no SMs are
+    visible here: the model assumes 148)."""
+    for B, Hkv in ((1, 1), (1, 8), (2, 8), (8, 8), (16, 8), (1, 32), (64, 8)):
+        for T_cap in (32, 8192, 8224, 16416, 24608, 65568, 131136, 139296):
+            D = _dims(B=B, Hkv=Hkv, Hq=4 * Hkv, T_cap=T_cap, F_cap=32)
+            assert _decode_records(D) >= -(-T_cap // 8192) + 1, (B, Hkv, T_cap)
+    # the shape that needs the extra record: the model gives 8224 positions two splits
+    assert _decode_records(_dims(B=8, Hkv=8, Hq=32, T_cap=8224, F_cap=32)) == 3
+
+
 def test_host_validation_rejects_before_launch(lib):
     D = _dims()
     C = _FakeCache()
