@@ -1,7 +1,8 @@
 """Benchmark: compressed-KV decode attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 4] [--t-cap T] [--no-cpu-baseline]
+                    [--workload 0..4] [--layers L] [--context T] [--t-cap T]
+                    [--quant 8|4] [--aware] [--seed S] [--no-cpu-baseline] [--no-clocks]
 
 The default workload is the largest one-GPU configuration: LLaMA-7B attention
 geometry (32 layers x 32 kv heads, MHA), 131072 tokens of context, ranks 48/64.
